@@ -1,0 +1,241 @@
+"""Pins of the oracle's 8-bit matrix products, the dequantizing epilogue, the
+composed Linear forward / dgrad and the SVDQuant branch."""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import svdquant
+
+
+def _rand_i8(shape, seed):
+    return np.random.default_rng(seed).integers(-128, 128, size=shape).astype(np.int8)
+
+
+# --------------------------------------------------------------------------- int GEMM
+def test_gemm_i8_bruteforce_tiny(orc):
+    A = _rand_i8((3, 5), 1)
+    B = _rand_i8((4, 5), 2)
+    acc = orc.gemm_i8_nt(A.view(np.uint8), B.view(np.uint8))
+    for m in range(3):
+        for n in range(4):
+            assert acc[m, n] == sum(int(A[m, k]) * int(B[n, k]) for k in range(5))
+
+
+@pytest.mark.parametrize("M,N,K", [(7, 9, 33), (64, 48, 256), (1, 300, 1024)])
+def test_gemm_i8_vs_numpy_int64(orc, M, N, K):
+    A = _rand_i8((M, K), M)
+    B = _rand_i8((N, K), N)
+    ref = A.astype(np.int64) @ B.astype(np.int64).T
+    assert np.array_equal(orc.gemm_i8_nt(A.view(np.uint8), B.view(np.uint8)), ref.astype(np.int32))
+    # contraction along B's rows (dgrad form): A2 [M,N] x B [N,K]
+    A2 = _rand_i8((M, N), K)
+    ref2 = A2.astype(np.int64) @ B.astype(np.int64)
+    assert np.array_equal(orc.gemm_i8_nn(A2.view(np.uint8), B.view(np.uint8)), ref2.astype(np.int32))
+
+
+def test_gemm_i8_int32_range_check(orc):
+    K = 140000   # 127*127*K > 2^31 - 1
+    A = np.full((1, K), 127, np.int8)
+    with pytest.raises(OverflowError):
+        orc.gemm_i8_nt(A.view(np.uint8), A.view(np.uint8))
+    # 12288 (the largest contraction of the DiT shapes) stays well inside
+    A = np.full((1, 12288), -127, np.int8)
+    assert orc.gemm_i8_nt(A.view(np.uint8), A.view(np.uint8))[0, 0] == 127 * 127 * 12288
+
+
+# --------------------------------------------------------------------------- e4m3 GEMM
+def test_gemm_e4m3_vs_numpy(orc):
+    rng = np.random.default_rng(3)
+    A = rng.integers(0, 256, size=(20, 96)).astype(np.uint8)
+    B = rng.integers(0, 256, size=(12, 96)).astype(np.uint8)
+    A[(A & 0x7F) == 0x7F] = 0x38   # no NaN codes
+    B[(B & 0x7F) == 0x7F] = 0x38
+    a = orc.e4m3_to_f32(A).astype(np.float64)
+    b = orc.e4m3_to_f32(B).astype(np.float64)
+    acc, absacc = orc.gemm_e4m3_nt(A, B)
+    assert np.allclose(acc, a @ b.T, rtol=1e-13, atol=1e-300)
+    assert np.allclose(absacc, np.abs(a) @ np.abs(b).T, rtol=1e-13)
+    acc2, _ = orc.gemm_e4m3_nn(A[:, :12], B[:, :50])
+    assert np.allclose(acc2, a[:, :12] @ b[:, :50], rtol=1e-13, atol=1e-300)
+
+
+# --------------------------------------------------------------------------- epilogue
+def _fp32_round(fr: Fraction) -> np.float32:
+    """Exact rational -> nearest fp32 (ties to even), via exact comparison."""
+    f = np.float32(float(fr))          # within one ulp; fix by exact comparison
+    lo = np.nextafter(f, np.float32(-np.inf))
+    hi = np.nextafter(f, np.float32(np.inf))
+    best = min((lo, f, hi), key=lambda c: (abs(Fraction(float(c)) - fr),
+                                           int(np.float32(c).view(np.uint32)) & 1))
+    return np.float32(best)
+
+
+def test_epilogue_closed_form(orc):
+    # powers of two and small integers: exact in every order
+    acc = np.array([[1000, -3, 0]], np.int32)
+    y, y32 = orc.epilogue(acc, np.float32([0.5]), np.float32([0.25]),
+                          workloads.to_u16(torch.tensor([1.0, 2.0, -1.5]).to(torch.bfloat16)))
+    assert y32.tolist() == [[126.0, 1.625, -1.5]]
+    # the fp64 (e4m3) form: same closed form
+    y, y32 = orc.epilogue(np.array([[1000.0, -3.0, 0.0]]), np.float32([0.5]), np.float32([0.25]),
+                          workloads.to_u16(torch.tensor([1.0, 2.0, -1.5]).to(torch.bfloat16)))
+    assert y32.tolist() == [[126.0, 1.625, -1.5]]
+
+
+def test_epilogue_rounds_each_operation(orc):
+    """((acc * s_row) * s_w) + bias with every step rounded to fp32 on its own:
+    checked against exact rational arithmetic rounded step by step."""
+    rng = np.random.default_rng(7)
+    acc = rng.integers(-2 ** 20, 2 ** 20, size=(16, 8)).astype(np.int32)
+    s_row = (rng.random(16).astype(np.float32) / np.float32(127))
+    s_w = np.float32([0.0123]) / np.float32(127)
+    bias_f = torch.tensor(rng.standard_normal(8) * 0.01, dtype=torch.float32).to(torch.bfloat16)
+    y, y32 = orc.epilogue(acc, s_row, s_w, workloads.to_u16(bias_f))
+    bias = bias_f.float().numpy()
+    for m in range(16):
+        for n in range(8):
+            t = _fp32_round(Fraction(int(acc[m, n])) * Fraction(float(s_row[m])))
+            u = _fp32_round(Fraction(float(t)) * Fraction(float(s_w[0])))
+            v = _fp32_round(Fraction(float(u)) + Fraction(float(bias[n])))
+            assert y32[m, n] == v, (m, n)
+    assert np.array_equal(y, orc.f32_to_bf16(y32))
+
+
+def test_epilogue_axis_scale_indexes_columns(orc):
+    acc = np.ones((2, 3), np.int32)
+    _, y32 = orc.epilogue(acc, np.float32([1.0, 2.0]), np.float32([1.0, 4.0, 16.0]))
+    assert y32.tolist() == [[1.0, 4.0, 16.0], [2.0, 8.0, 32.0]]
+
+
+# --------------------------------------------------------------------------- composed Linear
+def _integer_operands(M, N, K, seed):
+    """bf16 integer matrices whose every X row and W reach |127|: the token
+    scales and the tensor scale are exactly 1, so the W8A8 Linear reduces to
+    the textbook integer matmul."""
+    rng = np.random.default_rng(seed)
+    X = rng.integers(-127, 128, size=(M, K)).astype(np.float32)
+    X[:, 0] = 127.0
+    W = rng.integers(-127, 128, size=(N, K)).astype(np.float32)
+    W[0, 1] = -127.0
+    to = lambda a: workloads.to_u16(torch.from_numpy(a).to(torch.bfloat16))
+    return X, W, to(X), to(W)
+
+
+def test_linear_fwd_reduces_to_integer_matmul(orc):
+    M, N, K = 5, 7, 64      # non-square: a transposed operand cannot pass
+    X, W, xu, wu = _integer_operands(M, N, K, 8)
+    wq, sw = orc.quantize_weight(wu, orc.INT8, orc.TENSOR)
+    assert sw[0] == 1.0
+    out = orc.linear_fwd(xu, wq, sw)
+    ref = X.astype(np.int64) @ W.astype(np.int64).T
+    assert np.array_equal(out["acc"], ref)
+    assert np.all(out["sx"] == 1.0)
+    assert np.array_equal(out["y"], orc.f32_to_bf16(ref.astype(np.float32)))
+
+
+def test_linear_fwd_e4m3_reduces_to_float_matmul(orc):
+    """e4m3 with unit scales: codes of the e4m3 grid values come back exactly."""
+    rng = np.random.default_rng(9)
+    grid = orc.e4m3_to_f32(np.arange(0x30, 0x7F, dtype=np.uint8))   # 0.5 .. 448
+    X = rng.choice(np.concatenate([grid, -grid]), size=(4, 32)).astype(np.float32)
+    X[:, 3] = 448.0
+    W = rng.choice(np.concatenate([grid, -grid]), size=(6, 32)).astype(np.float32)
+    W[2, 2] = -448.0
+    to = lambda a: workloads.to_u16(torch.from_numpy(a).to(torch.bfloat16))
+    wq, sw = orc.quantize_weight(to(W), orc.E4M3, orc.TENSOR)
+    assert sw[0] == 1.0
+    out = orc.linear_fwd(to(X), wq, sw, qt=orc.E4M3)
+    ref = X.astype(np.float64) @ W.astype(np.float64).T
+    assert np.array_equal(out["acc"], ref)
+
+
+def test_linear_dgrad_reduces_to_integer_matmul(orc):
+    M, N, K = 6, 40, 24
+    dY, Wt, dyu, _ = _integer_operands(M, K, N, 10)    # dY [M,N], Wt [K,N]
+    W = np.ascontiguousarray(Wt.T)                      # W [N,K]
+    wu = workloads.to_u16(torch.from_numpy(W).to(torch.bfloat16))
+    wq, sw = orc.quantize_weight(wu, orc.INT8, orc.TENSOR)
+    assert sw[0] == 1.0
+    out = orc.linear_dgrad(dyu, wq, sw)
+    ref = dY.astype(np.int64) @ W.astype(np.int64)     # [M,N] x [N,K]
+    assert np.array_equal(out["acc"], ref)
+
+
+def test_dgrad_equals_forward_with_transposed_weight(orc):
+    """dgrad(dY, Wq) == forward GEMM against an explicit copy of Wq^T."""
+    dy = workloads.to_u16(workloads.normal((33, 80), 1e-3, 11))
+    wu = workloads.to_u16(workloads.normal((80, 48), 0.02, 12))
+    wq, sw = orc.quantize_weight(wu, orc.INT8, orc.TENSOR)
+    d = orc.linear_dgrad(dy, wq, sw)
+    f = orc.linear_fwd(dy, np.ascontiguousarray(wq.T), sw)
+    assert np.array_equal(d["acc"], f["acc"]) and np.array_equal(d["y"], f["y"])
+
+
+def test_linear_fwd_error_vs_bf16_matmul(orc):
+    """W8A8 error sanity: relative Frobenius error of the int8 Linear against
+    the fp64 product of the bf16 inputs stays at the 8-bit level."""
+    x = workloads.normal((64, 512), 1.0, 13)
+    w = workloads.normal((96, 512), 0.02, 14)
+    wq, sw = orc.quantize_weight(workloads.to_u16(w), orc.INT8, orc.TENSOR)
+    out = orc.linear_fwd(workloads.to_u16(x), wq, sw)
+    ref = x.double().numpy() @ w.double().numpy().T
+    rel = np.linalg.norm(out["y32"] - ref) / np.linalg.norm(ref)
+    assert 1e-3 < rel < 3e-2
+
+
+# --------------------------------------------------------------------------- SVDQuant
+def test_lowrank_vs_numpy(orc):
+    x = workloads.normal((9, 64), 1.0, 15)
+    l1 = workloads.normal((64, 8), 0.1, 16)
+    l2 = workloads.normal((8, 40), 0.1, 17)
+    t, t64 = orc.lowrank_down(workloads.to_u16(x), workloads.to_u16(l1))
+    ref = x.double().numpy() @ l1.double().numpy()
+    assert np.allclose(t64, ref, rtol=1e-12, atol=1e-15)
+    tb = torch.from_numpy(t.view(np.int16)).view(torch.bfloat16)
+    assert torch.equal(tb, torch.from_numpy(t64.astype(np.float32)).to(torch.bfloat16))
+    lr, lr_abs = orc.lowrank_up(t, workloads.to_u16(l2))
+    ref2 = tb.double().numpy() @ l2.double().numpy()
+    assert np.allclose(lr, ref2, rtol=1e-12, atol=1e-15)
+
+
+def test_svdq_zero_factors_is_int_linear(orc):
+    x = workloads.to_u16(workloads.with_outlier_channels((16, 256), 1.0, 18))
+    w = workloads.to_u16(workloads.normal((64, 256), 0.02, 19))
+    rq, sr = orc.quantize_weight(w, orc.INT8, orc.TENSOR)
+    z1 = np.zeros((256, 32), np.uint16)
+    z2 = np.zeros((32, 64), np.uint16)
+    s = orc.svdq_linear_fwd(x, rq, sr, z1, z2)
+    f = orc.linear_fwd(x, rq, sr)
+    assert np.array_equal(s["y"], f["y"])
+
+
+def test_svdq_split_reduces_weight_error(orc):
+    """With a rank-8 spike, the low-rank branch plus the int8 residual is a
+    better approximation of W than plain tensor-wise int8."""
+    w = workloads.rank_spike_weight(256, 320, 8, 0.5, 0.02, 20)
+    wu = workloads.to_u16(w)
+    prep = svdquant.prepare(wu, 32)
+    W = w.double().numpy()
+    lowrank = (orc.bf16_to_f32(prep["l1"]).astype(np.float64)
+               @ orc.bf16_to_f32(prep["l2"]).astype(np.float64)).T
+    deq_r = prep["rq"].view(np.int8).astype(np.float64) * prep["s_r"][0]
+    err_svd = np.linalg.norm(W - lowrank - deq_r)
+    wq, sw = orc.quantize_weight(wu, orc.INT8, orc.TENSOR)
+    err_plain = np.linalg.norm(W - wq.view(np.int8).astype(np.float64) * sw[0])
+    assert err_svd < 0.5 * err_plain
+    # the residual no longer holds the spike: its absmax is at the noise level
+    assert np.abs(orc.bf16_to_f32(prep["resid"])).max() < 0.2
+
+
+def test_svdq_exact_lowrank_weight(orc):
+    """A weight that is exactly rank 4 (bf16 factors, products exact) leaves a
+    residual at the bf16 rounding level."""
+    a = workloads.normal((48, 4), 0.25, 21).double()
+    b = workloads.normal((4, 40), 0.25, 22).double()
+    w = (a @ b).T.to(torch.bfloat16)     # [N=40, K=48]
+    prep = svdquant.prepare(workloads.to_u16(w), 8)
+    resid = orc.bf16_to_f32(prep["resid"])
+    assert np.abs(resid).max() < 0.02 * np.abs(w.float().numpy()).max()
