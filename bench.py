@@ -1,0 +1,501 @@
+#!/usr/bin/env python
+"""Benchmark of the W8A8 quantized Linear on B200.
+
+One step = the int W8A8 DiT MLP block, forward and input gradient, at
+M = 4608 tokens (4096 image + 512 text), hidden 3072, MLP 12288:
+    Y1  = Lin(X,   W1)    3072 -> 12288        quantize_rows + int8 GEMM
+    Y2  = Lin(Y1,  W2)    12288 -> 3072        quantize_rows + int8 GEMM
+    dX2 = Q(dY2) Q(W2)    dgrad                quantize_rows + int8 GEMM (MN-major W)
+    dX1 = Q(dX2) Q(W1)    dgrad                quantize_rows + int8 GEMM (MN-major W)
+with the weights quantized tensor-wise once, outside the timed region.
+Metric: TOPS = 4 * 2*M*N*K / step time (quant + GEMM + epilogue).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs the same per-GPU workload on its own seeded
+tokens (weak scaling, no data-path collective); the step time is the max over
+ranks.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W8A8 linear TOPS (quant+GEMM+epilogue) at DiT shapes; % of int8/fp8 TC peak"
+UNIT = "TOPS"
+M_TOK, HID, MLP = 4608, 3072, 12288
+OPS_PER_GEMM = 2 * M_TOK * HID * MLP
+OPS_PER_STEP = 4 * OPS_PER_GEMM
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic of one launch of the dominant kernel from an ncu capture, keyed
+# by the hash of the kernel source it was taken on (null when they differ).
+GEMM_TRAFFIC = {"source_sha": None, "bytes_per_launch": None, "note": ""}
+
+
+def gemm_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("gemm.cuh", "device.cuh"):
+        with open(os.path.join(ROOT, "w8a8_quantized_linear_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling of one GPU during the timed region."""
+    QUERY = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.out = ""
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    @staticmethod
+    def parse(text):
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        rows = [[c.strip() for c in r] for r in csv.reader(io.StringIO(text or "")) if len(r) >= 7]
+        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
+        mx = [num(r[1]) for r in rows if num(r[1]) is not None]
+        pw = [num(r[2]) for r in rows if num(r[2]) is not None]
+        reasons = sorted({ClockSampler.NAMES[i] for r in rows for i in range(4) if r[3 + i].lower() == "active"})
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        load = [v for v in sm if v >= 0.3 * max(mx or sm)] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None, "reasons": reasons, "samples": len(rows)}
+
+    def summary(self):
+        return self.parse(self.out)
+
+
+def gpu_selector(torch, dev) -> str:
+    """nvidia-smi -i argument for a torch device: its UUID, else its index."""
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        if u:
+            return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        pass
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [v for v in vis.split(",") if v.strip()]
+    idx = dev.index or 0
+    return ids[idx].strip() if idx < len(ids) else str(idx)
+
+
+# ----------------------------------------------------------------------------- oracle (CPU)
+def oracle_chain_rows(orc, wl, W1r, s1r, W2r, s2r, rows):
+    """The step on the CPU oracle for a subset of token rows (every step is
+    row-local).  Returns the int ops of the sample."""
+    import workloads
+    x = workloads.to_u16(wl["x"])[rows]
+    dy = workloads.to_u16(wl["dy2"])[rows]
+    r1 = orc.linear_fwd(x, W1r, s1r)
+    orc.linear_fwd(r1["y"], W2r, s2r)
+    g2 = orc.linear_dgrad(dy, W2r, s2r)
+    orc.linear_dgrad(g2["y"], W1r, s1r)
+    return 4 * 2 * len(rows) * HID * MLP
+
+
+def oracle_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def time_oracle(orc, wl, W1r, s1r, W2r, s2r, target_s):
+    import numpy as np
+    probe = np.arange(16)
+    t0 = time.perf_counter()
+    oracle_chain_rows(orc, wl, W1r, s1r, W2r, s2r, probe)
+    dt = time.perf_counter() - t0
+    n = int(min(M_TOK, max(16, 16 * target_s / max(dt, 1e-3))))
+    rows = np.linspace(0, M_TOK - 1, n).astype(np.int64)
+    t0 = time.perf_counter()
+    ops = oracle_chain_rows(orc, wl, W1r, s1r, W2r, s2r, rows)
+    dt = time.perf_counter() - t0
+    return ops / dt / 1e12, n, dt
+
+
+def oracle_weights(orc, wl):
+    import workloads
+    W1r, s1r = orc.quantize_weight(workloads.to_u16(wl["w1"]), orc.INT8, orc.TENSOR)
+    W2r, s2r = orc.quantize_weight(workloads.to_u16(wl["w2"]), orc.INT8, orc.TENSOR)
+    return W1r, s1r, W2r, s2r
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import oracle as orc
+    import workloads
+    orc.build()
+    wl = workloads.dit_mlp()
+    W1r, s1r, W2r, s2r = oracle_weights(orc, wl)
+    import numpy as np
+    # size each step so that warmup + steps end within about two minutes
+    probe = np.arange(8)
+    t0 = time.perf_counter()
+    oracle_chain_rows(orc, wl, W1r, s1r, W2r, s2r, probe)
+    per_row = (time.perf_counter() - t0) / 8
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    n = int(min(M_TOK, max(8, budget / max(per_row, 1e-6))))
+    rows = np.linspace(0, M_TOK - 1, n).astype(np.int64)
+    for _ in range(args.warmup):
+        oracle_chain_rows(orc, wl, W1r, s1r, W2r, s2r, rows)
+    t0 = time.perf_counter()
+    ops = 0
+    for _ in range(args.steps):
+        ops += oracle_chain_rows(orc, wl, W1r, s1r, W2r, s2r, rows)
+    dt = time.perf_counter() - t0
+    value = ops / dt / 1e12
+    sample = "%d of %d token rows per step (row-local step), all 4 GEMMs with quantize + epilogue" % (n, M_TOK)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+            "data": "synthetic", "config": workload_config(),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_cores(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config():
+    return {"workload": "int W8A8 DiT MLP block fwd+dgrad (up 3072->12288, down 12288->3072, "
+                        "dgrad through both), tensor-wise int8 W, token-wise int8 activations",
+            "M": M_TOK, "hidden": HID, "mlp": MLP, "global_batch_tokens_per_gpu": M_TOK,
+            "parallelism": "token-sharded replicas", "l2": "flushed (256 MiB write) between timed steps"}
+
+
+# ----------------------------------------------------------------------------- ours
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import workloads
+    import w8a8_quantized_linear_b200 as w8
+    from w8a8_quantized_linear_b200 import _build
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        dist = dist_mod
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if rank == 0:
+        _build.build()
+    if dist is not None:
+        dist.barrier()
+    w8.lib()
+
+    wl = workloads.dit_mlp()
+    if rank > 0:   # each rank its own tokens (weak scaling)
+        wl["x"] = workloads.with_outlier_channels((M_TOK, HID), 1.0, 21 + 1000 * rank)
+        wl["dy2"] = workloads.normal((M_TOK, HID), 1e-3, 24 + 1000 * rank)
+    X = wl["x"].to(dev)
+    dY2 = wl["dy2"].to(dev)
+    W1q, s1 = w8.quantize_weight(wl["w1"].to(dev), "int8", "tensor")
+    W2q, s2 = w8.quantize_weight(wl["w2"].to(dev), "int8", "tensor")
+    # pre-allocated codes, scales, outputs (no allocation inside the step)
+    u8 = lambda *s: torch.empty(*s, dtype=torch.int8, device=dev)
+    f32 = lambda *s: torch.empty(*s, dtype=torch.float32, device=dev)
+    b16 = lambda *s: torch.empty(*s, dtype=torch.bfloat16, device=dev)
+    xq1, sx1, Y1 = u8(M_TOK, HID), f32(M_TOK), b16(M_TOK, MLP)
+    xq2, sx2, Y2 = u8(M_TOK, MLP), f32(M_TOK), b16(M_TOK, HID)
+    gq2, sg2, dX2 = u8(M_TOK, HID), f32(M_TOK), b16(M_TOK, MLP)
+    gq1, sg1, dX1 = u8(M_TOK, MLP), f32(M_TOK), b16(M_TOK, HID)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    E = lambda: torch.cuda.Event(enable_timing=True)
+
+    def step(ev):
+        """ev: list of 10 events -> [start, q1, g1, q2, g2, q3, g3, q4, g4] boundaries."""
+        ev[0].record(stream)
+        w8.quantize_rows(X, "int8", out=xq1, scale=sx1); ev[1].record(stream)
+        w8.qgemm_fwd(xq1, sx1, W1q, s1, out=Y1); ev[2].record(stream)
+        w8.quantize_rows(Y1, "int8", out=xq2, scale=sx2); ev[3].record(stream)
+        w8.qgemm_fwd(xq2, sx2, W2q, s2, out=Y2); ev[4].record(stream)
+        w8.quantize_rows(dY2, "int8", out=gq2, scale=sg2); ev[5].record(stream)
+        w8.qgemm_dgrad(gq2, sg2, W2q, s2, out=dX2); ev[6].record(stream)
+        w8.quantize_rows(dX2, "int8", out=gq1, scale=sg1); ev[7].record(stream)
+        w8.qgemm_dgrad(gq1, sg1, W1q, s1, out=dX1); ev[8].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step([E() for _ in range(9)])
+    torch.cuda.synchronize()
+    assert w8.device_status() == 0, "device-side error during warm-up"
+
+    events = [[E() for _ in range(9)] for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_selector(torch, dev)) as clk:
+        wall0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)          # L2 flush, outside the step's events
+            step(events[i])
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+    if dist is not None:
+        dist.barrier()
+    step_ms = [ev[0].elapsed_time(ev[8]) for ev in events]
+    gemm_ms = [ev[k - 1].elapsed_time(ev[k]) for ev in events for k in (2, 4, 6, 8)]
+    quant_ms = [ev[k - 1].elapsed_time(ev[k]) for ev in events for k in (1, 3, 5, 7)]
+    total_ms = sum(step_ms)
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * OPS_PER_STEP * args.steps / (total_ms * 1e-3) / 1e12
+    assert w8.device_status() == 0, "device-side error during the timed steps"
+
+    # ---- end to end: pinned host inputs -> public API -> host result
+    e2e = None
+    if args.e2e_steps > 0:
+        hx = wl["x"].pin_memory()
+        hdy = wl["dy2"].pin_memory()
+        hy2 = torch.empty((M_TOK, HID), dtype=torch.bfloat16).pin_memory()
+        hdx1 = torch.empty((M_TOK, HID), dtype=torch.bfloat16).pin_memory()
+        ws = torch.empty(w8.workspace_bytes(w8.OP_LINEAR_FWD, M_TOK, MLP, MLP), dtype=torch.uint8, device=dev)
+        Xd, dYd = torch.empty_like(X), torch.empty_like(dY2)
+
+        def e2e_step():
+            Xd.copy_(hx, non_blocking=True)
+            dYd.copy_(hdy, non_blocking=True)
+            w8.linear_fwd(Xd, W1q, s1, out=Y1, ws=ws)
+            w8.linear_fwd(Y1, W2q, s2, out=Y2, ws=ws)
+            w8.linear_dgrad(dYd, W2q, s2, out=dX2, ws=ws)
+            w8.linear_dgrad(dX2, W1q, s1, out=dX1, ws=ws)
+            hy2.copy_(Y2, non_blocking=True)
+            hdx1.copy_(dX1, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        a, b = E(), E()
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b)
+        if dist is not None:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * OPS_PER_STEP * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": hx.numel() * 2 + hdy.numel() * 2,
+               "d2h_bytes_per_step": hy2.numel() * 2 + hdx1.numel() * 2,
+               "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps,
+               "api": "w8a8_linear_fwd x2 + w8a8_linear_dgrad x2 (pinned host buffers, copies timed)"}
+
+    if rank != 0:
+        return 0
+
+    peaks, src = load_peaks()
+    int8_peak = 2.0 * peaks["bf16_tflops_sustained"]   # int8 dense = 2 x bf16 dense (4.5 vs 2.25 PFLOP/s nominal)
+    gemm_avg = statistics.mean(gemm_ms)
+    achieved = OPS_PER_GEMM / (gemm_avg * 1e-3) / 1e12
+    sha = gemm_source_sha()
+    traffic = GEMM_TRAFFIC["bytes_per_launch"] if GEMM_TRAFFIC["source_sha"] == sha else None
+    roofline = {"bound": "tensor", "kernel": "gemm_kernel<i8> (tcgen05 kind::i8, fused epilogue)",
+                "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved / int8_peak,
+                "traffic": traffic,
+                "peak_source": "%s: 2 x bf16_tflops_sustained (int8 dense = 2x bf16 dense nominal)" % src,
+                "frac_of_burst": achieved / (2.0 * peaks["bf16_tflops"]),
+                "gemm_ms_avg": gemm_avg, "quantize_ms_avg": statistics.mean(quant_ms),
+                "quantize_share": sum(quant_ms) / sum(step_ms)}
+    clocks = clk.summary()
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic", "config": workload_config(),
+            "roofline": roofline, "e2e": e2e, "clocks": clocks, "gpu_launches": 8 * args.steps,
+            "wall_s_timed_region": wall}
+    if args.cpu_baseline and world == 1:
+        import oracle as orc
+        orc.build()
+        W1r, s1r, W2r, s2r = oracle_weights(orc, wl)
+        v, n, dt = time_oracle(orc, wl, W1r, s1r, W2r, s2r, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": oracle_cores(), "kind": "oracle",
+                                "sample": "%d of %d token rows of the same step (row-local), %.1f s" % (n, M_TOK, dt)}
+    if args.extras and world == 1:
+        line["extras"] = extras(w8, torch, workloads, dev, peaks, src)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _time(fn, reps, torch, stream, flush):
+    E = lambda: torch.cuda.Event(enable_timing=True)
+    fn()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(reps):
+        flush.fill_(3)
+        a, b = E(), E()
+        a.record(stream)
+        fn()
+        b.record(stream)
+        ms.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.median(x.elapsed_time(y) for x, y in ms)
+
+
+def extras(w8, torch, workloads, dev, peaks, src):
+    """The other rows of the hot path, each timed on its own (median of reps,
+    L2 flushed before each rep)."""
+    out = {}
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    hbm = peaks["hbm_gbs"]
+    tc8 = 2.0 * peaks["bf16_tflops"]
+    # token-wise quantize (K1) at 4608 x 12288
+    x = workloads.normal((M_TOK, MLP), 1.0, 5).to(dev)
+    q = torch.empty((M_TOK, MLP), dtype=torch.int8, device=dev)
+    s = torch.empty(M_TOK, dtype=torch.float32, device=dev)
+    ms = _time(lambda: w8.quantize_rows(x, "int8", out=q, scale=s), 20, torch, stream, flush)
+    gbs = (x.numel() * 3 + M_TOK * 4) / (ms * 1e-3) / 1e9
+    out["quantize_rows_4608x12288"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
+    del x, q
+    # float W8A8 forward (e4m3, bias) 4096 x 3072 x 3072
+    d = workloads.float_w8a8()
+    wq, sw = w8.quantize_weight(d["w"].to(dev), "e4m3", "tensor")
+    xx, bb = d["x"].to(dev), d["bias"].to(dev)
+    y = torch.empty((4096, 3072), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(w8.workspace_bytes(0, 4096, 3072, 3072), dtype=torch.uint8, device=dev)
+    ms = _time(lambda: w8.linear_fwd(xx, wq, sw, bias=bb, out=y, ws=ws), 20, torch, stream, flush)
+    xq, sx = w8.quantize_rows(xx, "e4m3")
+    gms = _time(lambda: w8.qgemm_fwd(xq, sx, wq, sw, bias=bb, out=y), 20, torch, stream, flush)
+    ops = 2 * 4096 * 3072 * 3072
+    out["float_w8a8_fwd_4096x3072x3072"] = {"ms": ms, "TOPS": ops / ms / 1e9, "gemm_ms": gms,
+                                            "gemm_TOPS": ops / gms / 1e9, "gemm_frac_fp8_burst": ops / gms / 1e9 / tc8}
+    # SVDQuant r=32, 4608 x 3072 x 3072
+    d = workloads.svdquant()
+    prep = w8.svdq_prepare(d["w"].to(dev), d["r"])
+    xx = d["x"].to(dev)
+    y = torch.empty((M_TOK, 3072), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(w8.workspace_bytes(2, M_TOK, 3072, 3072, 32), dtype=torch.uint8, device=dev)
+    ms = _time(lambda: w8.svdq_linear_fwd(xx, prep["rq"], prep["r_scale"], prep["l1"], prep["l2"], out=y, ws=ws),
+               20, torch, stream, flush)
+    ops = 2 * M_TOK * 3072 * 3072
+    out["svdquant_r32_fwd_4608x3072x3072"] = {"ms": ms, "TOPS_main": ops / ms / 1e9,
+                                              "lowrank_GFLOP": 2 * 2 * M_TOK * 3072 * 32 / 1e9}
+    # GGUF Q8_0: standalone quantize / dequantize of 2^28 fp32, requant, forward sweep
+    n = 1 << 28
+    xf = workloads.q8_0_standalone(n).to(dev)
+    blk = torch.empty(w8.q8_0_bytes(n), dtype=torch.uint8, device=dev)
+    ms = _time(lambda: w8.q8_0_quantize(xf, out=blk), 10, torch, stream, flush)
+    gbs = (4 * n + blk.numel()) / (ms * 1e-3) / 1e9
+    out["q8_0_quantize_2^28"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
+    ms = _time(lambda: w8.q8_0_dequantize(blk, n, out=xf), 10, torch, stream, flush)
+    gbs = (4 * n + blk.numel()) / (ms * 1e-3) / 1e9
+    out["q8_0_dequantize_2^28"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
+    del xf, blk
+    g = workloads.gguf_q8_0(M=max(workloads.GGUF_MS))
+    wb = w8.q8_0_quantize(g["w_f32"].reshape(-1).to(dev))
+    wq, sw = w8.q8_0_to_axis_int8(wb, MLP, HID)
+    ms = _time(lambda: w8.q8_0_to_axis_int8(wb, MLP, HID), 20, torch, stream, flush)
+    gbs = (wb.numel() + MLP * HID + MLP * 4) / (ms * 1e-3) / 1e9
+    out["q8_0_to_axis_int8_12288x3072"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
+    wt = workloads.normal((MLP, HID), 0.02, 9).to(dev)
+    ms = _time(lambda: w8.quantize_weight(wt, "int8", "tensor"), 20, torch, stream, flush)
+    out["quantize_weight_tensor_12288x3072"] = {"ms": ms, "GB/s": wt.numel() * 3 / (ms * 1e-3) / 1e9}
+    sweep = {}
+    xg = g["x"].to(dev)
+    for M in workloads.GGUF_MS:
+        xm = xg[:M].contiguous()
+        y = torch.empty((M, MLP), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(w8.workspace_bytes(0, M, MLP, HID), dtype=torch.uint8, device=dev)
+        ms = _time(lambda: w8.linear_fwd(xm, wq, sw, out=y, ws=ws), 20, torch, stream, flush)
+        sweep[str(M)] = {"ms": ms, "TOPS": 2 * M * MLP * HID / ms / 1e9,
+                         "weight_GB/s": MLP * HID / (ms * 1e-3) / 1e9}
+    out["gguf_a8_int_fwd_sweep_N12288_K3072"] = sweep
+    out["peaks"] = {"source": src, "hbm_gbs": hbm, "int8_burst_tops": tc8}
+    assert w8.device_status() == 0
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-extras", dest="extras", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

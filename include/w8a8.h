@@ -1,0 +1,225 @@
+/*
+ * w8a8.h - C ABI of libw8a8.so, a B200 (sm_100a) W8A8 quantized Linear.
+ *
+ * The operation (OneTrainer wiki "Quantization", int W8A8 and float W8A8
+ * paragraphs, "Technical:" lines): weights are quantized tensor-wise to int8
+ * or float8 e4m3, activations are quantized token-wise during training, and
+ * the Linear layer's matrix multiplication runs in int8 / float8.  The GGUF A8
+ * int paragraph adds weights re-quantized from GGUF blocks to int8 axis-wise;
+ * the SVDQuant paragraph adds a bfloat16 low-rank branch.
+ *
+ * Notation: X[M,K] bf16 activations, W[N,K] bf16 weight (nn.Linear layout),
+ * Y[M,N] = X W^T, all row-major.  Codes are int8 or OCP E4M3FN bytes; scales
+ * are fp32.  QMAX = 127 (int8) or 448 (e4m3).
+ *
+ * Conventions shared by every call
+ *  - Ownership: the caller owns every buffer.  All data pointers are DEVICE
+ *    pointers unless stated otherwise.  The library never allocates, frees or
+ *    synchronizes inside a compute call; workspace is passed in by the caller
+ *    (size from w8a8_workspace_bytes).
+ *  - Streams: all work is enqueued on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream).  Calls return as soon as the work is enqueued.
+ *  - Alignment: every device pointer must be 16-byte aligned
+ *    (W8A8_ERR_MISALIGNED otherwise) - the alignment to 16 that fixed the
+ *    misaligned-address offloading bug in OneTrainer PR #1034, Known issues.
+ *  - Shapes: M >= 0 (M == 0 is a no-op that returns W8A8_OK), N >= 1,
+ *    K >= 16 and K % 16 == 0 (tensor-copy row strides are 16-byte multiples;
+ *    cf. the cuBLASLt m/k shape limits in bitsandbytes #1401, Next steps).
+ *    Other shapes return W8A8_ERR_UNSUPPORTED_SHAPE before any launch.
+ *  - Inputs are finite (no NaN/Inf); results for non-finite inputs are
+ *    unspecified.
+ *  - Errors: argument errors return before any launch.  A failed launch
+ *    returns W8A8_ERR_CUDA.  A device that is not compute capability 10.0
+ *    returns W8A8_ERR_UNSUPPORTED_DEVICE; there is no CPU fallback.  Kernels
+ *    never trap: every wait on the GPU is bounded, and a wait that runs out
+ *    records W8A8_ERR_DEVICE_TIMEOUT in a per-device status word that
+ *    w8a8_device_status() reads.  w8a8_last_error() gives a message for the
+ *    last failing call of the calling thread.
+ */
+#ifndef W8A8_H
+#define W8A8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+struct CUstream_st;
+typedef struct CUstream_st* w8a8_stream_t;
+
+typedef enum {
+  W8A8_OK = 0,
+  W8A8_ERR_INVALID_ARG = 1,
+  W8A8_ERR_UNSUPPORTED_SHAPE = 2,
+  W8A8_ERR_MISALIGNED = 3,
+  W8A8_ERR_WORKSPACE = 4,
+  W8A8_ERR_CUDA = 5,
+  W8A8_ERR_DEVICE_TIMEOUT = 6,
+  W8A8_ERR_UNSUPPORTED_DEVICE = 7
+} w8a8_status;
+
+typedef enum { W8A8_INT8 = 0, W8A8_E4M3 = 1 } w8a8_qtype;
+typedef enum { W8A8_TENSOR = 0, W8A8_AXIS = 1 } w8a8_wgran;
+typedef enum {
+  W8A8_OP_LINEAR_FWD = 0,      /* w8a8_linear_fwd                          */
+  W8A8_OP_LINEAR_DGRAD = 1,    /* w8a8_linear_dgrad                        */
+  W8A8_OP_SVDQ_FWD = 2,        /* svdq_linear_fwd                          */
+  W8A8_OP_QUANTIZE_WEIGHT = 3  /* w8a8_quantize_weight (TENSOR needs 256 B) */
+} w8a8_op;
+
+/* ------------------------------------------------------------------------
+ * Token-wise calibrate + quantize (bitsandbytes #1401, Enhancements: the
+ * fused kernel for activation scale calibration and quantization,
+ * int8_vectorwise_quant; OneTrainer wiki: activations quantized token-wise).
+ * For every row m of X:  a = max_k |x[m,k]|,  s[m] = (a < 1e-10 ? 1e-10 :
+ * a / QMAX) (fp32 division),  q[m,k] = code(x[m,k] / s[m]) with int8 codes
+ * rounded half-to-even and clamped to +-127, e4m3 codes rounded to nearest
+ * even and saturated to +-448.  One pass over X.
+ *   x_bf16    [M, ldx] bf16, the first K columns are read; ldx % 8 == 0
+ *   q_out     [M, ldq] bytes (int8 or e4m3), ldq >= K, ldq % 16 == 0
+ *   row_scale [M] fp32
+ * ---------------------------------------------------------------------- */
+w8a8_status w8a8_quantize_rows(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                               w8a8_qtype qt, void* q_out, int64_t ldq, float* row_scale,
+                               w8a8_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Weight quantization (OneTrainer wiki, float8 / float W8A8 / int W8A8:
+ * "Tensor-wise quantization of weights"; GGUF A8: axis-wise).
+ *   TENSOR: one scale s = floor(absmax(W)) / QMAX for all N*K values; needs
+ *           ws_bytes >= w8a8_workspace_bytes(W8A8_OP_QUANTIZE_WEIGHT, ...)
+ *           (256 bytes, cleared by the call itself); scale is [1].
+ *   AXIS:   one scale per output row n, the token-wise rule applied to W's
+ *           rows; no workspace; scale is [N].
+ *   w_bf16 [N, K] contiguous bf16;  q_out [N, K] bytes.
+ * ---------------------------------------------------------------------- */
+w8a8_status w8a8_quantize_weight(const void* w_bf16, int64_t N, int64_t K, w8a8_qtype qt,
+                                 w8a8_wgran g, void* q_out, float* scale,
+                                 void* ws, size_t ws_bytes, w8a8_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * GGUF Q8_0 (entrenar 0.7.8, src/quant/gguf_quant/q8_0.rs: struct Q8_0 and
+ * Q8_0::quantize / Q8_0::dequantize).  A block holds 32 values in 34 bytes:
+ * the f16 scale (little-endian) followed by 32 int8 codes.  n values take
+ * ceil(n/32) blocks; a short last block is padded with zero codes.
+ *   quantize: per block max_abs = max|v|, scale = (max_abs < 1e-10 ? 1e-10 :
+ *             max_abs / 127) in fp32, code = clamp(round(v / scale), -128,
+ *             127) with round = ties away from zero; the stored scale is the
+ *             f16 (round-to-nearest-even) of the fp32 scale.
+ *   dequantize: y = f16 scale * code (exact in fp32), n values.
+ *   x / y: [n] fp32.  blocks: q8_0_bytes(n) bytes, 16-byte aligned base.
+ *   n >= 0 (0 is a no-op); no K constraint applies here.
+ * ---------------------------------------------------------------------- */
+size_t q8_0_bytes(int64_t n);
+w8a8_status q8_0_quantize(const float* x, int64_t n, void* blocks, w8a8_stream_t stream);
+w8a8_status q8_0_dequantize(const void* blocks, int64_t n, float* y, w8a8_stream_t stream);
+
+/* Re-quantize a Q8_0 weight to axis-wise int8 (OneTrainer wiki, GGUF A8 int:
+ * weights re-quantized from GGUF to int8 axis-wise).  Row n of W[N,K] is the
+ * K/32 consecutive blocks starting at block n*K/32.  Each value is
+ * dequantized exactly (f16 scale * code), then row n takes the token-wise
+ * int8 rule: s[n] = floor(max|deq|)/127, q = clamp(rne(deq/s[n]), +-127).
+ * K % 32 == 0 and K <= 131072.   q_out [N, K] int8;  scale [N] fp32. */
+w8a8_status q8_0_to_axis_int8(const void* blocks, int64_t N, int64_t K, int8_t* q_out,
+                              float* scale, w8a8_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * W8A8 Linear forward (OneTrainer wiki, int/float W8A8): quantize X
+ * token-wise (as w8a8_quantize_rows), multiply the codes with the weight
+ * codes on the 5th-generation tensor cores (int8 x int8 -> int32, or
+ * e4m3 x e4m3 -> fp32), then the fused epilogue
+ *     y = bf16( ((acc * s_x[m]) * w_scale[n or 0]) + bias[n] )
+ * with every product and sum rounded to fp32 on its own.
+ *   x_bf16 [M, K] contiguous;  wq [N, K] codes of qt;  w_scale [1] (TENSOR)
+ *   or [N] (AXIS);  bias_bf16 [N] or NULL;  y_bf16 [M, N] contiguous.
+ *   ws: w8a8_workspace_bytes(W8A8_OP_LINEAR_FWD, M, N, K, 0) bytes; holds
+ *   the activation codes and row scales of this call.
+ * ---------------------------------------------------------------------- */
+w8a8_status w8a8_linear_fwd(const void* x_bf16, int64_t M, int64_t N, int64_t K,
+                            w8a8_qtype qt, const void* wq, const float* w_scale, w8a8_wgran g,
+                            const void* bias_bf16, void* y_bf16,
+                            void* ws, size_t ws_bytes, w8a8_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * W8A8 Linear input gradient for LoRA training with frozen quantized weights
+ * (OneTrainer PR #1034: "train LoRA twice as fast"; wiki: activations are
+ * quantized token-wise during training):  dX = Q(dY) Q(W), i.e.
+ *     dx[m,k] = bf16( (acc[m,k] * s_dy[m]) * w_scale[0] ),
+ *     acc[m,k] = sum_n dyq[m,n] * wq[n,k].
+ * The tensor cores read the same wq[N,K] codes as the forward, with N as the
+ * contraction dimension (no transposed copy).  Tensor-wise weights only
+ * (g must be W8A8_TENSOR).  N % 16 == 0.
+ *   dy_bf16 [M, N];  wq [N, K];  dx_bf16 [M, K].
+ *   ws: w8a8_workspace_bytes(W8A8_OP_LINEAR_DGRAD, M, N, K, 0) bytes.
+ * ---------------------------------------------------------------------- */
+w8a8_status w8a8_linear_dgrad(const void* dy_bf16, int64_t M, int64_t N, int64_t K,
+                              w8a8_qtype qt, const void* wq, const float* w_scale, w8a8_wgran g,
+                              void* dx_bf16, void* ws, size_t ws_bytes, w8a8_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * SVDQuant int W8A8 forward (OneTrainer PR #1034, "SVDQuant", after arXiv
+ * 2411.05007; wiki: SVDQuant data type bfloat16):  W^T ~= L1 L2 + R^T with
+ * the residual R quantized int8 tensor-wise, so
+ *     T = bf16(X L1)                                   [M, r], fp32 sums
+ *     y = bf16( ((acc_R * s_x[m]) * r_scale) + bias[n] + sum_j T[m,j] L2[j,n] )
+ * where acc_R = Q(X) Q(R)^T on the tensor cores and the low-rank sum is an
+ * fp32 accumulation in the epilogue.  1 <= r <= 64.
+ *   rq [N, K] int8;  r_scale [1];  l1_bf16 [K, r];  l2_bf16 [r, N];
+ *   bias_bf16 [N] or NULL;  y_bf16 [M, N].
+ *   ws: w8a8_workspace_bytes(W8A8_OP_SVDQ_FWD, M, N, K, r) bytes; also
+ *   holds T.
+ * ---------------------------------------------------------------------- */
+w8a8_status svdq_linear_fwd(const void* x_bf16, int64_t M, int64_t N, int64_t K,
+                            const void* rq, const float* r_scale, int r,
+                            const void* l1_bf16, const void* l2_bf16, const void* bias_bf16,
+                            void* y_bf16, void* ws, size_t ws_bytes, w8a8_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * The two tensor-core products on codes that are already quantized (the
+ * second half of w8a8_linear_fwd / w8a8_linear_dgrad), for callers that
+ * quantize once and multiply many times.  Same epilogue and rules as above.
+ *   fwd:   xq [M, ldq] codes (ldq >= K, ldq % 16 == 0), x_scale [M], wq [N, K],
+ *          y [M, N] = epilogue( xq wq^T ).
+ *   dgrad: dyq [M, ldq] (ldq >= N, ldq % 16 == 0), dy_scale [M], wq [N, K],
+ *          dx [M, K] = epilogue( dyq wq ), tensor-wise w_scale only.
+ * ---------------------------------------------------------------------- */
+w8a8_status w8a8_qgemm_fwd(const void* xq, int64_t ldq, const float* x_scale,
+                           int64_t M, int64_t N, int64_t K, w8a8_qtype qt,
+                           const void* wq, const float* w_scale, w8a8_wgran g,
+                           const void* bias_bf16, void* y_bf16, w8a8_stream_t stream);
+w8a8_status w8a8_qgemm_dgrad(const void* dyq, int64_t ldq, const float* dy_scale,
+                             int64_t M, int64_t N, int64_t K, w8a8_qtype qt,
+                             const void* wq, const float* w_scale, void* dx_bf16,
+                             w8a8_stream_t stream);
+
+/* Workspace size in bytes for `op` at the given sizes (r only for SVDQ). */
+size_t w8a8_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r);
+
+/* ------------------------------------------------------------------------
+ * Device status and diagnostics (not on the pages; the failure-detection
+ * side of the library).
+ *  w8a8_device_status: synchronizes `stream`, then returns the first
+ *    device-side error recorded on the current device since the last reset
+ *    (W8A8_OK if none), and clears it when reset != 0.
+ *  w8a8_set_wait_limit_ns: bound of every device-side wait on the current
+ *    device (default 2e9 ns).  Synchronous; call outside stream capture.
+ *  w8a8_selftest_wait: launches one block that waits on a barrier which
+ *    nothing completes, bounded by `limit_ns`; the wait runs out, records
+ *    W8A8_ERR_DEVICE_TIMEOUT and the kernel returns normally.
+ *  w8a8_e4m3_encode: y[i] = E4M3FN code of x[i] (RNE, saturating), the same
+ *    device conversion the quantizers use.  x [n] fp32, y [n] bytes.
+ *  w8a8_last_error: message of the last failing call on this thread.
+ * ---------------------------------------------------------------------- */
+w8a8_status w8a8_device_status(w8a8_stream_t stream, int reset);
+w8a8_status w8a8_set_wait_limit_ns(uint64_t limit_ns);
+w8a8_status w8a8_selftest_wait(uint64_t limit_ns, w8a8_stream_t stream);
+w8a8_status w8a8_e4m3_encode(const float* x, int64_t n, uint8_t* y, w8a8_stream_t stream);
+const char* w8a8_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* W8A8_H */

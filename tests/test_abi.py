@@ -1,0 +1,120 @@
+"""The C-ABI library: it builds for sm_100a, loads, exports every function
+include/w8a8.h declares, and rejects bad arguments on the host before any
+CUDA call (so these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from w8a8_quantized_linear_b200 import _build
+    _build.build()
+    import w8a8_quantized_linear_b200 as w8
+    return w8.lib()
+
+
+def _header_functions():
+    text = open(os.path.join(ROOT, "include", "w8a8.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = _header_functions()
+    for want in ("w8a8_quantize_rows", "w8a8_quantize_weight", "q8_0_quantize", "q8_0_dequantize",
+                 "q8_0_to_axis_int8", "w8a8_linear_fwd", "w8a8_linear_dgrad", "svdq_linear_fwd"):
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    import w8a8_quantized_linear_b200 as w8
+    names = _header_functions()
+    assert set(names) == set(w8.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_library_is_built_for_sm100a():
+    from w8a8_quantized_linear_b200 import _build
+    cmd = _build.command()
+    assert "arch=compute_100a,code=sm_100a" in cmd
+
+
+def test_sizes(L):
+    assert L.q8_0_bytes(0) == 0
+    assert L.q8_0_bytes(1) == 34
+    assert L.q8_0_bytes(32) == 34
+    assert L.q8_0_bytes(33) == 68
+    assert L.q8_0_bytes(1 << 28) == (1 << 23) * 34
+    # workspace: codes then row scales, each on a 256-byte boundary
+    assert L.w8a8_workspace_bytes(0, 4608, 12288, 3072, 0) == 4608 * 3072 + 4608 * 4
+    assert L.w8a8_workspace_bytes(0, 3, 8, 16, 0) == 256 + 256
+    assert L.w8a8_workspace_bytes(1, 3, 40, 16, 0) == 256 + 256  # N padded to 48 -> 144 bytes
+    assert L.w8a8_workspace_bytes(2, 4608, 3072, 3072, 32) == 4608 * 3072 + 4608 * 4 + 4608 * 32 * 2
+    assert L.w8a8_workspace_bytes(3, 10, 10, 16, 0) == 256
+    assert L.w8a8_workspace_bytes(9, 1, 1, 16, 0) == 0
+
+
+A = ctypes.c_void_p(1 << 20)        # a 16-byte aligned stand-in pointer (never dereferenced)
+B = ctypes.c_void_p((1 << 20) + 8)  # misaligned
+
+
+def test_quantize_rows_validation(L):
+    # M == 0 is a no-op
+    assert L.w8a8_quantize_rows(A, 0, 64, 64, 0, A, 64, A, None) == 0
+    assert L.w8a8_quantize_rows(A, 4, 64, 64, 5, A, 64, A, None) == 1         # bad qtype
+    assert L.w8a8_quantize_rows(A, 4, 24, 24, 0, A, 32, A, None) == 2         # K % 16
+    assert L.w8a8_quantize_rows(A, 4, 0, 0, 0, A, 16, A, None) == 2           # K < 16
+    assert L.w8a8_quantize_rows(A, -1, 64, 64, 0, A, 64, A, None) == 2        # M < 0
+    assert L.w8a8_quantize_rows(A, 4, 64, 60, 0, A, 64, A, None) == 3         # ldx < K
+    assert L.w8a8_quantize_rows(A, 4, 64, 64, 0, A, 72, A, None) == 3         # ldq % 16
+    assert L.w8a8_quantize_rows(None, 4, 64, 64, 0, A, 64, A, None) == 1      # null
+    assert L.w8a8_quantize_rows(B, 4, 64, 64, 0, A, 64, A, None) == 3         # misaligned
+    assert b"16-byte" in L.w8a8_last_error()
+
+
+def test_linear_validation(L):
+    assert L.w8a8_linear_fwd(A, 8, 8, 24, 0, A, A, 0, None, A, A, 1 << 20, None) == 2
+    assert L.w8a8_linear_fwd(A, 8, 8, 32, 2, A, A, 0, None, A, A, 1 << 20, None) == 1
+    assert L.w8a8_linear_fwd(A, 8, 8, 32, 0, A, A, 0, B, A, A, 1 << 20, None) == 3   # bias misaligned
+    assert L.w8a8_linear_fwd(A, 8, 8, 32, 0, A, A, 0, None, A, A, 16, None) == 4     # workspace
+    assert L.w8a8_linear_fwd(A, 8, 8, 32, 0, A, A, 0, None, A, None, 0, None) == 4
+    assert L.w8a8_linear_fwd(A, 0, 8, 32, 0, A, A, 0, None, A, None, 0, None) == 0   # M == 0
+    assert L.w8a8_linear_fwd(A, 8, 0, 32, 0, A, A, 0, None, A, A, 1 << 20, None) == 2
+    # dgrad: tensor-wise only, N % 16
+    assert L.w8a8_linear_dgrad(A, 8, 32, 32, 0, A, A, 1, A, A, 1 << 20, None) == 1
+    assert L.w8a8_linear_dgrad(A, 8, 40, 32, 0, A, A, 0, A, A, 1 << 20, None) == 2
+    assert L.w8a8_linear_dgrad(A, 8, 32, 32, 0, A, A, 0, A, A, 8, None) == 4
+
+
+def test_svdq_validation(L):
+    assert L.svdq_linear_fwd(A, 8, 8, 32, A, A, 12, A, A, None, A, A, 1 << 20, None) == 2   # r % 8
+    assert L.svdq_linear_fwd(A, 8, 8, 32, A, A, 64, A, A, None, A, A, 1 << 20, None) == 2   # r > 32
+    assert L.svdq_linear_fwd(A, 8, 8, 32, A, A, 32, None, A, None, A, A, 1 << 20, None) == 1
+    assert L.svdq_linear_fwd(A, 8, 8, 32, A, A, 32, A, A, None, A, A, 64, None) == 4
+
+
+def test_q8_0_validation(L):
+    assert L.q8_0_quantize(A, 0, A, None) == 0
+    assert L.q8_0_quantize(A, -3, A, None) == 2
+    assert L.q8_0_quantize(None, 3, A, None) == 1
+    assert L.q8_0_quantize(A, 3, B, None) == 3
+    assert L.q8_0_dequantize(A, 3, B, None) == 3
+    assert L.q8_0_to_axis_int8(A, 4, 48, A, A, None) == 2      # K % 32
+    assert L.q8_0_to_axis_int8(A, 4, 1 << 18, A, A, None) == 2  # K too large
+    assert L.q8_0_to_axis_int8(A, 0, 64, A, A, None) == 2
+    assert L.w8a8_quantize_weight(A, 4, 64, 0, 0, A, A, None, 0, None) == 4   # tensor needs ws
+    assert L.w8a8_quantize_weight(A, 4, 64, 0, 7, A, A, None, 0, None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    import w8a8_quantized_linear_b200 as w8
+    monkeypatch.setattr(w8, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(w8, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        w8.lib()

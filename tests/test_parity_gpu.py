@@ -1,0 +1,306 @@
+"""GPU parity: every C-ABI call against the CPU oracle on the same seeded
+inputs.  Codes, scales, Q8_0 blocks and int-path outputs are compared bit
+for bit; e4m3 and low-rank outputs within the tolerances derived from the
+arithmetic (see the helpers below)."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from _tol import bf16_bits_to_f64, ulp_bf16
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def w8():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    from w8a8_quantized_linear_b200 import _build
+    _build.build()
+    import w8a8_quantized_linear_b200 as m
+    m.lib()
+    return m
+
+
+def u16(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def u8(t):
+    return t.detach().cpu().contiguous().view(torch.uint8).numpy()
+
+
+def f32(t):
+    return t.detach().cpu().numpy()
+
+
+QT = {"int8": 0, "e4m3": 1}
+
+
+# --------------------------------------------------------------------------- codecs
+def test_e4m3_device_conversion_matches_oracle(w8, orc):
+    grid = orc.bf16_to_f32(np.arange(1 << 16, dtype=np.uint32).astype(np.uint16))
+    grid = grid[np.isfinite(grid)]
+    scales = np.float32([1.0, 0.37, 3.1e-3, 117.0, 2.0 ** -12, 1e-10, 448.0 / 127.0])
+    vals = [grid / s for s in scales]
+    rng = np.random.default_rng(0)
+    bits = rng.integers(0, 1 << 32, size=1 << 22, dtype=np.uint64).astype(np.uint32).view(np.float32)
+    vals.append(bits[np.isfinite(bits)])
+    x = np.concatenate(vals).astype(np.float32)
+    with np.errstate(all="ignore"):
+        x = x[np.isfinite(x)]
+    got = u8(w8.e4m3_encode(torch.from_numpy(x).to(DEV)))
+    assert np.array_equal(got, orc.f32_to_e4m3(x))
+
+
+# --------------------------------------------------------------------------- quantize_rows
+ROW_SHAPES = [(1, 16), (5, 48), (127, 512), (129, 3072), (64, 12288), (3, 40000)]
+
+
+@pytest.mark.parametrize("qt", ["int8", "e4m3"])
+@pytest.mark.parametrize("M,K", ROW_SHAPES)
+def test_quantize_rows_parity(w8, orc, qt, M, K):
+    x = workloads.with_outlier_channels((M, K), 1.0, seed=M * 7 + K)
+    if M > 2:
+        x[1] = 0                       # all-zero row: the 1e-10 floor
+        x[2, :] = 1e-3
+        x[2, K // 3] = 3.0e4           # one huge value
+    q, s = w8.quantize_rows(x.to(DEV), qt)
+    qr, sr = orc.quantize_rows(workloads.to_u16(x), QT[qt])
+    assert np.array_equal(f32(s).view(np.uint32), sr.view(np.uint32))
+    assert np.array_equal(u8(q), qr)
+
+
+def test_quantize_rows_strided_input(w8, orc):
+    big = workloads.normal((40, 256), 1.0, 3)
+    x = big.to(DEV)[:, :160]           # ldx = 256 > K = 160
+    q, s = w8.quantize_rows(x, "int8")
+    qr, sr = orc.quantize_rows(workloads.to_u16(big[:, :160]), 0)
+    assert np.array_equal(u8(q), qr) and np.array_equal(f32(s), sr)
+
+
+# --------------------------------------------------------------------------- weights
+@pytest.mark.parametrize("qt", ["int8", "e4m3"])
+@pytest.mark.parametrize("gran", ["tensor", "axis"])
+@pytest.mark.parametrize("N,K", [(1, 16), (96, 160), (3072, 3072)])
+def test_quantize_weight_parity(w8, orc, qt, gran, N, K):
+    w = workloads.normal((N, K), 0.02, seed=N + K)
+    q, s = w8.quantize_weight(w.to(DEV), qt, gran)
+    qr, sr = orc.quantize_weight(workloads.to_u16(w), QT[qt], 0 if gran == "tensor" else 1)
+    assert np.array_equal(f32(s), sr)
+    assert np.array_equal(u8(q), qr)
+
+
+# --------------------------------------------------------------------------- Q8_0
+@pytest.mark.parametrize("n", [1, 31, 32, 33, 255, 256, 257, 1000, 65536 + 7, 1 << 22])
+def test_q8_0_parity(w8, orc, n):
+    x = workloads.q8_0_standalone(n, seed=n).numpy()
+    if n > 64:
+        x[32:64] = 0.0                 # a floor block
+        x[64:96] *= 1e-12
+    b = w8.q8_0_quantize(torch.from_numpy(x).to(DEV))
+    br, _ = orc.q8_0_quantize(x)
+    assert np.array_equal(u8(b), br)
+    y = w8.q8_0_dequantize(torch.from_numpy(br).to(DEV), n)
+    assert np.array_equal(f32(y).view(np.uint32), orc.q8_0_dequantize(br, n).view(np.uint32))
+
+
+def test_q8_0_standalone_full_size(w8, orc):
+    """2^28 fp32 values ~ N(0,1): every block bit-exact, every value exact."""
+    x = workloads.q8_0_standalone()
+    xd = x.to(DEV)
+    b = w8.q8_0_quantize(xd)
+    br, _ = orc.q8_0_quantize(x.numpy())
+    assert np.array_equal(u8(b), br)
+    del xd
+    y = w8.q8_0_dequantize(b, x.numel())
+    assert np.array_equal(f32(y).view(np.uint32), orc.q8_0_dequantize(br, x.numel()).view(np.uint32))
+
+
+@pytest.mark.parametrize("N,K", [(1, 32), (37, 96), (64, 512), (12288, 3072)])
+def test_q8_0_to_axis_int8_parity(w8, orc, N, K):
+    w = workloads.gguf_q8_0(N=N, K=K, M=1)["w_f32"].numpy().reshape(-1)
+    br, _ = orc.q8_0_quantize(w)
+    q, s = w8.q8_0_to_axis_int8(torch.from_numpy(br).to(DEV), N, K)
+    qr, sr = orc.q8_0_to_axis_int8(br, N, K)
+    assert np.array_equal(f32(s), sr)
+    assert np.array_equal(u8(q), qr.view(np.uint8))
+
+
+# --------------------------------------------------------------------------- Linear forward
+def _fp8_tol(ref, y):
+    """|y - y_ref| <= 1e-3 * s_x * s_w * sum|a*b| + 1 bf16 ulp."""
+    yr = bf16_bits_to_f64(ref["y"])
+    yg = bf16_bits_to_f64(y)
+    bound = 1e-3 * ref["sx"][:, None].astype(np.float64) * ref["sw"] * ref["absacc"]
+    bound = bound + ulp_bf16(np.maximum(np.abs(yr), np.abs(yg)))
+    return np.abs(yg - yr), bound
+
+
+LIN_SHAPES = [(256, 512, 512), (300, 520, 640), (1, 16, 16), (129, 257, 96), (7, 1000, 4096),
+              (128, 256, 128), (520, 300, 272)]
+
+
+@pytest.mark.parametrize("M,N,K", LIN_SHAPES)
+def test_linear_fwd_int8_parity(w8, orc, M, N, K):
+    x = workloads.with_outlier_channels((M, K), 1.0, seed=M + 3 * N + K)
+    w = workloads.normal((N, K), 0.02, seed=N + 5)
+    wq, sw = w8.quantize_weight(w.to(DEV), "int8", "tensor")
+    y = w8.linear_fwd(x.to(DEV), wq, sw)
+    wqr, swr = orc.quantize_weight(workloads.to_u16(w), 0, 0)
+    ref = orc.linear_fwd(workloads.to_u16(x), wqr, swr)
+    assert np.array_equal(u16(y), ref["y"])
+
+
+@pytest.mark.parametrize("M,N,K", [(200, 384, 256), (77, 130, 512)])
+def test_linear_fwd_int8_axis_bias_parity(w8, orc, M, N, K):
+    x = workloads.normal((M, K), 1.0, seed=11)
+    w = workloads.normal((N, K), 0.02, seed=12)
+    bias = workloads.normal((N,), 0.01, seed=13)
+    wq, sw = w8.quantize_weight(w.to(DEV), "int8", "axis")
+    y = w8.linear_fwd(x.to(DEV), wq, sw, bias=bias.to(DEV))
+    wqr, swr = orc.quantize_weight(workloads.to_u16(w), 0, 1)
+    ref = orc.linear_fwd(workloads.to_u16(x), wqr, swr, bias=workloads.to_u16(bias))
+    assert np.array_equal(u16(y), ref["y"])
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 512, 512), (300, 520, 640), (1, 16, 16), (129, 257, 96)])
+def test_linear_fwd_e4m3_parity(w8, orc, M, N, K):
+    x = workloads.with_outlier_channels((M, K), 1.0, seed=M + N)
+    w = workloads.normal((N, K), 0.02, seed=K + 1)
+    bias = workloads.normal((N,), 0.01, seed=N + 2)
+    wq, sw = w8.quantize_weight(w.to(DEV), "e4m3", "tensor")
+    y = w8.linear_fwd(x.to(DEV), wq, sw, bias=bias.to(DEV))
+    wqr, swr = orc.quantize_weight(workloads.to_u16(w), 1, 0)
+    assert np.array_equal(u8(wq), wqr)
+    ref = orc.linear_fwd(workloads.to_u16(x), wqr, swr, qt=1, bias=workloads.to_u16(bias))
+    ref["sw"] = swr[0]
+    err, bound = _fp8_tol(ref, u16(y))
+    assert np.all(err <= bound), float((err / bound).max())
+
+
+def test_qgemm_fwd_equals_linear(w8):
+    x = workloads.normal((300, 640), 1.0, 21).to(DEV)
+    wq, sw = w8.quantize_weight(workloads.normal((520, 640), 0.02, 22).to(DEV), "int8", "tensor")
+    xq, sx = w8.quantize_rows(x, "int8")
+    assert torch.equal(w8.qgemm_fwd(xq, sx, wq, sw), w8.linear_fwd(x, wq, sw))
+
+
+def test_linear_fwd_extreme_codes(w8, orc):
+    """Every code at +-127 and K = 12288: the int32 accumulator's largest sums."""
+    M, N, K = 130, 260, 12288
+    x = torch.full((M, K), 1.0)
+    x[::2] = -1.0
+    w = torch.full((N, K), 0.5)
+    w[1::3] = -0.5
+    xb, wb = x.to(torch.bfloat16), w.to(torch.bfloat16)
+    wq, sw = w8.quantize_weight(wb.to(DEV), "int8", "tensor")
+    y = w8.linear_fwd(xb.to(DEV), wq, sw)
+    wqr, swr = orc.quantize_weight(workloads.to_u16(wb), 0, 0)
+    ref = orc.linear_fwd(workloads.to_u16(xb), wqr, swr)
+    assert np.abs(ref["acc"]).max() == 127 * 127 * K
+    assert np.array_equal(u16(y), ref["y"])
+
+
+def test_linear_fwd_m0_noop(w8):
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device=DEV)
+    wq, sw = w8.quantize_weight(workloads.normal((32, 64), 0.02, 1).to(DEV), "int8", "tensor")
+    assert w8.linear_fwd(x, wq, sw).shape == (0, 32)
+
+
+def test_linear_fwd_deterministic(w8):
+    x = workloads.normal((1000, 1024), 1.0, 31).to(DEV)
+    wq, sw = w8.quantize_weight(workloads.normal((2048, 1024), 0.02, 32).to(DEV), "e4m3", "tensor")
+    a = w8.linear_fwd(x, wq, sw)
+    b = w8.linear_fwd(x, wq, sw)
+    assert torch.equal(a, b)
+
+
+# --------------------------------------------------------------------------- dgrad
+@pytest.mark.parametrize("qt", ["int8", "e4m3"])
+@pytest.mark.parametrize("M,N,K", [(64, 256, 512), (129, 96, 80), (300, 512, 272), (1, 16, 16)])
+def test_linear_dgrad_parity(w8, orc, qt, M, N, K):
+    dy = workloads.normal((M, N), 1e-3, seed=M + N)
+    w = workloads.normal((N, K), 0.02, seed=N * 3 + K)
+    wq, sw = w8.quantize_weight(w.to(DEV), qt, "tensor")
+    dx = w8.linear_dgrad(dy.to(DEV), wq, sw)
+    wqr, swr = orc.quantize_weight(workloads.to_u16(w), QT[qt], 0)
+    ref = orc.linear_dgrad(workloads.to_u16(dy), wqr, swr, qt=QT[qt])
+    if qt == "int8":
+        assert np.array_equal(u16(dx), ref["y"])
+    else:
+        ref["sw"] = swr[0]
+        err, bound = _fp8_tol(ref, u16(dx))
+        assert np.all(err <= bound), float((err / bound).max())
+
+
+def test_qgemm_dgrad_equals_linear(w8):
+    dy = workloads.normal((96, 256), 1e-3, 41).to(DEV)
+    wq, sw = w8.quantize_weight(workloads.normal((256, 160), 0.02, 42).to(DEV), "int8", "tensor")
+    dyq, sdy = w8.quantize_rows(dy, "int8")
+    assert torch.equal(w8.qgemm_dgrad(dyq, sdy, wq, sw), w8.linear_dgrad(dy, wq, sw))
+
+
+# --------------------------------------------------------------------------- SVDQuant
+def _svdq_check(w8, orc, x, w, r, bias=None, rows=None):
+    from oracle import svdquant
+    prep = svdquant.prepare(workloads.to_u16(w), r)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(DEV)
+    l1, l2 = to_dev(prep["l1"]), to_dev(prep["l2"])
+    rq = torch.from_numpy(prep["rq"].view(np.int8)).to(DEV)
+    rs = torch.from_numpy(prep["s_r"]).to(DEV)
+    M, K = x.shape
+    N = w.shape[0]
+    ws = torch.empty(w8.workspace_bytes(w8.OP_SVDQ_FWD, M, N, K, r), dtype=torch.uint8, device=DEV)
+    y = w8.svdq_linear_fwd(x.to(DEV), rq, rs, l1, l2, bias=None if bias is None else bias.to(DEV), ws=ws)
+    # T = bf16(X L1) as the kernel left it in the workspace
+    off = -(-(M * K) // 256) * 256 + -(-(M * 4) // 256) * 256
+    t_gpu = ws[off:off + M * r * 2].view(torch.bfloat16).view(M, r)
+    rows = np.arange(M) if rows is None else np.asarray(rows)
+    xs = workloads.to_u16(x)[rows]
+    ref = orc.svdq_linear_fwd(xs, prep["rq"], prep["s_r"], prep["l1"], prep["l2"],
+                              bias=None if bias is None else workloads.to_u16(bias))
+    # T: fp32 accumulation over K on the tensor cores, then one bf16 rounding
+    xabs = np.abs(orc.bf16_to_f32(xs).astype(np.float64)) @ np.abs(orc.bf16_to_f32(prep["l1"]).astype(np.float64))
+    gam = K * 2.0 ** -23 * xabs
+    tg = bf16_bits_to_f64(u16(t_gpu)[rows])
+    assert np.all(np.abs(tg - ref["t64"]) <= ulp_bf16(np.abs(ref["t64"]) + gam) + gam)
+    # y: the int part is exact; T may differ by its bound; lr sums in fp32
+    dt = ulp_bf16(np.abs(ref["t64"]) + gam) + gam
+    l2abs = np.abs(orc.bf16_to_f32(prep["l2"]).astype(np.float64))
+    yr = bf16_bits_to_f64(ref["y"])
+    yg = bf16_bits_to_f64(u16(y)[rows])
+    bound = dt @ l2abs + 2.0 ** -16 * ref["lr_abs"] + ulp_bf16(np.maximum(np.abs(yr), np.abs(yg)))
+    assert np.all(np.abs(yg - yr) <= bound), float((np.abs(yg - yr) / bound).max())
+    return y, ref
+
+
+@pytest.mark.parametrize("r", [8, 16, 32])
+def test_svdq_parity_small(w8, orc, r):
+    x = workloads.with_outlier_channels((200, 256), 1.0, seed=51 + r)
+    w = workloads.rank_spike_weight(320, 256, 8, 0.5, 0.02, seed=52)
+    bias = workloads.normal((320,), 0.01, seed=53)
+    _svdq_check(w8, orc, x, w, r, bias=bias)
+
+
+def test_svdq_zero_factors_equal_int_linear(w8):
+    x = workloads.normal((130, 256), 1.0, 61).to(DEV)
+    wq, sw = w8.quantize_weight(workloads.normal((300, 256), 0.02, 62).to(DEV), "int8", "tensor")
+    l1 = torch.zeros((256, 16), dtype=torch.bfloat16, device=DEV)
+    l2 = torch.zeros((16, 300), dtype=torch.bfloat16, device=DEV)
+    assert torch.equal(w8.svdq_linear_fwd(x, wq, sw, l1, l2), w8.linear_fwd(x, wq, sw))
+
+
+# --------------------------------------------------------------------------- diagnostics
+def test_device_status_clean_then_bounded_wait_times_out(w8):
+    assert w8.device_status(reset=True) == 0
+    w8.selftest_wait(50_000_000)                  # 50 ms wait on a barrier nothing completes
+    assert w8.device_status(reset=True) == 6      # W8A8_ERR_DEVICE_TIMEOUT, context intact
+    assert w8.device_status(reset=True) == 0
+    x = workloads.normal((64, 64), 1.0, 71).to(DEV)
+    wq, sw = w8.quantize_weight(workloads.normal((64, 64), 0.02, 72).to(DEV), "int8", "tensor")
+    w8.linear_fwd(x, wq, sw)
+    assert w8.device_status(reset=True) == 0

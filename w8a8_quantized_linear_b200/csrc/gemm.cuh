@@ -1,0 +1,297 @@
+// gemm.cuh - 8-bit (and bf16) GEMM on the sm_100a tensor cores with the
+// dequantizing epilogue fused.
+//
+//   D[m, n] = sum_k A[m, k] * B[n, k]       (B K-major: the forward, W[N,K])
+//   D[m, n] = sum_k A[m, k] * B[k, n]       (B MN-major: the dgrad, W[N,K] read
+//                                            with N as the contraction)
+//
+// One persistent CTA per SM, warp-specialized (192 threads; 320 with the
+// low-rank epilogue, which uses 8 epilogue warps):
+//   warp 0      TMA producer: A and B tiles into a ring of kStages shared-
+//               memory stages (128-byte swizzle), completion on mbarriers;
+//   warp 1      TMEM allocation; one thread issues tcgen05.mma (4 per stage)
+//               into one of two TMEM accumulators and commits the stage back;
+//   warps 2..   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
+//               lanes 32*(w%4)..+31 = tile rows), scales / bias / low-rank in
+//               fp32, bf16 stores.  Double buffering of the accumulator lets
+//               the epilogue of tile i overlap the MMAs of tile i+1.
+// Tile 128 x BN x 128 bytes of K per stage.  Every wait is bounded.
+#pragma once
+#include "device.cuh"
+
+namespace w8a8 {
+
+constexpr int kBM = 128;
+constexpr int kBKBytes = 128;
+constexpr int kStages = 4;
+
+enum { kKindI8 = 0, kKindE4M3 = 1, kKindBF16 = 2 };
+enum { kEpiScale = 0, kEpiLowRank = 1, kEpiPlain = 2 };
+
+struct EpiParams {
+  const float* s_row;            // [M] row (token) scales          (kEpiScale/LowRank)
+  const float* s_col;            // [1] or [N] weight scale
+  int s_col_axis;                // 1: s_col[n], 0: s_col[0]
+  const __nv_bfloat16* bias;     // [N] or nullptr
+  __nv_bfloat16* y;              // [M, ldy]
+  int64_t ldy;
+  const __nv_bfloat16* lr_t;     // T [M, r]                          (kEpiLowRank)
+  const __nv_bfloat16* lr_l2;    // L2 [r, N]
+  int r;
+};
+
+template <int KIND, int BN, int EPI>
+struct GemmCfg {
+  static constexpr int kElem = (KIND == kKindBF16) ? 2 : 1;
+  static constexpr int kBK = kBKBytes / kElem;            // K elements per stage
+  static constexpr int kMmaK = 32 / kElem;                // K elements per MMA
+  static constexpr int kABytes = kBM * kBKBytes;          // 16 KB
+  static constexpr int kBBytes = BN * kBKBytes;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kMaxRank = 32;
+  static constexpr int kLrBytes = (EPI == kEpiLowRank) ? kMaxRank * BN * 4 : 0;   // fp32 L2 tile
+  static constexpr int kEpiWarps = (EPI == kEpiLowRank) ? 8 : 4;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr size_t kSmem = 1024 /*alignment slack*/ + static_cast<size_t>(kStages) * kStageBytes +
+                                  kLrBytes + 256 /*barriers*/;
+};
+
+template <int KIND, bool B_MN, int BN, int EPI>
+__global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
+                int Kc, EpiParams ep) {
+  using C = GemmCfg<KIND, BN, EPI>;
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "tile N");
+  static_assert(!B_MN || (BN * C::kElem) % 128 == 0, "MN-major B needs whole 128-byte blocks");
+  constexpr uint32_t kIdesc = idesc<KIND>(kBM, BN, B_MN);
+  constexpr int kEpiThreads = 32 * C::kEpiWarps;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;                                        // kStages x kABytes
+  uint8_t* sB = smem + kStages * C::kABytes;                 // kStages x kBBytes
+  float* sLr = reinterpret_cast<float*>(smem + kStages * C::kStageBytes);   // [r][BN] fp32
+  uint8_t* tail = smem + kStages * C::kStageBytes + C::kLrBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(tail);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* teardown = tempty + 2;
+  uint64_t* lr_ready = teardown + 1;
+  uint64_t* lr_done = lr_ready + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lr_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t limit = g_wait_limit_ns;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], C::kEpiWarps);   // one arrival per epilogue warp
+    }
+    mbar_init(teardown, 1);
+    mbar_init(lr_ready, kEpiThreads);
+    mbar_init(lr_done, kEpiThreads);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int tiles_m = (M + kBM - 1) / kBM;
+  const int tiles_n = (N + BN - 1) / BN;
+  const int num_tiles = tiles_m * tiles_n;
+  const int num_kb = (Kc + C::kBK - 1) / C::kBK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, issued_phase = 0;   // per-stage bits, for teardown
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        const int m0 = (tile % tiles_m) * kBM, n0 = (tile / tiles_m) * BN;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, 0x100u | stage, limit)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          tma_load_2d(sA + stage * C::kABytes, &tmA, &full[stage], kb * C::kBK, m0);
+          uint8_t* b = sB + stage * C::kBBytes;
+          if constexpr (!B_MN) {
+            tma_load_2d(b, &tmB, &full[stage], kb * C::kBK, n0);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN * C::kElem / 128; ++j)
+              tma_load_2d(b + j * (C::kBK * 128), &tmB, &full[stage], n0 + j * (128 / C::kElem), kb * C::kBK);
+          }
+          issued |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Teardown: every copy this thread started has landed before the block
+      // can exit (a no-op on the normal path, where the MMAs consumed them).
+      for (int s = 0; s < kStages; ++s)
+        if (issued & (1u << s)) mbar_wait(&full[s], (issued_phase >> s) & 1u, nullptr, 0x180u | s, limit);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, 0x200u | acc, limit)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, 0x300u | stage, limit)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * C::kABytes);
+          const uint32_t b_base = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = sdesc_sw128(a_base + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? sdesc_sw128(b_base + k * (C::kMmaK * 128), C::kBK * 128, 1024)
+                                     : sdesc_sw128(b_base + k * 32, 16, 1024);
+            tc_mma<KIND>(d, ad, bd, kIdesc, (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      // Teardown: all MMAs issued by this thread have completed.
+      tc_commit(teardown);
+      mbar_wait(teardown, 0, nullptr, 0x380u, limit);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - 2;                       // epilogue warp index
+    const int quarter = warp & 3;                 // TMEM lanes this warp may read
+    const int group = e >> 2;                     // column-chunk interleave
+    constexpr int kGroups = C::kEpiWarps / 4;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+      const int m0 = (tile % tiles_m) * kBM, n0 = (tile / tiles_m) * BN;
+      if constexpr (EPI == kEpiLowRank) {
+        // L2[:, n0:n0+BN] as fp32 (zero outside N) for all epilogue warps.
+        if (local > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(lr_done, (local - 1) & 1, abort_flag, 0x500u, limit)))
+          break;
+        const int et = threadIdx.x - 64;
+        for (int i = et; i < ep.r * BN; i += kEpiThreads) {
+          const int j = i / BN, c = i % BN;
+          sLr[i] = (n0 + c < N) ? __bfloat162float(ep.lr_l2[static_cast<int64_t>(j) * N + n0 + c]) : 0.0f;
+        }
+        mbar_arrive(lr_ready);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(lr_ready, local & 1, abort_flag, 0x600u, limit))) break;
+      }
+      // Every lane polls; the warp then agrees (and reconverges) before the
+      // warp-collective tcgen05.ld, also when the wait ran out.
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[acc], acc_phase, abort_flag, 0x400u | acc, limit))) break;
+      tc_fence_after();
+      const int row = m0 + quarter * 32 + lane;
+      const bool row_ok = row < M;
+      float sx = 1.0f;
+      if constexpr (EPI != kEpiPlain) sx = row_ok ? ep.s_row[row] : 0.0f;
+      const float sw0 = (EPI != kEpiPlain && !ep.s_col_axis) ? ep.s_col[0] : 1.0f;
+      float t[C::kMaxRank];
+      if constexpr (EPI == kEpiLowRank) {
+#pragma unroll
+        for (int j = 0; j < C::kMaxRank; ++j)
+          t[j] = (row_ok && j < ep.r) ? __bfloat162float(ep.lr_t[static_cast<int64_t>(row) * ep.r + j]) : 0.0f;
+      }
+#pragma unroll 1
+      for (int c = group; c < BN / 32; c += kGroups) {
+        const int nc = n0 + c * 32;
+        if (nc >= N) break;                       // warp-uniform
+        uint32_t r[32];
+        tmem_ld_x32(tmem + lane_base + static_cast<uint32_t>(acc * BN + c * 32), r);
+        tmem_ld_wait();
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int>(r[j])) : __uint_as_float(r[j]);
+          if constexpr (EPI != kEpiPlain) {
+            const int n = nc + j;
+            const float sw = ep.s_col_axis ? ((n < N) ? __ldg(ep.s_col + n) : 0.0f) : sw0;
+            a = __fmul_rn(__fmul_rn(a, sx), sw);
+            if (ep.bias != nullptr && n < N) a = __fadd_rn(a, __bfloat162float(ep.bias[n]));
+          }
+          v[j] = a;
+        }
+        if constexpr (EPI == kEpiLowRank) {
+          float lr[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) lr[j] = 0.0f;
+#pragma unroll
+          for (int q = 0; q < C::kMaxRank; ++q) {
+            if (q >= ep.r) break;
+            const float4* l2row = reinterpret_cast<const float4*>(sLr + q * BN + c * 32);
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+              const float4 w = l2row[j4];
+              lr[4 * j4 + 0] = __fmaf_rn(t[q], w.x, lr[4 * j4 + 0]);
+              lr[4 * j4 + 1] = __fmaf_rn(t[q], w.y, lr[4 * j4 + 1]);
+              lr[4 * j4 + 2] = __fmaf_rn(t[q], w.z, lr[4 * j4 + 2]);
+              lr[4 * j4 + 3] = __fmaf_rn(t[q], w.w, lr[4 * j4 + 3]);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __fadd_rn(v[j], lr[j]);
+        }
+        if (row_ok) {
+          __nv_bfloat16* out = ep.y + static_cast<int64_t>(row) * ep.ldy + nc;
+          if (nc + 32 <= N && (ep.ldy & 7) == 0) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              uint4 p;
+              p.x = pack_bf16x2(v[j], v[j + 1]);
+              p.y = pack_bf16x2(v[j + 2], v[j + 3]);
+              p.z = pack_bf16x2(v[j + 4], v[j + 5]);
+              p.w = pack_bf16x2(v[j + 6], v[j + 7]);
+              *reinterpret_cast<uint4*>(out + j) = p;
+            }
+          } else {
+            for (int j = 0; j < 32; ++j)
+              if (nc + j < N) out[j] = __float2bfloat16_rn(v[j]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if constexpr (EPI == kEpiLowRank) mbar_arrive(lr_done);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace w8a8

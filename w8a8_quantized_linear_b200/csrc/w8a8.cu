@@ -1,0 +1,547 @@
+// w8a8.cu - the C ABI of libw8a8.so (declared in include/w8a8.h): argument
+// checks, workspace layout, TMA tensor maps and kernel launches.  One
+// translation unit holds every kernel, so the device status word and the
+// wait limit are single per-device symbols without relocatable device code.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "w8a8.h"
+#include "device.cuh"
+#include "gemm.cuh"
+#include "quantize.cuh"
+#include "q8_0.cuh"
+
+namespace w8a8 {
+namespace {
+
+thread_local std::string t_last_error;
+
+w8a8_status fail(w8a8_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+w8a8_status fail(w8a8_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return st;
+}
+
+w8a8_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(W8A8_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+constexpr int kMaxDevices = 64;
+
+// Compute capability 10.0 check and SM count, cached per device.
+struct DeviceInfo {
+  std::atomic<int> state{0};   // 0 unknown, 1 ok, 2 unsupported
+  int sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+w8a8_status current_device(int* dev_out, int* sms_out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(W8A8_ERR_UNSUPPORTED_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(W8A8_ERR_UNSUPPORTED_DEVICE, "device index %d out of range", dev);
+  DeviceInfo& di = g_dev[dev];
+  int st = di.state.load(std::memory_order_acquire);
+  if (st == 0) {
+    int major = 0, minor = 0, sms = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    di.sms = sms;
+    st = (major == 10 && minor == 0) ? 1 : 2;
+    di.state.store(st, std::memory_order_release);
+  }
+  if (st != 1) return fail(W8A8_ERR_UNSUPPORTED_DEVICE, "device %d is not compute capability 10.0 (sm_100a)", dev);
+  if (dev_out) *dev_out = dev;
+  if (sms_out) *sms_out = di.sms;
+  return W8A8_OK;
+}
+
+// ---------------------------------------------------------------- TMA maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [outer, inner] with `row_bytes` between rows, copied in
+// boxes of [box_outer, box_inner] elements with the 128-byte swizzle.
+w8a8_status make_map(CUtensorMap* map, CUtensorMapDataType dt, int elem, const void* base, int64_t inner,
+                     int64_t outer, int64_t row_bytes, int box_inner, int box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(W8A8_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  if (inner * elem > row_bytes || (row_bytes & 15) != 0 || !aligned16(base))
+    return fail(W8A8_ERR_MISALIGNED, "tensor map: base/stride not 16-byte aligned");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(W8A8_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return W8A8_OK;
+}
+
+// ---------------------------------------------------------------- launches
+template <typename Kernel>
+cudaError_t set_smem_once(Kernel k, size_t bytes, int dev, std::atomic<uint64_t>& mask) {
+  const uint64_t bit = 1ull << dev;
+  if (mask.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess) mask.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+template <int KIND, bool B_MN, int BN, int EPI>
+w8a8_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t M, int64_t N, int64_t Kc,
+                        const EpiParams& ep, cudaStream_t st) {
+  using C = GemmCfg<KIND, BN, EPI>;
+  static std::atomic<uint64_t> smem_set{0};
+  int dev = 0, sms = 0;
+  w8a8_status s = current_device(&dev, &sms);
+  if (s != W8A8_OK) return s;
+  auto kern = gemm_kernel<KIND, B_MN, BN, EPI>;
+  cudaError_t e = set_smem_once(kern, C::kSmem, dev, smem_set);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
+  const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  gemm_kernel<KIND, B_MN, BN, EPI><<<grid, C::kThreads, C::kSmem, st>>>(ta, tb, static_cast<int>(M),
+                                                                        static_cast<int>(N), static_cast<int>(Kc), ep);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "gemm launch");
+}
+
+w8a8_status launch_quantize_rows(const void* x, int64_t ldx, int64_t M, int64_t K, int qt, void* q, int64_t ldq,
+                                 float* s, cudaStream_t st) {
+  const int64_t nv = K / 8;
+  int64_t t = (nv + kRowVecs - 1) / kRowVecs;
+  t = round_up(t, 32);
+  if (t < 32) t = 32;
+  if (t > 1024) t = 1024;
+  const int grid = static_cast<int>(M < (1 << 20) ? M : (1 << 20));
+  const auto* xp = static_cast<const __nv_bfloat16*>(x);
+  auto* qp = static_cast<uint8_t*>(q);
+  if (qt == W8A8_E4M3)
+    quantize_rows_kernel<1><<<grid, static_cast<int>(t), 0, st>>>(xp, ldx, M, K, qp, ldq, s);
+  else
+    quantize_rows_kernel<0><<<grid, static_cast<int>(t), 0, st>>>(xp, ldx, M, K, qp, ldq, s);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "quantize_rows launch");
+}
+
+// Workspace carving: each piece starts on a 256-byte boundary.
+struct Carve {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carve(void* b) : base(static_cast<uint8_t*>(b)) {}
+  void* take(size_t bytes) {
+    void* p = base ? base + off : nullptr;
+    off += static_cast<size_t>(round_up(static_cast<int64_t>(bytes), 256));
+    return p;
+  }
+};
+
+size_t ws_linear(int64_t M, int64_t ld) {
+  Carve c(nullptr);
+  c.take(static_cast<size_t>(M * ld));
+  c.take(static_cast<size_t>(M) * 4);
+  return c.off;
+}
+size_t ws_svdq(int64_t M, int64_t K, int r) {
+  Carve c(nullptr);
+  c.take(static_cast<size_t>(M * K));
+  c.take(static_cast<size_t>(M) * 4);
+  c.take(static_cast<size_t>(M) * r * 2);
+  return c.off;
+}
+
+bool valid_qt(int qt) { return qt == W8A8_INT8 || qt == W8A8_E4M3; }
+bool valid_g(int g) { return g == W8A8_TENSOR || g == W8A8_AXIS; }
+
+CUtensorMapDataType code_type() { return CU_TENSOR_MAP_DATA_TYPE_UINT8; }
+
+// GEMM on codes.  fwd: A = xq [M, lda] K-major, B = wq [N, K] K-major.
+w8a8_status gemm_fwd(const void* xq, int64_t lda, const float* sx, int64_t M, int64_t N, int64_t K, int qt,
+                     const void* wq, const float* sw, int g, const void* bias, void* y, cudaStream_t st) {
+  alignas(64) CUtensorMap ta, tb;
+  w8a8_status s = make_map(&ta, code_type(), 1, xq, K, M, lda, kBKBytes, kBM);
+  if (s != W8A8_OK) return s;
+  s = make_map(&tb, code_type(), 1, wq, K, N, K, kBKBytes, 256);
+  if (s != W8A8_OK) return s;
+  EpiParams ep{};
+  ep.s_row = sx;
+  ep.s_col = sw;
+  ep.s_col_axis = (g == W8A8_AXIS);
+  ep.bias = static_cast<const __nv_bfloat16*>(bias);
+  ep.y = static_cast<__nv_bfloat16*>(y);
+  ep.ldy = N;
+  if (qt == W8A8_E4M3) return launch_gemm<kKindE4M3, false, 256, kEpiScale>(ta, tb, M, N, K, ep, st);
+  return launch_gemm<kKindI8, false, 256, kEpiScale>(ta, tb, M, N, K, ep, st);
+}
+
+// dgrad: A = dyq [M, lda] (contraction N), B = wq [N, K] read MN-major.
+w8a8_status gemm_dgrad(const void* dyq, int64_t lda, const float* sdy, int64_t M, int64_t N, int64_t K, int qt,
+                       const void* wq, const float* sw, void* dx, cudaStream_t st) {
+  alignas(64) CUtensorMap ta, tb;
+  w8a8_status s = make_map(&ta, code_type(), 1, dyq, N, M, lda, kBKBytes, kBM);
+  if (s != W8A8_OK) return s;
+  s = make_map(&tb, code_type(), 1, wq, K, N, K, 128, kBKBytes);
+  if (s != W8A8_OK) return s;
+  EpiParams ep{};
+  ep.s_row = sdy;
+  ep.s_col = sw;
+  ep.s_col_axis = 0;
+  ep.y = static_cast<__nv_bfloat16*>(dx);
+  ep.ldy = K;
+  if (qt == W8A8_E4M3) return launch_gemm<kKindE4M3, true, 256, kEpiScale>(ta, tb, M, K, N, ep, st);
+  return launch_gemm<kKindI8, true, 256, kEpiScale>(ta, tb, M, K, N, ep, st);
+}
+
+#define W8A8_CHECK(cond, status, ...) \
+  do {                                \
+    if (!(cond)) return fail(status, __VA_ARGS__); \
+  } while (0)
+
+w8a8_status check_k(int64_t K, const char* name) {
+  if (K < 16 || (K % 16) != 0)
+    return fail(W8A8_ERR_UNSUPPORTED_SHAPE, "%s = %lld: need >= 16 and a multiple of 16", name,
+                static_cast<long long>(K));
+  if (K > (1ll << 30)) return fail(W8A8_ERR_UNSUPPORTED_SHAPE, "%s too large", name);
+  return W8A8_OK;
+}
+
+}  // namespace
+}  // namespace w8a8
+
+using namespace w8a8;
+
+extern "C" {
+
+const char* w8a8_last_error(void) { return t_last_error.c_str(); }
+
+size_t q8_0_bytes(int64_t n) { return n <= 0 ? 0 : static_cast<size_t>((n + 31) / 32) * 34; }
+
+size_t w8a8_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
+  if (M < 0 || N < 0 || K < 0) return 0;
+  switch (op) {
+    case W8A8_OP_LINEAR_FWD: return ws_linear(M, K);
+    case W8A8_OP_LINEAR_DGRAD: return ws_linear(M, round_up(N, 16));
+    case W8A8_OP_SVDQ_FWD: return ws_svdq(M, K, r);
+    case W8A8_OP_QUANTIZE_WEIGHT: return 256;
+    default: return 0;
+  }
+}
+
+w8a8_status w8a8_quantize_rows(const void* x, int64_t M, int64_t K, int64_t ldx, w8a8_qtype qt, void* q,
+                               int64_t ldq, float* s, w8a8_stream_t stream) {
+  W8A8_CHECK(valid_qt(qt), W8A8_ERR_INVALID_ARG, "invalid qtype %d", static_cast<int>(qt));
+  W8A8_CHECK(M >= 0, W8A8_ERR_UNSUPPORTED_SHAPE, "M < 0");
+  w8a8_status st = check_k(K, "K");
+  if (st != W8A8_OK) return st;
+  W8A8_CHECK(ldx >= K && ldx % 8 == 0, W8A8_ERR_MISALIGNED, "ldx must be >= K and a multiple of 8");
+  W8A8_CHECK(ldq >= K && ldq % 16 == 0, W8A8_ERR_MISALIGNED, "ldq must be >= K and a multiple of 16");
+  W8A8_CHECK(x && q && s, W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(x) && aligned16(q) && aligned16(s), W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  if (M == 0) return W8A8_OK;
+  if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
+  return launch_quantize_rows(x, ldx, M, K, qt, q, ldq, s, reinterpret_cast<cudaStream_t>(stream));
+}
+
+w8a8_status w8a8_quantize_weight(const void* w, int64_t N, int64_t K, w8a8_qtype qt, w8a8_wgran g, void* q,
+                                 float* scale, void* ws, size_t ws_bytes, w8a8_stream_t stream) {
+  W8A8_CHECK(valid_qt(qt) && valid_g(g), W8A8_ERR_INVALID_ARG, "invalid qtype/granularity");
+  W8A8_CHECK(N >= 1, W8A8_ERR_UNSUPPORTED_SHAPE, "N < 1");
+  w8a8_status st = check_k(K, "K");
+  if (st != W8A8_OK) return st;
+  W8A8_CHECK(w && q && scale, W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(w) && aligned16(q) && aligned16(scale), W8A8_ERR_MISALIGNED,
+             "pointers must be 16-byte aligned");
+  if (g == W8A8_TENSOR) {
+    W8A8_CHECK(ws != nullptr && ws_bytes >= 256, W8A8_ERR_WORKSPACE, "tensor-wise quantization needs 256 B workspace");
+    W8A8_CHECK(aligned16(ws), W8A8_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+  }
+  int sms = 0;
+  if ((st = current_device(nullptr, &sms)) != W8A8_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (g == W8A8_AXIS) return launch_quantize_rows(w, K, N, K, qt, q, K, scale, s);
+  const int64_t nvec = N * K / 8;
+  unsigned* amax = static_cast<unsigned*>(ws);
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned), s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  int64_t blocks = (nvec + 255) / 256;
+  if (blocks > 8 * sms) blocks = 8 * sms;
+  absmax_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(static_cast<const uint4*>(w), nvec, amax);
+  if (qt == W8A8_E4M3)
+    quantize_tensor_kernel<1><<<static_cast<int>(blocks), 256, 0, s>>>(static_cast<const uint4*>(w), nvec, amax,
+                                                                       static_cast<uint2*>(q), scale);
+  else
+    quantize_tensor_kernel<0><<<static_cast<int>(blocks), 256, 0, s>>>(static_cast<const uint4*>(w), nvec, amax,
+                                                                       static_cast<uint2*>(q), scale);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "quantize_weight launch");
+}
+
+w8a8_status q8_0_quantize(const float* x, int64_t n, void* blocks, w8a8_stream_t stream) {
+  W8A8_CHECK(n >= 0, W8A8_ERR_UNSUPPORTED_SHAPE, "n < 0");
+  if (n == 0) return W8A8_OK;
+  W8A8_CHECK(x && blocks, W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(x) && aligned16(blocks), W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  int sms = 0;
+  w8a8_status st = current_device(nullptr, &sms);
+  if (st != W8A8_OK) return st;
+  const int64_t groups = (n + 255) / 256;
+  int64_t grid = (groups + kQ80WarpsPerBlock - 1) / kQ80WarpsPerBlock;
+  if (grid > 16 * sms) grid = 16 * sms;
+  q8_0_quantize_kernel<<<static_cast<int>(grid), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      x, n, static_cast<uint8_t*>(blocks));
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "q8_0_quantize launch");
+}
+
+w8a8_status q8_0_dequantize(const void* blocks, int64_t n, float* y, w8a8_stream_t stream) {
+  W8A8_CHECK(n >= 0, W8A8_ERR_UNSUPPORTED_SHAPE, "n < 0");
+  if (n == 0) return W8A8_OK;
+  W8A8_CHECK(y && blocks, W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(y) && aligned16(blocks), W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  int sms = 0;
+  w8a8_status st = current_device(nullptr, &sms);
+  if (st != W8A8_OK) return st;
+  const int64_t groups = (n + 255) / 256;
+  int64_t grid = (groups + kQ80WarpsPerBlock - 1) / kQ80WarpsPerBlock;
+  if (grid > 16 * sms) grid = 16 * sms;
+  q8_0_dequantize_kernel<<<static_cast<int>(grid), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(blocks), n, y);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "q8_0_dequantize launch");
+}
+
+w8a8_status q8_0_to_axis_int8(const void* blocks, int64_t N, int64_t K, int8_t* q, float* scale,
+                              w8a8_stream_t stream) {
+  W8A8_CHECK(N >= 1, W8A8_ERR_UNSUPPORTED_SHAPE, "N < 1");
+  W8A8_CHECK(K >= 32 && K % 32 == 0 && K <= 131072, W8A8_ERR_UNSUPPORTED_SHAPE,
+             "K must be a multiple of 32 in [32, 131072]");
+  W8A8_CHECK(blocks && q && scale, W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(blocks) && aligned16(q) && aligned16(scale), W8A8_ERR_MISALIGNED,
+             "pointers must be 16-byte aligned");
+  int dev = 0, sms = 0;
+  w8a8_status st = current_device(&dev, &sms);
+  if (st != W8A8_OK) return st;
+  const size_t smem = static_cast<size_t>(K / 32) * 34;
+  static std::atomic<uint64_t> smem_set{0};
+  cudaError_t e = set_smem_once(q8_0_to_axis_int8_kernel, 160 * 1024, dev, smem_set);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(requant)");
+  int64_t grid = N < 8 * sms ? N : 8 * sms;
+  q8_0_to_axis_int8_kernel<<<static_cast<int>(grid), 256, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(blocks), N, K, q, scale);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "q8_0_to_axis_int8 launch");
+}
+
+w8a8_status w8a8_qgemm_fwd(const void* xq, int64_t ldq, const float* sx, int64_t M, int64_t N, int64_t K,
+                           w8a8_qtype qt, const void* wq, const float* sw, w8a8_wgran g, const void* bias, void* y,
+                           w8a8_stream_t stream) {
+  W8A8_CHECK(valid_qt(qt) && valid_g(g), W8A8_ERR_INVALID_ARG, "invalid qtype/granularity");
+  W8A8_CHECK(M >= 0 && N >= 1 && M < (1ll << 31) && N < (1ll << 31), W8A8_ERR_UNSUPPORTED_SHAPE, "bad M/N");
+  w8a8_status st = check_k(K, "K");
+  if (st != W8A8_OK) return st;
+  W8A8_CHECK(ldq >= K && ldq % 16 == 0, W8A8_ERR_MISALIGNED, "ldq must be >= K and a multiple of 16");
+  W8A8_CHECK(xq && sx && wq && sw && y, W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(xq) && aligned16(sx) && aligned16(wq) && aligned16(sw) && aligned16(y) &&
+                 (bias == nullptr || aligned16(bias)),
+             W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  if (M == 0) return W8A8_OK;
+  if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
+  return gemm_fwd(xq, ldq, sx, M, N, K, qt, wq, sw, g, bias, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+w8a8_status w8a8_qgemm_dgrad(const void* dyq, int64_t ldq, const float* sdy, int64_t M, int64_t N, int64_t K,
+                             w8a8_qtype qt, const void* wq, const float* sw, void* dx, w8a8_stream_t stream) {
+  W8A8_CHECK(valid_qt(qt), W8A8_ERR_INVALID_ARG, "invalid qtype");
+  W8A8_CHECK(M >= 0 && M < (1ll << 31), W8A8_ERR_UNSUPPORTED_SHAPE, "bad M");
+  w8a8_status st = check_k(K, "K");
+  if (st != W8A8_OK) return st;
+  if ((st = check_k(N, "N")) != W8A8_OK) return st;
+  W8A8_CHECK(ldq >= N && ldq % 16 == 0, W8A8_ERR_MISALIGNED, "ldq must be >= N and a multiple of 16");
+  W8A8_CHECK(dyq && sdy && wq && sw && dx, W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(dyq) && aligned16(sdy) && aligned16(wq) && aligned16(sw) && aligned16(dx),
+             W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  if (M == 0) return W8A8_OK;
+  if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
+  return gemm_dgrad(dyq, ldq, sdy, M, N, K, qt, wq, sw, dx, reinterpret_cast<cudaStream_t>(stream));
+}
+
+w8a8_status w8a8_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, w8a8_qtype qt, const void* wq,
+                            const float* sw, w8a8_wgran g, const void* bias, void* y, void* ws, size_t ws_bytes,
+                            w8a8_stream_t stream) {
+  W8A8_CHECK(valid_qt(qt) && valid_g(g), W8A8_ERR_INVALID_ARG, "invalid qtype/granularity");
+  W8A8_CHECK(M >= 0 && N >= 1 && M < (1ll << 31) && N < (1ll << 31), W8A8_ERR_UNSUPPORTED_SHAPE, "bad M/N");
+  w8a8_status st = check_k(K, "K");
+  if (st != W8A8_OK) return st;
+  W8A8_CHECK(x && wq && sw && y, W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(x) && aligned16(wq) && aligned16(sw) && aligned16(y) && (bias == nullptr || aligned16(bias)),
+             W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  if (M == 0) return W8A8_OK;
+  W8A8_CHECK(ws != nullptr && ws_bytes >= ws_linear(M, K), W8A8_ERR_WORKSPACE, "workspace too small: need %zu bytes",
+             ws_linear(M, K));
+  W8A8_CHECK(aligned16(ws), W8A8_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+  if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Carve c(ws);
+  void* xq = c.take(static_cast<size_t>(M * K));
+  float* sx = static_cast<float*>(c.take(static_cast<size_t>(M) * 4));
+  if ((st = launch_quantize_rows(x, K, M, K, qt, xq, K, sx, s)) != W8A8_OK) return st;
+  return gemm_fwd(xq, K, sx, M, N, K, qt, wq, sw, g, bias, y, s);
+}
+
+w8a8_status w8a8_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, w8a8_qtype qt, const void* wq,
+                              const float* sw, w8a8_wgran g, void* dx, void* ws, size_t ws_bytes,
+                              w8a8_stream_t stream) {
+  W8A8_CHECK(valid_qt(qt) && valid_g(g), W8A8_ERR_INVALID_ARG, "invalid qtype/granularity");
+  W8A8_CHECK(g == W8A8_TENSOR, W8A8_ERR_INVALID_ARG, "dgrad reads a tensor-wise weight scale");
+  W8A8_CHECK(M >= 0 && M < (1ll << 31), W8A8_ERR_UNSUPPORTED_SHAPE, "bad M");
+  w8a8_status st = check_k(K, "K");
+  if (st != W8A8_OK) return st;
+  if ((st = check_k(N, "N")) != W8A8_OK) return st;
+  W8A8_CHECK(dy && wq && sw && dx, W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(dy) && aligned16(wq) && aligned16(sw) && aligned16(dx), W8A8_ERR_MISALIGNED,
+             "pointers must be 16-byte aligned");
+  if (M == 0) return W8A8_OK;
+  W8A8_CHECK(ws != nullptr && ws_bytes >= ws_linear(M, N), W8A8_ERR_WORKSPACE, "workspace too small: need %zu bytes",
+             ws_linear(M, N));
+  W8A8_CHECK(aligned16(ws), W8A8_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+  if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Carve c(ws);
+  void* dyq = c.take(static_cast<size_t>(M * N));
+  float* sdy = static_cast<float*>(c.take(static_cast<size_t>(M) * 4));
+  if ((st = launch_quantize_rows(dy, N, M, N, qt, dyq, N, sdy, s)) != W8A8_OK) return st;
+  return gemm_dgrad(dyq, N, sdy, M, N, K, qt, wq, sw, dx, s);
+}
+
+w8a8_status svdq_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, const void* rq, const float* r_scale,
+                            int r, const void* l1, const void* l2, const void* bias, void* y, void* ws,
+                            size_t ws_bytes, w8a8_stream_t stream) {
+  W8A8_CHECK(M >= 0 && N >= 1 && M < (1ll << 31) && N < (1ll << 31), W8A8_ERR_UNSUPPORTED_SHAPE, "bad M/N");
+  w8a8_status st = check_k(K, "K");
+  if (st != W8A8_OK) return st;
+  W8A8_CHECK(r >= 8 && r <= 32 && r % 8 == 0, W8A8_ERR_UNSUPPORTED_SHAPE, "rank r must be 8, 16, 24 or 32");
+  W8A8_CHECK(x && rq && r_scale && l1 && l2 && y, W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(x) && aligned16(rq) && aligned16(r_scale) && aligned16(l1) && aligned16(l2) && aligned16(y) &&
+                 (bias == nullptr || aligned16(bias)),
+             W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  if (M == 0) return W8A8_OK;
+  W8A8_CHECK(ws != nullptr && ws_bytes >= ws_svdq(M, K, r), W8A8_ERR_WORKSPACE,
+             "workspace too small: need %zu bytes", ws_svdq(M, K, r));
+  W8A8_CHECK(aligned16(ws), W8A8_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+  if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Carve c(ws);
+  void* xq = c.take(static_cast<size_t>(M * K));
+  float* sx = static_cast<float*>(c.take(static_cast<size_t>(M) * 4));
+  auto* t = static_cast<__nv_bfloat16*>(c.take(static_cast<size_t>(M) * r * 2));
+  if ((st = launch_quantize_rows(x, K, M, K, W8A8_INT8, xq, K, sx, s)) != W8A8_OK) return st;
+  // T = bf16(X L1): bf16 tensor-core GEMM, L1 [K, r] read MN-major.
+  {
+    alignas(64) CUtensorMap ta, tb;
+    if ((st = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, K, M, K * 2, 64, kBM)) != W8A8_OK) return st;
+    if ((st = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, l1, r, K, static_cast<int64_t>(r) * 2, 64, 64)) !=
+        W8A8_OK)
+      return st;
+    EpiParams ep{};
+    ep.y = t;
+    ep.ldy = r;
+    if ((st = launch_gemm<kKindBF16, true, 64, kEpiPlain>(ta, tb, M, r, K, ep, s)) != W8A8_OK) return st;
+  }
+  alignas(64) CUtensorMap ta, tb;
+  if ((st = make_map(&ta, code_type(), 1, xq, K, M, K, kBKBytes, kBM)) != W8A8_OK) return st;
+  if ((st = make_map(&tb, code_type(), 1, rq, K, N, K, kBKBytes, 256)) != W8A8_OK) return st;
+  EpiParams ep{};
+  ep.s_row = sx;
+  ep.s_col = r_scale;
+  ep.s_col_axis = 0;
+  ep.bias = static_cast<const __nv_bfloat16*>(bias);
+  ep.y = static_cast<__nv_bfloat16*>(y);
+  ep.ldy = N;
+  ep.lr_t = t;
+  ep.lr_l2 = static_cast<const __nv_bfloat16*>(l2);
+  ep.r = r;
+  return launch_gemm<kKindI8, false, 256, kEpiLowRank>(ta, tb, M, N, K, ep, s);
+}
+
+w8a8_status w8a8_device_status(w8a8_stream_t stream, int reset) {
+  w8a8_status st = current_device(nullptr, nullptr);
+  if (st != W8A8_OK) return st;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned v = 0, site = 0;
+  if ((e = cudaMemcpyFromSymbol(&v, g_status, sizeof(v))) != cudaSuccess) return cuda_fail(e, "read status");
+  cudaMemcpyFromSymbol(&site, g_status_site, sizeof(site));
+  if (reset) {
+    const unsigned z = 0;
+    cudaMemcpyToSymbol(g_status, &z, sizeof(z));
+    cudaMemcpyToSymbol(g_status_site, &z, sizeof(z));
+  }
+  if (v == kDevOk) return W8A8_OK;
+  if (v == kDevTimeout) return fail(W8A8_ERR_DEVICE_TIMEOUT, "device wait ran out (site 0x%x)", site);
+  return fail(W8A8_ERR_CUDA, "device status %u (site 0x%x)", v, site);
+}
+
+w8a8_status w8a8_set_wait_limit_ns(uint64_t limit_ns) {
+  w8a8_status st = current_device(nullptr, nullptr);
+  if (st != W8A8_OK) return st;
+  W8A8_CHECK(limit_ns > 0, W8A8_ERR_INVALID_ARG, "limit must be > 0");
+  unsigned long long v = limit_ns;
+  cudaError_t e = cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v));
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "set wait limit");
+}
+
+w8a8_status w8a8_selftest_wait(uint64_t limit_ns, w8a8_stream_t stream) {
+  W8A8_CHECK(limit_ns > 0 && limit_ns <= 10000000000ull, W8A8_ERR_INVALID_ARG, "limit must be in (0, 10 s]");
+  w8a8_status st = current_device(nullptr, nullptr);
+  if (st != W8A8_OK) return st;
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "selftest launch");
+}
+
+w8a8_status w8a8_e4m3_encode(const float* x, int64_t n, uint8_t* y, w8a8_stream_t stream) {
+  W8A8_CHECK(n >= 0, W8A8_ERR_UNSUPPORTED_SHAPE, "n < 0");
+  if (n == 0) return W8A8_OK;
+  W8A8_CHECK(x && y, W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(x) && aligned16(y), W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  int sms = 0;
+  w8a8_status st = current_device(nullptr, &sms);
+  if (st != W8A8_OK) return st;
+  int64_t grid = (n + 255) / 256;
+  if (grid > 16 * sms) grid = 16 * sms;
+  e4m3_encode_kernel<<<static_cast<int>(grid), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, n, y);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "e4m3 encode launch");
+}
+
+}  // extern "C"
