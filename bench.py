@@ -373,6 +373,38 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+def run_case(args):
+    """One quantize + GEMM pair of the step, warmup + steps times (profiling)."""
+    import torch
+    import workloads
+    import w8a8_quantized_linear_b200 as w8
+    dev = torch.device("cuda", 0)
+    wl = workloads.dit_mlp()
+    if args.case in ("up", "dgrad_up"):
+        wq, sw = w8.quantize_weight(wl["w1"].to(dev), "int8", "tensor")      # [12288, 3072]
+    else:
+        wq, sw = w8.quantize_weight(wl["w2"].to(dev), "int8", "tensor")      # [3072, 12288]
+    if args.case == "up":
+        x = wl["x"].to(dev)
+        fn = lambda xq, s: w8.qgemm_fwd(xq, s, wq, sw)
+    elif args.case == "down":
+        x = workloads.normal((M_TOK, MLP), 0.5, 25).to(dev)
+        fn = lambda xq, s: w8.qgemm_fwd(xq, s, wq, sw)
+    elif args.case == "dgrad_down":
+        x = wl["dy2"].to(dev)
+        fn = lambda xq, s: w8.qgemm_dgrad(xq, s, wq, sw)
+    else:
+        x = workloads.normal((M_TOK, MLP), 1e-3, 26).to(dev)
+        fn = lambda xq, s: w8.qgemm_dgrad(xq, s, wq, sw)
+    for _ in range(args.warmup + args.steps):
+        xq, s = w8.quantize_rows(x, "int8")
+        fn(xq, s)
+    torch.cuda.synchronize()
+    assert w8.device_status() == 0
+    print("case %s ok" % args.case)
+    return 0
+
+
 def _time(fn, reps, torch, stream, flush):
     E = lambda: torch.cuda.Event(enable_timing=True)
     fn()
@@ -473,6 +505,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-extras", dest="extras", action="store_false")
+    ap.add_argument("--case", choices=["up", "down", "dgrad_down", "dgrad_up"], default=None,
+                    help="run only one of the step's four quantize+GEMM pairs (for profiling), no JSON")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -482,6 +516,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.case:
+        return run_case(args)
     if world > 1:
         import datetime
         import torch

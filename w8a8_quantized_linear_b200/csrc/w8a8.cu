@@ -265,9 +265,9 @@ w8a8_status w8a8_quantize_rows(const void* x, int64_t M, int64_t K, int64_t ldx,
   if (st != W8A8_OK) return st;
   W8A8_CHECK(ldx >= K && ldx % 8 == 0, W8A8_ERR_MISALIGNED, "ldx must be >= K and a multiple of 8");
   W8A8_CHECK(ldq >= K && ldq % 16 == 0, W8A8_ERR_MISALIGNED, "ldq must be >= K and a multiple of 16");
+  if (M == 0) return W8A8_OK;   // empty tensors may carry null pointers
   W8A8_CHECK(x && q && s, W8A8_ERR_INVALID_ARG, "null pointer");
   W8A8_CHECK(aligned16(x) && aligned16(q) && aligned16(s), W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
-  if (M == 0) return W8A8_OK;
   if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
   return launch_quantize_rows(x, ldx, M, K, qt, q, ldq, s, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -370,11 +370,11 @@ w8a8_status w8a8_qgemm_fwd(const void* xq, int64_t ldq, const float* sx, int64_t
   w8a8_status st = check_k(K, "K");
   if (st != W8A8_OK) return st;
   W8A8_CHECK(ldq >= K && ldq % 16 == 0, W8A8_ERR_MISALIGNED, "ldq must be >= K and a multiple of 16");
+  if (M == 0) return W8A8_OK;
   W8A8_CHECK(xq && sx && wq && sw && y, W8A8_ERR_INVALID_ARG, "null pointer");
   W8A8_CHECK(aligned16(xq) && aligned16(sx) && aligned16(wq) && aligned16(sw) && aligned16(y) &&
                  (bias == nullptr || aligned16(bias)),
              W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
-  if (M == 0) return W8A8_OK;
   if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
   return gemm_fwd(xq, ldq, sx, M, N, K, qt, wq, sw, g, bias, y, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -387,10 +387,10 @@ w8a8_status w8a8_qgemm_dgrad(const void* dyq, int64_t ldq, const float* sdy, int
   if (st != W8A8_OK) return st;
   if ((st = check_k(N, "N")) != W8A8_OK) return st;
   W8A8_CHECK(ldq >= N && ldq % 16 == 0, W8A8_ERR_MISALIGNED, "ldq must be >= N and a multiple of 16");
+  if (M == 0) return W8A8_OK;
   W8A8_CHECK(dyq && sdy && wq && sw && dx, W8A8_ERR_INVALID_ARG, "null pointer");
   W8A8_CHECK(aligned16(dyq) && aligned16(sdy) && aligned16(wq) && aligned16(sw) && aligned16(dx),
              W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
-  if (M == 0) return W8A8_OK;
   if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
   return gemm_dgrad(dyq, ldq, sdy, M, N, K, qt, wq, sw, dx, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -402,10 +402,10 @@ w8a8_status w8a8_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, w8a8
   W8A8_CHECK(M >= 0 && N >= 1 && M < (1ll << 31) && N < (1ll << 31), W8A8_ERR_UNSUPPORTED_SHAPE, "bad M/N");
   w8a8_status st = check_k(K, "K");
   if (st != W8A8_OK) return st;
+  if (M == 0) return W8A8_OK;   // empty tensors may carry null pointers
   W8A8_CHECK(x && wq && sw && y, W8A8_ERR_INVALID_ARG, "null pointer");
   W8A8_CHECK(aligned16(x) && aligned16(wq) && aligned16(sw) && aligned16(y) && (bias == nullptr || aligned16(bias)),
              W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
-  if (M == 0) return W8A8_OK;
   W8A8_CHECK(ws != nullptr && ws_bytes >= ws_linear(M, K), W8A8_ERR_WORKSPACE, "workspace too small: need %zu bytes",
              ws_linear(M, K));
   W8A8_CHECK(aligned16(ws), W8A8_ERR_MISALIGNED, "workspace must be 16-byte aligned");
@@ -427,10 +427,10 @@ w8a8_status w8a8_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, w
   w8a8_status st = check_k(K, "K");
   if (st != W8A8_OK) return st;
   if ((st = check_k(N, "N")) != W8A8_OK) return st;
+  if (M == 0) return W8A8_OK;
   W8A8_CHECK(dy && wq && sw && dx, W8A8_ERR_INVALID_ARG, "null pointer");
   W8A8_CHECK(aligned16(dy) && aligned16(wq) && aligned16(sw) && aligned16(dx), W8A8_ERR_MISALIGNED,
              "pointers must be 16-byte aligned");
-  if (M == 0) return W8A8_OK;
   W8A8_CHECK(ws != nullptr && ws_bytes >= ws_linear(M, N), W8A8_ERR_WORKSPACE, "workspace too small: need %zu bytes",
              ws_linear(M, N));
   W8A8_CHECK(aligned16(ws), W8A8_ERR_MISALIGNED, "workspace must be 16-byte aligned");
@@ -450,11 +450,11 @@ w8a8_status svdq_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, cons
   w8a8_status st = check_k(K, "K");
   if (st != W8A8_OK) return st;
   W8A8_CHECK(r >= 8 && r <= 32 && r % 8 == 0, W8A8_ERR_UNSUPPORTED_SHAPE, "rank r must be 8, 16, 24 or 32");
+  if (M == 0) return W8A8_OK;
   W8A8_CHECK(x && rq && r_scale && l1 && l2 && y, W8A8_ERR_INVALID_ARG, "null pointer");
   W8A8_CHECK(aligned16(x) && aligned16(rq) && aligned16(r_scale) && aligned16(l1) && aligned16(l2) && aligned16(y) &&
                  (bias == nullptr || aligned16(bias)),
              W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
-  if (M == 0) return W8A8_OK;
   W8A8_CHECK(ws != nullptr && ws_bytes >= ws_svdq(M, K, r), W8A8_ERR_WORKSPACE,
              "workspace too small: need %zu bytes", ws_svdq(M, K, r));
   W8A8_CHECK(aligned16(ws), W8A8_ERR_MISALIGNED, "workspace must be 16-byte aligned");
