@@ -63,22 +63,23 @@ def load_peaks():
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling of one GPU during the timed region."""
-    QUERY = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+    """nvidia-smi clock / throttle sampling during the timed region, filtered
+    to one GPU by UUID (or by index when the UUID is unknown)."""
+    QUERY = ("uuid,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
              "clocks_event_reasons.sw_power_cap")
     NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_id: str):
-        self.gpu_id = gpu_id
+    def __init__(self, uuid: str, index: str):
+        self.uuid = (uuid or "").lower().replace("gpu-", "")
+        self.index = index
         self.proc = None
         self.out = ""
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + self.QUERY,
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.QUERY, "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
         return self
@@ -92,40 +93,41 @@ class ClockSampler:
                 self.proc.kill()
                 self.out, _ = self.proc.communicate()
 
-    @staticmethod
-    def parse(text):
+    def parse(self, text):
         def num(x):
             try:
                 return float(x)
             except ValueError:
                 return None
-        rows = [[c.strip() for c in r] for r in csv.reader(io.StringIO(text or "")) if len(r) >= 7]
-        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
-        mx = [num(r[1]) for r in rows if num(r[1]) is not None]
-        pw = [num(r[2]) for r in rows if num(r[2]) is not None]
-        reasons = sorted({ClockSampler.NAMES[i] for r in rows for i in range(4) if r[3 + i].lower() == "active"})
+        rows = [[c.strip() for c in r] for r in csv.reader(io.StringIO(text or "")) if len(r) >= 9]
+        mine = [r for r in rows if self.uuid and r[0].lower().replace("gpu-", "") == self.uuid]
+        if not mine:
+            mine = [r for r in rows if r[1] == self.index]
+        sm = [num(r[2]) for r in mine if num(r[2]) is not None]
+        mx = [num(r[3]) for r in mine if num(r[3]) is not None]
+        pw = [num(r[4]) for r in mine if num(r[4]) is not None]
+        reasons = sorted({self.NAMES[i] for r in mine for i in range(4) if r[5 + i].lower() == "active"})
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
         load = [v for v in sm if v >= 0.3 * max(mx or sm)] or sm
         return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(mx) if mx else None,
-                "power_w_max": max(pw) if pw else None, "reasons": reasons, "samples": len(rows)}
+                "power_w_max": max(pw) if pw else None, "reasons": reasons, "samples": len(mine)}
 
     def summary(self):
         return self.parse(self.out)
 
 
-def gpu_selector(torch, dev) -> str:
-    """nvidia-smi -i argument for a torch device: its UUID, else its index."""
+def gpu_identity(torch, dev):
+    """(uuid, nvidia-smi index) of a torch device."""
+    uuid = ""
     try:
-        u = str(torch.cuda.get_device_properties(dev).uuid)
-        if u:
-            return u if u.startswith("GPU-") else "GPU-" + u
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         pass
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
-    ids = [v for v in vis.split(",") if v.strip()]
+    vis = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
     idx = dev.index or 0
-    return ids[idx].strip() if idx < len(ids) else str(idx)
+    index = vis[idx] if idx < len(vis) and vis[idx].isdigit() else str(idx)
+    return uuid, index
 
 
 # ----------------------------------------------------------------------------- oracle (CPU)
@@ -276,7 +278,7 @@ def run_ours(args, rank, world, local_rank):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(gpu_selector(torch, dev)) as clk:
+    with ClockSampler(*gpu_identity(torch, dev)) as clk:
         wall0 = time.perf_counter()
         for i in range(args.steps):
             flush.fill_(i & 0xFF)          # L2 flush, outside the step's events
@@ -508,7 +510,7 @@ def main():
     ap.add_argument("--case", choices=["up", "down", "dgrad_down", "dgrad_up"], default=None,
                     help="run only one of the step's four quantize+GEMM pairs (for profiling), no JSON")
     args = ap.parse_args()
-    if args.warmup < 3:
+    if args.warmup < 3 and not args.case:
         ap.error("--warmup must be >= 3")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
