@@ -195,6 +195,43 @@ w8a8_status w8a8_qgemm_dgrad(const void* dyq, int64_t ldq, const float* dy_scale
                              const void* wq, const float* w_scale, void* dx_bf16,
                              w8a8_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * w8a8_linear_fwd without a caller workspace.  (No counterpart on the pages:
+ * this is a calling convenience of this library.)
+ *
+ * Some callers cannot hand the library device memory for scratch: code that
+ * runs where allocating is not allowed or not possible (an embedding runtime
+ * or plugin host that owns all device memory and exposes no allocator, a
+ * latency-critical path that must not call cudaMalloc because it can
+ * synchronize the device, a language binding with no CUDA allocator).  This
+ * entry point computes exactly what w8a8_linear_fwd computes, but keeps the
+ * activation codes and row scales in a fixed scratch array that is part of
+ * the library itself (a file-scope __device__ array of
+ * W8A8_NOALLOC_SCRATCH_BYTES; every GPU that loads the library holds it
+ * until the process exits).  It calls no cudaMalloc / cudaFree and no
+ * allocating library routine.  The caller still passes x, wq, w_scale, bias
+ * and the output y.
+ *
+ * Limits: M * K <= W8A8_NOALLOC_MAX_CODES and M <= W8A8_NOALLOC_MAX_ROWS;
+ * larger problems return W8A8_ERR_WORKSPACE before any launch (use
+ * w8a8_linear_fwd with a workspace instead).
+ * Set-up: the first call on each device looks up the scratch array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.
+ * Sharing: all calls on a device use the same scratch, which keeps the last
+ * call's contents (every byte a call reads was written earlier by the same
+ * call, so nothing needs clearing).  Calls whose kernels overlap on the GPU
+ * (different streams, or graphs replayed concurrently) race on the scratch;
+ * order them on one stream.
+ * ---------------------------------------------------------------------- */
+#define W8A8_NOALLOC_MAX_CODES (64ull << 20)
+#define W8A8_NOALLOC_MAX_ROWS 65536ll
+#define W8A8_NOALLOC_SCRATCH_BYTES (W8A8_NOALLOC_MAX_CODES + 4ull * W8A8_NOALLOC_MAX_ROWS)
+w8a8_status w8a8_linear_fwd_noalloc(const void* x_bf16, int64_t M, int64_t N, int64_t K,
+                                    w8a8_qtype qt, const void* wq, const float* w_scale,
+                                    w8a8_wgran g, const void* bias_bf16, void* y_bf16,
+                                    w8a8_stream_t stream);
+
 /* Workspace size in bytes for `op` at the given sizes (r only for SVDQ). */
 size_t w8a8_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r);
 

@@ -34,7 +34,7 @@ EXPORTS = ("w8a8_quantize_rows", "w8a8_quantize_weight", "q8_0_bytes", "q8_0_qua
            "q8_0_dequantize", "q8_0_to_axis_int8", "w8a8_linear_fwd", "w8a8_linear_dgrad",
            "svdq_linear_fwd", "w8a8_qgemm_fwd", "w8a8_qgemm_dgrad", "w8a8_workspace_bytes",
            "w8a8_device_status", "w8a8_set_wait_limit_ns", "w8a8_selftest_wait",
-           "w8a8_e4m3_encode", "w8a8_last_error")
+           "w8a8_e4m3_encode", "w8a8_last_error", "w8a8_linear_fwd_noalloc")
 
 
 class W8A8Error(RuntimeError):
@@ -70,6 +70,7 @@ def lib() -> ctypes.CDLL:
             "w8a8_set_wait_limit_ns": [_U64],
             "w8a8_selftest_wait": [_U64, _P],
             "w8a8_e4m3_encode": [_P, _I64, _P, _P],
+            "w8a8_linear_fwd_noalloc": [_P, _I64, _I64, _I64, _I, _P, _P, _I, _P, _P, _P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -223,6 +224,20 @@ def linear_fwd(x, wq, w_scale, bias=None, out=None, ws=None):
     _check(lib().w8a8_linear_fwd(_ptr(x), M, N, K, qt, _ptr(_as_bytes(wq)), _ptr(w_scale), g, _ptr(bias),
                                  _ptr(y), _ptr(ws), ws.numel(), _stream(x.device)))
     return y
+
+
+def linear_fwd_noalloc(x, wq, w_scale, out, bias=None):
+    """linear_fwd for callers that cannot provide scratch memory: the library
+    keeps the activation codes in its own fixed device array (M*K and M are
+    bounded; see include/w8a8.h).  The output `out` [M, N] bf16 is the caller's."""
+    _cuda_2d(x, torch.bfloat16, "x")
+    qt = _qt(wq.dtype)
+    M, K = x.shape
+    N = wq.shape[0]
+    g = AXIS if w_scale.numel() > 1 else TENSOR
+    _check(lib().w8a8_linear_fwd_noalloc(_ptr(x), M, N, K, qt, _ptr(_as_bytes(wq)), _ptr(w_scale), g,
+                                         _ptr(bias), _ptr(out), _stream(x.device)))
+    return out
 
 
 def linear_dgrad(dy, wq, w_scale, out=None, ws=None):

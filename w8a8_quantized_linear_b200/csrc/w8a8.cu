@@ -235,6 +235,27 @@ w8a8_status check_k(int64_t K, const char* name) {
   return W8A8_OK;
 }
 
+// Scratch of w8a8_linear_fwd_noalloc: activation codes at offset 0, row
+// scales at offset W8A8_NOALLOC_MAX_CODES (both 256-byte aligned).  Host code
+// only sees a stand-in for this symbol; its device address comes from
+// cudaGetSymbolAddress, once per device, with that device current.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[W8A8_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+w8a8_status noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return W8A8_OK;
+}
+
 }  // namespace
 }  // namespace w8a8
 
@@ -414,6 +435,33 @@ w8a8_status w8a8_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, w8a8
   Carve c(ws);
   void* xq = c.take(static_cast<size_t>(M * K));
   float* sx = static_cast<float*>(c.take(static_cast<size_t>(M) * 4));
+  if ((st = launch_quantize_rows(x, K, M, K, qt, xq, K, sx, s)) != W8A8_OK) return st;
+  return gemm_fwd(xq, K, sx, M, N, K, qt, wq, sw, g, bias, y, s);
+}
+
+w8a8_status w8a8_linear_fwd_noalloc(const void* x, int64_t M, int64_t N, int64_t K, w8a8_qtype qt, const void* wq,
+                                    const float* sw, w8a8_wgran g, const void* bias, void* y, w8a8_stream_t stream) {
+  W8A8_CHECK(valid_qt(qt) && valid_g(g), W8A8_ERR_INVALID_ARG, "invalid qtype/granularity");
+  W8A8_CHECK(M >= 0 && N >= 1 && M < (1ll << 31) && N < (1ll << 31), W8A8_ERR_UNSUPPORTED_SHAPE, "bad M/N");
+  w8a8_status st = check_k(K, "K");
+  if (st != W8A8_OK) return st;
+  if (M == 0) return W8A8_OK;
+  W8A8_CHECK(M <= W8A8_NOALLOC_MAX_ROWS && static_cast<uint64_t>(M) * static_cast<uint64_t>(K) <= W8A8_NOALLOC_MAX_CODES,
+             W8A8_ERR_WORKSPACE,
+             "w8a8_linear_fwd_noalloc: M=%lld, M*K=%lld exceed the built-in scratch (M <= %lld, M*K <= %llu); "
+             "use w8a8_linear_fwd with a workspace",
+             static_cast<long long>(M), static_cast<long long>(M * K), static_cast<long long>(W8A8_NOALLOC_MAX_ROWS),
+             static_cast<unsigned long long>(W8A8_NOALLOC_MAX_CODES));
+  W8A8_CHECK(x && wq && sw && y, W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(x) && aligned16(wq) && aligned16(sw) && aligned16(y) && (bias == nullptr || aligned16(bias)),
+             W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  int dev = 0;
+  if ((st = current_device(&dev, nullptr)) != W8A8_OK) return st;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(dev, &scratch)) != W8A8_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  void* xq = scratch;
+  float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + W8A8_NOALLOC_MAX_CODES);
   if ((st = launch_quantize_rows(x, K, M, K, qt, xq, K, sx, s)) != W8A8_OK) return st;
   return gemm_fwd(xq, K, sx, M, N, K, qt, wq, sw, g, bias, y, s);
 }
