@@ -77,21 +77,33 @@ class ClockSampler:
         self.out = ""
 
     def __enter__(self):
-        try:
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="w8a8_clocks_", suffix=".csv")
+        os.close(fd)
+        try:   # -f: nvidia-smi writes (and flushes) every sample to the file itself
             self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.QUERY, "--format=csv,noheader,nounits",
-                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                                          "-lms", "200", "-f", self.path],
+                                         stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+        time.sleep(0.5)   # first sample before the timed region
         return self
 
     def __exit__(self, *a):
         if self.proc is not None:
+            time.sleep(0.3)
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                self.out, _ = self.proc.communicate()
+                self.proc.wait()
+        try:
+            with open(self.path) as fh:
+                self.out = fh.read()
+            os.unlink(self.path)
+        except OSError:
+            self.out = ""
 
     def parse(self, text):
         def num(x):
@@ -343,7 +355,10 @@ def run_ours(args, rank, world, local_rank):
         return 0
 
     peaks, src = load_peaks()
-    int8_peak = 2.0 * peaks["bf16_tflops_sustained"]   # int8 dense = 2 x bf16 dense (4.5 vs 2.25 PFLOP/s nominal)
+    # int8 dense = 2 x bf16 dense (4.5 vs 2.25 PFLOP/s nominal).  The timed
+    # region lasts tens of milliseconds, so the burst figure applies; the
+    # sustained fraction is reported beside it.
+    int8_peak = 2.0 * peaks["bf16_tflops"]
     gemm_avg = statistics.mean(gemm_ms)
     achieved = OPS_PER_GEMM / (gemm_avg * 1e-3) / 1e12
     sha = gemm_source_sha()
@@ -351,8 +366,8 @@ def run_ours(args, rank, world, local_rank):
     roofline = {"bound": "tensor", "kernel": "gemm_kernel<i8> (tcgen05 kind::i8, fused epilogue)",
                 "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved / int8_peak,
                 "traffic": traffic,
-                "peak_source": "%s: 2 x bf16_tflops_sustained (int8 dense = 2x bf16 dense nominal)" % src,
-                "frac_of_burst": achieved / (2.0 * peaks["bf16_tflops"]),
+                "peak_source": "%s: 2 x bf16_tflops (burst; int8 dense = 2x bf16 dense nominal)" % src,
+                "frac_of_sustained": achieved / (2.0 * peaks["bf16_tflops_sustained"]),
                 "gemm_ms_avg": gemm_avg, "quantize_ms_avg": statistics.mean(quant_ms),
                 "quantize_share": sum(quant_ms) / sum(step_ms)}
     clocks = clk.summary()

@@ -5,15 +5,15 @@
 //   D[m, n] = sum_k A[m, k] * B[k, n]       (B MN-major: the dgrad, W[N,K] read
 //                                            with N as the contraction)
 //
-// One persistent CTA per SM, warp-specialized (192 threads; 320 with the
-// low-rank epilogue, which uses 8 epilogue warps):
+// One persistent CTA per SM, warp-specialized, 320 threads:
 //   warp 0      TMA producer: A and B tiles into a ring of kStages shared-
 //               memory stages (128-byte swizzle), completion on mbarriers;
 //   warp 1      TMEM allocation; one thread issues tcgen05.mma (4 per stage)
 //               into one of two TMEM accumulators and commits the stage back;
-//   warps 2..   epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
-//               lanes 32*(w%4)..+31 = tile rows), scales / bias / low-rank in
-//               fp32, bf16 stores.  Double buffering of the accumulator lets
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
+//               lanes 32*(w%4)..+31 = tile rows; the two warps of a lane
+//               quarter take alternate 32-column chunks), scales / bias /
+//               low-rank in fp32, bf16 stores.  Double buffering of the accumulator lets
 //               the epilogue of tile i overlap the MMAs of tile i+1.
 // Tile 128 x BN x 128 bytes of K per stage.  Every wait is bounded.
 #pragma once
@@ -23,7 +23,6 @@ namespace w8a8 {
 
 constexpr int kBM = 128;
 constexpr int kBKBytes = 128;
-constexpr int kStages = 4;
 
 enum { kKindI8 = 0, kKindE4M3 = 1, kKindBF16 = 2 };
 enum { kEpiScale = 0, kEpiLowRank = 1, kEpiPlain = 2 };
@@ -35,6 +34,7 @@ struct EpiParams {
   const __nv_bfloat16* bias;     // [N] or nullptr
   __nv_bfloat16* y;              // [M, ldy]
   int64_t ldy;
+  int tma_store;                 // 1: Y goes out through the tmY tensor map (ldy % 8 == 0)
   const __nv_bfloat16* lr_t;     // T [M, r]                          (kEpiLowRank)
   const __nv_bfloat16* lr_l2;    // L2 [r, N]
   int r;
@@ -51,28 +51,35 @@ struct GemmCfg {
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kMaxRank = 32;
   static constexpr int kLrBytes = (EPI == kEpiLowRank) ? kMaxRank * BN * 4 : 0;   // fp32 L2 tile
-  static constexpr int kEpiWarps = (EPI == kEpiLowRank) ? 8 : 4;
+  static constexpr int kEpiWarps = 8;   // two per TMEM lane quarter, splitting the column chunks
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kStages = (EPI == kEpiLowRank) ? 3 : 4;
+  // per epilogue warp, two 32 x 32 bf16 staging buffers for the TMA store
+  static constexpr int kOutBufBytes = 32 * 32 * 2;
+  static constexpr int kOutBytes = kEpiWarps * 2 * kOutBufBytes;
   static constexpr size_t kSmem = 1024 /*alignment slack*/ + static_cast<size_t>(kStages) * kStageBytes +
-                                  kLrBytes + 256 /*barriers*/;
+                                  kLrBytes + kOutBytes + 256 /*barriers*/;
 };
 
 template <int KIND, bool B_MN, int BN, int EPI>
 __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
-                int Kc, EpiParams ep) {
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmY, int M, int N, int Kc, EpiParams ep) {
   using C = GemmCfg<KIND, BN, EPI>;
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "tile N");
   static_assert(!B_MN || (BN * C::kElem) % 128 == 0, "MN-major B needs whole 128-byte blocks");
   constexpr uint32_t kIdesc = idesc<KIND>(kBM, BN, B_MN);
   constexpr int kEpiThreads = 32 * C::kEpiWarps;
+  constexpr bool kAxisOk = (EPI == kEpiScale);   // per-column weight scales (the low-rank path is tensor-wise)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int kStages = C::kStages;
   uint8_t* sA = smem;                                        // kStages x kABytes
   uint8_t* sB = smem + kStages * C::kABytes;                 // kStages x kBBytes
   float* sLr = reinterpret_cast<float*>(smem + kStages * C::kStageBytes);   // [r][BN] fp32
-  uint8_t* tail = smem + kStages * C::kStageBytes + C::kLrBytes;
+  uint8_t* sOut = smem + kStages * C::kStageBytes + C::kLrBytes;             // epilogue staging
+  uint8_t* tail = sOut + C::kOutBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(tail);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
@@ -102,6 +109,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (ep.tma_store) tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
@@ -191,6 +199,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     int local = 0;
+    uint32_t out_iter = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       const int m0 = (tile % tiles_m) * kBM, n0 = (tile / tiles_m) * BN;
       if constexpr (EPI == kEpiLowRank) {
@@ -224,6 +233,38 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
       for (int c = group; c < BN / 32; c += kGroups) {
         const int nc = n0 + c * 32;
         if (nc >= N) break;                       // warp-uniform
+        const bool full_chunk = nc + 32 <= N;
+        // Column parameters of the chunk, loaded before the TMEM load so that
+        // their latency overlaps it: 16-byte vectors, the same addresses in
+        // every lane (broadcast).
+        float sw[32], bs[32];
+        if constexpr (EPI != kEpiPlain) {
+          if (kAxisOk && ep.s_col_axis) {
+            if (full_chunk) {
+#pragma unroll
+              for (int j = 0; j < 32; j += 4) {
+                const float4 f = __ldg(reinterpret_cast<const float4*>(ep.s_col + nc + j));
+                sw[j] = f.x; sw[j + 1] = f.y; sw[j + 2] = f.z; sw[j + 3] = f.w;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) sw[j] = (nc + j < N) ? __ldg(ep.s_col + nc + j) : 0.0f;
+            }
+          }
+          if (ep.bias != nullptr) {
+            if (full_chunk) {
+#pragma unroll
+              for (int j = 0; j < 32; j += 8) {
+                const uint4 b = __ldg(reinterpret_cast<const uint4*>(ep.bias + nc + j));
+                bs[j] = bf16_lo(b.x); bs[j + 1] = bf16_hi(b.x); bs[j + 2] = bf16_lo(b.y); bs[j + 3] = bf16_hi(b.y);
+                bs[j + 4] = bf16_lo(b.z); bs[j + 5] = bf16_hi(b.z); bs[j + 6] = bf16_lo(b.w); bs[j + 7] = bf16_hi(b.w);
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) bs[j] = (nc + j < N) ? __bfloat162float(ep.bias[nc + j]) : 0.0f;
+            }
+          }
+        }
         uint32_t r[32];
         tmem_ld_x32(tmem + lane_base + static_cast<uint32_t>(acc * BN + c * 32), r);
         tmem_ld_wait();
@@ -232,10 +273,8 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
         for (int j = 0; j < 32; ++j) {
           float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int>(r[j])) : __uint_as_float(r[j]);
           if constexpr (EPI != kEpiPlain) {
-            const int n = nc + j;
-            const float sw = ep.s_col_axis ? ((n < N) ? __ldg(ep.s_col + n) : 0.0f) : sw0;
-            a = __fmul_rn(__fmul_rn(a, sx), sw);
-            if (ep.bias != nullptr && n < N) a = __fadd_rn(a, __bfloat162float(ep.bias[n]));
+            a = __fmul_rn(__fmul_rn(a, sx), (kAxisOk && ep.s_col_axis) ? sw[j] : sw0);
+            if (ep.bias != nullptr) a = __fadd_rn(a, bs[j]);
           }
           v[j] = a;
         }
@@ -259,7 +298,30 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __fadd_rn(v[j], lr[j]);
         }
-        if (row_ok) {
+        if (ep.tma_store) {
+          // Stage the warp's 32 x 32 bf16 block in shared memory with the 64-byte
+          // swizzle (16-byte unit j of row l at unit j ^ ((l >> 1) & 3)), then
+          // one lane stores it with TMA; the box is clipped at M and N.
+          uint8_t* buf = sOut + ((e * 2 + (out_iter & 1)) * C::kOutBufBytes);
+          if (lane == 0) bulk_wait_read<1>();     // this buffer's previous store has read it
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 p;
+            p.x = pack_bf16x2(v[8 * j], v[8 * j + 1]);
+            p.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+            p.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+            p.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+            *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) = p;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && m0 + quarter * 32 < M) {   // skip blocks wholly below the last row
+            tma_store_2d(&tmY, buf, nc, m0 + quarter * 32);
+            bulk_commit();
+          }
+          ++out_iter;
+        } else if (row_ok) {
           __nv_bfloat16* out = ep.y + static_cast<int64_t>(row) * ep.ldy + nc;
           if (nc + 32 <= N && (ep.ldy & 7) == 0) {
 #pragma unroll
@@ -283,6 +345,8 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
       if constexpr (EPI == kEpiLowRank) mbar_arrive(lr_done);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    // the staging buffers must outlive the stores that read them
+    if (ep.tma_store && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();

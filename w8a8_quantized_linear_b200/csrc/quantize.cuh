@@ -1,15 +1,14 @@
 // quantize.cuh - token-wise absmax calibration + quantization in one pass
 // (the fused row calibrate-and-quantize of bitsandbytes #1401), and the
 // tensor-wise weight quantizer.  Bandwidth-bound: 16-byte coalesced loads and
-// stores, warp-shuffle reductions, no tensor cores.
+// stores, packed bf16x2 absmax, warp-shuffle reductions, no tensor cores.
 #pragma once
 #include "device.cuh"
 
 namespace w8a8 {
 
-constexpr int kRowVecs = 4;   // 16-byte vectors per thread kept in registers
+constexpr int kRowVecs = 8;   // 16-byte vectors per thread kept in registers
 
-// Code of v for the two activation formats.
 template <int QT>
 __device__ __forceinline__ float qmax_of() { return QT == 1 ? 448.0f : 127.0f; }
 
@@ -19,37 +18,89 @@ __device__ __forceinline__ float absmax_scale(float a) {
   return (a < 1e-10f) ? 1e-10f : __fdiv_rn(a, qmax_of<QT>());
 }
 
-// 8 bf16 (one uint4) -> 8 codes (one uint2), each x / s divided in fp32.
-template <int QT>
-__device__ __forceinline__ uint2 encode8(uint4 v, float s) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t out[2];
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const float a0 = __fdiv_rn(bf16_lo(w[2 * h]), s), a1 = __fdiv_rn(bf16_hi(w[2 * h]), s);
-    const float a2 = __fdiv_rn(bf16_lo(w[2 * h + 1]), s), a3 = __fdiv_rn(bf16_hi(w[2 * h + 1]), s);
-    if constexpr (QT == 1) {
-      out[h] = static_cast<uint32_t>(cvt_e4m3x2(a0, a1)) | (static_cast<uint32_t>(cvt_e4m3x2(a2, a3)) << 16);
-    } else {
-      out[h] = int8_code(a0) | (int8_code(a1) << 8) | (int8_code(a2) << 16) | (int8_code(a3) << 24);
-    }
-  }
-  return make_uint2(out[0], out[1]);
+// Exact codes of fl(v / s) without a division in the common case.
+//
+// rcp = fl(1/s) is correctly rounded, so t = fl(v * rcp) lies within
+// 3.0001 ulp (relative to |v / s|) of fl(v / s).
+//
+// int8: t is rounded to the nearest integer, ties to even, by adding
+// 1.5 * 2^23 (an fp32 add rounds exactly there for |t| < 2^22); the low byte
+// of the sum's bit pattern is then the two's-complement code.  The remainder
+// d = t - rne(t) is exact; when |d| < 0.5 - 2^-14 no rounding boundary lies
+// within 2^-14 > 3.0001 ulp * 127.5 of t, so fl(v / s) rounds to the same
+// integer.  |v / s| <= 127 (1 + 2^-23) with the absmax scale, so no clamp is
+// reached.  A group of values with any |d| at the margin is recomputed with
+// IEEE divisions (the rare slow path).
+//
+// e4m3: the codes of t * (1 - 2^-21) and t * (1 + 2^-21) - the ends of a
+// +-8 ulp interval that contains fl(v / s) - are compared; e4m3 rounding with
+// saturation is monotonic, so when they agree they are the code of fl(v / s).
+constexpr float kRneMagic = 12582912.0f;            // 1.5 * 2^23
+constexpr float kNearHalf = 0.49993896484375f;      // 0.5 - 2^-14
+
+__device__ __forceinline__ uint32_t rne_low_byte(float t, bool& near) {
+  const float big = __fadd_rn(t, kRneMagic);
+  const float d = __fsub_rn(t, __fsub_rn(big, kRneMagic));
+  near |= fabsf(d) > kNearHalf;
+  return __float_as_uint(big) & 0xFFu;
+}
+__device__ __forceinline__ uint32_t int8_code_exact(float v, float s) {   // RNE, clamp +-127
+  int q = __float2int_rn(__fdiv_rn(v, s));
+  q = max(-127, min(127, q));
+  return static_cast<uint32_t>(q) & 0xFFu;
+}
+__device__ __forceinline__ uint32_t e4m3_code_exact(float v, float s) {
+  return static_cast<uint32_t>(cvt_e4m3x2(__fdiv_rn(v, s), 0.0f)) & 0xFFu;
+}
+__device__ __forceinline__ uint32_t e4m3_code_fast(float t, bool& near) {
+  const uint32_t pair = cvt_e4m3x2(__fmul_rn(t, 1.0f - 0x1p-21f), __fmul_rn(t, 1.0f + 0x1p-21f));
+  near |= (pair & 0xFFu) != (pair >> 8);
+  return pair & 0xFFu;
 }
 
-__device__ __forceinline__ float absmax8(uint4 v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  float a = 0.0f;
+// 8 values -> 8 codes (one uint2), fast path with one exactness flag.
+template <int QT>
+__device__ __forceinline__ uint2 encode8f(const float (&v)[8], float s, float rcp) {
+  bool near = false;
+  uint32_t c[8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) a = fmaxf(a, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
-  return a;
+  for (int i = 0; i < 8; ++i) {
+    const float t = __fmul_rn(v[i], rcp);
+    c[i] = (QT == 1) ? e4m3_code_fast(t, near) : rne_low_byte(t, near);
+  }
+  if (near) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = (QT == 1) ? e4m3_code_exact(v[i], s) : int8_code_exact(v[i], s);
+  }
+  return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24), c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
 }
+
+// 8 bf16 (one uint4) -> 8 codes (one uint2).
+template <int QT>
+__device__ __forceinline__ uint2 encode8(uint4 w, float s, float rcp) {
+  const float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                      bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+  return encode8f<QT>(v, s, rcp);
+}
+
+// Packed absmax of 8 bf16 (finite inputs).
+__device__ __forceinline__ __nv_bfloat162 absmax8_bf2(uint4 v, __nv_bfloat162 m) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m = __hmax2(m, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[i])));
+  return m;
+}
+__device__ __forceinline__ float bf2_max(__nv_bfloat162 m) {
+  return fmaxf(__bfloat162float(m.x), __bfloat162float(m.y));
+}
+__device__ __forceinline__ __nv_bfloat162 bf2_zero() { return __floats2bfloat162_rn(0.0f, 0.0f); }
 
 // Block-wide max; every thread gets the result.  red: >= 32 floats of smem.
 __device__ __forceinline__ float block_max(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = (blockDim.x + 31) >> 5;
+  if (nw == 1) return v;
   __syncthreads();                 // red may still be read from the previous row
   if (lane == 0) red[warp] = v;
   __syncthreads();
@@ -71,28 +122,29 @@ __global__ void __launch_bounds__(1024) quantize_rows_kernel(const __nv_bfloat16
   for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
     const uint4* row = reinterpret_cast<const uint4*>(x + m * ldx);
     uint4 keep[kRowVecs];
-    float a = 0.0f;
+    __nv_bfloat162 mb = bf2_zero();
 #pragma unroll
     for (int j = 0; j < kRowVecs; ++j) {
       const int64_t v = threadIdx.x + static_cast<int64_t>(j) * blockDim.x;
       if (v < nv) {
         keep[j] = __ldg(row + v);
-        a = fmaxf(a, absmax8(keep[j]));
+        mb = absmax8_bf2(keep[j], mb);
       }
     }
     for (int64_t v = threadIdx.x + static_cast<int64_t>(kRowVecs) * blockDim.x; v < nv; v += blockDim.x)
-      a = fmaxf(a, absmax8(__ldg(row + v)));
-    a = block_max(a, red);
+      mb = absmax8_bf2(__ldg(row + v), mb);
+    const float a = block_max(bf2_max(mb), red);
     const float s = absmax_scale<QT>(a);
+    const float rcp = __frcp_rn(s);
     if (threadIdx.x == 0) scale[m] = s;
     uint2* out = reinterpret_cast<uint2*>(q + m * ldq);
 #pragma unroll
     for (int j = 0; j < kRowVecs; ++j) {
       const int64_t v = threadIdx.x + static_cast<int64_t>(j) * blockDim.x;
-      if (v < nv) out[v] = encode8<QT>(keep[j], s);
+      if (v < nv) out[v] = encode8<QT>(keep[j], s, rcp);
     }
     for (int64_t v = threadIdx.x + static_cast<int64_t>(kRowVecs) * blockDim.x; v < nv; v += blockDim.x)
-      out[v] = encode8<QT>(__ldg(row + v), s);
+      out[v] = encode8<QT>(__ldg(row + v), s, rcp);
   }
 }
 
@@ -101,11 +153,11 @@ __global__ void __launch_bounds__(1024) quantize_rows_kernel(const __nv_bfloat16
 __global__ void __launch_bounds__(256) absmax_kernel(const uint4* __restrict__ w, int64_t nvec,
                                                      unsigned* __restrict__ amax_bits) {
   __shared__ float red[32];
-  float a = 0.0f;
+  __nv_bfloat162 mb = bf2_zero();
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nvec;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    a = fmaxf(a, absmax8(__ldg(w + i)));
-  a = block_max(a, red);
+    mb = absmax8_bf2(__ldg(w + i), mb);
+  const float a = block_max(bf2_max(mb), red);
   if (threadIdx.x == 0) atomicMax(amax_bits, __float_as_uint(a));
 }
 
@@ -115,10 +167,11 @@ __global__ void __launch_bounds__(256) quantize_tensor_kernel(const uint4* __res
                                                               const unsigned* __restrict__ amax_bits,
                                                               uint2* __restrict__ q, float* __restrict__ scale) {
   const float s = absmax_scale<QT>(__uint_as_float(*amax_bits));
+  const float rcp = __frcp_rn(s);
   if (blockIdx.x == 0 && threadIdx.x == 0) scale[0] = s;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nvec;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    q[i] = encode8<QT>(__ldg(w + i), s);
+    q[i] = encode8<QT>(__ldg(w + i), s, rcp);
 }
 
 // fp32 -> E4M3FN codes with the quantizers' conversion.

@@ -89,9 +89,11 @@ EncodeTiledFn encode_fn() {
 }
 
 // 2-D row-major tensor [outer, inner] with `row_bytes` between rows, copied in
-// boxes of [box_outer, box_inner] elements with the 128-byte swizzle.
+// boxes of [box_outer, box_inner] elements with the given swizzle (128-byte
+// for the operand tiles, 64-byte for the epilogue's output blocks).
 w8a8_status make_map(CUtensorMap* map, CUtensorMapDataType dt, int elem, const void* base, int64_t inner,
-                     int64_t outer, int64_t row_bytes, int box_inner, int box_outer) {
+                     int64_t outer, int64_t row_bytes, int box_inner, int box_outer,
+                     CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(W8A8_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   if (inner * elem > row_bytes || (row_bytes & 15) != 0 || !aligned16(base))
@@ -101,7 +103,7 @@ w8a8_status make_map(CUtensorMap* map, CUtensorMapDataType dt, int elem, const v
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(W8A8_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return W8A8_OK;
@@ -117,9 +119,25 @@ cudaError_t set_smem_once(Kernel k, size_t bytes, int dev, std::atomic<uint64_t>
   return e;
 }
 
+// Output tensor map for the epilogue's TMA stores: bf16 [M, ldy] in 32 x 32
+// boxes with the 64-byte swizzle.  Used only when ldy % 8 == 0 (16-byte row
+// stride); otherwise the epilogue stores directly and the map is not read.
+w8a8_status make_out_map(CUtensorMap* map, EpiParams* ep, int64_t M, int64_t N) {
+  ep->tma_store = (ep->ldy % 8) == 0 ? 1 : 0;
+  if (!ep->tma_store) {
+    std::memset(map, 0, sizeof(*map));
+    return W8A8_OK;
+  }
+  return make_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ep->y, N, M, ep->ldy * 2, 32, 32,
+                  CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
 template <int KIND, bool B_MN, int BN, int EPI>
 w8a8_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t M, int64_t N, int64_t Kc,
-                        const EpiParams& ep, cudaStream_t st) {
+                        EpiParams ep, cudaStream_t st) {
+  alignas(64) CUtensorMap ty;
+  w8a8_status ms = make_out_map(&ty, &ep, M, N);
+  if (ms != W8A8_OK) return ms;
   using C = GemmCfg<KIND, BN, EPI>;
   static std::atomic<uint64_t> smem_set{0};
   int dev = 0, sms = 0;
@@ -130,7 +148,7 @@ w8a8_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t M,
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
   const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  gemm_kernel<KIND, B_MN, BN, EPI><<<grid, C::kThreads, C::kSmem, st>>>(ta, tb, static_cast<int>(M),
+  gemm_kernel<KIND, B_MN, BN, EPI><<<grid, C::kThreads, C::kSmem, st>>>(ta, tb, ty, static_cast<int>(M),
                                                                         static_cast<int>(N), static_cast<int>(Kc), ep);
   e = cudaGetLastError();
   return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "gemm launch");
@@ -335,8 +353,8 @@ w8a8_status q8_0_quantize(const float* x, int64_t n, void* blocks, w8a8_stream_t
   int sms = 0;
   w8a8_status st = current_device(nullptr, &sms);
   if (st != W8A8_OK) return st;
-  const int64_t groups = (n + 255) / 256;
-  int64_t grid = (groups + kQ80WarpsPerBlock - 1) / kQ80WarpsPerBlock;
+  const int64_t chunks = (n + 256 * kQ80Unroll - 1) / (256 * kQ80Unroll);
+  int64_t grid = (chunks + kQ80WarpsPerBlock - 1) / kQ80WarpsPerBlock;
   if (grid > 16 * sms) grid = 16 * sms;
   q8_0_quantize_kernel<<<static_cast<int>(grid), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       x, n, static_cast<uint8_t*>(blocks));
@@ -352,8 +370,8 @@ w8a8_status q8_0_dequantize(const void* blocks, int64_t n, float* y, w8a8_stream
   int sms = 0;
   w8a8_status st = current_device(nullptr, &sms);
   if (st != W8A8_OK) return st;
-  const int64_t groups = (n + 255) / 256;
-  int64_t grid = (groups + kQ80WarpsPerBlock - 1) / kQ80WarpsPerBlock;
+  const int64_t chunks = (n + 256 * kQ80Unroll - 1) / (256 * kQ80Unroll);
+  int64_t grid = (chunks + kQ80WarpsPerBlock - 1) / kQ80WarpsPerBlock;
   if (grid > 16 * sms) grid = 16 * sms;
   q8_0_dequantize_kernel<<<static_cast<int>(grid), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint8_t*>(blocks), n, y);
@@ -372,12 +390,17 @@ w8a8_status q8_0_to_axis_int8(const void* blocks, int64_t N, int64_t K, int8_t* 
   int dev = 0, sms = 0;
   w8a8_status st = current_device(&dev, &sms);
   if (st != W8A8_OK) return st;
-  const size_t smem = static_cast<size_t>(K / 32) * 34;
+  // one warp per row; each warp stages its row (rounded to 16 bytes) in shared memory
+  const size_t row_stride = (static_cast<size_t>(K / 32) * 34 + 15) & ~static_cast<size_t>(15);
+  int warps = static_cast<int>((200 * 1024) / row_stride);
+  warps = warps < 1 ? 1 : (warps > kRequantMaxWarps ? kRequantMaxWarps : warps);
+  const size_t smem = row_stride * warps;
   static std::atomic<uint64_t> smem_set{0};
-  cudaError_t e = set_smem_once(q8_0_to_axis_int8_kernel, 160 * 1024, dev, smem_set);
+  cudaError_t e = set_smem_once(q8_0_to_axis_int8_kernel, 200 * 1024, dev, smem_set);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(requant)");
-  int64_t grid = N < 8 * sms ? N : 8 * sms;
-  q8_0_to_axis_int8_kernel<<<static_cast<int>(grid), 256, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
+  int64_t grid = (N + warps - 1) / warps;
+  if (grid > 32 * sms) grid = 32 * sms;
+  q8_0_to_axis_int8_kernel<<<static_cast<int>(grid), 32 * warps, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint8_t*>(blocks), N, K, q, scale);
   e = cudaGetLastError();
   return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "q8_0_to_axis_int8 launch");
