@@ -58,7 +58,9 @@ def test_e4m3_device_conversion_matches_oracle(w8, orc):
 
 
 # --------------------------------------------------------------------------- quantize_rows
-ROW_SHAPES = [(1, 16), (5, 48), (127, 512), (129, 3072), (64, 12288), (3, 40000)]
+# rows up to 200 KB take the bulk-copy kernel; (2, 110016) is past that and
+# exercises the register kernel
+ROW_SHAPES = [(1, 16), (5, 48), (127, 512), (129, 3072), (64, 12288), (3, 40000), (2, 110016)]
 
 
 @pytest.mark.parametrize("qt", ["int8", "e4m3"])
@@ -73,6 +75,44 @@ def test_quantize_rows_parity(w8, orc, qt, M, K):
     qr, sr = orc.quantize_rows(workloads.to_u16(x), QT[qt])
     assert np.array_equal(f32(s).view(np.uint32), sr.view(np.uint32))
     assert np.array_equal(u8(q), qr)
+
+
+GOLDEN_ROWS = __import__("json").load(open(__import__("os").path.join(
+    __import__("os").path.dirname(__file__), "golden", "quantize_rows.json")))["cases"]
+
+
+@pytest.mark.parametrize("case", GOLDEN_ROWS, ids=lambda c: c["name"])
+def test_quantize_rows_golden_on_gpu(w8, case):
+    """The hand-derived golden rows (ties, floors, e4m3 grid points) through
+    the device kernels, zero-padded to K = 16 (zeros change no absmax)."""
+    vals = case["x"] + [0.0] * (16 - len(case["x"]))
+    x = torch.tensor([vals], dtype=torch.float32).to(torch.bfloat16).to(DEV)
+    q, s = w8.quantize_rows(x, case["qt"])
+    assert float(s[0]) == float(np.float32(case["scale"]))
+    got = u8(q)[0, :len(case["codes"])]
+    want = np.array(case["codes"], dtype=np.int64)
+    want = (want & 0xFF).astype(np.uint8)
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("qt", ["int8", "e4m3"])
+def test_quantize_rows_exact_ties(w8, orc, qt):
+    """Rows whose quotients x/s fall exactly on rounding boundaries (every
+    half-integer for int8, e4m3 midpoints): the exactness check must route
+    them to the exact division."""
+    if qt == "int8":
+        base = np.arange(-127, 127, dtype=np.float32) + 0.5        # all ties, s = 1 via the 127 entry
+        row = np.concatenate([[127.0], base]).astype(np.float32)
+        row = np.concatenate([row, np.zeros((-row.size) % 16, np.float32)])
+    else:
+        grid = orc.e4m3_to_f32(np.arange(1, 126, dtype=np.uint8)).astype(np.float64)
+        mids = ((grid[1:] + grid[:-1]) / 2).astype(np.float32)      # midpoints, s = 1 via 448
+        row = np.concatenate([[448.0], mids, -mids]).astype(np.float32)
+        row = np.concatenate([row, np.zeros((-row.size) % 16, np.float32)])
+    xb = torch.from_numpy(np.tile(row, (40, 1))).to(torch.bfloat16)
+    q, s = w8.quantize_rows(xb.to(DEV), qt)
+    qr, sr = orc.quantize_rows(workloads.to_u16(xb), QT[qt])
+    assert np.array_equal(f32(s), sr) and np.array_equal(u8(q), qr)
 
 
 def test_quantize_rows_strided_input(w8, orc):

@@ -50,7 +50,8 @@ struct GemmCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;
   static constexpr int kMaxRank = 32;
-  static constexpr int kLrBytes = (EPI == kEpiLowRank) ? kMaxRank * BN * 4 : 0;   // fp32 L2 tile
+  static constexpr int kLrStride = 40;   // bf16 per row of the transposed L2 tile (32 ranks + 8 pad: no bank conflicts)
+  static constexpr int kLrBytes = (EPI == kEpiLowRank) ? BN * kLrStride * 2 : 0;
   static constexpr int kEpiWarps = 8;   // two per TMEM lane quarter, splitting the column chunks
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kStages = (EPI == kEpiLowRank) ? 3 : 4;
@@ -58,7 +59,7 @@ struct GemmCfg {
   static constexpr int kOutBufBytes = 32 * 32 * 2;
   static constexpr int kOutBytes = kEpiWarps * 2 * kOutBufBytes;
   static constexpr size_t kSmem = 1024 /*alignment slack*/ + static_cast<size_t>(kStages) * kStageBytes +
-                                  kLrBytes + kOutBytes + 256 /*barriers*/;
+                                  ((kLrBytes + 1023) & ~1023) + kOutBytes + 256 /*barriers*/;
 };
 
 template <int KIND, bool B_MN, int BN, int EPI>
@@ -77,8 +78,8 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
   constexpr int kStages = C::kStages;
   uint8_t* sA = smem;                                        // kStages x kABytes
   uint8_t* sB = smem + kStages * C::kABytes;                 // kStages x kBBytes
-  float* sLr = reinterpret_cast<float*>(smem + kStages * C::kStageBytes);   // [r][BN] fp32
-  uint8_t* sOut = smem + kStages * C::kStageBytes + C::kLrBytes;             // epilogue staging
+  uint16_t* sLr = reinterpret_cast<uint16_t*>(smem + kStages * C::kStageBytes);   // L2^T [BN][kLrStride] bf16
+  uint8_t* sOut = smem + kStages * C::kStageBytes + ((C::kLrBytes + 1023) & ~1023);   // epilogue staging
   uint8_t* tail = sOut + C::kOutBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(tail);
   uint64_t* empty = full + kStages;
@@ -203,13 +204,19 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
       const int m0 = (tile % tiles_m) * kBM, n0 = (tile / tiles_m) * BN;
       if constexpr (EPI == kEpiLowRank) {
-        // L2[:, n0:n0+BN] as fp32 (zero outside N) for all epilogue warps.
+        // Every epilogue thread is done with the previous tile's L2^T before it
+        // is overwritten.
         if (local > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(lr_done, (local - 1) & 1, abort_flag, 0x500u, limit)))
           break;
+        // L2^T for the tile: sLr[n][k] = L2[k][n0 + n] (bf16), zero for k >= r
+        // or n0 + n >= N.  Consecutive threads read consecutive n (coalesced).
         const int et = threadIdx.x - 64;
-        for (int i = et; i < ep.r * BN; i += kEpiThreads) {
-          const int j = i / BN, c = i % BN;
-          sLr[i] = (n0 + c < N) ? __bfloat162float(ep.lr_l2[static_cast<int64_t>(j) * N + n0 + c]) : 0.0f;
+        for (int i = et; i < C::kMaxRank * BN; i += kEpiThreads) {
+          const int k = i / BN, n = i % BN;
+          uint16_t v = 0;
+          if (k < ep.r && n0 + n < N)
+            v = __bfloat16_as_ushort(ep.lr_l2[static_cast<int64_t>(k) * N + n0 + n]);
+          sLr[n * C::kLrStride + k] = v;
         }
         mbar_arrive(lr_ready);
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(lr_ready, local & 1, abort_flag, 0x600u, limit))) break;
@@ -218,124 +225,204 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
       // warp-collective tcgen05.ld, also when the wait ran out.
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[acc], acc_phase, abort_flag, 0x400u | acc, limit))) break;
       tc_fence_after();
-      const int row = m0 + quarter * 32 + lane;
-      const bool row_ok = row < M;
-      float sx = 1.0f;
-      if constexpr (EPI != kEpiPlain) sx = row_ok ? ep.s_row[row] : 0.0f;
-      const float sw0 = (EPI != kEpiPlain && !ep.s_col_axis) ? ep.s_col[0] : 1.0f;
-      float t[C::kMaxRank];
       if constexpr (EPI == kEpiLowRank) {
+        // Accumulator read in the m16n8 fragment layout (16x256b loads), the
+        // layout of warp-level bf16 MMAs that compute T * L2 on the tensor
+        // cores for the same elements.
+        const int g = lane >> 2, tq = lane & 3;
+        const int rbase = m0 + quarter * 32;
+        const float sw0 = ep.s_col[0];    // the residual's tensor-wise scale
+        uint32_t afr[2][2][4];            // T fragments [m16 tile][k16 step][4]
+        float sxr[2][2];                  // s_x of rows g and g + 8 in each m16 tile
 #pragma unroll
-        for (int j = 0; j < C::kMaxRank; ++j)
-          t[j] = (row_ok && j < ep.r) ? __bfloat162float(ep.lr_t[static_cast<int64_t>(row) * ep.r + j]) : 0.0f;
-      }
+        for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int rr = rbase + mt * 16 + g + hh * 8;
+            sxr[mt][hh] = rr < M ? ep.s_row[rr] : 0.0f;
+          }
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const int rr = rbase + mt * 16 + g + (q4 & 1) * 8;
+              const int kk = ks * 16 + 2 * tq + (q4 >> 1) * 8;
+              afr[mt][ks][q4] = (rr < M && kk < ep.r)
+                                    ? *reinterpret_cast<const uint32_t*>(ep.lr_t + static_cast<int64_t>(rr) * ep.r + kk)
+                                    : 0u;
+            }
+          }
+        }
+        const int nks = (ep.r + 15) / 16;
 #pragma unroll 1
-      for (int c = group; c < BN / 32; c += kGroups) {
-        const int nc = n0 + c * 32;
-        if (nc >= N) break;                       // warp-uniform
-        const bool full_chunk = nc + 32 <= N;
-        // Column parameters of the chunk, loaded before the TMEM load so that
-        // their latency overlaps it: 16-byte vectors, the same addresses in
-        // every lane (broadcast).
-        float sw[32], bs[32];
-        if constexpr (EPI != kEpiPlain) {
-          if (kAxisOk && ep.s_col_axis) {
-            if (full_chunk) {
+        for (int c = group; c < BN / 32; c += kGroups) {
+          const int nc = n0 + c * 32;
+          if (nc >= N) break;                       // warp-uniform
+          float bcol[4][2];
 #pragma unroll
-              for (int j = 0; j < 32; j += 4) {
-                const float4 f = __ldg(reinterpret_cast<const float4*>(ep.s_col + nc + j));
-                sw[j] = f.x; sw[j + 1] = f.y; sw[j + 2] = f.z; sw[j + 3] = f.w;
-              }
-            } else {
+          for (int i = 0; i < 4; ++i) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j) sw[j] = (nc + j < N) ? __ldg(ep.s_col + nc + j) : 0.0f;
+            for (int u = 0; u < 2; ++u) {
+              const int n = nc + 8 * i + 2 * tq + u;
+              bcol[i][u] = (ep.bias != nullptr && n < N) ? __bfloat162float(ep.bias[n]) : 0.0f;
             }
           }
-          if (ep.bias != nullptr) {
-            if (full_chunk) {
+          uint32_t rfr[2][16];
 #pragma unroll
-              for (int j = 0; j < 32; j += 8) {
-                const uint4 b = __ldg(reinterpret_cast<const uint4*>(ep.bias + nc + j));
-                bs[j] = bf16_lo(b.x); bs[j + 1] = bf16_hi(b.x); bs[j + 2] = bf16_lo(b.y); bs[j + 3] = bf16_hi(b.y);
-                bs[j + 4] = bf16_lo(b.z); bs[j + 5] = bf16_hi(b.z); bs[j + 6] = bf16_lo(b.w); bs[j + 7] = bf16_hi(b.w);
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) bs[j] = (nc + j < N) ? __bfloat162float(ep.bias[nc + j]) : 0.0f;
-            }
-          }
-        }
-        uint32_t r[32];
-        tmem_ld_x32(tmem + lane_base + static_cast<uint32_t>(acc * BN + c * 32), r);
-        tmem_ld_wait();
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int>(r[j])) : __uint_as_float(r[j]);
-          if constexpr (EPI != kEpiPlain) {
-            a = __fmul_rn(__fmul_rn(a, sx), (kAxisOk && ep.s_col_axis) ? sw[j] : sw0);
-            if (ep.bias != nullptr) a = __fadd_rn(a, bs[j]);
-          }
-          v[j] = a;
-        }
-        if constexpr (EPI == kEpiLowRank) {
-          float lr[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) lr[j] = 0.0f;
-#pragma unroll
-          for (int q = 0; q < C::kMaxRank; ++q) {
-            if (q >= ep.r) break;
-            const float4* l2row = reinterpret_cast<const float4*>(sLr + q * BN + c * 32);
-#pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4) {
-              const float4 w = l2row[j4];
-              lr[4 * j4 + 0] = __fmaf_rn(t[q], w.x, lr[4 * j4 + 0]);
-              lr[4 * j4 + 1] = __fmaf_rn(t[q], w.y, lr[4 * j4 + 1]);
-              lr[4 * j4 + 2] = __fmaf_rn(t[q], w.z, lr[4 * j4 + 2]);
-              lr[4 * j4 + 3] = __fmaf_rn(t[q], w.w, lr[4 * j4 + 3]);
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __fadd_rn(v[j], lr[j]);
-        }
-        if (ep.tma_store) {
-          // Stage the warp's 32 x 32 bf16 block in shared memory with the 64-byte
-          // swizzle (16-byte unit j of row l at unit j ^ ((l >> 1) & 3)), then
-          // one lane stores it with TMA; the box is clipped at M and N.
+          for (int mt = 0; mt < 2; ++mt)
+            tmem_ld_16x256b_x4(tmem + (static_cast<uint32_t>(quarter * 32 + mt * 16) << 16) +
+                                   static_cast<uint32_t>(acc * BN + c * 32),
+                               rfr[mt]);
+          tmem_ld_wait();
           uint8_t* buf = sOut + ((e * 2 + (out_iter & 1)) * C::kOutBufBytes);
-          if (lane == 0) bulk_wait_read<1>();     // this buffer's previous store has read it
-          __syncwarp();
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint4 p;
-            p.x = pack_bf16x2(v[8 * j], v[8 * j + 1]);
-            p.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-            p.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-            p.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
-            *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) = p;
+          if (ep.tma_store) {
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && m0 + quarter * 32 < M) {   // skip blocks wholly below the last row
-            tma_store_2d(&tmY, buf, nc, m0 + quarter * 32);
-            bulk_commit();
-          }
-          ++out_iter;
-        } else if (row_ok) {
-          __nv_bfloat16* out = ep.y + static_cast<int64_t>(row) * ep.ldy + nc;
-          if (nc + 32 <= N && (ep.ldy & 7) == 0) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 8) {
-              uint4 p;
-              p.x = pack_bf16x2(v[j], v[j + 1]);
-              p.y = pack_bf16x2(v[j + 2], v[j + 3]);
-              p.z = pack_bf16x2(v[j + 4], v[j + 5]);
-              p.w = pack_bf16x2(v[j + 6], v[j + 7]);
-              *reinterpret_cast<uint4*>(out + j) = p;
+          for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              // lr = T * L2 on the tensor cores from a zero accumulator (the
+              // MMA does not add an fp32 C operand at full precision), then
+              // y = (((acc * s_x) * s_w) + bias) + lr, each an fp32 RN operation.
+              float lr[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+              const uint16_t* brow = sLr + (c * 32 + 8 * i + g) * C::kLrStride + 2 * tq;
+#pragma unroll
+              for (int ks = 0; ks < 2; ++ks) {
+                if (ks < nks)
+                  mma_bf16_m16n8k16(lr, afr[mt][ks], *reinterpret_cast<const uint32_t*>(brow + ks * 16),
+                                    *reinterpret_cast<const uint32_t*>(brow + ks * 16 + 8));
+              }
+              float d[4];
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                float a = __int2float_rn(static_cast<int>(rfr[mt][4 * i + q4]));
+                a = __fmul_rn(__fmul_rn(a, sxr[mt][q4 >> 1]), sw0);
+                if (ep.bias != nullptr) a = __fadd_rn(a, bcol[i][q4 & 1]);
+                d[q4] = __fadd_rn(a, lr[q4]);
+              }
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                const int rl = mt * 16 + g + hh * 8;            // row within the warp's 32-row block
+                if (ep.tma_store) {
+                  *reinterpret_cast<uint32_t*>(buf + rl * 64 + ((i ^ ((rl >> 1) & 3)) << 4) + 4 * tq) =
+                      pack_bf16x2(d[2 * hh], d[2 * hh + 1]);
+                } else {   // row stride not a 16-byte multiple: guarded 2-byte stores
+                  const int rr = rbase + rl, n = nc + 8 * i + 2 * tq;
+                  if (rr < M) {
+                    __nv_bfloat16* out = ep.y + static_cast<int64_t>(rr) * ep.ldy;
+                    if (n < N) out[n] = __float2bfloat16_rn(d[2 * hh]);
+                    if (n + 1 < N) out[n + 1] = __float2bfloat16_rn(d[2 * hh + 1]);
+                  }
+                }
+              }
             }
-          } else {
-            for (int j = 0; j < 32; ++j)
-              if (nc + j < N) out[j] = __float2bfloat16_rn(v[j]);
+          }
+          if (ep.tma_store) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && rbase < M) {
+              tma_store_2d(&tmY, buf, nc, rbase);
+              bulk_commit();
+            }
+            ++out_iter;
+          }
+        }
+      } else {
+        const int row = m0 + quarter * 32 + lane;
+        const bool row_ok = row < M;
+        float sx = 1.0f;
+        if constexpr (EPI != kEpiPlain) sx = row_ok ? ep.s_row[row] : 0.0f;
+        const float sw0 = (EPI != kEpiPlain && !ep.s_col_axis) ? ep.s_col[0] : 1.0f;
+  #pragma unroll 1
+        for (int c = group; c < BN / 32; c += kGroups) {
+          const int nc = n0 + c * 32;
+          if (nc >= N) break;                       // warp-uniform
+          const bool full_chunk = nc + 32 <= N;
+          // Column parameters of the chunk, loaded before the TMEM load so that
+          // their latency overlaps it: 16-byte vectors, the same addresses in
+          // every lane (broadcast).
+          float sw[32], bs[32];
+          if constexpr (EPI != kEpiPlain) {
+            if (kAxisOk && ep.s_col_axis) {
+              if (full_chunk) {
+  #pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                  const float4 f = __ldg(reinterpret_cast<const float4*>(ep.s_col + nc + j));
+                  sw[j] = f.x; sw[j + 1] = f.y; sw[j + 2] = f.z; sw[j + 3] = f.w;
+                }
+              } else {
+  #pragma unroll
+                for (int j = 0; j < 32; ++j) sw[j] = (nc + j < N) ? __ldg(ep.s_col + nc + j) : 0.0f;
+              }
+            }
+            if (ep.bias != nullptr) {
+              if (full_chunk) {
+  #pragma unroll
+                for (int j = 0; j < 32; j += 8) {
+                  const uint4 b = __ldg(reinterpret_cast<const uint4*>(ep.bias + nc + j));
+                  bs[j] = bf16_lo(b.x); bs[j + 1] = bf16_hi(b.x); bs[j + 2] = bf16_lo(b.y); bs[j + 3] = bf16_hi(b.y);
+                  bs[j + 4] = bf16_lo(b.z); bs[j + 5] = bf16_hi(b.z); bs[j + 6] = bf16_lo(b.w); bs[j + 7] = bf16_hi(b.w);
+                }
+              } else {
+  #pragma unroll
+                for (int j = 0; j < 32; ++j) bs[j] = (nc + j < N) ? __bfloat162float(ep.bias[nc + j]) : 0.0f;
+              }
+            }
+          }
+          uint32_t r[32];
+          tmem_ld_x32(tmem + lane_base + static_cast<uint32_t>(acc * BN + c * 32), r);
+          tmem_ld_wait();
+          float v[32];
+  #pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int>(r[j])) : __uint_as_float(r[j]);
+            if constexpr (EPI != kEpiPlain) {
+              a = __fmul_rn(__fmul_rn(a, sx), (kAxisOk && ep.s_col_axis) ? sw[j] : sw0);
+              if (ep.bias != nullptr) a = __fadd_rn(a, bs[j]);
+            }
+            v[j] = a;
+          }
+          if (ep.tma_store) {
+            // Stage the warp's 32 x 32 bf16 block in shared memory with the 64-byte
+            // swizzle (16-byte unit j of row l at unit j ^ ((l >> 1) & 3)), then
+            // one lane stores it with TMA; the box is clipped at M and N.
+            uint8_t* buf = sOut + ((e * 2 + (out_iter & 1)) * C::kOutBufBytes);
+            if (lane == 0) bulk_wait_read<1>();     // this buffer's previous store has read it
+            __syncwarp();
+  #pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 p;
+              p.x = pack_bf16x2(v[8 * j], v[8 * j + 1]);
+              p.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+              p.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+              p.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+              *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) = p;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && m0 + quarter * 32 < M) {   // skip blocks wholly below the last row
+              tma_store_2d(&tmY, buf, nc, m0 + quarter * 32);
+              bulk_commit();
+            }
+            ++out_iter;
+          } else if (row_ok) {
+            __nv_bfloat16* out = ep.y + static_cast<int64_t>(row) * ep.ldy + nc;
+            if (nc + 32 <= N && (ep.ldy & 7) == 0) {
+  #pragma unroll
+              for (int j = 0; j < 32; j += 8) {
+                uint4 p;
+                p.x = pack_bf16x2(v[j], v[j + 1]);
+                p.y = pack_bf16x2(v[j + 2], v[j + 3]);
+                p.z = pack_bf16x2(v[j + 4], v[j + 5]);
+                p.w = pack_bf16x2(v[j + 6], v[j + 7]);
+                *reinterpret_cast<uint4*>(out + j) = p;
+              }
+            } else {
+              for (int j = 0; j < 32; ++j)
+                if (nc + j < N) out[j] = __float2bfloat16_rn(v[j]);
+            }
           }
         }
       }

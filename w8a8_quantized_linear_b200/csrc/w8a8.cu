@@ -156,18 +156,44 @@ w8a8_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t M,
 
 w8a8_status launch_quantize_rows(const void* x, int64_t ldx, int64_t M, int64_t K, int qt, void* q, int64_t ldq,
                                  float* s, cudaStream_t st) {
-  const int64_t nv = K / 8;
-  int64_t t = (nv + kRowVecs - 1) / kRowVecs;
-  t = round_up(t, 32);
-  if (t < 32) t = 32;
-  if (t > 1024) t = 1024;
-  const int grid = static_cast<int>(M < (1 << 20) ? M : (1 << 20));
   const auto* xp = static_cast<const __nv_bfloat16*>(x);
   auto* qp = static_cast<uint8_t*>(q);
-  if (qt == W8A8_E4M3)
-    quantize_rows_kernel<1><<<grid, static_cast<int>(t), 0, st>>>(xp, ldx, M, K, qp, ldq, s);
-  else
-    quantize_rows_kernel<0><<<grid, static_cast<int>(t), 0, st>>>(xp, ldx, M, K, qp, ldq, s);
+  const int64_t nv = K / 8;
+  const int64_t tw = (nv + 32 * kTeamVecs - 1) / (32 * kTeamVecs);   // warps per row
+  if (tw <= 8) {
+    int team_w = 1;
+    while (team_w < tw) team_w *= 2;
+    const int64_t teams = 8 / team_w;
+    const int grid = static_cast<int>((M + teams - 1) / teams < (1 << 20) ? (M + teams - 1) / teams : (1 << 20));
+#define W8A8_TEAM_LAUNCH(QT, TW) \
+  quantize_rows_team_kernel<QT, TW><<<grid, 256, 0, st>>>(xp, ldx, M, K, qp, ldq, s)
+    if (qt == W8A8_E4M3) {
+      switch (team_w) {
+        case 1: W8A8_TEAM_LAUNCH(1, 1); break;
+        case 2: W8A8_TEAM_LAUNCH(1, 2); break;
+        case 4: W8A8_TEAM_LAUNCH(1, 4); break;
+        default: W8A8_TEAM_LAUNCH(1, 8); break;
+      }
+    } else {
+      switch (team_w) {
+        case 1: W8A8_TEAM_LAUNCH(0, 1); break;
+        case 2: W8A8_TEAM_LAUNCH(0, 2); break;
+        case 4: W8A8_TEAM_LAUNCH(0, 4); break;
+        default: W8A8_TEAM_LAUNCH(0, 8); break;
+      }
+    }
+#undef W8A8_TEAM_LAUNCH
+  } else {
+    int64_t t = (nv + kRowVecs - 1) / kRowVecs;
+    t = round_up(t, 32);
+    if (t < 32) t = 32;
+    if (t > 1024) t = 1024;
+    const int grid = static_cast<int>(M < (1 << 20) ? M : (1 << 20));
+    if (qt == W8A8_E4M3)
+      quantize_rows_kernel<1><<<grid, static_cast<int>(t), 0, st>>>(xp, ldx, M, K, qp, ldq, s);
+    else
+      quantize_rows_kernel<0><<<grid, static_cast<int>(t), 0, st>>>(xp, ldx, M, K, qp, ldq, s);
+  }
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "quantize_rows launch");
 }
