@@ -54,12 +54,18 @@ struct GemmCfg {
   static constexpr int kLrBytes = (EPI == kEpiLowRank) ? BN * kLrStride * 2 : 0;
   static constexpr int kEpiWarps = 8;   // two per TMEM lane quarter, splitting the column chunks
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
-  static constexpr int kStages = (EPI == kEpiLowRank) ? 3 : 4;
+  // as many pipeline stages as the shared memory holds (4 for 128x256 tiles,
+  // 8 for 128x64 tiles, whose CTAs must keep more bytes in flight), at most 8
+  static constexpr int kFixedBytes = 1024 + ((kLrBytes + 1023) & ~1023) + kEpiWarps * 2 * 32 * 32 * 2 + 256;
+  static constexpr int kStagesFit = (232448 - kFixedBytes) / kStageBytes;
+  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   // per epilogue warp, two 32 x 32 bf16 staging buffers for the TMA store
   static constexpr int kOutBufBytes = 32 * 32 * 2;
   static constexpr int kOutBytes = kEpiWarps * 2 * kOutBufBytes;
   static constexpr size_t kSmem = 1024 /*alignment slack*/ + static_cast<size_t>(kStages) * kStageBytes +
                                   ((kLrBytes + 1023) & ~1023) + kOutBytes + 256 /*barriers*/;
+  static constexpr int kCtasPerSm = 1;
+  static_assert(kSmem <= 232448, "shared memory per block");
 };
 
 template <int KIND, bool B_MN, int BN, int EPI>

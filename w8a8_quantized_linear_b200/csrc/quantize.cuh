@@ -83,61 +83,45 @@ __device__ __forceinline__ uint2 encode8(uint4 w, float s, float rcp) {
   return encode8f<QT>(v, s, rcp);
 }
 
-// The same codes with packed fp32 pair arithmetic (two values per multiply
-// and add); the exactness flag is the largest |remainder| of the group for
-// int8, and a code mismatch between the two ends of the interval for e4m3.
+// The same codes, four fp32 operations per value.  int8: the exact product
+// x * rcp is rounded once, to an integer, by fma(x, rcp, 1.5 * 2^23) (ties
+// to even), and its exact remainder d = fma(x, rcp, -rne) is rounded once.
+// x * rcp lies within 2 ulp of fl(x / s), so |d| < 0.5 - 2^-14 proves that
+// fl(x / s) rounds to the same integer; a group with any |d| at the margin
+// takes the exact division.  e4m3: as encode8 (interval ends compared).
 template <int QT>
-__device__ __forceinline__ uint2 encode8_x2(uint4 w, float s, float rcp) {
-  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-  const uint64_t rcp2 = f2_pack(rcp, rcp);
-  uint32_t out[2];
+__device__ __forceinline__ uint2 encode8_fast(uint4 w, float s, float rcp) {
+  const float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                      bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+  uint32_t c[8];
   bool near = false;
   if constexpr (QT == 1) {
-    const uint64_t lo_f = f2_pack(1.0f - 0x1p-21f, 1.0f - 0x1p-21f);
-    const uint64_t hi_f = f2_pack(1.0f + 0x1p-21f, 1.0f + 0x1p-21f);
-    uint32_t pairs[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint64_t t = f2_mul(bf16x2_to_f2(ws[i]), rcp2);
-      float a0, a1, b0, b1;
-      f2_unpack(f2_mul(t, lo_f), a0, a1);
-      f2_unpack(f2_mul(t, hi_f), b0, b1);
-      const uint32_t ca = cvt_e4m3x2(a0, a1), cb = cvt_e4m3x2(b0, b1);   // codes of both elements, each end
+    for (int i = 0; i < 8; i += 2) {
+      const float t0 = __fmul_rn(v[i], rcp), t1 = __fmul_rn(v[i + 1], rcp);
+      const uint32_t ca = cvt_e4m3x2(__fmul_rn(t0, 1.0f - 0x1p-21f), __fmul_rn(t1, 1.0f - 0x1p-21f));
+      const uint32_t cb = cvt_e4m3x2(__fmul_rn(t0, 1.0f + 0x1p-21f), __fmul_rn(t1, 1.0f + 0x1p-21f));
       near |= ca != cb;
-      pairs[i] = ca;
+      c[i] = ca & 0xFFu;
+      c[i + 1] = ca >> 8;
     }
-    out[0] = prmt(pairs[0], pairs[1], 0x5410u);
-    out[1] = prmt(pairs[2], pairs[3], 0x5410u);
   } else {
-    const uint64_t magic2 = f2_pack(kRneMagic, kRneMagic);
     float dmax = 0.0f;
-    uint32_t big[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint64_t t = f2_mul(bf16x2_to_f2(ws[i]), rcp2);
-      const uint64_t b = f2_add(t, magic2);
-      const uint64_t d = f2_sub(t, f2_sub(b, magic2));
-      float b0, b1, d0, d1;
-      f2_unpack(b, b0, b1);
-      f2_unpack(d, d0, d1);
-      dmax = fmaxf(dmax, fmaxf(fabsf(d0), fabsf(d1)));
-      big[2 * i] = __float_as_uint(b0);
-      big[2 * i + 1] = __float_as_uint(b1);
+    for (int i = 0; i < 8; ++i) {
+      const float big = __fmaf_rn(v[i], rcp, kRneMagic);
+      const float d = __fmaf_rn(v[i], rcp, -__fsub_rn(big, kRneMagic));
+      dmax = fmaxf(dmax, fabsf(d));
+      c[i] = __float_as_uint(big);
     }
     near = dmax > kNearHalf;
-    out[0] = prmt(prmt(big[0], big[1], 0x0040u), prmt(big[2], big[3], 0x0040u), 0x5410u);
-    out[1] = prmt(prmt(big[4], big[5], 0x0040u), prmt(big[6], big[7], 0x0040u), 0x5410u);
   }
   if (near) {
-    const float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
-                        bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
-    uint32_t c[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) c[i] = (QT == 1) ? e4m3_code_exact(v[i], s) : int8_code_exact(v[i], s);
-    out[0] = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-    out[1] = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
   }
-  return make_uint2(out[0], out[1]);
+  return make_uint2(prmt(prmt(c[0], c[1], 0x0040u), prmt(c[2], c[3], 0x0040u), 0x5410u),
+                    prmt(prmt(c[4], c[5], 0x0040u), prmt(c[6], c[7], 0x0040u), 0x5410u));
 }
 
 // Packed absmax of 8 bf16 (finite inputs).
@@ -209,9 +193,9 @@ __global__ void __launch_bounds__(1024) quantize_rows_kernel(const __nv_bfloat16
 // row, every lane holding up to kTeamVecs vectors of the row in registers
 // (one pass over HBM).  Teams reduce the absmax with warp shuffles and, for
 // TW > 1, a per-team named barrier over double-buffered shared slots.
-constexpr int kTeamVecs = 12;
+constexpr int kTeamVecs = 8;
 template <int QT, int TW>
-__global__ void __launch_bounds__(256) quantize_rows_team_kernel(const __nv_bfloat16* __restrict__ x, int64_t ldx,
+__global__ void __launch_bounds__(256, 4) quantize_rows_team_kernel(const __nv_bfloat16* __restrict__ x, int64_t ldx,
                                                                  int64_t M, int64_t K, uint8_t* __restrict__ q,
                                                                  int64_t ldq, float* __restrict__ scale) {
   __shared__ float red[2][8];
@@ -219,7 +203,7 @@ __global__ void __launch_bounds__(256) quantize_rows_team_kernel(const __nv_bflo
   const int team = warp / TW, tw = warp % TW;
   const int teams = (blockDim.x >> 5) / TW;
   const int tl = tw * 32 + lane;
-  const int64_t nv = K >> 3;
+  const int nv = static_cast<int>(K >> 3);
   int iter = 0;
   for (int64_t m = blockIdx.x * static_cast<int64_t>(teams) + team; m < M;
        m += static_cast<int64_t>(gridDim.x) * teams, ++iter) {
@@ -227,13 +211,13 @@ __global__ void __launch_bounds__(256) quantize_rows_team_kernel(const __nv_bflo
     uint4 keep[kTeamVecs];
 #pragma unroll
     for (int j = 0; j < kTeamVecs; ++j) {
-      const int64_t v = tl + static_cast<int64_t>(j) * (32 * TW);
+      const int v = tl + j * (32 * TW);
       if (v < nv) keep[j] = __ldg(row + v);
     }
     __nv_bfloat162 mb = bf2_zero();
 #pragma unroll
     for (int j = 0; j < kTeamVecs; ++j)
-      if (tl + static_cast<int64_t>(j) * (32 * TW) < nv) mb = absmax8_bf2(keep[j], mb);
+      if (tl + j * (32 * TW) < nv) mb = absmax8_bf2(keep[j], mb);
     float a = bf2_max(mb);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
@@ -249,8 +233,8 @@ __global__ void __launch_bounds__(256) quantize_rows_team_kernel(const __nv_bflo
     uint2* out = reinterpret_cast<uint2*>(q + m * ldq);
 #pragma unroll
     for (int j = 0; j < kTeamVecs; ++j) {
-      const int64_t v = tl + static_cast<int64_t>(j) * (32 * TW);
-      if (v < nv) out[v] = encode8_x2<QT>(keep[j], s, rcp);
+      const int v = tl + j * (32 * TW);
+      if (v < nv) out[v] = encode8_fast<QT>(keep[j], s, rcp);
     }
   }
 }
@@ -278,7 +262,7 @@ __global__ void __launch_bounds__(256) quantize_tensor_kernel(const uint4* __res
   if (blockIdx.x == 0 && threadIdx.x == 0) scale[0] = s;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nvec;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    q[i] = encode8_x2<QT>(__ldg(w + i), s, rcp);
+    q[i] = encode8_fast<QT>(__ldg(w + i), s, rcp);
 }
 
 // fp32 -> E4M3FN codes with the quantizers' conversion.

@@ -147,7 +147,8 @@ w8a8_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t M,
   cudaError_t e = set_smem_once(kern, C::kSmem, dev, smem_set);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
   const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  const int64_t slots = static_cast<int64_t>(sms) * C::kCtasPerSm;
+  const int grid = static_cast<int>(tiles < slots ? tiles : slots);
   gemm_kernel<KIND, B_MN, BN, EPI><<<grid, C::kThreads, C::kSmem, st>>>(ta, tb, ty, static_cast<int>(M),
                                                                         static_cast<int>(N), static_cast<int>(Kc), ep);
   e = cudaGetLastError();
