@@ -142,6 +142,29 @@ def gpu_identity(torch, dev):
     return uuid, index
 
 
+# ----------------------------------------------------------------------------- ranks
+def rank_workload(rank: int):
+    """Per-rank step inputs: every rank quantizes its own seeded tokens (the
+    path shards by tokens) against the same weights."""
+    import workloads
+    wl = workloads.dit_mlp()
+    if rank > 0:
+        wl["x"] = workloads.with_outlier_channels((M_TOK, HID), 1.0, 21 + 1000 * rank)
+        wl["dy2"] = workloads.normal((M_TOK, HID), 1e-3, 24 + 1000 * rank)
+    return wl
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest of the ranks' values (timings are taken as the slowest
+    rank's); the identity without a process group."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ----------------------------------------------------------------------------- oracle (CPU)
 def oracle_chain_rows(orc, wl, W1r, s1r, W2r, s2r, rows):
     """The step on the CPU oracle for a subset of token rows (every step is
@@ -226,7 +249,7 @@ def workload_config():
     return {"workload": "int W8A8 DiT MLP block fwd+dgrad (up 3072->12288, down 12288->3072, "
                         "dgrad through both), tensor-wise int8 W, token-wise int8 activations",
             "M": M_TOK, "hidden": HID, "mlp": MLP, "global_batch_tokens_per_gpu": M_TOK,
-            "parallelism": "token-sharded replicas", "l2": "flushed (256 MiB write) between timed steps"}
+            "parallelism": "token-sharded replicas", "l2": "flushed between timed steps: 256 MiB written, then read back (outside the step's events)"}
 
 
 # ----------------------------------------------------------------------------- ours
@@ -248,10 +271,7 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     w8.lib()
 
-    wl = workloads.dit_mlp()
-    if rank > 0:   # each rank its own tokens (weak scaling)
-        wl["x"] = workloads.with_outlier_channels((M_TOK, HID), 1.0, 21 + 1000 * rank)
-        wl["dy2"] = workloads.normal((M_TOK, HID), 1e-3, 24 + 1000 * rank)
+    wl = rank_workload(rank)
     X = wl["x"].to(dev)
     dY2 = wl["dy2"].to(dev)
     W1q, s1 = w8.quantize_weight(wl["w1"].to(dev), "int8", "tensor")
@@ -282,6 +302,7 @@ def run_ours(args, rank, world, local_rank):
 
     for _ in range(args.warmup):
         flush.fill_(1)
+        flush_sum = flush.view(torch.int64).sum()
         step([E() for _ in range(9)])
     torch.cuda.synchronize()
     assert w8.device_status() == 0, "device-side error during warm-up"
@@ -293,7 +314,8 @@ def run_ours(args, rank, world, local_rank):
     with ClockSampler(*gpu_identity(torch, dev)) as clk:
         wall0 = time.perf_counter()
         for i in range(args.steps):
-            flush.fill_(i & 0xFF)          # L2 flush, outside the step's events
+            flush.fill_(i & 0xFF)          # L2 flush (write, then read back so that no dirty
+            flush_sum = flush.view(torch.int64).sum()   # lines are left for the step), outside the step's events
             step(events[i])
         torch.cuda.synchronize()
         wall = time.perf_counter() - wall0
@@ -302,54 +324,67 @@ def run_ours(args, rank, world, local_rank):
     step_ms = [ev[0].elapsed_time(ev[8]) for ev in events]
     gemm_ms = [ev[k - 1].elapsed_time(ev[k]) for ev in events for k in (2, 4, 6, 8)]
     quant_ms = [ev[k - 1].elapsed_time(ev[k]) for ev in events for k in (1, 3, 5, 7)]
-    total_ms = sum(step_ms)
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, dev)
     ms_per_step = total_ms / args.steps
     value = world * OPS_PER_STEP * args.steps / (total_ms * 1e-3) / 1e12
     assert w8.device_status() == 0, "device-side error during the timed steps"
 
-    # ---- end to end: pinned host inputs -> public API -> host result
+    # ---- end to end: pinned host inputs -> public API -> pinned host results.
+    # Three streams: the host->device copies of step i+1 and the device->host
+    # copies of step i-1 overlap the compute of step i (double-buffered device
+    # inputs and outputs); every step copies its inputs in and its results out.
     e2e = None
     if args.e2e_steps > 0:
         hx = wl["x"].pin_memory()
         hdy = wl["dy2"].pin_memory()
-        hy2 = torch.empty((M_TOK, HID), dtype=torch.bfloat16).pin_memory()
-        hdx1 = torch.empty((M_TOK, HID), dtype=torch.bfloat16).pin_memory()
+        hy2 = [torch.empty((M_TOK, HID), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        hdx1 = [torch.empty((M_TOK, HID), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
         ws = torch.empty(w8.workspace_bytes(w8.OP_LINEAR_FWD, M_TOK, MLP, MLP), dtype=torch.uint8, device=dev)
-        Xd, dYd = torch.empty_like(X), torch.empty_like(dY2)
+        Xd = [torch.empty_like(X) for _ in range(2)]
+        dYd = [torch.empty_like(dY2) for _ in range(2)]
+        Y2d = [torch.empty_like(Y2) for _ in range(2)]
+        dX1d = [torch.empty_like(dX1) for _ in range(2)]
+        s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        ev = lambda: torch.cuda.Event()
+        in_done, cmp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
 
-        def e2e_step():
-            Xd.copy_(hx, non_blocking=True)
-            dYd.copy_(hdy, non_blocking=True)
-            w8.linear_fwd(Xd, W1q, s1, out=Y1, ws=ws)
-            w8.linear_fwd(Y1, W2q, s2, out=Y2, ws=ws)
-            w8.linear_dgrad(dYd, W2q, s2, out=dX2, ws=ws)
-            w8.linear_dgrad(dX2, W1q, s1, out=dX1, ws=ws)
-            hy2.copy_(Y2, non_blocking=True)
-            hdx1.copy_(dX1, non_blocking=True)
+        def e2e_steps(n):
+            for i in range(n):
+                b = i & 1
+                with torch.cuda.stream(s_in):
+                    s_in.wait_event(cmp_done[b])            # step i-2 finished reading this input buffer
+                    Xd[b].copy_(hx, non_blocking=True)
+                    dYd[b].copy_(hdy, non_blocking=True)
+                    in_done[b].record(s_in)
+                with torch.cuda.stream(s_cmp):
+                    s_cmp.wait_event(in_done[b])
+                    s_cmp.wait_event(out_done[b])           # step i-2's results have left this buffer
+                    w8.linear_fwd(Xd[b], W1q, s1, out=Y1, ws=ws)
+                    w8.linear_fwd(Y1, W2q, s2, out=Y2d[b], ws=ws)
+                    w8.linear_dgrad(dYd[b], W2q, s2, out=dX2, ws=ws)
+                    w8.linear_dgrad(dX2, W1q, s1, out=dX1d[b], ws=ws)
+                    cmp_done[b].record(s_cmp)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(cmp_done[b])
+                    hy2[b].copy_(Y2d[b], non_blocking=True)
+                    hdx1[b].copy_(dX1d[b], non_blocking=True)
+                    out_done[b].record(s_out)
 
-        for _ in range(2):
-            e2e_step()
+        e2e_steps(3)
         torch.cuda.synchronize()
         a, b = E(), E()
-        a.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        b.record(stream)
+        a.record(s_in)
+        e2e_steps(args.e2e_steps)
+        s_in.wait_stream(s_out)
+        b.record(s_in)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b)
-        if dist is not None:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(a.elapsed_time(b), dist, dev)
         e2e = {"value": world * OPS_PER_STEP * args.e2e_steps / (e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": hx.numel() * 2 + hdy.numel() * 2,
-               "d2h_bytes_per_step": hy2.numel() * 2 + hdx1.numel() * 2,
+               "d2h_bytes_per_step": hy2[0].numel() * 2 + hdx1[0].numel() * 2,
                "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps,
-               "api": "w8a8_linear_fwd x2 + w8a8_linear_dgrad x2 (pinned host buffers, copies timed)"}
+               "api": "w8a8_linear_fwd x2 + w8a8_linear_dgrad x2 per step; pinned host buffers; "
+                      "copies in and out timed, overlapped with compute across steps (3 streams)"}
 
     if rank != 0:
         return 0
@@ -429,6 +464,7 @@ def _time(fn, reps, torch, stream, flush):
     ms = []
     for _ in range(reps):
         flush.fill_(3)
+        flush_sum = flush.view(torch.int64).sum()
         a, b = E(), E()
         a.record(stream)
         fn()
@@ -518,7 +554,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-extras", dest="extras", action="store_false")
