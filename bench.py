@@ -459,93 +459,146 @@ def run_case(args):
     return 0
 
 
-def _time(fn, reps, torch, stream, flush):
+L2_BYTES = 126 << 20
+
+
+def _nsets(set_bytes):
+    """Copies of a buffer set to rotate through so that each is touched once
+    per cycle over at least 3x the L2 size (no set is L2-resident when used)."""
+    return max(2, -(-3 * L2_BYTES // max(1, int(set_bytes))))
+
+
+def _time_rot(fns, reps, torch, stream):
+    """Mean time of one call, cycling through ``fns`` (each on its own buffers)
+    back to back between two events on the launching stream."""
+    for f in fns:
+        f()
+    torch.cuda.synchronize()
     E = lambda: torch.cuda.Event(enable_timing=True)
-    fn()
+    a, b = E(), E()
+    a.record(stream)
+    for i in range(reps):
+        fns[i % len(fns)]()
+    b.record(stream)
     torch.cuda.synchronize()
-    ms = []
-    for _ in range(reps):
-        flush.fill_(3)
-        flush_sum = flush.view(torch.int64).sum()
-        a, b = E(), E()
-        a.record(stream)
-        fn()
-        b.record(stream)
-        ms.append((a, b))
-    torch.cuda.synchronize()
-    return statistics.median(x.elapsed_time(y) for x, y in ms)
+    return a.elapsed_time(b) / reps
 
 
 def extras(w8, torch, workloads, dev, peaks, src):
-    """The other rows of the hot path, each timed on its own (median of reps,
-    L2 flushed before each rep)."""
+    """The other rows of the hot path, each timed on its own: mean over reps
+    launched back to back, rotating through copies of the inputs and outputs
+    whose footprint is at least 3x the L2 size."""
     out = {}
     stream = torch.cuda.current_stream(dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     hbm = peaks["hbm_gbs"]
     tc8 = 2.0 * peaks["bf16_tflops"]
+    nbytes = lambda *ts: sum(t.numel() * t.element_size() for t in ts)
     # token-wise quantize (K1) at 4608 x 12288
-    x = workloads.normal((M_TOK, MLP), 1.0, 5).to(dev)
-    q = torch.empty((M_TOK, MLP), dtype=torch.int8, device=dev)
-    s = torch.empty(M_TOK, dtype=torch.float32, device=dev)
-    ms = _time(lambda: w8.quantize_rows(x, "int8", out=q, scale=s), 20, torch, stream, flush)
-    gbs = (x.numel() * 3 + M_TOK * 4) / (ms * 1e-3) / 1e9
+    x0 = workloads.normal((M_TOK, MLP), 1.0, 5).to(dev)
+    sets = []
+    for i in range(_nsets(nbytes(x0) * 1.5)):
+        x = x0.clone()
+        q = torch.empty((M_TOK, MLP), dtype=torch.int8, device=dev)
+        s = torch.empty(M_TOK, dtype=torch.float32, device=dev)
+        sets.append(lambda x=x, q=q, s=s: w8.quantize_rows(x, "int8", out=q, scale=s))
+    ms = _time_rot(sets, 30, torch, stream)
+    gbs = (x0.numel() * 3 + M_TOK * 4) / (ms * 1e-3) / 1e9
     out["quantize_rows_4608x12288"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
-    del x, q
+    del x0, sets
     # float W8A8 forward (e4m3, bias) 4096 x 3072 x 3072
     d = workloads.float_w8a8()
-    wq, sw = w8.quantize_weight(d["w"].to(dev), "e4m3", "tensor")
-    xx, bb = d["x"].to(dev), d["bias"].to(dev)
-    y = torch.empty((4096, 3072), dtype=torch.bfloat16, device=dev)
-    ws = torch.empty(w8.workspace_bytes(0, 4096, 3072, 3072), dtype=torch.uint8, device=dev)
-    ms = _time(lambda: w8.linear_fwd(xx, wq, sw, bias=bb, out=y, ws=ws), 20, torch, stream, flush)
-    xq, sx = w8.quantize_rows(xx, "e4m3")
-    gms = _time(lambda: w8.qgemm_fwd(xq, sx, wq, sw, bias=bb, out=y), 20, torch, stream, flush)
+    wq0, sw = w8.quantize_weight(d["w"].to(dev), "e4m3", "tensor")
+    xx0, bb = d["x"].to(dev), d["bias"].to(dev)
+    xq0, sx0 = w8.quantize_rows(xx0, "e4m3")
+    fsets, gsets = [], []
+    for i in range(_nsets(nbytes(xx0, wq0) + 4096 * 3072 * 2)):
+        xx, wq, xq = xx0.clone(), wq0.clone(), xq0.clone()
+        y = torch.empty((4096, 3072), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(w8.workspace_bytes(0, 4096, 3072, 3072), dtype=torch.uint8, device=dev)
+        fsets.append(lambda xx=xx, wq=wq, y=y, ws=ws: w8.linear_fwd(xx, wq, sw, bias=bb, out=y, ws=ws))
+        gsets.append(lambda xq=xq, wq=wq, y=y: w8.qgemm_fwd(xq, sx0, wq, sw, bias=bb, out=y))
+    ms = _time_rot(fsets, 30, torch, stream)
+    gms = _time_rot(gsets, 30, torch, stream)
     ops = 2 * 4096 * 3072 * 3072
     out["float_w8a8_fwd_4096x3072x3072"] = {"ms": ms, "TOPS": ops / ms / 1e9, "gemm_ms": gms,
                                             "gemm_TOPS": ops / gms / 1e9, "gemm_frac_fp8_burst": ops / gms / 1e9 / tc8}
+    del fsets, gsets
     # SVDQuant r=32, 4608 x 3072 x 3072
     d = workloads.svdquant()
-    prep = w8.svdq_prepare(d["w"].to(dev), d["r"])
-    xx = d["x"].to(dev)
-    y = torch.empty((M_TOK, 3072), dtype=torch.bfloat16, device=dev)
-    ws = torch.empty(w8.workspace_bytes(2, M_TOK, 3072, 3072, 32), dtype=torch.uint8, device=dev)
-    ms = _time(lambda: w8.svdq_linear_fwd(xx, prep["rq"], prep["r_scale"], prep["l1"], prep["l2"], out=y, ws=ws),
-               20, torch, stream, flush)
+    prep0 = w8.svdq_prepare(d["w"].to(dev), d["r"])
+    xx0 = d["x"].to(dev)
+    sets = []
+    for i in range(_nsets(nbytes(xx0, prep0["rq"]) + M_TOK * 3072 * 2)):
+        xx = xx0.clone()
+        rq, l1, l2 = prep0["rq"].clone(), prep0["l1"].clone(), prep0["l2"].clone()
+        y = torch.empty((M_TOK, 3072), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(w8.workspace_bytes(2, M_TOK, 3072, 3072, 32), dtype=torch.uint8, device=dev)
+        sets.append(lambda xx=xx, rq=rq, l1=l1, l2=l2, y=y, ws=ws:
+                    w8.svdq_linear_fwd(xx, rq, prep0["r_scale"], l1, l2, out=y, ws=ws))
+    ms = _time_rot(sets, 30, torch, stream)
     ops = 2 * M_TOK * 3072 * 3072
     out["svdquant_r32_fwd_4608x3072x3072"] = {"ms": ms, "TOPS_main": ops / ms / 1e9,
                                               "lowrank_GFLOP": 2 * 2 * M_TOK * 3072 * 32 / 1e9}
-    # GGUF Q8_0: standalone quantize / dequantize of 2^28 fp32, requant, forward sweep
+    del sets
+    # GGUF Q8_0: standalone quantize / dequantize of 2^28 fp32 (each 1.3 GB of traffic)
     n = 1 << 28
-    xf = workloads.q8_0_standalone(n).to(dev)
-    blk = torch.empty(w8.q8_0_bytes(n), dtype=torch.uint8, device=dev)
-    ms = _time(lambda: w8.q8_0_quantize(xf, out=blk), 10, torch, stream, flush)
-    gbs = (4 * n + blk.numel()) / (ms * 1e-3) / 1e9
+    xf0 = workloads.q8_0_standalone(n).to(dev)
+    qsets, dsets = [], []
+    for i in range(2):
+        xf = xf0 if i == 0 else xf0.clone()
+        blk = torch.empty(w8.q8_0_bytes(n), dtype=torch.uint8, device=dev)
+        w8.q8_0_quantize(xf, out=blk)
+        yf = torch.empty_like(xf)
+        qsets.append(lambda xf=xf, blk=blk: w8.q8_0_quantize(xf, out=blk))
+        dsets.append(lambda blk=blk, yf=yf: w8.q8_0_dequantize(blk, n, out=yf))
+    nb = w8.q8_0_bytes(n)
+    ms = _time_rot(qsets, 10, torch, stream)
+    gbs = (4 * n + nb) / (ms * 1e-3) / 1e9
     out["q8_0_quantize_2^28"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
-    ms = _time(lambda: w8.q8_0_dequantize(blk, n, out=xf), 10, torch, stream, flush)
-    gbs = (4 * n + blk.numel()) / (ms * 1e-3) / 1e9
+    ms = _time_rot(dsets, 10, torch, stream)
+    gbs = (4 * n + nb) / (ms * 1e-3) / 1e9
     out["q8_0_dequantize_2^28"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
-    del xf, blk
+    del xf0, qsets, dsets
+    # requant Q8_0 -> axis int8 (K10), 12288 x 3072
     g = workloads.gguf_q8_0(M=max(workloads.GGUF_MS))
-    wb = w8.q8_0_quantize(g["w_f32"].reshape(-1).to(dev))
-    wq, sw = w8.q8_0_to_axis_int8(wb, MLP, HID)
-    ms = _time(lambda: w8.q8_0_to_axis_int8(wb, MLP, HID), 20, torch, stream, flush)
-    gbs = (wb.numel() + MLP * HID + MLP * 4) / (ms * 1e-3) / 1e9
+    wb0 = w8.q8_0_quantize(g["w_f32"].reshape(-1).to(dev))
+    wq0, sw = w8.q8_0_to_axis_int8(wb0, MLP, HID)
+    sets = []
+    for i in range(_nsets(nbytes(wb0, wq0))):
+        wb = wb0.clone()
+        q = torch.empty_like(wq0)
+        s = torch.empty(MLP, dtype=torch.float32, device=dev)
+        sets.append(lambda wb=wb, q=q, s=s: w8.q8_0_to_axis_int8(wb, MLP, HID, out=q, scale=s))
+    ms = _time_rot(sets, 30, torch, stream)
+    gbs = (wb0.numel() + MLP * HID + MLP * 4) / (ms * 1e-3) / 1e9
     out["q8_0_to_axis_int8_12288x3072"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
-    wt = workloads.normal((MLP, HID), 0.02, 9).to(dev)
-    ms = _time(lambda: w8.quantize_weight(wt, "int8", "tensor"), 20, torch, stream, flush)
-    out["quantize_weight_tensor_12288x3072"] = {"ms": ms, "GB/s": wt.numel() * 3 / (ms * 1e-3) / 1e9}
+    del sets
+    # tensor-wise weight quantization (load time), 12288 x 3072
+    wt0 = workloads.normal((MLP, HID), 0.02, 9).to(dev)
+    sets = [lambda wt=(wt0 if i == 0 else wt0.clone()): w8.quantize_weight(wt, "int8", "tensor")
+            for i in range(_nsets(nbytes(wt0) * 1.5))]
+    ms = _time_rot(sets, 30, torch, stream)
+    out["quantize_weight_tensor_12288x3072"] = {"ms": ms, "GB/s": wt0.numel() * 3 / (ms * 1e-3) / 1e9}
+    del sets, wt0
+    # GGUF A8 int forward sweep over M: the weight is rotated too, so that
+    # small M streams it from HBM as it would in a model
     sweep = {}
     xg = g["x"].to(dev)
     for M in workloads.GGUF_MS:
-        xm = xg[:M].contiguous()
-        y = torch.empty((M, MLP), dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(w8.workspace_bytes(0, M, MLP, HID), dtype=torch.uint8, device=dev)
-        ms = _time(lambda: w8.linear_fwd(xm, wq, sw, out=y, ws=ws), 20, torch, stream, flush)
+        xm0 = xg[:M].contiguous()
+        sets = []
+        for i in range(_nsets(nbytes(xm0, wq0) + M * MLP * 2)):
+            xm, wq = xm0.clone(), wq0.clone()
+            y = torch.empty((M, MLP), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(w8.workspace_bytes(0, M, MLP, HID), dtype=torch.uint8, device=dev)
+            sets.append(lambda xm=xm, wq=wq, y=y, ws=ws: w8.linear_fwd(xm, wq, sw, out=y, ws=ws))
+        ms = _time_rot(sets, 30, torch, stream)
         sweep[str(M)] = {"ms": ms, "TOPS": 2 * M * MLP * HID / ms / 1e9,
                          "weight_GB/s": MLP * HID / (ms * 1e-3) / 1e9}
+        del sets
     out["gguf_a8_int_fwd_sweep_N12288_K3072"] = sweep
     out["peaks"] = {"source": src, "hbm_gbs": hbm, "int8_burst_tops": tc8}
+    out["method"] = "mean over back-to-back reps rotating through >= 3x L2 of input/output copies"
     assert w8.device_status() == 0
     return out
 

@@ -161,13 +161,25 @@ def test_q8_0_standalone_full_size(w8, orc):
     assert np.array_equal(f32(y).view(np.uint32), orc.q8_0_dequantize(br, x.numel()).view(np.uint32))
 
 
-@pytest.mark.parametrize("N,K", [(1, 32), (37, 96), (64, 512), (12288, 3072)])
+@pytest.mark.parametrize("N,K", [(1, 32), (37, 96), (64, 512), (12288, 3072), (5, 4096), (7, 12288),
+                                 (3, 32768), (2, 131072)])
 def test_q8_0_to_axis_int8_parity(w8, orc, N, K):
     w = workloads.gguf_q8_0(N=N, K=K, M=1)["w_f32"].numpy().reshape(-1)
     br, _ = orc.q8_0_quantize(w)
     q, s = w8.q8_0_to_axis_int8(torch.from_numpy(br).to(DEV), N, K)
     qr, sr = orc.q8_0_to_axis_int8(br, N, K)
     assert np.array_equal(f32(s), sr)
+    assert np.array_equal(u8(q), qr.view(np.uint8))
+
+
+@pytest.mark.parametrize("N,K", [(13, 256), (50, 3072), (11, 4096), (6, 12288), (4, 32768), (9, 96)])
+def test_q8_0_to_axis_int8_arbitrary_blocks(w8, orc, N, K):
+    """Blocks not produced by a quantizer: -128 codes, zero, negative and
+    subnormal f16 scales, rows sharing one scale (codes come back unchanged)."""
+    br = workloads.raw_q8_0_blocks(N, K, seed=61 + K)
+    q, s = w8.q8_0_to_axis_int8(br.to(DEV), N, K)
+    qr, sr = orc.q8_0_to_axis_int8(br.numpy(), N, K)
+    assert np.array_equal(f32(s).view(np.uint32), sr.view(np.uint32))
     assert np.array_equal(u8(q), qr.view(np.uint8))
 
 

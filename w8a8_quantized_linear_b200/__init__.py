@@ -196,14 +196,16 @@ def q8_0_dequantize(blocks: torch.Tensor, n: int, out=None):
     return y
 
 
-def q8_0_to_axis_int8(blocks: torch.Tensor, N: int, K: int):
+def q8_0_to_axis_int8(blocks: torch.Tensor, N: int, K: int, out=None, scale=None):
     """Q8_0 weight [N, K/32 blocks] -> (int8 codes [N, K], per-row scales [N])."""
     if not (blocks.is_cuda and blocks.dtype == torch.uint8 and blocks.is_contiguous()):
         raise ValueError("blocks must be a contiguous uint8 CUDA tensor")
     if blocks.numel() < q8_0_bytes(N * K):
         raise ValueError("blocks hold fewer than N*K values")
-    q = torch.empty((N, K), dtype=torch.int8, device=blocks.device)
-    s = torch.empty((N,), dtype=torch.float32, device=blocks.device)
+    q = torch.empty((N, K), dtype=torch.int8, device=blocks.device) if out is None else out
+    s = torch.empty((N,), dtype=torch.float32, device=blocks.device) if scale is None else scale
+    if q.shape != (N, K) or q.dtype != torch.int8 or not q.is_contiguous() or s.numel() < N:
+        raise ValueError("out must be a contiguous int8 [N, K] tensor and scale hold N floats")
     _check(lib().q8_0_to_axis_int8(_ptr(blocks), N, K, _ptr(q), _ptr(s), _stream(blocks.device)))
     return q, s
 

@@ -224,4 +224,183 @@ __global__ void __launch_bounds__(32 * kRequantMaxWarps) q8_0_to_axis_int8_kerne
   }
 }
 
+// ----------------------------------------------------------------------------
+// Q8_0 -> axis int8 for rows whose blocks fill whole 16-byte units
+// (K % 256 == 0): a team of TW warps per row, thread t of the team taking
+// blocks t, t + 32 TW, ...  Each team copies its next row into shared memory
+// (cp.async, double-buffered) while it processes the current one.
+//
+// A block b starts at byte 34 b of the row, i.e. on a word boundary when b is
+// even and 2 bytes past one when b is odd; its 34 bytes lie in the 9 words
+// from word floor(34 b / 4), and prmt selects the f16 scale and the 32 codes
+// from them.  Pass 1 takes max |q| of each block on sign-extended 16-bit
+// pairs (max/min.s16x2); max |d q| = |d| max |q| exactly.  Pass 2 rounds
+// q * fl(d / s') as rne_low_byte does, with the exact product inside an fma;
+// a group of 8 within 2^-14 of a tie takes the IEEE division out of line.
+// ----------------------------------------------------------------------------
+constexpr int kRqThreads = 256;
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ uint32_t vmax_s16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.s16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t vmin_s16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.s16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+template <int TW>
+__device__ __forceinline__ void team_sync(int team) {
+  if constexpr (TW == 1) {
+    __syncwarp();
+  } else {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(32 * TW) : "memory");
+  }
+}
+
+// The 9 words holding block b of a staged row.
+__device__ __forceinline__ void rq_block_words(const uint8_t* row, int b, uint32_t (&w)[9]) {
+  const uint32_t* p = reinterpret_cast<const uint32_t*>(row) + ((17 * b) >> 1);
+#pragma unroll
+  for (int i = 0; i < 9; ++i) w[i] = p[i];
+}
+
+// max |q| over the 32 codes of a block.
+__device__ __forceinline__ int rq_block_maxabs(const uint32_t (&w)[9], bool odd) {
+  const uint32_t s0 = odd ? 0xD5C4u : 0xB3A2u, s1 = odd ? 0xF7E6u : 0xD5C4u;
+  uint32_t mx = 0x80008000u, mn = 0x7FFF7FFFu;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t p0 = prmt(w[k], w[k + 1], s0), p1 = prmt(w[k], w[k + 1], s1);
+    mx = vmax_s16x2(mx, vmax_s16x2(p0, p1));
+    mn = vmin_s16x2(mn, vmin_s16x2(p0, p1));
+  }
+  const int hi = max(static_cast<int>(static_cast<int16_t>(mx & 0xFFFFu)), static_cast<int>(static_cast<int16_t>(mx >> 16)));
+  const int lo = min(static_cast<int>(static_cast<int16_t>(mn & 0xFFFFu)), static_cast<int>(static_cast<int16_t>(mn >> 16)));
+  return max(hi, -lo);
+}
+
+__device__ __forceinline__ float rq_block_scale(const uint32_t (&w)[9], bool odd) {
+  return __half2float(__ushort_as_half(static_cast<uint16_t>(prmt(w[0], 0u, odd ? 0x4432u : 0x4410u))));
+}
+
+// The rare exact path, kept out of line so that the hot loop stays small:
+// codes of fl(d q) / s by IEEE division for 8 values.
+__device__ __noinline__ uint2 rq_codes8_exact(float d, float s, float q0, float q1, float q2, float q3, float q4,
+                                              float q5, float q6, float q7) {
+  const float v[8] = {q0, q1, q2, q3, q4, q5, q6, q7};
+  uint32_t c[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) c[i] = int8_code_exact(__fmul_rn(d, v[i]), s);
+  return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24), c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
+}
+
+// 32 codes of a block -> 32 axis int8 codes (8 words).
+__device__ __forceinline__ void rq_block_codes(const uint32_t (&w)[9], bool odd, float d, float s, float rcp,
+                                               uint32_t (&out)[8]) {
+  const uint32_t csel = odd ? 0x7654u : 0x5432u;
+  const float drcp = __fmul_rn(d, rcp);
+  uint32_t c[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) c[k] = prmt(w[k], w[k + 1], csel);
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    float qf[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) qf[i] = static_cast<float>(static_cast<int8_t>(c[2 * g + i / 4] >> (8 * (i & 3))));
+    uint32_t big[8];
+    float dmax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float b = __fmaf_rn(qf[i], drcp, kRneMagic);
+      const float r = __fmaf_rn(qf[i], drcp, -__fsub_rn(b, kRneMagic));
+      dmax = fmaxf(dmax, fabsf(r));
+      big[i] = __float_as_uint(b);
+    }
+    if (dmax > kNearHalf) {
+      const uint2 e = rq_codes8_exact(d, s, qf[0], qf[1], qf[2], qf[3], qf[4], qf[5], qf[6], qf[7]);
+      out[2 * g] = e.x;
+      out[2 * g + 1] = e.y;
+    } else {
+      out[2 * g] = prmt(prmt(big[0], big[1], 0x0040u), prmt(big[2], big[3], 0x0040u), 0x5410u);
+      out[2 * g + 1] = prmt(prmt(big[4], big[5], 0x0040u), prmt(big[6], big[7], 0x0040u), 0x5410u);
+    }
+  }
+}
+
+template <int TW>
+__global__ void __launch_bounds__(kRqThreads) q8_0_to_axis_int8_team_kernel(const uint8_t* __restrict__ blocks,
+                                                                           int64_t N, int64_t K,
+                                                                           int8_t* __restrict__ q,
+                                                                           float* __restrict__ scale) {
+  extern __shared__ __align__(16) uint8_t rq_smem[];
+  __shared__ float red[2][8];
+  constexpr int T = 32 * TW;
+  constexpr int kTeams = kRqThreads / T;
+  const int team = threadIdx.x / T, t = threadIdx.x % T;
+  const int nblk = static_cast<int>(K >> 5);
+  const int row_bytes = nblk * kQ80Bytes;   // a multiple of 16
+  const int nvec = row_bytes >> 4;
+  uint8_t* const buf = rq_smem + 2 * team * row_bytes;   // two row buffers per team
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kTeams;
+  int64_t n = blockIdx.x * static_cast<int64_t>(kTeams) + team;
+  if (n < N) {
+    const uint8_t* src = blocks + n * row_bytes;
+    for (int i = t; i < nvec; i += T) cp_async16(buf + 16 * i, src + 16 * i);
+  }
+  cp_async_commit();
+  for (int it = 0; n < N; n += stride, ++it) {
+    const uint8_t* cur = buf + (it & 1) * row_bytes;
+    if (n + stride < N) {
+      const uint8_t* src = blocks + (n + stride) * row_bytes;
+      uint8_t* dst = buf + ((it + 1) & 1) * row_bytes;
+      for (int i = t; i < nvec; i += T) cp_async16(dst + 16 * i, src + 16 * i);
+    }
+    cp_async_commit();
+    cp_async_wait<1>();
+    team_sync<TW>(team);
+    float a = 0.0f;
+#pragma unroll 1
+    for (int b = t; b < nblk; b += T) {
+      uint32_t w[9];
+      rq_block_words(cur, b, w);
+      const bool odd = b & 1;
+      a = fmaxf(a, __fmul_rn(fabsf(rq_block_scale(w, odd)), static_cast<float>(rq_block_maxabs(w, odd))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+    if constexpr (TW > 1) {
+      if ((t & 31) == 0) red[it & 1][threadIdx.x >> 5] = a;
+      team_sync<TW>(team);
+#pragma unroll
+      for (int i = 0; i < TW; ++i) a = fmaxf(a, red[it & 1][team * TW + i]);
+    }
+    const float s = (a < 1e-10f) ? 1e-10f : __fdiv_rn(a, 127.0f);
+    const float rcp = __frcp_rn(s);
+    if (t == 0) scale[n] = s;
+#pragma unroll 1
+    for (int b = t; b < nblk; b += T) {
+      uint32_t w[9];
+      rq_block_words(cur, b, w);
+      const bool odd = b & 1;
+      uint32_t o[8];
+      rq_block_codes(w, odd, rq_block_scale(w, odd), s, rcp, o);
+      uint4* dst = reinterpret_cast<uint4*>(q + n * K + 32 * static_cast<int64_t>(b));
+      dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+    team_sync<TW>(team);   // the buffer of this row is refilled two rows on
+  }
+  cp_async_wait<0>();
+}
+
 }  // namespace w8a8

@@ -83,6 +83,18 @@ __device__ __forceinline__ uint2 encode8(uint4 w, float s, float rcp) {
   return encode8f<QT>(v, s, rcp);
 }
 
+// The exact codes of 8 bf16 by IEEE division: the rare path of encode8_fast,
+// kept out of line so that the hot loops stay small.
+template <int QT>
+__device__ __noinline__ uint2 encode8_exact(uint4 w, float s) {
+  const float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                      bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+  uint32_t c[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) c[i] = (QT == 1) ? e4m3_code_exact(v[i], s) : int8_code_exact(v[i], s);
+  return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24), c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
+}
+
 // The same codes, four fp32 operations per value.  int8: the exact product
 // x * rcp is rounded once, to an integer, by fma(x, rcp, 1.5 * 2^23) (ties
 // to even), and its exact remainder d = fma(x, rcp, -rne) is rounded once.
@@ -116,10 +128,7 @@ __device__ __forceinline__ uint2 encode8_fast(uint4 w, float s, float rcp) {
     }
     near = dmax > kNearHalf;
   }
-  if (near) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) c[i] = (QT == 1) ? e4m3_code_exact(v[i], s) : int8_code_exact(v[i], s);
-  }
+  if (near) return encode8_exact<QT>(w, s);
   return make_uint2(prmt(prmt(c[0], c[1], 0x0040u), prmt(c[2], c[3], 0x0040u), 0x5410u),
                     prmt(prmt(c[4], c[5], 0x0040u), prmt(c[6], c[7], 0x0040u), 0x5410u));
 }

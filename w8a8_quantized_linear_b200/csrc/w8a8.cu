@@ -417,7 +417,37 @@ w8a8_status q8_0_to_axis_int8(const void* blocks, int64_t N, int64_t K, int8_t* 
   int dev = 0, sms = 0;
   w8a8_status st = current_device(&dev, &sms);
   if (st != W8A8_OK) return st;
-  // one warp per row; each warp stages its row (rounded to 16 bytes) in shared memory
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t nblk = K / 32;
+  if (K % 256 == 0) {
+    // rows of whole 16-byte units: a team of TW warps per row, double-buffered rows
+    int tw = 1;
+    while (tw < 8 && tw * 48 < nblk) tw *= 2;
+    const size_t smem = static_cast<size_t>(2 * (8 / tw)) * static_cast<size_t>(nblk * 34);
+    if (smem <= 200 * 1024) {
+      int per_sm = static_cast<int>((220 * 1024) / (smem + 1024));
+      per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
+      int64_t grid = (N + (8 / tw) - 1) / (8 / tw);
+      if (grid > static_cast<int64_t>(per_sm) * sms) grid = static_cast<int64_t>(per_sm) * sms;
+      static std::atomic<uint64_t> team_smem_set[4] = {};
+      cudaError_t e = cudaSuccess;
+      const auto* bp = static_cast<const uint8_t*>(blocks);
+#define W8A8_RQ_TEAM(TW, IDX)                                                                              \
+  e = set_smem_once(q8_0_to_axis_int8_team_kernel<TW>, 200 * 1024, dev, team_smem_set[IDX]);               \
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(requant)");                             \
+  q8_0_to_axis_int8_team_kernel<TW><<<static_cast<int>(grid), kRqThreads, smem, cs>>>(bp, N, K, q, scale)
+      switch (tw) {
+        case 1: W8A8_RQ_TEAM(1, 0); break;
+        case 2: W8A8_RQ_TEAM(2, 1); break;
+        case 4: W8A8_RQ_TEAM(4, 2); break;
+        default: W8A8_RQ_TEAM(8, 3); break;
+      }
+#undef W8A8_RQ_TEAM
+      e = cudaGetLastError();
+      return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "q8_0_to_axis_int8 launch");
+    }
+  }
+  // other rows: one warp per row; each warp stages its row (rounded to 16 bytes) in shared memory
   const size_t row_stride = (static_cast<size_t>(K / 32) * 34 + 15) & ~static_cast<size_t>(15);
   int warps = static_cast<int>((200 * 1024) / row_stride);
   warps = warps < 1 ? 1 : (warps > kRequantMaxWarps ? kRequantMaxWarps : warps);
@@ -427,7 +457,7 @@ w8a8_status q8_0_to_axis_int8(const void* blocks, int64_t N, int64_t K, int8_t* 
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(requant)");
   int64_t grid = (N + warps - 1) / warps;
   if (grid > 32 * sms) grid = 32 * sms;
-  q8_0_to_axis_int8_kernel<<<static_cast<int>(grid), 32 * warps, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
+  q8_0_to_axis_int8_kernel<<<static_cast<int>(grid), 32 * warps, smem, cs>>>(
       static_cast<const uint8_t*>(blocks), N, K, q, scale);
   e = cudaGetLastError();
   return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "q8_0_to_axis_int8 launch");

@@ -98,6 +98,38 @@ def q8_0_standalone(n=1 << 28, seed=51):
     return torch.randn(n, generator=_gen(seed), dtype=torch.float32)
 
 
+def raw_q8_0_blocks(N: int, K: int, seed: int) -> torch.Tensor:
+    """Arbitrary Q8_0 block bytes for N rows of K values (K % 32 == 0): each
+    34-byte block is an f16 scale followed by 32 int8 codes, both drawn at
+    random rather than produced by a quantizer.  Row n % 6 picks the kind:
+    0 one shared scale with +-127 present, 1 all scales zero, 2 random scales
+    of both signs, 3 codes that include -128, 4 all codes zero, 5 scales in
+    the f16 subnormal range."""
+    nb = K // 32
+    g = _gen(seed)
+    codes = torch.round(torch.randn(N, nb, 32, generator=g) * 40.0).clamp_(-128, 127)
+    scales = torch.rand(N, nb, generator=g) * 2e-3 + 1e-5
+    signs = torch.where(torch.rand(N, nb, generator=g) < 0.1, -1.0, 1.0)
+    kind = torch.arange(N) % 6
+    scales = torch.where((kind == 2)[:, None], scales * signs, scales)
+    scales = torch.where((kind == 0)[:, None], torch.full_like(scales, 0.02 / 127), scales)
+    scales = torch.where((kind == 1)[:, None], torch.zeros_like(scales), scales)
+    scales = torch.where((kind == 5)[:, None], scales * 1e-3, scales)
+    idx = torch.arange(nb) % 32
+    spike = torch.where(torch.arange(nb) % 2 == 0, 127.0, -127.0)
+    rows0 = torch.nonzero(kind == 0).reshape(-1)
+    codes[rows0] = codes[rows0].clamp(-126, 126)
+    for n in rows0.tolist():
+        codes[n, torch.arange(nb), idx] = spike
+    neg = torch.rand(N, nb, 32, generator=g) < 1.0 / 64
+    codes = torch.where((kind == 3)[:, None, None] & neg, torch.full_like(codes, -128.0), codes)
+    codes = torch.where((kind == 4)[:, None, None], torch.zeros_like(codes), codes)
+    out = torch.empty(N, nb, 34, dtype=torch.uint8)
+    out[:, :, :2] = scales.to(torch.float16).contiguous().view(torch.uint8).view(N, nb, 2)
+    out[:, :, 2:] = codes.to(torch.int8).view(torch.uint8)
+    return out.reshape(-1)
+
+
 def to_u16(t: torch.Tensor):
     """bf16 tensor -> numpy uint16 bit patterns (for the oracle)."""
     return t.contiguous().view(torch.int16).numpy().view("uint16")
