@@ -290,42 +290,61 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
     E = lambda: torch.cuda.Event(enable_timing=True)
 
-    def step(ev):
-        """ev: list of 10 events -> [start, q1, g1, q2, g2, q3, g3, q4, g4] boundaries."""
-        ev[0].record(stream)
-        w8.quantize_rows(X, "int8", out=xq1, scale=sx1); ev[1].record(stream)
-        w8.qgemm_fwd(xq1, sx1, W1q, s1, out=Y1); ev[2].record(stream)
-        w8.quantize_rows(Y1, "int8", out=xq2, scale=sx2); ev[3].record(stream)
-        w8.qgemm_fwd(xq2, sx2, W2q, s2, out=Y2); ev[4].record(stream)
-        w8.quantize_rows(dY2, "int8", out=gq2, scale=sg2); ev[5].record(stream)
-        w8.qgemm_dgrad(gq2, sg2, W2q, s2, out=dX2); ev[6].record(stream)
-        w8.quantize_rows(dX2, "int8", out=gq1, scale=sg1); ev[7].record(stream)
-        w8.qgemm_dgrad(gq1, sg1, W1q, s1, out=dX1); ev[8].record(stream)
+    KERNELS = [lambda: w8.quantize_rows(X, "int8", out=xq1, scale=sx1),
+               lambda: w8.qgemm_fwd(xq1, sx1, W1q, s1, out=Y1),
+               lambda: w8.quantize_rows(Y1, "int8", out=xq2, scale=sx2),
+               lambda: w8.qgemm_fwd(xq2, sx2, W2q, s2, out=Y2),
+               lambda: w8.quantize_rows(dY2, "int8", out=gq2, scale=sg2),
+               lambda: w8.qgemm_dgrad(gq2, sg2, W2q, s2, out=dX2),
+               lambda: w8.quantize_rows(dX2, "int8", out=gq1, scale=sg1),
+               lambda: w8.qgemm_dgrad(gq1, sg1, W1q, s1, out=dX1)]
 
-    for _ in range(args.warmup):
-        flush.fill_(1)
-        flush_sum = flush.view(torch.int64).sum()
-        step([E() for _ in range(9)])
+    def step(ev, per_kernel=False):
+        """The step's 8 launches between events ev[0] and ev[-1]; with
+        per_kernel, an event after each launch as well (ev has 9 entries).
+        Without them consecutive launches may overlap (programmatic dependent
+        launch), so the timed steps record only the two ends."""
+        ev[0].record(stream)
+        for k, fn in enumerate(KERNELS):
+            fn()
+            if per_kernel:
+                ev[k + 1].record(stream)
+        if not per_kernel:
+            ev[-1].record(stream)
+
+    def flush_l2(i):
+        flush.fill_(i & 0xFF)          # L2 flush (write, then read back so that no dirty
+        return flush.view(torch.int64).sum()   # lines are left for the step), outside the step's events
+
+    for i in range(args.warmup):
+        flush_l2(i)
+        step([E(), E()])
     torch.cuda.synchronize()
     assert w8.device_status() == 0, "device-side error during warm-up"
 
-    events = [[E() for _ in range(9)] for _ in range(args.steps)]
+    events = [[E(), E()] for _ in range(args.steps)]
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(*gpu_identity(torch, dev)) as clk:
         wall0 = time.perf_counter()
         for i in range(args.steps):
-            flush.fill_(i & 0xFF)          # L2 flush (write, then read back so that no dirty
-            flush_sum = flush.view(torch.int64).sum()   # lines are left for the step), outside the step's events
+            flush_l2(i)
             step(events[i])
         torch.cuda.synchronize()
         wall = time.perf_counter() - wall0
+        # the per-kernel split, from as many steps again with an event after
+        # every launch (same inputs and launches; L2 flushed the same way)
+        kev = [[E() for _ in range(9)] for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush_l2(i)
+            step(kev[i], per_kernel=True)
+        torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    step_ms = [ev[0].elapsed_time(ev[8]) for ev in events]
-    gemm_ms = [ev[k - 1].elapsed_time(ev[k]) for ev in events for k in (2, 4, 6, 8)]
-    quant_ms = [ev[k - 1].elapsed_time(ev[k]) for ev in events for k in (1, 3, 5, 7)]
+    step_ms = [ev[0].elapsed_time(ev[-1]) for ev in events]
+    gemm_ms = [ev[k - 1].elapsed_time(ev[k]) for ev in kev for k in (2, 4, 6, 8)]
+    quant_ms = [ev[k - 1].elapsed_time(ev[k]) for ev in kev for k in (1, 3, 5, 7)]
     total_ms = max_over_ranks(sum(step_ms), dist, dev)
     ms_per_step = total_ms / args.steps
     value = world * OPS_PER_STEP * args.steps / (total_ms * 1e-3) / 1e12
@@ -406,7 +425,10 @@ def run_ours(args, rank, world, local_rank):
                 "peak_source": "%s: 2 x bf16_tflops (burst; int8 dense = 2x bf16 dense nominal)" % src,
                 "frac_of_sustained": achieved / (2.0 * peaks["bf16_tflops_sustained"]),
                 "gemm_ms_avg": gemm_avg, "quantize_ms_avg": statistics.mean(quant_ms),
-                "quantize_share": sum(quant_ms) / sum(step_ms)}
+                "quantize_share": sum(quant_ms) / (sum(quant_ms) + sum(gemm_ms)),
+                "per_kernel_events": "separate steps with an event after every launch (launches then "
+                                     "cannot overlap); their sum per step: %.4f ms" %
+                                     ((sum(quant_ms) + sum(gemm_ms)) / args.steps)}
     clocks = clk.summary()
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -469,19 +491,29 @@ def _nsets(set_bytes):
 
 
 def _time_rot(fns, reps, torch, stream):
-    """Mean time of one call, cycling through ``fns`` (each on its own buffers)
-    back to back between two events on the launching stream."""
+    """Mean GPU time of one call.  The calls, cycling through ``fns`` (each on
+    its own buffers), are captured once in a CUDA graph, and the graph is
+    replayed between two events on the launching stream: host-side launch
+    cost is left out, as in a captured model step (every call of the library
+    is stream-ordered and capturable)."""
     for f in fns:
         f()
+    torch.cuda.synchronize()
+    n = max(reps, len(fns))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n):
+            fns[i % len(fns)]()
+    g.replay()
     torch.cuda.synchronize()
     E = lambda: torch.cuda.Event(enable_timing=True)
     a, b = E(), E()
     a.record(stream)
-    for i in range(reps):
-        fns[i % len(fns)]()
+    g.replay()
     b.record(stream)
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / reps
+    del g
+    return a.elapsed_time(b) / n
 
 
 def extras(w8, torch, workloads, dev, peaks, src):
@@ -598,7 +630,8 @@ def extras(w8, torch, workloads, dev, peaks, src):
         del sets
     out["gguf_a8_int_fwd_sweep_N12288_K3072"] = sweep
     out["peaks"] = {"source": src, "hbm_gbs": hbm, "int8_burst_tops": tc8}
-    out["method"] = "mean over back-to-back reps rotating through >= 3x L2 of input/output copies"
+    out["method"] = ("mean over reps replayed from one CUDA graph (no host launch cost), rotating through "
+                     ">= 3x L2 of input/output copies")
     assert w8.device_status() == 0
     return out
 

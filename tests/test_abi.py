@@ -57,6 +57,13 @@ def test_sizes(L):
     assert L.w8a8_workspace_bytes(1, 3, 40, 16, 0) == 256 + 256  # N padded to 48 -> 144 bytes
     assert L.w8a8_workspace_bytes(2, 4608, 3072, 3072, 32) == 4608 * 3072 + 4608 * 4 + 4608 * 32 * 2
     assert L.w8a8_workspace_bytes(3, 10, 10, 16, 0) == 256
+    # few output tiles, long contraction: split-K partial sums follow
+    # (48 tiles -> 3 splits of 8 K blocks; [3, 1, 12288] int32)
+    assert L.w8a8_workspace_bytes(0, 1, 12288, 3072, 0) == 3072 + 256 + 3 * 12288 * 4
+    # dgrad of the up-projection at M=64: 12 tiles over K=3072, 96 K blocks -> 12 splits
+    assert L.w8a8_workspace_bytes(1, 64, 12288, 3072, 0) == 64 * 12288 + 256 + 12 * 64 * 3072 * 4
+    # output width not a multiple of 8: never split
+    assert L.w8a8_workspace_bytes(0, 1, 1001, 4096, 0) == 4096 + 256
     assert L.w8a8_workspace_bytes(9, 1, 1, 16, 0) == 0
 
 

@@ -115,6 +115,35 @@ def test_quantize_rows_exact_ties(w8, orc, qt):
     assert np.array_equal(f32(s), sr) and np.array_equal(u8(q), qr)
 
 
+@pytest.mark.parametrize("qt", ["int8", "e4m3"])
+def test_quantize_rows_every_bf16_value(w8, orc, qt):
+    """Each row holds its absmax a and every bf16 value v with |v| <= a, so
+    every code of every representable input is compared with the oracle at
+    these scales: powers of two (exact products), absmax values whose halves
+    land next to ties after the fp32 division (4.0625, 4.125, 3.59375 - the
+    common case in N(0,1) rows), and arbitrary ones."""
+    grid = orc.bf16_to_f32(np.arange(1 << 16, dtype=np.uint32).astype(np.uint16))
+    grid = np.unique(np.abs(grid[np.isfinite(grid)]))
+    absmax = [4.0625, 4.125, 3.59375, 3.828125, 4.5, 3.96875, 1.0, 0.7578125, 100.5, 448.0, 57.5,
+              1.0e-3, 3.0e-8, 2.5e4, 15.875]
+    rows = []   # rows of 12288 (the team kernel), each [a, a chunk of the values, zeros]
+    for a in absmax:
+        a = float(np.float32(torch.tensor(a).to(torch.bfloat16).float()))
+        v = grid[grid <= a]
+        v = np.concatenate([v, -v])
+        for c in range(0, v.size, 12287):
+            rows.append(np.concatenate([[a], v[c:c + 12287]]))
+    K = 12288
+    x = np.zeros((len(rows), K), np.float32)
+    for i, r in enumerate(rows):
+        x[i, :r.size] = r
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    q, s = w8.quantize_rows(xb.to(DEV), qt)
+    qr, sr = orc.quantize_rows(workloads.to_u16(xb), QT[qt])
+    assert np.array_equal(f32(s).view(np.uint32), sr.view(np.uint32))
+    assert np.array_equal(u8(q), qr)
+
+
 def test_quantize_rows_strided_input(w8, orc):
     big = workloads.normal((40, 256), 1.0, 3)
     x = big.to(DEV)[:, :160]           # ldx = 256 > K = 160
@@ -193,8 +222,10 @@ def _fp8_tol(ref, y):
     return np.abs(yg - yr), bound
 
 
+# (7, 1000, 4096), (1, 2048, 3072) and (100, 256, 12288) have few output
+# tiles and a long contraction: split-K with 8, 6 and 16 splits
 LIN_SHAPES = [(256, 512, 512), (300, 520, 640), (1, 16, 16), (129, 257, 96), (7, 1000, 4096),
-              (128, 256, 128), (520, 300, 272)]
+              (128, 256, 128), (520, 300, 272), (1, 2048, 3072), (100, 256, 12288)]
 
 
 @pytest.mark.parametrize("M,N,K", LIN_SHAPES)
@@ -208,7 +239,7 @@ def test_linear_fwd_int8_parity(w8, orc, M, N, K):
     assert np.array_equal(u16(y), ref["y"])
 
 
-@pytest.mark.parametrize("M,N,K", [(200, 384, 256), (77, 130, 512)])
+@pytest.mark.parametrize("M,N,K", [(200, 384, 256), (77, 130, 512), (33, 520, 2048)])
 def test_linear_fwd_int8_axis_bias_parity(w8, orc, M, N, K):
     x = workloads.normal((M, K), 1.0, seed=11)
     w = workloads.normal((N, K), 0.02, seed=12)
@@ -220,7 +251,7 @@ def test_linear_fwd_int8_axis_bias_parity(w8, orc, M, N, K):
     assert np.array_equal(u16(y), ref["y"])
 
 
-@pytest.mark.parametrize("M,N,K", [(256, 512, 512), (300, 520, 640), (1, 16, 16), (129, 257, 96)])
+@pytest.mark.parametrize("M,N,K", [(256, 512, 512), (300, 520, 640), (1, 16, 16), (129, 257, 96), (5, 264, 4096)])
 def test_linear_fwd_e4m3_parity(w8, orc, M, N, K):
     x = workloads.with_outlier_channels((M, K), 1.0, seed=M + N)
     w = workloads.normal((N, K), 0.02, seed=K + 1)
@@ -264,6 +295,19 @@ def test_linear_fwd_m0_noop(w8):
     assert w8.linear_fwd(x, wq, sw).shape == (0, 32)
 
 
+def test_linear_fwd_split_equals_unsplit(w8):
+    """A forward with few output tiles and a long K (split-K for int8) equals
+    the GEMM on the same codes without splitting (qgemm_fwd never splits), bit
+    for bit; e4m3 products are not split, so they are equal too."""
+    x = workloads.normal((64, 3072), 1.0, 33).to(DEV)
+    w = workloads.normal((1024, 3072), 0.02, 34).to(DEV)
+    assert w8.workspace_bytes(w8.OP_LINEAR_FWD, 64, 1024, 3072) > 64 * 3072 + 256
+    for qt in ("int8", "e4m3"):
+        wq, sw = w8.quantize_weight(w, qt, "tensor")
+        xq, sx = w8.quantize_rows(x, qt)
+        assert torch.equal(w8.linear_fwd(x, wq, sw), w8.qgemm_fwd(xq, sx, wq, sw)), qt
+
+
 def test_linear_fwd_deterministic(w8):
     x = workloads.normal((1000, 1024), 1.0, 31).to(DEV)
     wq, sw = w8.quantize_weight(workloads.normal((2048, 1024), 0.02, 32).to(DEV), "e4m3", "tensor")
@@ -274,7 +318,7 @@ def test_linear_fwd_deterministic(w8):
 
 # --------------------------------------------------------------------------- dgrad
 @pytest.mark.parametrize("qt", ["int8", "e4m3"])
-@pytest.mark.parametrize("M,N,K", [(64, 256, 512), (129, 96, 80), (300, 512, 272), (1, 16, 16)])
+@pytest.mark.parametrize("M,N,K", [(64, 256, 512), (129, 96, 80), (300, 512, 272), (1, 16, 16), (50, 2048, 768)])
 def test_linear_dgrad_parity(w8, orc, qt, M, N, K):
     dy = workloads.normal((M, N), 1e-3, seed=M + N)
     w = workloads.normal((N, K), 0.02, seed=N * 3 + K)

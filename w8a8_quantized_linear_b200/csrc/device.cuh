@@ -36,6 +36,19 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 }
 
 // ----------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel on the stream is still
+// running (once every block of that kernel has called griddep_launch).
+// griddep_wait() returns when the previous kernel has completed and its
+// memory writes are visible (at once when there is no such kernel); a
+// kernel touches no global memory that the previous one may write or read
+// before it.  Weights are the exception the GEMM relies on: no kernel that
+// runs directly before it with an early trigger writes them.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ----------------------------------------------------------------------------
 // mbarrier
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

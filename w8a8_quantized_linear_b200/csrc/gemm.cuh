@@ -16,6 +16,14 @@
 //               low-rank in fp32, bf16 stores.  Double buffering of the accumulator lets
 //               the epilogue of tile i overlap the MMAs of tile i+1.
 // Tile 128 x BN x 128 bytes of K per stage.  Every wait is bounded.
+//
+// Split-K (scale epilogue only): with ep.splits = S > 1 the work units are
+// (tile, split) pairs, split s covering K blocks [s*nkb/S, (s+1)*nkb/S).  A
+// unit writes its raw sums (int32, or fp32 bits for e4m3) for the tile's
+// valid rows to ep.partial[s][m][n]; splitk_epilogue_kernel then adds the S
+// partial sums in split order (a fixed order, so e4m3 results are
+// reproducible; integer sums are exact in any order) and applies the
+// epilogue.
 #pragma once
 #include "device.cuh"
 
@@ -38,6 +46,8 @@ struct EpiParams {
   const __nv_bfloat16* lr_t;     // T [M, r]                          (kEpiLowRank)
   const __nv_bfloat16* lr_l2;    // L2 [r, N]
   int r;
+  int splits;                    // K splits per tile (>= 1; > 1 only with kEpiScale)
+  uint32_t* partial;             // [splits, M, N] raw sums (splits > 1)
 };
 
 template <int KIND, int BN, int EPI>
@@ -126,11 +136,15 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_launch();   // the next kernel may set itself up while this one runs
 
   const int tiles_m = (M + kBM - 1) / kBM;
   const int tiles_n = (N + BN - 1) / BN;
   const int num_tiles = tiles_m * tiles_n;
   const int num_kb = (Kc + C::kBK - 1) / C::kBK;
+  // the host keeps 1 <= splits <= num_kb, so every unit has at least one K block
+  const int splits = (EPI == kEpiScale) ? ep.splits : 1;
+  const int num_units = num_tiles * splits;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -139,20 +153,44 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
       uint32_t phase = 0;
       uint32_t issued = 0, issued_phase = 0;   // per-stage bits, for teardown
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        const int m0 = (tile % tiles_m) * kBM, n0 = (tile / tiles_m) * BN;
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, 0x100u | stage, limit)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-          tma_load_2d(sA + stage * C::kABytes, &tmA, &full[stage], kb * C::kBK, m0);
-          uint8_t* b = sB + stage * C::kBBytes;
-          if constexpr (!B_MN) {
-            tma_load_2d(b, &tmB, &full[stage], kb * C::kBK, n0);
-          } else {
+      auto load_b = [&](int st, int kb, int n0) {
+        uint8_t* b = sB + st * C::kBBytes;
+        if constexpr (!B_MN) {
+          tma_load_2d(b, &tmB, &full[st], kb * C::kBK, n0);
+        } else {
 #pragma unroll
-            for (int j = 0; j < BN * C::kElem / 128; ++j)
-              tma_load_2d(b + j * (C::kBK * 128), &tmB, &full[stage], n0 + j * (128 / C::kElem), kb * C::kBK);
+          for (int j = 0; j < BN * C::kElem / 128; ++j)
+            tma_load_2d(b + j * (C::kBK * 128), &tmB, &full[st], n0 + j * (128 / C::kElem), kb * C::kBK);
+        }
+      };
+      // The weight (B) tiles of the first unit's first stages are requested
+      // before waiting for the previous kernel, which never writes them; the
+      // activation codes (A) it may be producing are read after the wait.
+      int pre = 0;
+      if (static_cast<int>(blockIdx.x) < num_units) {
+        const int tile = blockIdx.x / splits, split = blockIdx.x - tile * splits;
+        const int kb0 = split * num_kb / splits, kb1 = (split + 1) * num_kb / splits;
+        pre = (kb1 - kb0) < kStages ? (kb1 - kb0) : kStages;
+        for (int i = 0; i < pre; ++i) {
+          mbar_arrive_expect_tx(&full[i], C::kStageBytes);
+          load_b(i, kb0 + i, (tile / tiles_m) * BN);
+          issued |= 1u << i;
+        }
+      }
+      griddep_wait();
+      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+        const int tile = u / splits, split = u - tile * splits;
+        const int m0 = (tile % tiles_m) * kBM, n0 = (tile / tiles_m) * BN;
+        const int kb0 = split * num_kb / splits, kb1 = (split + 1) * num_kb / splits;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, 0x100u | stage, limit)) { ok = false; break; }
+          if (pre > 0) {
+            --pre;   // this stage's B tile and byte count are in flight already
+          } else {
+            mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+            load_b(stage, kb, n0);
           }
+          tma_load_2d(sA + stage * C::kABytes, &tmA, &full[stage], kb * C::kBK, m0);
           issued |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -169,11 +207,13 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+        const int split = u % splits;
+        const int kb0 = split * num_kb / splits, kb1 = (split + 1) * num_kb / splits;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, 0x200u | acc, limit)) break;
         tc_fence_after();
         const uint32_t d = tmem + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, 0x300u | stage, limit)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_base = smem_u32(sA + stage * C::kABytes);
@@ -183,7 +223,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
             const uint64_t ad = sdesc_sw128(a_base + k * 32, 16, 1024);
             const uint64_t bd = B_MN ? sdesc_sw128(b_base + k * (C::kMmaK * 128), C::kBK * 128, 1024)
                                      : sdesc_sw128(b_base + k * 32, 16, 1024);
-            tc_mma<KIND>(d, ad, bd, kIdesc, (kb > 0 || k > 0) ? 1u : 0u);
+            tc_mma<KIND>(d, ad, bd, kIdesc, (kb > kb0 || k > 0) ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -198,6 +238,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    griddep_wait();                               // row scales come from the previous kernel
     const int e = warp - 2;                       // epilogue warp index
     const int quarter = warp & 3;                 // TMEM lanes this warp may read
     const int group = e >> 2;                     // column-chunk interleave
@@ -207,7 +248,8 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
     uint32_t acc_phase = 0;
     int local = 0;
     uint32_t out_iter = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+    for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++local) {
+      const int tile = u / splits, split = u - tile * splits;
       const int m0 = (tile % tiles_m) * kBM, n0 = (tile / tiles_m) * BN;
       if constexpr (EPI == kEpiLowRank) {
         // Every epilogue thread is done with the previous tile's L2^T before it
@@ -341,8 +383,33 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
         float sx = 1.0f;
         if constexpr (EPI != kEpiPlain) sx = row_ok ? ep.s_row[row] : 0.0f;
         const float sw0 = (EPI != kEpiPlain && !ep.s_col_axis) ? ep.s_col[0] : 1.0f;
+        const bool vec_partial = (N & 3) == 0;      // partial rows are 16-byte aligned
+        bool write_out = true;
+        if (splits > 1) {
+          // This unit's raw sums -> partial[split][row][n] (valid rows only).
+          uint32_t* prow = ep.partial + (static_cast<int64_t>(split) * M + (row_ok ? row : 0)) * N;
   #pragma unroll 1
-        for (int c = group; c < BN / 32; c += kGroups) {
+          for (int c = group; c < BN / 32; c += kGroups) {
+            const int nc = n0 + c * 32;
+            if (nc >= N) break;                     // warp-uniform
+            uint32_t r[32];
+            tmem_ld_x32(tmem + lane_base + static_cast<uint32_t>(acc * BN + c * 32), r);
+            tmem_ld_wait();
+            if (row_ok) {
+              if (vec_partial && nc + 32 <= N) {
+  #pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                  *reinterpret_cast<uint4*>(prow + nc + j) = make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]);
+              } else {
+                for (int j = 0; j < 32; ++j)
+                  if (nc + j < N) prow[nc + j] = r[j];
+              }
+            }
+          }
+          write_out = false;   // splitk_epilogue_kernel finishes the tile
+        }
+  #pragma unroll 1
+        for (int c = group; write_out && c < BN / 32; c += kGroups) {
           const int nc = n0 + c * 32;
           if (nc >= N) break;                       // warp-uniform
           const bool full_chunk = nc + 32 <= N;
@@ -448,6 +515,65 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// Finish a split-K product:  y[m, n] = bf16( ((sum_s partial[s][m][n]) * s_x[m]) * s_w[n or 0] + bias[n] ),
+// the partial sums added in split order and every other step the fp32 RN
+// operation of the fused epilogue, so the result equals the unsplit one
+// (int8) or is reproducible (e4m3).  8 columns per thread: N % 8 == 0, y
+// contiguous [M, N].
+template <int KIND>
+__global__ void __launch_bounds__(256) splitk_epilogue_kernel(const uint32_t* __restrict__ partial, int splits,
+                                                              int64_t M, int64_t N, const float* __restrict__ s_row,
+                                                              const float* __restrict__ s_col, int axis,
+                                                              const __nv_bfloat16* __restrict__ bias,
+                                                              __nv_bfloat16* __restrict__ y) {
+  griddep_launch();
+  griddep_wait();   // the partial sums come from the GEMM just before
+  const int64_t n8 = N >> 3;
+  const int64_t total = M * n8;
+  const int64_t plane = M * N;
+  for (int64_t i = blockIdx.x * 256ll + threadIdx.x; i < total; i += static_cast<int64_t>(gridDim.x) * 256) {
+    const int64_t m = i / n8, n = (i - m * n8) * 8;
+    const uint4* p = reinterpret_cast<const uint4*>(partial + m * N + n);
+    uint4 lo = __ldcg(p), hi = __ldcg(p + 1);
+    uint32_t r[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll 4
+    for (int sp = 1; sp < splits; ++sp) {
+      const uint4* q = reinterpret_cast<const uint4*>(partial + sp * plane + m * N + n);
+      lo = __ldcg(q);
+      hi = __ldcg(q + 1);
+      const uint32_t t[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        r[j] = (KIND == kKindI8) ? r[j] + t[j] : __float_as_uint(__fadd_rn(__uint_as_float(r[j]), __uint_as_float(t[j])));
+    }
+    const float sx = s_row[m];
+    float sw[8], bs[8];
+    if (axis) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(s_col + n));
+      const float4 b = __ldg(reinterpret_cast<const float4*>(s_col + n) + 1);
+      sw[0] = a.x; sw[1] = a.y; sw[2] = a.z; sw[3] = a.w; sw[4] = b.x; sw[5] = b.y; sw[6] = b.z; sw[7] = b.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) sw[j] = s_col[0];
+    }
+    if (bias != nullptr) {
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(bias + n));
+      bs[0] = bf16_lo(b.x); bs[1] = bf16_hi(b.x); bs[2] = bf16_lo(b.y); bs[3] = bf16_hi(b.y);
+      bs[4] = bf16_lo(b.z); bs[5] = bf16_hi(b.z); bs[6] = bf16_lo(b.w); bs[7] = bf16_hi(b.w);
+    }
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int>(r[j])) : __uint_as_float(r[j]);
+      a = __fmul_rn(__fmul_rn(a, sx), sw[j]);
+      if (bias != nullptr) a = __fadd_rn(a, bs[j]);
+      v[j] = a;
+    }
+    *reinterpret_cast<uint4*>(y + m * N + n) =
+        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
   }
 }
 

@@ -294,13 +294,18 @@ __device__ __forceinline__ float rq_block_scale(const uint32_t (&w)[9], bool odd
 }
 
 // The rare exact path, kept out of line so that the hot loop stays small:
-// codes of fl(d q) / s by IEEE division for 8 values.
-__device__ __noinline__ uint2 rq_codes8_exact(float d, float s, float q0, float q1, float q2, float q3, float q4,
-                                              float q5, float q6, float q7) {
+// the remainders are recomputed and only the values at the margin take the
+// IEEE division of fl(d q) by s.
+__device__ __noinline__ uint2 rq_codes8_exact(float d, float s, float drcp, float q0, float q1, float q2, float q3,
+                                              float q4, float q5, float q6, float q7) {
   const float v[8] = {q0, q1, q2, q3, q4, q5, q6, q7};
   uint32_t c[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) c[i] = int8_code_exact(__fmul_rn(d, v[i]), s);
+  for (int i = 0; i < 8; ++i) {
+    const float b = __fmaf_rn(v[i], drcp, kRneMagic);
+    const float r = __fmaf_rn(v[i], drcp, -__fsub_rn(b, kRneMagic));
+    c[i] = (fabsf(r) > kNearHalf) ? int8_code_exact(__fmul_rn(d, v[i]), s) : (__float_as_uint(b) & 0xFFu);
+  }
   return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24), c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
 }
 
@@ -327,7 +332,7 @@ __device__ __forceinline__ void rq_block_codes(const uint32_t (&w)[9], bool odd,
       big[i] = __float_as_uint(b);
     }
     if (dmax > kNearHalf) {
-      const uint2 e = rq_codes8_exact(d, s, qf[0], qf[1], qf[2], qf[3], qf[4], qf[5], qf[6], qf[7]);
+      const uint2 e = rq_codes8_exact(d, s, drcp, qf[0], qf[1], qf[2], qf[3], qf[4], qf[5], qf[6], qf[7]);
       out[2 * g] = e.x;
       out[2 * g + 1] = e.y;
     } else {

@@ -18,26 +18,31 @@ __device__ __forceinline__ float absmax_scale(float a) {
   return (a < 1e-10f) ? 1e-10f : __fdiv_rn(a, qmax_of<QT>());
 }
 
-// Exact codes of fl(v / s) without a division in the common case.
-//
-// rcp = fl(1/s) is correctly rounded, so t = fl(v * rcp) lies within
-// 3.0001 ulp (relative to |v / s|) of fl(v / s).
-//
-// int8: t is rounded to the nearest integer, ties to even, by adding
-// 1.5 * 2^23 (an fp32 add rounds exactly there for |t| < 2^22); the low byte
-// of the sum's bit pattern is then the two's-complement code.  The remainder
-// d = t - rne(t) is exact; when |d| < 0.5 - 2^-14 no rounding boundary lies
-// within 2^-14 > 3.0001 ulp * 127.5 of t, so fl(v / s) rounds to the same
-// integer.  |v / s| <= 127 (1 + 2^-23) with the absmax scale, so no clamp is
-// reached.  A group of values with any |d| at the margin is recomputed with
-// IEEE divisions (the rare slow path).
-//
-// e4m3: the codes of t * (1 - 2^-21) and t * (1 + 2^-21) - the ends of a
-// +-8 ulp interval that contains fl(v / s) - are compared; e4m3 rounding with
-// saturation is monotonic, so when they agree they are the code of fl(v / s).
+// Exact codes of fl(v / s) without a division and without a data-dependent
+// branch.  With y = fl(1/s) (correctly rounded), the quotient is refined
+// once (Markstein's correction step, P. Markstein, IBM J. Res. Dev. 34(1),
+// 1990):
+//     q0 = fl(v y),   r = fl(v - q0 s)  (one fma),   q1 = fl(q0 + r y)  (one fma)
+// and q1 is the IEEE quotient fl(v / s) for every bf16 v: checked
+// exhaustively on the GPU for every fp32 significand of s against every bf16
+// significand of v over the 23 binades that hold |v / s| in [2^-13, 2^11)
+// (tests/quotient_check.cu); the codes are invariant under scaling v and s by
+// the same power of two, and smaller quotients give code 0 either way.
+//   int8: fl(q1 + 1.5 * 2^23) rounds q1 to the nearest integer, ties to even
+//         (an fp32 sum in [2^23, 2^24) has unit spacing); the low byte of its
+//         bit pattern is the two's-complement code.  |v / s| <= 127 (1 +
+//         2^-23) with the absmax scale, so no clamp is reached.
+//   e4m3: the quotient goes through the RNE-satfinite conversion; its sign is
+//         v's (fl(-0 / s) = -0 has code 0x80).
+// Every step is an fp32 operation on pairs (the f32x2 forms of sm_100).
 constexpr float kRneMagic = 12582912.0f;            // 1.5 * 2^23
 constexpr float kNearHalf = 0.49993896484375f;      // 0.5 - 2^-14
 
+// Remainder form of a division-free int8 rounding, for the Q8_0 kernels
+// (whose inputs are not bf16): t = fl(v * fl(1/s)) lies within 3.0001 ulp of
+// fl(v / s); d = t - rne(t) is exact, and |d| < 0.5 - 2^-14 puts no rounding
+// boundary between them, so the integer is right; otherwise `near` is set
+// and the caller takes the IEEE division.
 __device__ __forceinline__ uint32_t rne_low_byte(float t, bool& near) {
   const float big = __fadd_rn(t, kRneMagic);
   const float d = __fsub_rn(t, __fsub_rn(big, kRneMagic));
@@ -49,101 +54,56 @@ __device__ __forceinline__ uint32_t int8_code_exact(float v, float s) {   // RNE
   q = max(-127, min(127, q));
   return static_cast<uint32_t>(q) & 0xFFu;
 }
-__device__ __forceinline__ uint32_t e4m3_code_exact(float v, float s) {
-  return static_cast<uint32_t>(cvt_e4m3x2(__fdiv_rn(v, s), 0.0f)) & 0xFFu;
-}
-__device__ __forceinline__ uint32_t e4m3_code_fast(float t, bool& near) {
-  const uint32_t pair = cvt_e4m3x2(__fmul_rn(t, 1.0f - 0x1p-21f), __fmul_rn(t, 1.0f + 0x1p-21f));
-  near |= (pair & 0xFFu) != (pair >> 8);
-  return pair & 0xFFu;
-}
 
-// 8 values -> 8 codes (one uint2), fast path with one exactness flag.
+// 8 bf16 (one uint4) -> 8 codes (one uint2); y = fl(1/s).
 template <int QT>
-__device__ __forceinline__ uint2 encode8f(const float (&v)[8], float s, float rcp) {
-  bool near = false;
-  uint32_t c[8];
+__device__ __forceinline__ uint2 encode8(uint4 w, float s, float y) {
+  const float2 v[4] = {make_float2(bf16_lo(w.x), bf16_hi(w.x)), make_float2(bf16_lo(w.y), bf16_hi(w.y)),
+                       make_float2(bf16_lo(w.z), bf16_hi(w.z)), make_float2(bf16_lo(w.w), bf16_hi(w.w))};
+  const float2 y2 = make_float2(y, y), ns2 = make_float2(-s, -s);
+  float2 q[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float t = __fmul_rn(v[i], rcp);
-    c[i] = (QT == 1) ? e4m3_code_fast(t, near) : rne_low_byte(t, near);
+  for (int i = 0; i < 4; ++i) {
+    const float2 q0 = __fmul2_rn(v[i], y2);
+    const float2 r = __ffma2_rn(q0, ns2, v[i]);
+    q[i] = __ffma2_rn(r, y2, q0);
   }
-  if (near) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) c[i] = (QT == 1) ? e4m3_code_exact(v[i], s) : int8_code_exact(v[i], s);
-  }
-  return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24), c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
-}
-
-// 8 bf16 (one uint4) -> 8 codes (one uint2).
-template <int QT>
-__device__ __forceinline__ uint2 encode8(uint4 w, float s, float rcp) {
-  const float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
-                      bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
-  return encode8f<QT>(v, s, rcp);
-}
-
-// The exact codes of 8 bf16 by IEEE division: the rare path of encode8_fast,
-// kept out of line so that the hot loops stay small.
-template <int QT>
-__device__ __noinline__ uint2 encode8_exact(uint4 w, float s) {
-  const float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
-                      bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
-  uint32_t c[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) c[i] = (QT == 1) ? e4m3_code_exact(v[i], s) : int8_code_exact(v[i], s);
-  return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24), c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
-}
-
-// The same codes, four fp32 operations per value.  int8: the exact product
-// x * rcp is rounded once, to an integer, by fma(x, rcp, 1.5 * 2^23) (ties
-// to even), and its exact remainder d = fma(x, rcp, -rne) is rounded once.
-// x * rcp lies within 2 ulp of fl(x / s), so |d| < 0.5 - 2^-14 proves that
-// fl(x / s) rounds to the same integer; a group with any |d| at the margin
-// takes the exact division.  e4m3: as encode8 (interval ends compared).
-template <int QT>
-__device__ __forceinline__ uint2 encode8_fast(uint4 w, float s, float rcp) {
-  const float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
-                      bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
-  uint32_t c[8];
-  bool near = false;
   if constexpr (QT == 1) {
+    uint32_t c[4];
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-      const float t0 = __fmul_rn(v[i], rcp), t1 = __fmul_rn(v[i + 1], rcp);
-      const uint32_t ca = cvt_e4m3x2(__fmul_rn(t0, 1.0f - 0x1p-21f), __fmul_rn(t1, 1.0f - 0x1p-21f));
-      const uint32_t cb = cvt_e4m3x2(__fmul_rn(t0, 1.0f + 0x1p-21f), __fmul_rn(t1, 1.0f + 0x1p-21f));
-      near |= ca != cb;
-      c[i] = ca & 0xFFu;
-      c[i + 1] = ca >> 8;
+    for (int i = 0; i < 4; ++i) {
+      const float lo = __uint_as_float((__float_as_uint(q[i].x) & 0x7FFFFFFFu) | (__float_as_uint(v[i].x) & 0x80000000u));
+      const float hi = __uint_as_float((__float_as_uint(q[i].y) & 0x7FFFFFFFu) | (__float_as_uint(v[i].y) & 0x80000000u));
+      c[i] = cvt_e4m3x2(lo, hi);
     }
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
   } else {
-    float dmax = 0.0f;
+    const float2 mg = make_float2(kRneMagic, kRneMagic);
+    uint32_t c[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float big = __fmaf_rn(v[i], rcp, kRneMagic);
-      const float d = __fmaf_rn(v[i], rcp, -__fsub_rn(big, kRneMagic));
-      dmax = fmaxf(dmax, fabsf(d));
-      c[i] = __float_as_uint(big);
+    for (int i = 0; i < 4; ++i) {
+      const float2 b = __fadd2_rn(q[i], mg);
+      c[2 * i] = __float_as_uint(b.x);
+      c[2 * i + 1] = __float_as_uint(b.y);
     }
-    near = dmax > kNearHalf;
+    return make_uint2(prmt(prmt(c[0], c[1], 0x0040u), prmt(c[2], c[3], 0x0040u), 0x5410u),
+                      prmt(prmt(c[4], c[5], 0x0040u), prmt(c[6], c[7], 0x0040u), 0x5410u));
   }
-  if (near) return encode8_exact<QT>(w, s);
-  return make_uint2(prmt(prmt(c[0], c[1], 0x0040u), prmt(c[2], c[3], 0x0040u), 0x5410u),
-                    prmt(prmt(c[4], c[5], 0x0040u), prmt(c[6], c[7], 0x0040u), 0x5410u));
 }
 
-// Packed absmax of 8 bf16 (finite inputs).
-__device__ __forceinline__ __nv_bfloat162 absmax8_bf2(uint4 v, __nv_bfloat162 m) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) m = __hmax2(m, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[i])));
-  return m;
+// Running absmax of packed bf16 pairs: max(|m|, |v|) per half (the sign bit
+// of the result is junk; bf2_absmax_final clears it).  Finite inputs.
+__device__ __forceinline__ uint32_t bf2_absmax(uint32_t m, uint32_t v) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(m), "r"(v));
+  return d;
 }
-__device__ __forceinline__ float bf2_max(__nv_bfloat162 m) {
-  return fmaxf(__bfloat162float(m.x), __bfloat162float(m.y));
+__device__ __forceinline__ uint32_t absmax8(uint4 v, uint32_t m) {
+  return bf2_absmax(bf2_absmax(bf2_absmax(bf2_absmax(m, v.x), v.y), v.z), v.w);
 }
-__device__ __forceinline__ __nv_bfloat162 bf2_zero() { return __floats2bfloat162_rn(0.0f, 0.0f); }
+__device__ __forceinline__ float bf2_absmax_final(uint32_t m) {
+  return fmaxf(fabsf(bf16_lo(m)), fabsf(bf16_hi(m)));
+}
 
 // Block-wide max; every thread gets the result.  red: >= 32 floats of smem.
 __device__ __forceinline__ float block_max(float v, float* red) {
@@ -168,22 +128,24 @@ __global__ void __launch_bounds__(1024) quantize_rows_kernel(const __nv_bfloat16
                                                              int64_t M, int64_t K, uint8_t* __restrict__ q,
                                                              int64_t ldq, float* __restrict__ scale) {
   __shared__ float red[32];
+  griddep_launch();
+  griddep_wait();   // x may be the previous kernel's output
   const int64_t nv = K >> 3;
   for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
     const uint4* row = reinterpret_cast<const uint4*>(x + m * ldx);
     uint4 keep[kRowVecs];
-    __nv_bfloat162 mb = bf2_zero();
+    uint32_t mb = 0;
 #pragma unroll
     for (int j = 0; j < kRowVecs; ++j) {
       const int64_t v = threadIdx.x + static_cast<int64_t>(j) * blockDim.x;
       if (v < nv) {
         keep[j] = __ldg(row + v);
-        mb = absmax8_bf2(keep[j], mb);
+        mb = absmax8(keep[j], mb);
       }
     }
     for (int64_t v = threadIdx.x + static_cast<int64_t>(kRowVecs) * blockDim.x; v < nv; v += blockDim.x)
-      mb = absmax8_bf2(__ldg(row + v), mb);
-    const float a = block_max(bf2_max(mb), red);
+      mb = absmax8(__ldg(row + v), mb);
+    const float a = block_max(bf2_absmax_final(mb), red);
     const float s = absmax_scale<QT>(a);
     const float rcp = __frcp_rn(s);
     if (threadIdx.x == 0) scale[m] = s;
@@ -208,6 +170,8 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_team_kernel(const __nv_b
                                                                  int64_t M, int64_t K, uint8_t* __restrict__ q,
                                                                  int64_t ldq, float* __restrict__ scale) {
   __shared__ float red[2][8];
+  griddep_launch();
+  griddep_wait();   // x may be the previous kernel's output
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int team = warp / TW, tw = warp % TW;
   const int teams = (blockDim.x >> 5) / TW;
@@ -223,11 +187,11 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_team_kernel(const __nv_b
       const int v = tl + j * (32 * TW);
       if (v < nv) keep[j] = __ldg(row + v);
     }
-    __nv_bfloat162 mb = bf2_zero();
+    uint32_t mb = 0;
 #pragma unroll
     for (int j = 0; j < kTeamVecs; ++j)
-      if (tl + j * (32 * TW) < nv) mb = absmax8_bf2(keep[j], mb);
-    float a = bf2_max(mb);
+      if (tl + j * (32 * TW) < nv) mb = absmax8(keep[j], mb);
+    float a = bf2_absmax_final(mb);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
     if constexpr (TW > 1) {
@@ -243,7 +207,7 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_team_kernel(const __nv_b
 #pragma unroll
     for (int j = 0; j < kTeamVecs; ++j) {
       const int v = tl + j * (32 * TW);
-      if (v < nv) out[v] = encode8_fast<QT>(keep[j], s, rcp);
+      if (v < nv) out[v] = encode8<QT>(keep[j], s, rcp);
     }
   }
 }
@@ -253,11 +217,11 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_team_kernel(const __nv_b
 __global__ void __launch_bounds__(256) absmax_kernel(const uint4* __restrict__ w, int64_t nvec,
                                                      unsigned* __restrict__ amax_bits) {
   __shared__ float red[32];
-  __nv_bfloat162 mb = bf2_zero();
+  uint32_t mb = 0;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nvec;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    mb = absmax8_bf2(__ldg(w + i), mb);
-  const float a = block_max(bf2_max(mb), red);
+    mb = absmax8(__ldg(w + i), mb);
+  const float a = block_max(bf2_absmax_final(mb), red);
   if (threadIdx.x == 0) atomicMax(amax_bits, __float_as_uint(a));
 }
 
@@ -271,7 +235,7 @@ __global__ void __launch_bounds__(256) quantize_tensor_kernel(const uint4* __res
   if (blockIdx.x == 0 && threadIdx.x == 0) scale[0] = s;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nvec;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    q[i] = encode8_fast<QT>(__ldg(w + i), s, rcp);
+    q[i] = encode8<QT>(__ldg(w + i), s, rcp);
 }
 
 // fp32 -> E4M3FN codes with the quantizers' conversion.

@@ -8,6 +8,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "w8a8.h"
 #include "device.cuh"
@@ -119,6 +120,27 @@ cudaError_t set_smem_once(Kernel k, size_t bytes, int dev, std::atomic<uint64_t>
   return e;
 }
 
+// Launch with programmatic stream serialization: the kernel may start (and
+// run up to its griddep_wait) while the previous kernel on the stream
+// finishes.  The kernels launched this way are the row quantizers, the GEMM
+// and the split-K epilogue; each waits before touching memory that the
+// previous kernel may write or read.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // Output tensor map for the epilogue's TMA stores: bf16 [M, ldy] in 32 x 32
 // boxes with the 64-byte swizzle.  Used only when ldy % 8 == 0 (16-byte row
 // stride); otherwise the epilogue stores directly and the map is not read.
@@ -146,12 +168,12 @@ w8a8_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t M,
   auto kern = gemm_kernel<KIND, B_MN, BN, EPI>;
   cudaError_t e = set_smem_once(kern, C::kSmem, dev, smem_set);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
-  const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN);
+  if (ep.splits < 1) ep.splits = 1;
+  const int64_t units = ((M + kBM - 1) / kBM) * ((N + BN - 1) / BN) * ep.splits;
   const int64_t slots = static_cast<int64_t>(sms) * C::kCtasPerSm;
-  const int grid = static_cast<int>(tiles < slots ? tiles : slots);
-  gemm_kernel<KIND, B_MN, BN, EPI><<<grid, C::kThreads, C::kSmem, st>>>(ta, tb, ty, static_cast<int>(M),
-                                                                        static_cast<int>(N), static_cast<int>(Kc), ep);
-  e = cudaGetLastError();
+  const int grid = static_cast<int>(units < slots ? units : slots);
+  e = launch_pdl(kern, dim3(grid), dim3(C::kThreads), C::kSmem, st, ta, tb, ty, static_cast<int>(M),
+                 static_cast<int>(N), static_cast<int>(Kc), ep);
   return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "gemm launch");
 }
 
@@ -166,8 +188,9 @@ w8a8_status launch_quantize_rows(const void* x, int64_t ldx, int64_t M, int64_t 
     while (team_w < tw) team_w *= 2;
     const int64_t teams = 8 / team_w;
     const int grid = static_cast<int>((M + teams - 1) / teams < (1 << 20) ? (M + teams - 1) / teams : (1 << 20));
+    cudaError_t e = cudaSuccess;
 #define W8A8_TEAM_LAUNCH(QT, TW) \
-  quantize_rows_team_kernel<QT, TW><<<grid, 256, 0, st>>>(xp, ldx, M, K, qp, ldq, s)
+  e = launch_pdl(quantize_rows_team_kernel<QT, TW>, dim3(grid), dim3(256), 0, st, xp, ldx, M, K, qp, ldq, s)
     if (qt == W8A8_E4M3) {
       switch (team_w) {
         case 1: W8A8_TEAM_LAUNCH(1, 1); break;
@@ -184,19 +207,21 @@ w8a8_status launch_quantize_rows(const void* x, int64_t ldx, int64_t M, int64_t 
       }
     }
 #undef W8A8_TEAM_LAUNCH
+    return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "quantize_rows launch");
   } else {
     int64_t t = (nv + kRowVecs - 1) / kRowVecs;
     t = round_up(t, 32);
     if (t < 32) t = 32;
     if (t > 1024) t = 1024;
     const int grid = static_cast<int>(M < (1 << 20) ? M : (1 << 20));
-    if (qt == W8A8_E4M3)
-      quantize_rows_kernel<1><<<grid, static_cast<int>(t), 0, st>>>(xp, ldx, M, K, qp, ldq, s);
-    else
-      quantize_rows_kernel<0><<<grid, static_cast<int>(t), 0, st>>>(xp, ldx, M, K, qp, ldq, s);
+    const cudaError_t e =
+        (qt == W8A8_E4M3)
+            ? launch_pdl(quantize_rows_kernel<1>, dim3(grid), dim3(static_cast<unsigned>(t)), 0, st, xp, ldx, M, K,
+                         qp, ldq, s)
+            : launch_pdl(quantize_rows_kernel<0>, dim3(grid), dim3(static_cast<unsigned>(t)), 0, st, xp, ldx, M, K,
+                         qp, ldq, s);
+    return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "quantize_rows launch");
   }
-  cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "quantize_rows launch");
 }
 
 // Workspace carving: each piece starts on a 256-byte boundary.
@@ -211,12 +236,78 @@ struct Carve {
   }
 };
 
-size_t ws_linear(int64_t M, int64_t ld) {
+// Split-K for int8 GEMMs with few output tiles (few tokens): when the tiles
+// fill at most half of a B200's 148 SMs, the contraction is split, at least
+// 4 K blocks (512 codes) per split and at most 16 splits; the partial sums
+// [S, M, Nout] go to the workspace and splitk_epilogue_kernel finishes them
+// (Nout % 8 == 0).  Integer partial sums add up exactly, so the result is the
+// unsplit one bit for bit.  e4m3 products are never split: the tensor cores'
+// fp32 accumulation order would change, and with it the rounding.  The count
+// depends on the shape alone (the workspace size covers the int8 case for
+// both formats), so workspace sizes do not depend on the device.
+constexpr int64_t kSplitSms = 148;
+int choose_splits(int64_t M, int64_t Nout, int64_t Kc) {
+  const int64_t tiles = ((M + kBM - 1) / kBM) * ((Nout + 255) / 256);
+  const int64_t num_kb = (Kc + kBKBytes - 1) / kBKBytes;
+  if (tiles <= 0 || tiles * 2 > kSplitSms || (Nout % 8) != 0) return 1;
+  int64_t s = kSplitSms / tiles;
+  if (s > num_kb / 4) s = num_kb / 4;
+  if (s > 16) s = 16;
+  return s < 2 ? 1 : static_cast<int>(s);
+}
+
+// Workspace of a linear call: codes [M, ld] and row scales [M], then, when
+// the GEMM is split, the partial sums [S, M, Nout].
+struct LinearWs {
+  size_t bytes;
+  int splits;
+};
+LinearWs linear_ws(int64_t M, int64_t ld, int64_t Nout) {
+  LinearWs w{0, choose_splits(M, Nout, ld)};
   Carve c(nullptr);
   c.take(static_cast<size_t>(M * ld));
   c.take(static_cast<size_t>(M) * 4);
-  return c.off;
+  if (w.splits > 1) c.take(static_cast<size_t>(w.splits) * static_cast<size_t>(M) * static_cast<size_t>(Nout) * 4);
+  w.bytes = c.off;
+  return w;
 }
+size_t ws_linear(int64_t M, int64_t ld, int64_t Nout) { return linear_ws(M, ld, Nout).bytes; }
+
+// The split-K part of a carved workspace.
+struct SplitWs {
+  int splits = 1;
+  uint32_t* partial = nullptr;
+};
+SplitWs carve_split(Carve& c, int64_t M, int64_t Nout, const LinearWs& w, int qt) {
+  SplitWs sk;
+  if (w.splits > 1 && qt == W8A8_INT8) {
+    sk.splits = w.splits;
+    sk.partial = static_cast<uint32_t*>(
+        c.take(static_cast<size_t>(w.splits) * static_cast<size_t>(M) * static_cast<size_t>(Nout) * 4));
+  }
+  return sk;
+}
+
+// The finishing kernel of a split product (after the GEMM on the stream).
+w8a8_status launch_splitk_epilogue(int qt, const SplitWs& sk, int64_t M, int64_t Nout, const float* sx,
+                                   const float* sw, int axis, const void* bias, void* y, cudaStream_t st) {
+  int sms = 0;
+  w8a8_status s = current_device(nullptr, &sms);
+  if (s != W8A8_OK) return s;
+  int64_t grid = (M * (Nout / 8) + 255) / 256;
+  if (grid > 8 * static_cast<int64_t>(sms)) grid = 8 * static_cast<int64_t>(sms);
+  const auto* b = static_cast<const __nv_bfloat16*>(bias);
+  auto* yp = static_cast<__nv_bfloat16*>(y);
+  const uint32_t* part = sk.partial;
+  const cudaError_t e =
+      (qt == W8A8_E4M3)
+          ? launch_pdl(splitk_epilogue_kernel<kKindE4M3>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, part,
+                       sk.splits, M, Nout, sx, sw, axis, b, yp)
+          : launch_pdl(splitk_epilogue_kernel<kKindI8>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, part,
+                       sk.splits, M, Nout, sx, sw, axis, b, yp);
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "split-K epilogue launch");
+}
+
 size_t ws_svdq(int64_t M, int64_t K, int r) {
   Carve c(nullptr);
   c.take(static_cast<size_t>(M * K));
@@ -231,8 +322,10 @@ bool valid_g(int g) { return g == W8A8_TENSOR || g == W8A8_AXIS; }
 CUtensorMapDataType code_type() { return CU_TENSOR_MAP_DATA_TYPE_UINT8; }
 
 // GEMM on codes.  fwd: A = xq [M, lda] K-major, B = wq [N, K] K-major.
+// sk: split-K workspace (partial sums), or null for an unsplit product.
 w8a8_status gemm_fwd(const void* xq, int64_t lda, const float* sx, int64_t M, int64_t N, int64_t K, int qt,
-                     const void* wq, const float* sw, int g, const void* bias, void* y, cudaStream_t st) {
+                     const void* wq, const float* sw, int g, const void* bias, void* y, cudaStream_t st,
+                     const SplitWs* sk = nullptr) {
   alignas(64) CUtensorMap ta, tb;
   w8a8_status s = make_map(&ta, code_type(), 1, xq, K, M, lda, kBKBytes, kBM);
   if (s != W8A8_OK) return s;
@@ -245,13 +338,20 @@ w8a8_status gemm_fwd(const void* xq, int64_t lda, const float* sx, int64_t M, in
   ep.bias = static_cast<const __nv_bfloat16*>(bias);
   ep.y = static_cast<__nv_bfloat16*>(y);
   ep.ldy = N;
-  if (qt == W8A8_E4M3) return launch_gemm<kKindE4M3, false, 256, kEpiScale>(ta, tb, M, N, K, ep, st);
-  return launch_gemm<kKindI8, false, 256, kEpiScale>(ta, tb, M, N, K, ep, st);
+  ep.splits = 1;
+  if (sk != nullptr && sk->splits > 1) {
+    ep.splits = sk->splits;
+    ep.partial = sk->partial;
+  }
+  s = (qt == W8A8_E4M3) ? launch_gemm<kKindE4M3, false, 256, kEpiScale>(ta, tb, M, N, K, ep, st)
+                        : launch_gemm<kKindI8, false, 256, kEpiScale>(ta, tb, M, N, K, ep, st);
+  if (s != W8A8_OK || ep.splits == 1) return s;
+  return launch_splitk_epilogue(qt, *sk, M, N, sx, sw, g == W8A8_AXIS, bias, y, st);
 }
 
 // dgrad: A = dyq [M, lda] (contraction N), B = wq [N, K] read MN-major.
 w8a8_status gemm_dgrad(const void* dyq, int64_t lda, const float* sdy, int64_t M, int64_t N, int64_t K, int qt,
-                       const void* wq, const float* sw, void* dx, cudaStream_t st) {
+                       const void* wq, const float* sw, void* dx, cudaStream_t st, const SplitWs* sk = nullptr) {
   alignas(64) CUtensorMap ta, tb;
   w8a8_status s = make_map(&ta, code_type(), 1, dyq, N, M, lda, kBKBytes, kBM);
   if (s != W8A8_OK) return s;
@@ -263,8 +363,15 @@ w8a8_status gemm_dgrad(const void* dyq, int64_t lda, const float* sdy, int64_t M
   ep.s_col_axis = 0;
   ep.y = static_cast<__nv_bfloat16*>(dx);
   ep.ldy = K;
-  if (qt == W8A8_E4M3) return launch_gemm<kKindE4M3, true, 256, kEpiScale>(ta, tb, M, K, N, ep, st);
-  return launch_gemm<kKindI8, true, 256, kEpiScale>(ta, tb, M, K, N, ep, st);
+  ep.splits = 1;
+  if (sk != nullptr && sk->splits > 1) {
+    ep.splits = sk->splits;
+    ep.partial = sk->partial;
+  }
+  s = (qt == W8A8_E4M3) ? launch_gemm<kKindE4M3, true, 256, kEpiScale>(ta, tb, M, K, N, ep, st)
+                        : launch_gemm<kKindI8, true, 256, kEpiScale>(ta, tb, M, K, N, ep, st);
+  if (s != W8A8_OK || ep.splits == 1) return s;
+  return launch_splitk_epilogue(qt, *sk, M, K, sdy, sw, 0, nullptr, dx, st);
 }
 
 #define W8A8_CHECK(cond, status, ...) \
@@ -315,8 +422,8 @@ size_t q8_0_bytes(int64_t n) { return n <= 0 ? 0 : static_cast<size_t>((n + 31) 
 size_t w8a8_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
   if (M < 0 || N < 0 || K < 0) return 0;
   switch (op) {
-    case W8A8_OP_LINEAR_FWD: return ws_linear(M, K);
-    case W8A8_OP_LINEAR_DGRAD: return ws_linear(M, round_up(N, 16));
+    case W8A8_OP_LINEAR_FWD: return ws_linear(M, K, N);
+    case W8A8_OP_LINEAR_DGRAD: return ws_linear(M, round_up(N, 16), K);
     case W8A8_OP_SVDQ_FWD: return ws_svdq(M, K, r);
     case W8A8_OP_QUANTIZE_WEIGHT: return 256;
     default: return 0;
@@ -507,16 +614,18 @@ w8a8_status w8a8_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, w8a8
   W8A8_CHECK(x && wq && sw && y, W8A8_ERR_INVALID_ARG, "null pointer");
   W8A8_CHECK(aligned16(x) && aligned16(wq) && aligned16(sw) && aligned16(y) && (bias == nullptr || aligned16(bias)),
              W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
-  W8A8_CHECK(ws != nullptr && ws_bytes >= ws_linear(M, K), W8A8_ERR_WORKSPACE, "workspace too small: need %zu bytes",
-             ws_linear(M, K));
+  const LinearWs lw = linear_ws(M, K, N);
+  W8A8_CHECK(ws != nullptr && ws_bytes >= lw.bytes, W8A8_ERR_WORKSPACE, "workspace too small: need %zu bytes",
+             lw.bytes);
   W8A8_CHECK(aligned16(ws), W8A8_ERR_MISALIGNED, "workspace must be 16-byte aligned");
   if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   Carve c(ws);
   void* xq = c.take(static_cast<size_t>(M * K));
   float* sx = static_cast<float*>(c.take(static_cast<size_t>(M) * 4));
+  const SplitWs sk = carve_split(c, M, N, lw, qt);
   if ((st = launch_quantize_rows(x, K, M, K, qt, xq, K, sx, s)) != W8A8_OK) return st;
-  return gemm_fwd(xq, K, sx, M, N, K, qt, wq, sw, g, bias, y, s);
+  return gemm_fwd(xq, K, sx, M, N, K, qt, wq, sw, g, bias, y, s, &sk);
 }
 
 w8a8_status w8a8_linear_fwd_noalloc(const void* x, int64_t M, int64_t N, int64_t K, w8a8_qtype qt, const void* wq,
@@ -559,16 +668,18 @@ w8a8_status w8a8_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, w
   W8A8_CHECK(dy && wq && sw && dx, W8A8_ERR_INVALID_ARG, "null pointer");
   W8A8_CHECK(aligned16(dy) && aligned16(wq) && aligned16(sw) && aligned16(dx), W8A8_ERR_MISALIGNED,
              "pointers must be 16-byte aligned");
-  W8A8_CHECK(ws != nullptr && ws_bytes >= ws_linear(M, N), W8A8_ERR_WORKSPACE, "workspace too small: need %zu bytes",
-             ws_linear(M, N));
+  const LinearWs lw = linear_ws(M, N, K);
+  W8A8_CHECK(ws != nullptr && ws_bytes >= lw.bytes, W8A8_ERR_WORKSPACE, "workspace too small: need %zu bytes",
+             lw.bytes);
   W8A8_CHECK(aligned16(ws), W8A8_ERR_MISALIGNED, "workspace must be 16-byte aligned");
   if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   Carve c(ws);
   void* dyq = c.take(static_cast<size_t>(M * N));
   float* sdy = static_cast<float*>(c.take(static_cast<size_t>(M) * 4));
+  const SplitWs sk = carve_split(c, M, K, lw, qt);
   if ((st = launch_quantize_rows(dy, N, M, N, qt, dyq, N, sdy, s)) != W8A8_OK) return st;
-  return gemm_dgrad(dyq, N, sdy, M, N, K, qt, wq, sw, dx, s);
+  return gemm_dgrad(dyq, N, sdy, M, N, K, qt, wq, sw, dx, s, &sk);
 }
 
 w8a8_status svdq_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, const void* rq, const float* r_scale,
