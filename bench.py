@@ -450,11 +450,14 @@ def run_ours(args, rank, world, local_rank):
 
 
 def run_case(args):
-    """One quantize + GEMM pair of the step, warmup + steps times (profiling)."""
+    """One quantize + GEMM pair of the step, or one other kernel of the path,
+    warmup + steps times (profiling)."""
     import torch
     import workloads
     import w8a8_quantized_linear_b200 as w8
     dev = torch.device("cuda", 0)
+    if args.case in ("requant", "gguf_m1", "gguf_m64", "svdq"):
+        return run_other_case(args, torch, workloads, w8, dev)
     wl = workloads.dit_mlp()
     if args.case in ("up", "dgrad_up"):
         wq, sw = w8.quantize_weight(wl["w1"].to(dev), "int8", "tensor")      # [12288, 3072]
@@ -475,6 +478,33 @@ def run_case(args):
     for _ in range(args.warmup + args.steps):
         xq, s = w8.quantize_rows(x, "int8")
         fn(xq, s)
+    torch.cuda.synchronize()
+    assert w8.device_status() == 0
+    print("case %s ok" % args.case)
+    return 0
+
+
+def run_other_case(args, torch, workloads, w8, dev):
+    """requant: Q8_0 -> axis int8 of the 12288 x 3072 GGUF weight;
+    gguf_m1 / gguf_m64: the GGUF A8 int forward at M = 1 / 64;
+    svdq: the SVDQuant r = 32 forward at 4608 x 3072 x 3072."""
+    if args.case == "svdq":
+        d = workloads.svdquant()
+        prep = w8.svdq_prepare(d["w"].to(dev), d["r"])
+        x = d["x"].to(dev)
+        fn = lambda: w8.svdq_linear_fwd(x, prep["rq"], prep["r_scale"], prep["l1"], prep["l2"])
+    else:
+        g = workloads.gguf_q8_0(M=64)
+        N, K = g["w_f32"].shape
+        blk = w8.q8_0_quantize(g["w_f32"].reshape(-1).to(dev))
+        if args.case == "requant":
+            fn = lambda: w8.q8_0_to_axis_int8(blk, N, K)
+        else:
+            wq, sw = w8.q8_0_to_axis_int8(blk, N, K)
+            x = g["x"][:1 if args.case == "gguf_m1" else 64].to(dev)
+            fn = lambda: w8.linear_fwd(x, wq, sw)
+    for _ in range(args.warmup + args.steps):
+        fn()
     torch.cuda.synchronize()
     assert w8.device_status() == 0
     print("case %s ok" % args.case)
@@ -646,8 +676,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-extras", dest="extras", action="store_false")
-    ap.add_argument("--case", choices=["up", "down", "dgrad_down", "dgrad_up"], default=None,
-                    help="run only one of the step's four quantize+GEMM pairs (for profiling), no JSON")
+    ap.add_argument("--case", choices=["up", "down", "dgrad_down", "dgrad_up", "requant", "gguf_m1", "gguf_m64", "svdq"],
+                    default=None, help="run only one of the step's four quantize+GEMM pairs, or one other kernel "
+                                       "of the path (for profiling), no JSON")
     args = ap.parse_args()
     if args.warmup < 3 and not args.case:
         ap.error("--warmup must be >= 3")

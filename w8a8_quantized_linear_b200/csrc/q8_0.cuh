@@ -227,16 +227,17 @@ __global__ void __launch_bounds__(32 * kRequantMaxWarps) q8_0_to_axis_int8_kerne
 // ----------------------------------------------------------------------------
 // Q8_0 -> axis int8 for rows whose blocks fill whole 16-byte units
 // (K % 256 == 0): a team of TW warps per row, thread t of the team taking
-// blocks t, t + 32 TW, ...  Each team copies its next row into shared memory
-// (cp.async, double-buffered) while it processes the current one.
+// blocks t, t + 32 TW, ...  Each team keeps its next S - 1 rows in flight
+// into a ring of S shared-memory row buffers (cp.async) while it processes
+// the current one.
 //
 // A block b starts at byte 34 b of the row, i.e. on a word boundary when b is
 // even and 2 bytes past one when b is odd; its 34 bytes lie in the 9 words
 // from word floor(34 b / 4), and prmt selects the f16 scale and the 32 codes
 // from them.  Pass 1 takes max |q| of each block on sign-extended 16-bit
-// pairs (max/min.s16x2); max |d q| = |d| max |q| exactly.  Pass 2 rounds
-// q * fl(d / s') as rne_low_byte does, with the exact product inside an fma;
-// a group of 8 within 2^-14 of a tie takes the IEEE division out of line.
+// pairs (max/min.s16x2); max |d q| = |d| max |q| exactly.  Pass 2 forms
+// the codes with the refined quotient of rq_block_codes (no division, no
+// data-dependent branch).
 // ----------------------------------------------------------------------------
 constexpr int kRqThreads = 256;
 
@@ -293,56 +294,41 @@ __device__ __forceinline__ float rq_block_scale(const uint32_t (&w)[9], bool odd
   return __half2float(__ushort_as_half(static_cast<uint16_t>(prmt(w[0], 0u, odd ? 0x4432u : 0x4410u))));
 }
 
-// The rare exact path, kept out of line so that the hot loop stays small:
-// the remainders are recomputed and only the values at the margin take the
-// IEEE division of fl(d q) by s.
-__device__ __noinline__ uint2 rq_codes8_exact(float d, float s, float drcp, float q0, float q1, float q2, float q3,
-                                              float q4, float q5, float q6, float q7) {
-  const float v[8] = {q0, q1, q2, q3, q4, q5, q6, q7};
-  uint32_t c[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float b = __fmaf_rn(v[i], drcp, kRneMagic);
-    const float r = __fmaf_rn(v[i], drcp, -__fsub_rn(b, kRneMagic));
-    c[i] = (fabsf(r) > kNearHalf) ? int8_code_exact(__fmul_rn(d, v[i]), s) : (__float_as_uint(b) & 0xFFu);
-  }
-  return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24), c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
-}
-
-// 32 codes of a block -> 32 axis int8 codes (8 words).
-__device__ __forceinline__ void rq_block_codes(const uint32_t (&w)[9], bool odd, float d, float s, float rcp,
+// 32 codes of a block -> 32 axis int8 codes (8 words).  Each value
+// fl(d q) = d q is exact (an 11-bit by 8-bit product); its code is
+// fl(d q / s) rounded half to even, with the quotient refined from
+// y = fl(1/s) as in the row quantizers (encode8): q0 = fl(x y),
+// r = fl(x - q0 s), q1 = fl(q0 + r y) is the IEEE quotient for every value
+// a Q8_0 block can hold and every scale s = fl(a / 127) such values give
+// (checked exhaustively on the GPU), so no value needs a division and no
+// data-dependent branch is taken.  |x / s| <= 127 (1 + 2^-23): no clamp.
+__device__ __forceinline__ void rq_block_codes(const uint32_t (&w)[9], bool odd, float d, float s, float y,
                                                uint32_t (&out)[8]) {
   const uint32_t csel = odd ? 0x7654u : 0x5432u;
-  const float drcp = __fmul_rn(d, rcp);
   uint32_t c[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) c[k] = prmt(w[k], w[k + 1], csel);
+  const float2 d2 = make_float2(d, d), y2 = make_float2(y, y), ns2 = make_float2(-s, -s);
+  const float2 mg = make_float2(kRneMagic, kRneMagic);
 #pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    float qf[8];
+  for (int k = 0; k < 8; ++k) {
+    uint32_t b[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) qf[i] = static_cast<float>(static_cast<int8_t>(c[2 * g + i / 4] >> (8 * (i & 3))));
-    uint32_t big[8];
-    float dmax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float b = __fmaf_rn(qf[i], drcp, kRneMagic);
-      const float r = __fmaf_rn(qf[i], drcp, -__fsub_rn(b, kRneMagic));
-      dmax = fmaxf(dmax, fabsf(r));
-      big[i] = __float_as_uint(b);
+    for (int h = 0; h < 2; ++h) {
+      const float2 qv = make_float2(static_cast<float>(static_cast<int8_t>(c[k] >> (16 * h))),
+                                    static_cast<float>(static_cast<int8_t>(c[k] >> (16 * h + 8))));
+      const float2 x = __fmul2_rn(qv, d2);
+      const float2 q0 = __fmul2_rn(x, y2);
+      const float2 r = __ffma2_rn(q0, ns2, x);
+      const float2 q1 = __fadd2_rn(__ffma2_rn(r, y2, q0), mg);
+      b[2 * h] = __float_as_uint(q1.x);
+      b[2 * h + 1] = __float_as_uint(q1.y);
     }
-    if (dmax > kNearHalf) {
-      const uint2 e = rq_codes8_exact(d, s, drcp, qf[0], qf[1], qf[2], qf[3], qf[4], qf[5], qf[6], qf[7]);
-      out[2 * g] = e.x;
-      out[2 * g + 1] = e.y;
-    } else {
-      out[2 * g] = prmt(prmt(big[0], big[1], 0x0040u), prmt(big[2], big[3], 0x0040u), 0x5410u);
-      out[2 * g + 1] = prmt(prmt(big[4], big[5], 0x0040u), prmt(big[6], big[7], 0x0040u), 0x5410u);
-    }
+    out[k] = prmt(prmt(b[0], b[1], 0x0040u), prmt(b[2], b[3], 0x0040u), 0x5410u);
   }
 }
 
-template <int TW>
+template <int TW, int S>
 __global__ void __launch_bounds__(kRqThreads) q8_0_to_axis_int8_team_kernel(const uint8_t* __restrict__ blocks,
                                                                            int64_t N, int64_t K,
                                                                            int8_t* __restrict__ q,
@@ -355,24 +341,24 @@ __global__ void __launch_bounds__(kRqThreads) q8_0_to_axis_int8_team_kernel(cons
   const int nblk = static_cast<int>(K >> 5);
   const int row_bytes = nblk * kQ80Bytes;   // a multiple of 16
   const int nvec = row_bytes >> 4;
-  uint8_t* const buf = rq_smem + 2 * team * row_bytes;   // two row buffers per team
+  uint8_t* const buf = rq_smem + S * team * row_bytes;   // a ring of S row buffers per team
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kTeams;
   int64_t n = blockIdx.x * static_cast<int64_t>(kTeams) + team;
-  if (n < N) {
-    const uint8_t* src = blocks + n * row_bytes;
-    for (int i = t; i < nvec; i += T) cp_async16(buf + 16 * i, src + 16 * i);
-  }
-  cp_async_commit();
-  for (int it = 0; n < N; n += stride, ++it) {
-    const uint8_t* cur = buf + (it & 1) * row_bytes;
-    if (n + stride < N) {
-      const uint8_t* src = blocks + (n + stride) * row_bytes;
-      uint8_t* dst = buf + ((it + 1) & 1) * row_bytes;
+  auto fetch = [&](int64_t row, int slot) {   // one commit group per call, empty past the last row
+    if (row < N) {
+      const uint8_t* src = blocks + row * row_bytes;
+      uint8_t* dst = buf + slot * row_bytes;
       for (int i = t; i < nvec; i += T) cp_async16(dst + 16 * i, src + 16 * i);
     }
     cp_async_commit();
-    cp_async_wait<1>();
-    team_sync<TW>(team);
+  };
+#pragma unroll
+  for (int p = 0; p < S - 1; ++p) fetch(n + p * stride, p);
+  for (int it = 0; n < N; n += stride, ++it) {
+    const uint8_t* cur = buf + (it % S) * row_bytes;
+    fetch(n + (S - 1) * stride, (it + S - 1) % S);
+    cp_async_wait<S - 1>();   // this thread's copies of the current row have landed
+    team_sync<TW>(team);      // ... and every other thread's
     float a = 0.0f;
 #pragma unroll 1
     for (int b = t; b < nblk; b += T) {
@@ -403,7 +389,7 @@ __global__ void __launch_bounds__(kRqThreads) q8_0_to_axis_int8_team_kernel(cons
       dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
       dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
     }
-    team_sync<TW>(team);   // the buffer of this row is refilled two rows on
+    team_sync<TW>(team);   // this row's buffer is refilled on the next iteration
   }
   cp_async_wait<0>();
 }
