@@ -78,6 +78,111 @@ struct GemmCfg {
   static_assert(kSmem <= 232448, "shared memory per block");
 };
 
+// One epilogue warp's chunks of a 128-row x BN-column accumulator tile:
+// the warp reads the 32 TMEM lanes of its quarter (rows m0 + 32 quarter +
+// lane) for the 32-column chunks c = group, group + kGroups, ... at TMEM
+// address tacc; y = bf16(((acc * s_x) * s_w) + bias), each step an fp32 RN
+// operation; the warp's 32 x 32 bf16 block goes out through one of its two
+// swizzled staging buffers (sOutWarp) with a TMA store, or directly when the
+// row stride is not a multiple of 8.
+template <int KIND, int EPI, int BN, int kGroups, bool kAxisOk>
+__device__ __forceinline__ void epilogue_scale_chunks(const EpiParams& ep, const CUtensorMap* tmY, uint32_t tacc, int m0,
+                                                      int n0, int M, int N, int quarter, int group, int lane, float sx,
+                                                      float sw0, uint8_t* sOutWarp, uint32_t& out_iter) {
+  const int row = m0 + quarter * 32 + lane;
+  const bool row_ok = row < M;
+  #pragma unroll 1
+  for (int c = group; c < BN / 32; c += kGroups) {
+    const int nc = n0 + c * 32;
+    if (nc >= N) break;                       // warp-uniform
+    const bool full_chunk = nc + 32 <= N;
+    // Column parameters of the chunk, loaded before the TMEM load so that
+    // their latency overlaps it: 16-byte vectors, the same addresses in
+    // every lane (broadcast).
+    float sw[32], bs[32];
+    if constexpr (EPI != kEpiPlain) {
+      if (kAxisOk && ep.s_col_axis) {
+        if (full_chunk) {
+  #pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            const float4 f = __ldg(reinterpret_cast<const float4*>(ep.s_col + nc + j));
+            sw[j] = f.x; sw[j + 1] = f.y; sw[j + 2] = f.z; sw[j + 3] = f.w;
+          }
+        } else {
+  #pragma unroll
+          for (int j = 0; j < 32; ++j) sw[j] = (nc + j < N) ? __ldg(ep.s_col + nc + j) : 0.0f;
+        }
+      }
+      if (ep.bias != nullptr) {
+        if (full_chunk) {
+  #pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            const uint4 b = __ldg(reinterpret_cast<const uint4*>(ep.bias + nc + j));
+            bs[j] = bf16_lo(b.x); bs[j + 1] = bf16_hi(b.x); bs[j + 2] = bf16_lo(b.y); bs[j + 3] = bf16_hi(b.y);
+            bs[j + 4] = bf16_lo(b.z); bs[j + 5] = bf16_hi(b.z); bs[j + 6] = bf16_lo(b.w); bs[j + 7] = bf16_hi(b.w);
+          }
+        } else {
+  #pragma unroll
+          for (int j = 0; j < 32; ++j) bs[j] = (nc + j < N) ? __bfloat162float(ep.bias[nc + j]) : 0.0f;
+        }
+      }
+    }
+    uint32_t r[32];
+    tmem_ld_x32(tacc + static_cast<uint32_t>(c * 32), r);
+    tmem_ld_wait();
+    float v[32];
+  #pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int>(r[j])) : __uint_as_float(r[j]);
+      if constexpr (EPI != kEpiPlain) {
+        a = __fmul_rn(__fmul_rn(a, sx), (kAxisOk && ep.s_col_axis) ? sw[j] : sw0);
+        if (ep.bias != nullptr) a = __fadd_rn(a, bs[j]);
+      }
+      v[j] = a;
+    }
+    if (ep.tma_store) {
+      // Stage the warp's 32 x 32 bf16 block in shared memory with the 64-byte
+      // swizzle (16-byte unit j of row l at unit j ^ ((l >> 1) & 3)), then
+      // one lane stores it with TMA; the box is clipped at M and N.
+      uint8_t* buf = sOutWarp + (out_iter & 1) * (32 * 32 * 2);
+      if (lane == 0) bulk_wait_read<1>();     // this buffer's previous store has read it
+      __syncwarp();
+  #pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint4 p;
+        p.x = pack_bf16x2(v[8 * j], v[8 * j + 1]);
+        p.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+        p.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+        p.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+        *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) = p;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && m0 + quarter * 32 < M) {   // skip blocks wholly below the last row
+        tma_store_2d(tmY, buf, nc, m0 + quarter * 32);
+        bulk_commit();
+      }
+      ++out_iter;
+    } else if (row_ok) {
+      __nv_bfloat16* out = ep.y + static_cast<int64_t>(row) * ep.ldy + nc;
+      if (nc + 32 <= N && (ep.ldy & 7) == 0) {
+  #pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          uint4 p;
+          p.x = pack_bf16x2(v[j], v[j + 1]);
+          p.y = pack_bf16x2(v[j + 2], v[j + 3]);
+          p.z = pack_bf16x2(v[j + 4], v[j + 5]);
+          p.w = pack_bf16x2(v[j + 6], v[j + 7]);
+          *reinterpret_cast<uint4*>(out + j) = p;
+        }
+      } else {
+        for (int j = 0; j < 32; ++j)
+          if (nc + j < N) out[j] = __float2bfloat16_rn(v[j]);
+      }
+    }
+  }
+}
+
 template <int KIND, bool B_MN, int BN, int EPI>
 __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -408,96 +513,10 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
           }
           write_out = false;   // splitk_epilogue_kernel finishes the tile
         }
-  #pragma unroll 1
-        for (int c = group; write_out && c < BN / 32; c += kGroups) {
-          const int nc = n0 + c * 32;
-          if (nc >= N) break;                       // warp-uniform
-          const bool full_chunk = nc + 32 <= N;
-          // Column parameters of the chunk, loaded before the TMEM load so that
-          // their latency overlaps it: 16-byte vectors, the same addresses in
-          // every lane (broadcast).
-          float sw[32], bs[32];
-          if constexpr (EPI != kEpiPlain) {
-            if (kAxisOk && ep.s_col_axis) {
-              if (full_chunk) {
-  #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                  const float4 f = __ldg(reinterpret_cast<const float4*>(ep.s_col + nc + j));
-                  sw[j] = f.x; sw[j + 1] = f.y; sw[j + 2] = f.z; sw[j + 3] = f.w;
-                }
-              } else {
-  #pragma unroll
-                for (int j = 0; j < 32; ++j) sw[j] = (nc + j < N) ? __ldg(ep.s_col + nc + j) : 0.0f;
-              }
-            }
-            if (ep.bias != nullptr) {
-              if (full_chunk) {
-  #pragma unroll
-                for (int j = 0; j < 32; j += 8) {
-                  const uint4 b = __ldg(reinterpret_cast<const uint4*>(ep.bias + nc + j));
-                  bs[j] = bf16_lo(b.x); bs[j + 1] = bf16_hi(b.x); bs[j + 2] = bf16_lo(b.y); bs[j + 3] = bf16_hi(b.y);
-                  bs[j + 4] = bf16_lo(b.z); bs[j + 5] = bf16_hi(b.z); bs[j + 6] = bf16_lo(b.w); bs[j + 7] = bf16_hi(b.w);
-                }
-              } else {
-  #pragma unroll
-                for (int j = 0; j < 32; ++j) bs[j] = (nc + j < N) ? __bfloat162float(ep.bias[nc + j]) : 0.0f;
-              }
-            }
-          }
-          uint32_t r[32];
-          tmem_ld_x32(tmem + lane_base + static_cast<uint32_t>(acc * BN + c * 32), r);
-          tmem_ld_wait();
-          float v[32];
-  #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int>(r[j])) : __uint_as_float(r[j]);
-            if constexpr (EPI != kEpiPlain) {
-              a = __fmul_rn(__fmul_rn(a, sx), (kAxisOk && ep.s_col_axis) ? sw[j] : sw0);
-              if (ep.bias != nullptr) a = __fadd_rn(a, bs[j]);
-            }
-            v[j] = a;
-          }
-          if (ep.tma_store) {
-            // Stage the warp's 32 x 32 bf16 block in shared memory with the 64-byte
-            // swizzle (16-byte unit j of row l at unit j ^ ((l >> 1) & 3)), then
-            // one lane stores it with TMA; the box is clipped at M and N.
-            uint8_t* buf = sOut + ((e * 2 + (out_iter & 1)) * C::kOutBufBytes);
-            if (lane == 0) bulk_wait_read<1>();     // this buffer's previous store has read it
-            __syncwarp();
-  #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              uint4 p;
-              p.x = pack_bf16x2(v[8 * j], v[8 * j + 1]);
-              p.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-              p.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-              p.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
-              *reinterpret_cast<uint4*>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) = p;
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0 && m0 + quarter * 32 < M) {   // skip blocks wholly below the last row
-              tma_store_2d(&tmY, buf, nc, m0 + quarter * 32);
-              bulk_commit();
-            }
-            ++out_iter;
-          } else if (row_ok) {
-            __nv_bfloat16* out = ep.y + static_cast<int64_t>(row) * ep.ldy + nc;
-            if (nc + 32 <= N && (ep.ldy & 7) == 0) {
-  #pragma unroll
-              for (int j = 0; j < 32; j += 8) {
-                uint4 p;
-                p.x = pack_bf16x2(v[j], v[j + 1]);
-                p.y = pack_bf16x2(v[j + 2], v[j + 3]);
-                p.z = pack_bf16x2(v[j + 4], v[j + 5]);
-                p.w = pack_bf16x2(v[j + 6], v[j + 7]);
-                *reinterpret_cast<uint4*>(out + j) = p;
-              }
-            } else {
-              for (int j = 0; j < 32; ++j)
-                if (nc + j < N) out[j] = __float2bfloat16_rn(v[j]);
-            }
-          }
-        }
+        if (write_out)
+          epilogue_scale_chunks<KIND, EPI, BN, kGroups, kAxisOk>(ep, &tmY, tmem + lane_base + static_cast<uint32_t>(acc * BN),
+                                                                 m0, n0, M, N, quarter, group, lane, sx, sw0,
+                                                                 sOut + e * 2 * C::kOutBufBytes, out_iter);
       }
       tc_fence_before();
       __syncwarp();

@@ -1,0 +1,222 @@
+// gemm_pair.cuh - the 8-bit GEMM with the scale epilogue on CTA pairs: a
+// cluster of two CTAs on two SMs computes a 256 x 256 tile with one
+// tcgen05.mma.cta_group::2 stream (M = 256: 128 rows in each CTA's shared
+// memory and TMEM; B split along N, 128 rows or columns in each CTA).  Per
+// SM this moves 32 KB per 128-byte K step instead of the 48 KB of the
+// single-SM 128 x 256 tile, for the same MMA work.
+//
+//   D[m, n] = sum_k A[m, k] * B[n, k]    (B K-major: the forward)
+//   D[m, n] = sum_k A[m, k] * B[k, n]    (B MN-major: the dgrad)
+//
+// Roles per CTA (320 threads), as in gemm_kernel:
+//   warp 0      TMA producer: this CTA's A rows and B half into its own stage
+//               ring; the bytes of both CTAs complete on the even CTA's
+//               `full` barrier, whose one arrival (with the byte count of
+//               both) comes from the even CTA's producer;
+//   warp 1      TMEM (cta_group::2 allocation in both CTAs); in the even CTA
+//               one thread issues the pair's MMAs and commits each stage to
+//               the `empty` barriers of both CTAs, each finished tile to the
+//               `tfull` barriers of both;
+//   warps 2..9  epilogue on this CTA's 128 rows x 256 columns (the code of
+//               gemm_kernel), releasing the accumulator on the even CTA's
+//               `tempty` barrier (16 warps arrive per tile).
+// At the end the two CTAs hand over (bounded waits) before TMEM is freed:
+// the odd CTA's epilogue is done, the even CTA's MMAs have completed.
+// Every wait is bounded; no TMA multicast.
+#pragma once
+#include "gemm.cuh"
+
+namespace w8a8 {
+
+template <int KIND>
+struct PairCfg {
+  static constexpr int kBN = 256;                  // pair tile N (each CTA holds 128 of it)
+  static constexpr int kBK = kBKBytes;             // 128 codes per stage
+  static constexpr int kABytes = kBM * kBKBytes;   // 16 KB: this CTA's 128 rows of A
+  static constexpr int kBBytes = 128 * kBKBytes;   // 16 KB: this CTA's half of B
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = 6;
+  static constexpr int kTmemCols = 2 * kBN;        // two accumulators of 256 columns
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kOutBufBytes = 32 * 32 * 2;
+  static constexpr int kOutBytes = kEpiWarps * 2 * kOutBufBytes;
+  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * kStageBytes + kOutBytes + 256;
+  static_assert(kSmem <= 232448, "shared memory per block");
+};
+
+template <int KIND, bool B_MN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KIND>::kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmY, int M, int N, int Kc, EpiParams ep) {
+  using C = PairCfg<KIND>;
+  constexpr int BN = C::kBN;
+  constexpr uint32_t kIdesc = idesc<KIND>(2 * kBM, BN, B_MN);
+  constexpr int kStages = C::kStages;
+  constexpr int kGroups = C::kEpiWarps / 4;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;                                  // kStages x 16 KB
+  uint8_t* sB = smem + kStages * C::kABytes;           // kStages x 16 KB
+  uint8_t* sOut = smem + kStages * C::kStageBytes;     // epilogue staging
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + C::kOutBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* teardown = tempty + 2;
+  uint64_t* handover = teardown + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(handover + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();   // 0: issues the MMAs
+  const bool leader = rank == 0;
+  const uint64_t limit = g_wait_limit_ns;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * C::kEpiWarps);   // the epilogue warps of both CTAs
+    }
+    mbar_init(teardown, 1);
+    mbar_init(handover, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    if (ep.tma_store) tma_prefetch_desc(&tmY);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();   // both CTAs' barriers exist before either reaches the other's
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_launch();
+
+  const int tiles_m = (M + 2 * kBM - 1) / (2 * kBM);
+  const int tiles_n = (N + BN - 1) / BN;
+  const int num_tiles = tiles_m * tiles_n;
+  const int num_kb = (Kc + C::kBK - 1) / C::kBK;
+  const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, issued_phase = 0;
+      bool ok = true;
+      griddep_wait();
+      for (int tile = pair; ok && tile < num_tiles; tile += num_pairs) {
+        const int m0 = (tile % tiles_m) * (2 * kBM) + static_cast<int>(rank) * kBM;
+        const int nh = (tile / tiles_m) * BN + static_cast<int>(rank) * 128;   // this CTA's half of B
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, 0x100u | stage, limit)) { ok = false; break; }
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
+          const uint32_t fb = mapa_shared(&full[stage], 0);   // the even CTA's full[stage]
+          tma_load_2d_pair(sA + stage * C::kABytes, &tmA, fb, kb * C::kBK, m0);
+          if constexpr (!B_MN)
+            tma_load_2d_pair(sB + stage * C::kBBytes, &tmB, fb, kb * C::kBK, nh);
+          else
+            tma_load_2d_pair(sB + stage * C::kBBytes, &tmB, fb, nh, kb * C::kBK);
+          issued |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // Teardown (even CTA): every stage filled has completed.  The odd
+      // CTA's copies complete on the even CTA's barriers; the hand-over at
+      // the end keeps it resident until the MMAs have read them.
+      if (leader)
+        for (int s = 0; s < kStages; ++s)
+          if (issued & (1u << s)) mbar_wait(&full[s], (issued_phase >> s) & 1u, nullptr, 0x180u | s, limit);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (leader && lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < num_tiles; tile += num_pairs) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, 0x200u | acc, limit)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, 0x300u | stage, limit)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * C::kABytes);
+          const uint32_t b_base = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = sdesc_sw128(a_base + k * 32, 16, 1024);
+            const uint64_t bd = B_MN ? sdesc_sw128(b_base + k * (32 * 128), 16, 1024) : sdesc_sw128(b_base + k * 32, 16, 1024);
+            tc_mma_pair<KIND>(d, ad, bd, kIdesc, (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          tc_commit_pair_mc(&empty[stage], 0x3);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(&tfull[acc], 0x3);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      tc_commit_pair(teardown);
+      mbar_wait(teardown, 0, nullptr, 0x380u, limit);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    griddep_wait();
+    const int e = warp - 2;
+    const int quarter = warp & 3;
+    const int group = e >> 2;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    uint32_t out_iter = 0;
+    for (int tile = pair; tile < num_tiles; tile += num_pairs) {
+      const int m0 = (tile % tiles_m) * (2 * kBM) + static_cast<int>(rank) * kBM;
+      const int n0 = (tile / tiles_m) * BN;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[acc], acc_phase, abort_flag, 0x400u | acc, limit))) break;
+      tc_fence_after();
+      const int row = m0 + quarter * 32 + lane;
+      const float sx = row < M ? ep.s_row[row] : 0.0f;
+      const float sw0 = ep.s_col_axis ? 1.0f : ep.s_col[0];
+      epilogue_scale_chunks<KIND, kEpiScale, BN, kGroups, true>(ep, &tmY, tmem + lane_base + static_cast<uint32_t>(acc * BN),
+                                                                m0, n0, M, N, quarter, group, lane, sx, sw0,
+                                                                sOut + e * 2 * C::kOutBufBytes, out_iter);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(&tempty[acc], 0));   // the even CTA's barrier
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    if (ep.tma_store && lane == 0) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  // Hand-over: the odd CTA reports that its epilogue is done; the even CTA
+  // (whose MMAs have completed) answers; then both free the pair's TMEM.
+  if (warp == 1) {
+    if (lane == 0) {
+      if (!leader) {
+        mbar_arrive_cluster(mapa_shared(handover, 0));
+        mbar_wait(handover, 0, nullptr, 0x600u, limit);
+      } else {
+        mbar_wait(handover, 0, nullptr, 0x600u, limit);
+        mbar_arrive_cluster(mapa_shared(handover, 1));
+      }
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace w8a8

@@ -13,6 +13,7 @@
 #include "w8a8.h"
 #include "device.cuh"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "quantize.cuh"
 #include "q8_0.cuh"
 
@@ -176,6 +177,34 @@ w8a8_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t M,
                  static_cast<int>(N), static_cast<int>(Kc), ep);
   return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "gemm launch");
 }
+
+// The CTA-pair GEMM (256 x 256 tiles, clusters of two), persistent over
+// tile pairs.
+template <int KIND, bool B_MN>
+w8a8_status launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, int64_t M, int64_t N, int64_t Kc,
+                             EpiParams ep, cudaStream_t st) {
+  alignas(64) CUtensorMap ty;
+  w8a8_status ms = make_out_map(&ty, &ep, M, N);
+  if (ms != W8A8_OK) return ms;
+  using C = PairCfg<KIND>;
+  static std::atomic<uint64_t> smem_set{0};
+  int dev = 0, sms = 0;
+  w8a8_status s = current_device(&dev, &sms);
+  if (s != W8A8_OK) return s;
+  auto kern = gemm_pair_kernel<KIND, B_MN>;
+  cudaError_t e = set_smem_once(kern, C::kSmem, dev, smem_set);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm pair)");
+  const int64_t tiles = ((M + 2 * kBM - 1) / (2 * kBM)) * ((N + C::kBN - 1) / C::kBN);
+  const int64_t pairs = sms / 2;
+  const int grid = static_cast<int>(2 * (tiles < pairs ? tiles : pairs));
+  ep.splits = 1;
+  e = launch_pdl(kern, dim3(grid), dim3(C::kThreads), C::kSmem, st, ta, tb, ty, static_cast<int>(M),
+                 static_cast<int>(N), static_cast<int>(Kc), ep);
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "gemm pair launch");
+}
+
+// Products with at least this many rows (and no split) run on CTA pairs.
+constexpr int64_t kPairMinRows = 512;
 
 w8a8_status launch_quantize_rows(const void* x, int64_t ldx, int64_t M, int64_t K, int qt, void* q, int64_t ldq,
                                  float* s, cudaStream_t st) {
@@ -343,6 +372,12 @@ w8a8_status gemm_fwd(const void* xq, int64_t lda, const float* sx, int64_t M, in
     ep.splits = sk->splits;
     ep.partial = sk->partial;
   }
+  if (ep.splits == 1 && M >= kPairMinRows) {
+    // B in halves of 128 rows, one per CTA of the pair
+    if ((s = make_map(&tb, code_type(), 1, wq, K, N, K, kBKBytes, 128)) != W8A8_OK) return s;
+    return (qt == W8A8_E4M3) ? launch_gemm_pair<kKindE4M3, false>(ta, tb, M, N, K, ep, st)
+                             : launch_gemm_pair<kKindI8, false>(ta, tb, M, N, K, ep, st);
+  }
   s = (qt == W8A8_E4M3) ? launch_gemm<kKindE4M3, false, 256, kEpiScale>(ta, tb, M, N, K, ep, st)
                         : launch_gemm<kKindI8, false, 256, kEpiScale>(ta, tb, M, N, K, ep, st);
   if (s != W8A8_OK || ep.splits == 1) return s;
@@ -368,6 +403,9 @@ w8a8_status gemm_dgrad(const void* dyq, int64_t lda, const float* sdy, int64_t M
     ep.splits = sk->splits;
     ep.partial = sk->partial;
   }
+  if (ep.splits == 1 && M >= kPairMinRows)
+    return (qt == W8A8_E4M3) ? launch_gemm_pair<kKindE4M3, true>(ta, tb, M, K, N, ep, st)
+                             : launch_gemm_pair<kKindI8, true>(ta, tb, M, K, N, ep, st);
   s = (qt == W8A8_E4M3) ? launch_gemm<kKindE4M3, true, 256, kEpiScale>(ta, tb, M, K, N, ep, st)
                         : launch_gemm<kKindI8, true, 256, kEpiScale>(ta, tb, M, K, N, ep, st);
   if (s != W8A8_OK || ep.splits == 1) return s;
