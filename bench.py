@@ -41,14 +41,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic of one launch of the dominant kernel from an ncu capture, keyed
 # by the hash of the kernel source it was taken on (null when they differ).
-GEMM_TRAFFIC = {"source_sha": "54b23fe168e0b881", "bytes_per_launch": 124640256,
+GEMM_TRAFFIC = {"source_sha": "a2771761740e0d61", "bytes_per_launch": 123282688,
                 "note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one up-proj launch "
-                        "(bench.py --case up): 51.97 MB read + 72.67 MB written"}
+                        "(bench.py --case up): 52.02 MB read + 71.26 MB written"}
 
 
 def gemm_source_sha() -> str:
     h = hashlib.sha256()
-    for f in ("gemm.cuh", "device.cuh"):
+    for f in ("gemm_pair.cuh", "gemm.cuh", "device.cuh"):
         with open(os.path.join(ROOT, "w8a8_quantized_linear_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -419,7 +419,7 @@ def run_ours(args, rank, world, local_rank):
     achieved = OPS_PER_GEMM / (gemm_avg * 1e-3) / 1e12
     sha = gemm_source_sha()
     traffic = GEMM_TRAFFIC["bytes_per_launch"] if GEMM_TRAFFIC["source_sha"] == sha else None
-    roofline = {"bound": "tensor", "kernel": "gemm_kernel<i8> (tcgen05 kind::i8, fused epilogue)",
+    roofline = {"bound": "tensor", "kernel": "gemm_pair_kernel<i8> (tcgen05 cta_group::2 kind::i8, fused epilogue)",
                 "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s", "frac": achieved / int8_peak,
                 "traffic": traffic,
                 "peak_source": "%s: 2 x bf16_tflops (burst; int8 dense = 2x bf16 dense nominal)" % src,
