@@ -55,7 +55,10 @@ def test_sizes(L):
     assert L.w8a8_workspace_bytes(0, 4608, 12288, 3072, 0) == 4608 * 3072 + 4608 * 4
     assert L.w8a8_workspace_bytes(0, 3, 8, 16, 0) == 256 + 256
     assert L.w8a8_workspace_bytes(1, 3, 40, 16, 0) == 256 + 256  # N padded to 48 -> 144 bytes
-    assert L.w8a8_workspace_bytes(2, 4608, 3072, 3072, 32) == 4608 * 3072 + 4608 * 4 + 4608 * 32 * 2
+    # SVDQuant: codes, row scales, T [M, r] bf16, then T's split-K partial sums
+    # (36 row tiles over a 3072-long contraction: 4 splits, [4, 4608, 32] fp32)
+    assert L.w8a8_workspace_bytes(2, 4608, 3072, 3072, 32) == 4608 * 3072 + 4608 * 4 + 4608 * 32 * 2 + 4 * 4608 * 32 * 4
+    assert L.w8a8_workspace_bytes(2, 200, 320, 256, 32) == 200 * 256 + 1024 + 200 * 32 * 2   # unsplit
     assert L.w8a8_workspace_bytes(3, 10, 10, 16, 0) == 256
     # few output tiles, long contraction: split-K partial sums follow
     # (48 tiles -> 3 splits of 8 K blocks; [3, 1, 12288] int32)

@@ -383,11 +383,24 @@ def test_svdq_parity_small(w8, orc, r):
     _svdq_check(w8, orc, x, w, r, bias=bias)
 
 
-def test_svdq_zero_factors_equal_int_linear(w8):
-    x = workloads.normal((130, 256), 1.0, 61).to(DEV)
-    wq, sw = w8.quantize_weight(workloads.normal((300, 256), 0.02, 62).to(DEV), "int8", "tensor")
+@pytest.mark.parametrize("M,N,K,r", [(600, 520, 512, 8), (777, 264, 384, 24), (1024, 1024, 1024, 32),
+                                     (520, 136, 256, 16), (530, 300, 256, 16)])
+def test_svdq_parity_pairs(w8, orc, M, N, K, r):
+    """M >= 512 with N % 8 == 0 runs the CTA-pair kernel, whose low-rank sum
+    is a second tensor-core product (256 x 128 tiles, ragged edges, r padded
+    to the MMA's K steps); (530, 300) keeps the single-SM form."""
+    x = workloads.with_outlier_channels((M, K), 1.0, seed=M + r)
+    w = workloads.rank_spike_weight(N, K, 8, 0.5, 0.02, seed=N + K)
+    bias = workloads.normal((N,), 0.01, seed=N + 7)
+    _svdq_check(w8, orc, x, w, r, bias=bias)
+
+
+@pytest.mark.parametrize("M", [130, 600])
+def test_svdq_zero_factors_equal_int_linear(w8, M):
+    x = workloads.normal((M, 256), 1.0, 61).to(DEV)
+    wq, sw = w8.quantize_weight(workloads.normal((304, 256), 0.02, 62).to(DEV), "int8", "tensor")
     l1 = torch.zeros((256, 16), dtype=torch.bfloat16, device=DEV)
-    l2 = torch.zeros((16, 300), dtype=torch.bfloat16, device=DEV)
+    l2 = torch.zeros((16, 304), dtype=torch.bfloat16, device=DEV)
     assert torch.equal(w8.svdq_linear_fwd(x, wq, sw, l1, l2), w8.linear_fwd(x, wq, sw))
 
 

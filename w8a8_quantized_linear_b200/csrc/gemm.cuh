@@ -17,7 +17,7 @@
 //               the epilogue of tile i overlap the MMAs of tile i+1.
 // Tile 128 x BN x 128 bytes of K per stage.  Every wait is bounded.
 //
-// Split-K (scale epilogue only): with ep.splits = S > 1 the work units are
+// Split-K (scale and plain epilogues): with ep.splits = S > 1 the work units are
 // (tile, split) pairs, split s covering K blocks [s*nkb/S, (s+1)*nkb/S).  A
 // unit writes its raw sums (int32, or fp32 bits for e4m3) for the tile's
 // valid rows to ep.partial[s][m][n]; splitk_epilogue_kernel then adds the S
@@ -46,7 +46,7 @@ struct EpiParams {
   const __nv_bfloat16* lr_t;     // T [M, r]                          (kEpiLowRank)
   const __nv_bfloat16* lr_l2;    // L2 [r, N]
   int r;
-  int splits;                    // K splits per tile (>= 1; > 1 only with kEpiScale)
+  int splits;                    // K splits per tile (>= 1; > 1 not with kEpiLowRank)
   uint32_t* partial;             // [splits, M, N] raw sums (splits > 1)
 };
 
@@ -82,13 +82,15 @@ struct GemmCfg {
 // the warp reads the 32 TMEM lanes of its quarter (rows m0 + 32 quarter +
 // lane) for the 32-column chunks c = group, group + kGroups, ... at TMEM
 // address tacc; y = bf16(((acc * s_x) * s_w) + bias), each step an fp32 RN
-// operation; the warp's 32 x 32 bf16 block goes out through one of its two
-// swizzled staging buffers (sOutWarp) with a TMA store, or directly when the
-// row stride is not a multiple of 8.
-template <int KIND, int EPI, int BN, int kGroups, bool kAxisOk>
+// operation, and with LR one more RN add of the fp32 low-rank sum read at
+// TMEM address tlr; the warp's 32 x 32 bf16 block goes out through one of
+// its two swizzled staging buffers (sOutWarp) with a TMA store, or directly
+// when the row stride is not a multiple of 8.
+template <int KIND, int EPI, int BN, int kGroups, bool kAxisOk, bool LR = false>
 __device__ __forceinline__ void epilogue_scale_chunks(const EpiParams& ep, const CUtensorMap* tmY, uint32_t tacc, int m0,
                                                       int n0, int M, int N, int quarter, int group, int lane, float sx,
-                                                      float sw0, uint8_t* sOutWarp, uint32_t& out_iter) {
+                                                      float sw0, uint8_t* sOutWarp, uint32_t& out_iter,
+                                                      uint32_t tlr = 0) {
   const int row = m0 + quarter * 32 + lane;
   const bool row_ok = row < M;
   #pragma unroll 1
@@ -129,6 +131,8 @@ __device__ __forceinline__ void epilogue_scale_chunks(const EpiParams& ep, const
     }
     uint32_t r[32];
     tmem_ld_x32(tacc + static_cast<uint32_t>(c * 32), r);
+    uint32_t lr[LR ? 32 : 1];
+    if constexpr (LR) tmem_ld_x32(tlr + static_cast<uint32_t>(c * 32), lr);
     tmem_ld_wait();
     float v[32];
   #pragma unroll
@@ -138,6 +142,7 @@ __device__ __forceinline__ void epilogue_scale_chunks(const EpiParams& ep, const
         a = __fmul_rn(__fmul_rn(a, sx), (kAxisOk && ep.s_col_axis) ? sw[j] : sw0);
         if (ep.bias != nullptr) a = __fadd_rn(a, bs[j]);
       }
+      if constexpr (LR) a = __fadd_rn(a, __uint_as_float(lr[j]));
       v[j] = a;
     }
     if (ep.tma_store) {
@@ -248,7 +253,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
   const int num_tiles = tiles_m * tiles_n;
   const int num_kb = (Kc + C::kBK - 1) / C::kBK;
   // the host keeps 1 <= splits <= num_kb, so every unit has at least one K block
-  const int splits = (EPI == kEpiScale) ? ep.splits : 1;
+  const int splits = (EPI != kEpiLowRank) ? ep.splits : 1;
   const int num_units = num_tiles * splits;
 
   if (warp == 0) {
@@ -540,8 +545,9 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
 // Finish a split-K product:  y[m, n] = bf16( ((sum_s partial[s][m][n]) * s_x[m]) * s_w[n or 0] + bias[n] ),
 // the partial sums added in split order and every other step the fp32 RN
 // operation of the fused epilogue, so the result equals the unsplit one
-// (int8) or is reproducible (e4m3).  8 columns per thread: N % 8 == 0, y
-// contiguous [M, N].
+// (int8) or is reproducible (e4m3).  KIND = kKindBF16 is the plain form:
+// y = bf16(sum_s partial), fp32 sums in split order, no scales.  8 columns
+// per thread: N % 8 == 0, y contiguous [M, N].
 template <int KIND>
 __global__ void __launch_bounds__(256) splitk_epilogue_kernel(const uint32_t* __restrict__ partial, int splits,
                                                               int64_t M, int64_t N, const float* __restrict__ s_row,
@@ -567,6 +573,14 @@ __global__ void __launch_bounds__(256) splitk_epilogue_kernel(const uint32_t* __
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         r[j] = (KIND == kKindI8) ? r[j] + t[j] : __float_as_uint(__fadd_rn(__uint_as_float(r[j]), __uint_as_float(t[j])));
+    }
+    if constexpr (KIND == kKindBF16) {
+      *reinterpret_cast<uint4*>(y + m * N + n) =
+          make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                     pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                     pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                     pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
+      continue;
     }
     const float sx = s_row[m];
     float sw[8], bs[8];

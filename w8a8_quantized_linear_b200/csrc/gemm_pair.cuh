@@ -28,45 +28,64 @@
 
 namespace w8a8 {
 
-template <int KIND>
+// LR: the SVDQuant form.  TMEM holds one buffer of the int32 sums (256
+// columns) and the fp32 low-rank sums T L2 (256 columns), so the epilogue
+// of a tile does not overlap the next tile's MMAs; the stage ring is one
+// stage shorter to make room for the T and L2 tiles.  Per tile, after the
+// int8 MMAs, bf16 MMAs (r <= 32 in K steps of 16) multiply the tile's T
+// [128 rows x r per CTA] by its L2 [r x 128 columns per CTA], both brought
+// in by TMA once per tile (r padded to 64 columns and 32 rows by the TMA
+// zero fill).
+template <int KIND, bool LR>
 struct PairCfg {
-  static constexpr int kBN = 256;                  // pair tile N (each CTA holds 128 of it)
+  static constexpr int kBN = 256;                  // pair tile N (each CTA holds 128 rows or columns of B)
+  static constexpr int kBHalf = kBN / 2;
   static constexpr int kBK = kBKBytes;             // 128 codes per stage
   static constexpr int kABytes = kBM * kBKBytes;   // 16 KB: this CTA's 128 rows of A
-  static constexpr int kBBytes = 128 * kBKBytes;   // 16 KB: this CTA's half of B
+  static constexpr int kBBytes = kBHalf * kBKBytes;   // 16 KB: this CTA's half of B
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = 6;
-  static constexpr int kTmemCols = 2 * kBN;        // two accumulators of 256 columns
+  static constexpr int kStages = LR ? 5 : 6;
+  static constexpr int kAccBufs = LR ? 1 : 2;      // TMEM buffers of 256 columns (+ 256 low-rank with LR)
+  static constexpr int kTmemCols = 512;
+  static constexpr int kTBytes = LR ? kBM * 128 : 0;       // T tile: 128 rows x 64 bf16 (r zero-padded)
+  static constexpr int kL2Bytes = LR ? 2 * 32 * 128 : 0;   // L2 tile: 32 rows x 128 bf16 (two 64-column boxes)
   static constexpr int kEpiWarps = 8;
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kOutBufBytes = 32 * 32 * 2;
   static constexpr int kOutBytes = kEpiWarps * 2 * kOutBufBytes;
-  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * kStageBytes + kOutBytes + 256;
+  static constexpr size_t kSmem =
+      1024 + static_cast<size_t>(kStages) * kStageBytes + kTBytes + kL2Bytes + kOutBytes + 256;
   static_assert(kSmem <= 232448, "shared memory per block");
 };
 
-template <int KIND, bool B_MN>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KIND>::kThreads, 1)
+template <int KIND, bool B_MN, bool LR = false>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KIND, LR>::kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmY, int M, int N, int Kc, EpiParams ep) {
-  using C = PairCfg<KIND>;
+                     const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmT,
+                     const __grid_constant__ CUtensorMap tmL2, int M, int N, int Kc, EpiParams ep) {
+  using C = PairCfg<KIND, LR>;
   constexpr int BN = C::kBN;
   constexpr uint32_t kIdesc = idesc<KIND>(2 * kBM, BN, B_MN);
+  constexpr uint32_t kIdescLr = idesc<kKindBF16>(2 * kBM, BN, true);   // T K-major, L2 MN-major
   constexpr int kStages = C::kStages;
   constexpr int kGroups = C::kEpiWarps / 4;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;                                  // kStages x 16 KB
-  uint8_t* sB = smem + kStages * C::kABytes;           // kStages x 16 KB
-  uint8_t* sOut = smem + kStages * C::kStageBytes;     // epilogue staging
+  uint8_t* sB = smem + kStages * C::kABytes;           // kStages x kBBytes
+  uint8_t* sT = smem + kStages * C::kStageBytes;       // LR: 16 KB
+  uint8_t* sL2 = sT + C::kTBytes;                      // LR: 8 KB
+  uint8_t* sOut = sL2 + C::kL2Bytes;                   // epilogue staging
   uint64_t* full = reinterpret_cast<uint64_t*>(sOut + C::kOutBytes);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* teardown = tempty + 2;
   uint64_t* handover = teardown + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(handover + 1);
+  uint64_t* lrfull = handover + 1;                     // LR: T and L2 tiles landed (even CTA's)
+  uint64_t* lrempty = lrfull + 1;                      // LR: the low-rank MMAs read them
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lrempty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -85,11 +104,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KIND>::kThre
     }
     mbar_init(teardown, 1);
     mbar_init(handover, 1);
+    mbar_init(lrfull, 1);
+    mbar_init(lrempty, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     if (ep.tma_store) tma_prefetch_desc(&tmY);
+    if constexpr (LR) {
+      tma_prefetch_desc(&tmT);
+      tma_prefetch_desc(&tmL2);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, C::kTmemCols);
@@ -113,11 +138,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KIND>::kThre
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0, issued_phase = 0;
+      uint32_t lr_phase = 0;
+      bool lr_issued = false;
       bool ok = true;
       griddep_wait();
       for (int tile = pair; ok && tile < num_tiles; tile += num_pairs) {
         const int m0 = (tile % tiles_m) * (2 * kBM) + static_cast<int>(rank) * kBM;
-        const int nh = (tile / tiles_m) * BN + static_cast<int>(rank) * 128;   // this CTA's half of B
+        const int nh = (tile / tiles_m) * BN + static_cast<int>(rank) * C::kBHalf;   // this CTA's half of B
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, 0x100u | stage, limit)) { ok = false; break; }
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
@@ -131,24 +158,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KIND>::kThre
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
+        if constexpr (LR) {
+          // This tile's T rows and L2 columns, once the previous tile's
+          // low-rank MMAs have read the buffers (long done by now: they ran
+          // before this tile's first MMA).
+          if (ok && !mbar_wait(lrempty, lr_phase ^ 1u, abort_flag, 0x700u, limit)) ok = false;
+          if (ok) {
+            if (leader) mbar_arrive_expect_tx(lrfull, 2 * (C::kTBytes + C::kL2Bytes));
+            const uint32_t lb = mapa_shared(lrfull, 0);
+            tma_load_2d_pair(sT, &tmT, lb, 0, m0);
+            tma_load_2d_pair(sL2, &tmL2, lb, nh, 0);
+            tma_load_2d_pair(sL2 + 32 * 128, &tmL2, lb, nh + 64, 0);
+            lr_issued = true;
+            lr_phase ^= 1u;
+          }
+        }
       }
       // Teardown (even CTA): every stage filled has completed.  The odd
       // CTA's copies complete on the even CTA's barriers; the hand-over at
       // the end keeps it resident until the MMAs have read them.
-      if (leader)
+      if (leader) {
         for (int s = 0; s < kStages; ++s)
           if (issued & (1u << s)) mbar_wait(&full[s], (issued_phase >> s) & 1u, nullptr, 0x180u | s, limit);
+        if (LR && lr_issued) mbar_wait(lrfull, lr_phase ^ 1u, nullptr, 0x780u, limit);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (leader && lane == 0) {
       int stage = 0, acc = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      uint32_t phase = 0, acc_phase = 0, lr_phase = 0;
       bool ok = true;
       for (int tile = pair; ok && tile < num_tiles; tile += num_pairs) {
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, 0x200u | acc, limit)) break;
         tc_fence_after();
-        const uint32_t d = tmem + static_cast<uint32_t>(acc * BN);
+        const uint32_t d = tmem + static_cast<uint32_t>(acc * 256);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, 0x300u | stage, limit)) { ok = false; break; }
           tc_fence_after();
@@ -164,8 +208,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KIND>::kThre
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
+        if constexpr (LR) {
+          // T L2 into the buffer's second 128 columns, from zero, fp32
+          if (!mbar_wait(lrfull, lr_phase, abort_flag, 0x800u, limit)) break;
+          tc_fence_after();
+          const uint32_t t_base = smem_u32(sT), l_base = smem_u32(sL2);
+          const int nks = (ep.r + 15) / 16;
+          for (int k = 0; k < nks; ++k)
+            tc_mma_pair<kKindBF16>(d + BN, sdesc_sw128(t_base + k * 32, 16, 1024),
+                                   sdesc_sw128(l_base + k * (16 * 128), 32 * 128, 1024), kIdescLr, k > 0 ? 1u : 0u);
+          tc_commit_pair_mc(lrempty, 0x3);
+          lr_phase ^= 1u;
+        }
         tc_commit_pair_mc(&tfull[acc], 0x3);
-        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        if (++acc == C::kAccBufs) { acc = 0; acc_phase ^= 1u; }
       }
       tc_commit_pair(teardown);
       mbar_wait(teardown, 0, nullptr, 0x380u, limit);
@@ -188,13 +244,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KIND>::kThre
       const int row = m0 + quarter * 32 + lane;
       const float sx = row < M ? ep.s_row[row] : 0.0f;
       const float sw0 = ep.s_col_axis ? 1.0f : ep.s_col[0];
-      epilogue_scale_chunks<KIND, kEpiScale, BN, kGroups, true>(ep, &tmY, tmem + lane_base + static_cast<uint32_t>(acc * BN),
-                                                                m0, n0, M, N, quarter, group, lane, sx, sw0,
-                                                                sOut + e * 2 * C::kOutBufBytes, out_iter);
+      const uint32_t tacc = tmem + lane_base + static_cast<uint32_t>(acc * 256);
+      epilogue_scale_chunks<KIND, kEpiScale, BN, kGroups, !LR, LR>(ep, &tmY, tacc, m0, n0, M, N, quarter, group, lane,
+                                                                    sx, sw0, sOut + e * 2 * C::kOutBufBytes, out_iter,
+                                                                    tacc + BN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(&tempty[acc], 0));   // the even CTA's barrier
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if (++acc == C::kAccBufs) { acc = 0; acc_phase ^= 1u; }
     }
     if (ep.tma_store && lane == 0) bulk_wait_all();
   }

@@ -178,28 +178,31 @@ w8a8_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t M,
   return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "gemm launch");
 }
 
-// The CTA-pair GEMM (256 x 256 tiles, clusters of two), persistent over
-// tile pairs.
-template <int KIND, bool B_MN>
+// The CTA-pair GEMM (256-row tiles, clusters of two), persistent over tile
+// pairs.  tt / tl2: the T and L2 maps of the low-rank form (LR), unused
+// otherwise.
+template <int KIND, bool B_MN, bool LR = false>
 w8a8_status launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, int64_t M, int64_t N, int64_t Kc,
-                             EpiParams ep, cudaStream_t st) {
-  alignas(64) CUtensorMap ty;
+                             EpiParams ep, cudaStream_t st, const CUtensorMap* tt = nullptr,
+                             const CUtensorMap* tl2 = nullptr) {
+  alignas(64) CUtensorMap ty, tz;
   w8a8_status ms = make_out_map(&ty, &ep, M, N);
   if (ms != W8A8_OK) return ms;
-  using C = PairCfg<KIND>;
+  std::memset(&tz, 0, sizeof(tz));
+  using C = PairCfg<KIND, LR>;
   static std::atomic<uint64_t> smem_set{0};
   int dev = 0, sms = 0;
   w8a8_status s = current_device(&dev, &sms);
   if (s != W8A8_OK) return s;
-  auto kern = gemm_pair_kernel<KIND, B_MN>;
+  auto kern = gemm_pair_kernel<KIND, B_MN, LR>;
   cudaError_t e = set_smem_once(kern, C::kSmem, dev, smem_set);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm pair)");
   const int64_t tiles = ((M + 2 * kBM - 1) / (2 * kBM)) * ((N + C::kBN - 1) / C::kBN);
   const int64_t pairs = sms / 2;
   const int grid = static_cast<int>(2 * (tiles < pairs ? tiles : pairs));
   ep.splits = 1;
-  e = launch_pdl(kern, dim3(grid), dim3(C::kThreads), C::kSmem, st, ta, tb, ty, static_cast<int>(M),
-                 static_cast<int>(N), static_cast<int>(Kc), ep);
+  e = launch_pdl(kern, dim3(grid), dim3(C::kThreads), C::kSmem, st, ta, tb, ty, LR ? *tt : tz, LR ? *tl2 : tz,
+                 static_cast<int>(M), static_cast<int>(N), static_cast<int>(Kc), ep);
   return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "gemm pair launch");
 }
 
@@ -337,11 +340,27 @@ w8a8_status launch_splitk_epilogue(int qt, const SplitWs& sk, int64_t M, int64_t
   return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "split-K epilogue launch");
 }
 
+// Split count of the SVDQuant low-rank input T = X L1 (a bf16 product with
+// r <= 32 columns: one output tile per 128 rows), as choose_splits with
+// 64-element K blocks.
+int t_splits(int64_t M, int64_t K) {
+  const int64_t tiles = (M + kBM - 1) / kBM;
+  const int64_t num_kb = (K + 63) / 64;
+  if (tiles * 2 > kSplitSms) return 1;
+  int64_t s = kSplitSms / tiles;
+  if (s > num_kb / 4) s = num_kb / 4;
+  if (s > 16) s = 16;
+  return s < 2 ? 1 : static_cast<int>(s);
+}
+// Workspace of svdq_linear_fwd: codes [M, K], row scales [M], T [M, r]
+// bf16, then T's split-K partial sums [S, M, r] fp32 when split.
 size_t ws_svdq(int64_t M, int64_t K, int r) {
   Carve c(nullptr);
   c.take(static_cast<size_t>(M * K));
   c.take(static_cast<size_t>(M) * 4);
   c.take(static_cast<size_t>(M) * r * 2);
+  const int s = t_splits(M, K);
+  if (s > 1) c.take(static_cast<size_t>(s) * static_cast<size_t>(M) * static_cast<size_t>(r) * 4);
   return c.off;
 }
 
@@ -742,8 +761,17 @@ w8a8_status svdq_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, cons
   void* xq = c.take(static_cast<size_t>(M * K));
   float* sx = static_cast<float*>(c.take(static_cast<size_t>(M) * 4));
   auto* t = static_cast<__nv_bfloat16*>(c.take(static_cast<size_t>(M) * r * 2));
+  const int tsplit = t_splits(M, K);
+  SplitWs tsk;
+  if (tsplit > 1) {
+    tsk.splits = tsplit;
+    tsk.partial = static_cast<uint32_t*>(
+        c.take(static_cast<size_t>(tsplit) * static_cast<size_t>(M) * static_cast<size_t>(r) * 4));
+  }
   if ((st = launch_quantize_rows(x, K, M, K, W8A8_INT8, xq, K, sx, s)) != W8A8_OK) return st;
-  // T = bf16(X L1): bf16 tensor-core GEMM, L1 [K, r] read MN-major.
+  // T = bf16(X L1): bf16 tensor-core GEMM, L1 [K, r] read MN-major; split
+  // along K when the rows make few tiles (fp32 partial sums, added in split
+  // order, then one bf16 rounding).
   {
     alignas(64) CUtensorMap ta, tb;
     if ((st = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, K, M, K * 2, 64, kBM)) != W8A8_OK) return st;
@@ -753,11 +781,26 @@ w8a8_status svdq_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, cons
     EpiParams ep{};
     ep.y = t;
     ep.ldy = r;
+    ep.splits = tsk.splits;
+    ep.partial = tsk.partial;
     if ((st = launch_gemm<kKindBF16, true, 64, kEpiPlain>(ta, tb, M, r, K, ep, s)) != W8A8_OK) return st;
+    if (tsk.splits > 1) {
+      int sms = 0;
+      if ((st = current_device(nullptr, &sms)) != W8A8_OK) return st;
+      int64_t grid = (M * (r / 8) + 255) / 256;
+      if (grid > 8 * static_cast<int64_t>(sms)) grid = 8 * static_cast<int64_t>(sms);
+      const uint32_t* part = tsk.partial;
+      const cudaError_t e = launch_pdl(splitk_epilogue_kernel<kKindBF16>, dim3(static_cast<unsigned>(grid)), dim3(256), 0,
+                                       s, part, tsk.splits, M, static_cast<int64_t>(r), static_cast<const float*>(nullptr),
+                                       static_cast<const float*>(nullptr), 0, static_cast<const __nv_bfloat16*>(nullptr),
+                                       t);
+      if (e != cudaSuccess) return cuda_fail(e, "split-K epilogue launch");
+    }
   }
   alignas(64) CUtensorMap ta, tb;
   if ((st = make_map(&ta, code_type(), 1, xq, K, M, K, kBKBytes, kBM)) != W8A8_OK) return st;
-  if ((st = make_map(&tb, code_type(), 1, rq, K, N, K, kBKBytes, 256)) != W8A8_OK) return st;
+  const bool pair = M >= kPairMinRows && (N % 8) == 0;   // L2 rows must be 16-byte multiples for its tensor map
+  if ((st = make_map(&tb, code_type(), 1, rq, K, N, K, kBKBytes, pair ? 128 : 256)) != W8A8_OK) return st;
   EpiParams ep{};
   ep.s_row = sx;
   ep.s_col = r_scale;
@@ -768,6 +811,16 @@ w8a8_status svdq_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, cons
   ep.lr_t = t;
   ep.lr_l2 = static_cast<const __nv_bfloat16*>(l2);
   ep.r = r;
+  if (pair) {
+    // T [M, r] and L2 [r, N] tiles for the tensor-core low-rank product:
+    // 64 bf16 (128 bytes) wide, r zero-padded by the copy
+    alignas(64) CUtensorMap tt, tl2;
+    if ((st = make_map(&tt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, t, r, M, static_cast<int64_t>(r) * 2, 64, kBM)) !=
+        W8A8_OK)
+      return st;
+    if ((st = make_map(&tl2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, l2, N, r, N * 2, 64, 32)) != W8A8_OK) return st;
+    return launch_gemm_pair<kKindI8, false, true>(ta, tb, M, N, K, ep, s, &tt, &tl2);
+  }
   return launch_gemm<kKindI8, false, 256, kEpiLowRank>(ta, tb, M, N, K, ep, s);
 }
 
