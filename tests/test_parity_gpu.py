@@ -295,6 +295,25 @@ def test_linear_fwd_m0_noop(w8):
     assert w8.linear_fwd(x, wq, sw).shape == (0, 32)
 
 
+@pytest.mark.parametrize("M,N,K", [(1, 7, 16), (2, 300, 48), (5, 1000, 3072), (8, 513, 16384), (3, 64, 16400)])
+@pytest.mark.parametrize("gran", ["tensor", "axis"])
+def test_linear_fwd_few_tokens(w8, orc, M, N, K, gran):
+    """M <= 8 int8 forwards run as one weight-streaming launch (dp4a on the
+    CUDA cores, the rows quantized inside it; K <= 16384, else the GEMM):
+    bit-exact with the oracle and with the tensor-core product on the same
+    codes."""
+    x = workloads.with_outlier_channels((M, K), 1.0, seed=M * 31 + K)
+    w = workloads.normal((N, K), 0.02, seed=N + 17)
+    bias = workloads.normal((N,), 0.01, seed=N + 18)
+    wq, sw = w8.quantize_weight(w.to(DEV), "int8", gran)
+    y = w8.linear_fwd(x.to(DEV), wq, sw, bias=bias.to(DEV))
+    wqr, swr = orc.quantize_weight(workloads.to_u16(w), 0, 1 if gran == "axis" else 0)
+    ref = orc.linear_fwd(workloads.to_u16(x), wqr, swr, bias=workloads.to_u16(bias))
+    assert np.array_equal(u16(y), ref["y"])
+    xq, sx = w8.quantize_rows(x.to(DEV), "int8")
+    assert torch.equal(y, w8.qgemm_fwd(xq, sx, wq, sw, bias=bias.to(DEV)))
+
+
 def test_linear_fwd_split_equals_unsplit(w8):
     """A forward with few output tiles and a long K (split-K for int8) equals
     the GEMM on the same codes without splitting (qgemm_fwd never splits), bit

@@ -16,6 +16,7 @@
 #include "gemm_pair.cuh"
 #include "quantize.cuh"
 #include "q8_0.cuh"
+#include "gemv.cuh"
 
 namespace w8a8 {
 namespace {
@@ -204,6 +205,41 @@ w8a8_status launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, int64
   e = launch_pdl(kern, dim3(grid), dim3(C::kThreads), C::kSmem, st, ta, tb, ty, LR ? *tt : tz, LR ? *tl2 : tz,
                  static_cast<int>(M), static_cast<int>(N), static_cast<int>(Kc), ep);
   return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "gemm pair launch");
+}
+
+// The few-token int8 forward in one launch (gemv.cuh): M <= kGemvMaxRows,
+// K <= kGemvMaxK; each block quantizes the M rows itself.
+w8a8_status launch_gemv(const void* x, int64_t M, int64_t N, int64_t K, const void* wq, const float* sw, int axis,
+                        const void* bias, void* y, cudaStream_t st) {
+  int dev = 0, sms = 0;
+  w8a8_status s = current_device(&dev, &sms);
+  if (s != W8A8_OK) return s;
+  static std::atomic<uint64_t> smem_set[kGemvMaxRows] = {};
+  const size_t smem = static_cast<size_t>(M * K);
+  // up to 4 blocks per SM (as shared memory allows) keep the weight stream's
+  // loads in flight
+  int64_t per_sm = static_cast<int64_t>(200 * 1024) / static_cast<int64_t>(smem + 1024);
+  per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
+  int64_t grid = (N + kGemvThreads / 32 - 1) / (kGemvThreads / 32);
+  if (grid > per_sm * sms) grid = per_sm * sms;
+  const auto* xp = static_cast<const __nv_bfloat16*>(x);
+  const auto* wp = static_cast<const int8_t*>(wq);
+  const auto* bp = static_cast<const __nv_bfloat16*>(bias);
+  auto* yp = static_cast<__nv_bfloat16*>(y);
+  cudaError_t e = cudaSuccess;
+#define W8A8_GEMV(MM)                                                                                            \
+  case MM:                                                                                                       \
+    e = set_smem_once(gemv_int8_kernel<MM>, static_cast<size_t>(MM) * kGemvMaxK, dev, smem_set[MM - 1]);         \
+    if (e == cudaSuccess)                                                                                        \
+      e = launch_pdl(gemv_int8_kernel<MM>, dim3(static_cast<unsigned>(grid)), dim3(kGemvThreads), smem, st, xp, K, \
+                     static_cast<int>(N), static_cast<int>(K), wp, sw, axis, bp, yp);                            \
+    break;
+  switch (M) {
+    W8A8_GEMV(1) W8A8_GEMV(2) W8A8_GEMV(3) W8A8_GEMV(4) W8A8_GEMV(5) W8A8_GEMV(6) W8A8_GEMV(7) W8A8_GEMV(8)
+    default: return fail(W8A8_ERR_UNSUPPORTED_SHAPE, "gemv rows");
+  }
+#undef W8A8_GEMV
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "gemv launch");
 }
 
 // Products with at least this many rows (and no split) run on CTA pairs.
@@ -678,6 +714,8 @@ w8a8_status w8a8_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, w8a8
   W8A8_CHECK(aligned16(ws), W8A8_ERR_MISALIGNED, "workspace must be 16-byte aligned");
   if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (qt == W8A8_INT8 && M <= kGemvMaxRows && K <= kGemvMaxK)   // a few tokens: one weight-streaming launch
+    return launch_gemv(x, M, N, K, wq, sw, g == W8A8_AXIS, bias, y, s);
   Carve c(ws);
   void* xq = c.take(static_cast<size_t>(M * K));
   float* sx = static_cast<float*>(c.take(static_cast<size_t>(M) * 4));
