@@ -229,7 +229,8 @@ __global__ void __launch_bounds__(32 * kRequantMaxWarps) q8_0_to_axis_int8_kerne
 // (K % 256 == 0): a team of TW warps per row, thread t of the team taking
 // blocks t, t + 32 TW, ...  Each team keeps its next S - 1 rows in flight
 // into a ring of S shared-memory row buffers (cp.async) while it processes
-// the current one.
+// the current one; with S = 1 a row is loaded just before its turn and the
+// other teams on the SM (up to 8 blocks) hide the latency.
 //
 // A block b starts at byte 34 b of the row, i.e. on a word boundary when b is
 // even and 2 bytes past one when b is odd; its 34 bytes lie in the 9 words

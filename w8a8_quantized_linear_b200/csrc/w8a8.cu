@@ -621,22 +621,23 @@ w8a8_status q8_0_to_axis_int8(const void* blocks, int64_t N, int64_t K, int8_t* 
   const int64_t nblk = K / 32;
   if (K % 256 == 0) {
     // rows of whole 16-byte units: a team of TW warps per row (at least 3
-    // blocks per thread), double-buffered rows
+    // blocks per thread), one row buffer per team and up to 8 blocks per SM
+    // (more warps in flight beat a deeper prefetch ring here)
     int tw = 1;
     while (tw < 8 && tw * 2 * 96 <= nblk) tw *= 2;
-    const size_t smem = static_cast<size_t>(2 * (8 / tw)) * static_cast<size_t>(nblk * 34);
+    const size_t smem = static_cast<size_t>(8 / tw) * static_cast<size_t>(nblk * 34);
     if (smem <= 200 * 1024) {
       int per_sm = static_cast<int>((220 * 1024) / (smem + 1024));
-      per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
+      per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
       int64_t grid = (N + (8 / tw) - 1) / (8 / tw);
       if (grid > static_cast<int64_t>(per_sm) * sms) grid = static_cast<int64_t>(per_sm) * sms;
       static std::atomic<uint64_t> team_smem_set[4] = {};
       cudaError_t e = cudaSuccess;
       const auto* bp = static_cast<const uint8_t*>(blocks);
 #define W8A8_RQ_TEAM(TW, IDX)                                                                              \
-  e = set_smem_once(q8_0_to_axis_int8_team_kernel<TW, 2>, 200 * 1024, dev, team_smem_set[IDX]);            \
+  e = set_smem_once(q8_0_to_axis_int8_team_kernel<TW, 1>, 200 * 1024, dev, team_smem_set[IDX]);            \
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(requant)");                             \
-  q8_0_to_axis_int8_team_kernel<TW, 2><<<static_cast<int>(grid), kRqThreads, smem, cs>>>(bp, N, K, q, scale)
+  q8_0_to_axis_int8_team_kernel<TW, 1><<<static_cast<int>(grid), kRqThreads, smem, cs>>>(bp, N, K, q, scale)
       switch (tw) {
         case 1: W8A8_RQ_TEAM(1, 0); break;
         case 2: W8A8_RQ_TEAM(2, 1); break;
