@@ -395,4 +395,75 @@ __global__ void __launch_bounds__(kRqThreads) q8_0_to_axis_int8_team_kernel(cons
   cp_async_wait<0>();
 }
 
+// The same computation for rows of at most HOLD * 32 * TW blocks: pass 1
+// keeps each thread's blocks (9 words each) in registers, so the row buffer
+// is free as soon as pass 1 has read it - the next row's copy is issued then
+// and overlaps the arithmetic of pass 2, which needs no shared memory.
+template <int TW, int HOLD, int MINB = 1>
+__global__ void __launch_bounds__(kRqThreads, MINB) q8_0_to_axis_int8_hold_kernel(const uint8_t* __restrict__ blocks,
+                                                                           int64_t N, int64_t K,
+                                                                           int8_t* __restrict__ q,
+                                                                           float* __restrict__ scale) {
+  extern __shared__ __align__(16) uint8_t rq_smem[];
+  __shared__ float red[2][8];
+  constexpr int T = 32 * TW;
+  constexpr int kTeams = kRqThreads / T;
+  const int team = threadIdx.x / T, t = threadIdx.x % T;
+  const int nblk = static_cast<int>(K >> 5);
+  const int row_bytes = nblk * kQ80Bytes;   // a multiple of 16
+  const int nvec = row_bytes >> 4;
+  uint8_t* const buf = rq_smem + team * row_bytes;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * kTeams;
+  int64_t n = blockIdx.x * static_cast<int64_t>(kTeams) + team;
+  auto fetch = [&](int64_t row) {
+    if (row < N) {
+      const uint8_t* src = blocks + row * row_bytes;
+      for (int i = t; i < nvec; i += T) cp_async16(buf + 16 * i, src + 16 * i);
+    }
+    cp_async_commit();
+  };
+  fetch(n);
+  for (int it = 0; n < N; n += stride, ++it) {
+    cp_async_wait<0>();
+    team_sync<TW>(team);   // the row has landed
+    uint32_t w[HOLD][9];
+    float a = 0.0f;
+#pragma unroll
+    for (int h = 0; h < HOLD; ++h) {
+      const int b = t + h * T;
+      if (b < nblk) {
+        rq_block_words(buf, b, w[h]);
+        const bool odd = b & 1;
+        a = fmaxf(a, __fmul_rn(fabsf(rq_block_scale(w[h], odd)), static_cast<float>(rq_block_maxabs(w[h], odd))));
+      }
+    }
+    team_sync<TW>(team);   // every thread has its words: refill the buffer
+    fetch(n + stride);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+    if constexpr (TW > 1) {
+      if ((t & 31) == 0) red[it & 1][threadIdx.x >> 5] = a;
+      team_sync<TW>(team);
+#pragma unroll
+      for (int i = 0; i < TW; ++i) a = fmaxf(a, red[it & 1][team * TW + i]);
+    }
+    const float s = (a < 1e-10f) ? 1e-10f : __fdiv_rn(a, 127.0f);
+    const float rcp = __frcp_rn(s);
+    if (t == 0) scale[n] = s;
+#pragma unroll
+    for (int h = 0; h < HOLD; ++h) {
+      const int b = t + h * T;
+      if (b < nblk) {
+        const bool odd = b & 1;
+        uint32_t o[8];
+        rq_block_codes(w[h], odd, rq_block_scale(w[h], odd), s, rcp, o);
+        uint4* dst = reinterpret_cast<uint4*>(q + n * K + 32 * static_cast<int64_t>(b));
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+      }
+    }
+  }
+  cp_async_wait<0>();
+}
+
 }  // namespace w8a8

@@ -619,6 +619,32 @@ w8a8_status q8_0_to_axis_int8(const void* blocks, int64_t N, int64_t K, int8_t* 
   if (st != W8A8_OK) return st;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const int64_t nblk = K / 32;
+  if (K % 256 == 0 && nblk <= 8 * 96) {
+    // rows of whole 16-byte units and at most 3 blocks per thread of a team
+    // of TW warps: blocks held in registers between the two passes, one row
+    // per team
+    int tw = 1;
+    while (tw * 96 < nblk) tw *= 2;
+    const size_t smem = static_cast<size_t>(8 / tw) * static_cast<size_t>(nblk * 34);
+    int64_t grid = (N + (8 / tw) - 1) / (8 / tw);
+    if (grid > 16 * static_cast<int64_t>(sms)) grid = 16 * static_cast<int64_t>(sms);
+    static std::atomic<uint64_t> hold_smem_set[4] = {};
+    cudaError_t e = cudaSuccess;
+    const auto* bp = static_cast<const uint8_t*>(blocks);
+#define W8A8_RQ_HOLD(TW, IDX)                                                                              \
+  e = set_smem_once(q8_0_to_axis_int8_hold_kernel<TW, 3, 4>, 64 * 1024, dev, hold_smem_set[IDX]);          \
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(requant)");                             \
+  q8_0_to_axis_int8_hold_kernel<TW, 3, 4><<<static_cast<int>(grid), kRqThreads, smem, cs>>>(bp, N, K, q, scale)
+    switch (tw) {
+      case 1: W8A8_RQ_HOLD(1, 0); break;
+      case 2: W8A8_RQ_HOLD(2, 1); break;
+      case 4: W8A8_RQ_HOLD(4, 2); break;
+      default: W8A8_RQ_HOLD(8, 3); break;
+    }
+#undef W8A8_RQ_HOLD
+    e = cudaGetLastError();
+    return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "q8_0_to_axis_int8 launch");
+  }
   if (K % 256 == 0) {
     // rows of whole 16-byte units: a team of TW warps per row (at least 3
     // blocks per thread), one row buffer per team and up to 8 blocks per SM
