@@ -41,9 +41,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic of one launch of the dominant kernel from an ncu capture, keyed
 # by the hash of the kernel source it was taken on (null when they differ).
-GEMM_TRAFFIC = {"source_sha": "a2771761740e0d61", "bytes_per_launch": 123282688,
+GEMM_TRAFFIC = {"source_sha": "8f7b3f8153ef2a77", "bytes_per_launch": 124070400,
                 "note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one up-proj launch "
-                        "(bench.py --case up): 52.02 MB read + 71.26 MB written"}
+                        "(bench.py --case up): 52.00 MB read + 72.07 MB written"}
 
 
 def gemm_source_sha() -> str:
@@ -351,9 +351,12 @@ def run_ours(args, rank, world, local_rank):
     assert w8.device_status() == 0, "device-side error during the timed steps"
 
     # ---- end to end: pinned host inputs -> public API -> pinned host results.
-    # Three streams: the host->device copies of step i+1 and the device->host
-    # copies of step i-1 overlap the compute of step i (double-buffered device
-    # inputs and outputs); every step copies its inputs in and its results out.
+    # Three streams, double-buffered device inputs and outputs: the copies of
+    # step i + 1's inputs and of step i - 1's results overlap step i's
+    # compute.  Dependencies are per tensor: the forward waits only for X,
+    # the input gradient only for dY; Y2 leaves as soon as the forward is
+    # done; an input buffer is refilled once its one reader has finished.
+    # Every step copies all of its inputs in and all of its results out.
     e2e = None
     if args.e2e_steps > 0:
         hx = wl["x"].pin_memory()
@@ -367,36 +370,54 @@ def run_ours(args, rank, world, local_rank):
         dX1d = [torch.empty_like(dX1) for _ in range(2)]
         s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
         ev = lambda: torch.cuda.Event()
-        in_done, cmp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        x_in, dy_in = [ev(), ev()], [ev(), ev()]             # inputs landed
+        x_read, dy_read = [ev(), ev()], [ev(), ev()]         # inputs consumed
+        y2_done, dx1_done = [ev(), ev()], [ev(), ev()]       # results computed
+        y2_out, dx1_out = [ev(), ev()], [ev(), ev()]         # results copied out
 
-        def e2e_steps(n):
+        def e2e_steps(n, first):
             for i in range(n):
                 b = i & 1
+                reuse = not (first and i < 2)                 # buffer b was used two steps ago
                 with torch.cuda.stream(s_in):
-                    s_in.wait_event(cmp_done[b])            # step i-2 finished reading this input buffer
+                    if reuse:
+                        s_in.wait_event(x_read[b])
                     Xd[b].copy_(hx, non_blocking=True)
+                    x_in[b].record(s_in)
+                    if reuse:
+                        s_in.wait_event(dy_read[b])
                     dYd[b].copy_(hdy, non_blocking=True)
-                    in_done[b].record(s_in)
+                    dy_in[b].record(s_in)
                 with torch.cuda.stream(s_cmp):
-                    s_cmp.wait_event(in_done[b])
-                    s_cmp.wait_event(out_done[b])           # step i-2's results have left this buffer
+                    s_cmp.wait_event(x_in[b])
+                    if reuse:
+                        s_cmp.wait_event(y2_out[b])
                     w8.linear_fwd(Xd[b], W1q, s1, out=Y1, ws=ws)
+                    x_read[b].record(s_cmp)
                     w8.linear_fwd(Y1, W2q, s2, out=Y2d[b], ws=ws)
+                    y2_done[b].record(s_cmp)
+                    s_cmp.wait_event(dy_in[b])
+                    if reuse:
+                        s_cmp.wait_event(dx1_out[b])
                     w8.linear_dgrad(dYd[b], W2q, s2, out=dX2, ws=ws)
+                    dy_read[b].record(s_cmp)
                     w8.linear_dgrad(dX2, W1q, s1, out=dX1d[b], ws=ws)
-                    cmp_done[b].record(s_cmp)
+                    dx1_done[b].record(s_cmp)
                 with torch.cuda.stream(s_out):
-                    s_out.wait_event(cmp_done[b])
+                    s_out.wait_event(y2_done[b])
                     hy2[b].copy_(Y2d[b], non_blocking=True)
+                    y2_out[b].record(s_out)
+                    s_out.wait_event(dx1_done[b])
                     hdx1[b].copy_(dX1d[b], non_blocking=True)
-                    out_done[b].record(s_out)
+                    dx1_out[b].record(s_out)
 
-        e2e_steps(3)
+        e2e_steps(3, True)
         torch.cuda.synchronize()
         a, b = E(), E()
         a.record(s_in)
-        e2e_steps(args.e2e_steps)
+        e2e_steps(args.e2e_steps, False)
         s_in.wait_stream(s_out)
+        s_in.wait_stream(s_cmp)
         b.record(s_in)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(a.elapsed_time(b), dist, dev)
@@ -405,7 +426,8 @@ def run_ours(args, rank, world, local_rank):
                "d2h_bytes_per_step": hy2[0].numel() * 2 + hdx1[0].numel() * 2,
                "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps,
                "api": "w8a8_linear_fwd x2 + w8a8_linear_dgrad x2 per step; pinned host buffers; "
-                      "copies in and out timed, overlapped with compute across steps (3 streams)"}
+                      "copies in and out timed, overlapped with compute across steps (3 streams, "
+                      "per-tensor dependencies)"}
 
     if rank != 0:
         return 0
