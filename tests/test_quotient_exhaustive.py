@@ -1,7 +1,10 @@
-"""The row quantizers compute fl(x / s) without a division (a refined
-quotient, see quantize.cuh).  This runs the exhaustive proof of that step on
-the GPU: every fp32 scale significand against every bf16 significand over all
-binades the codes depend on (about 2.5e10 pairs, a couple of seconds)."""
+"""The row quantizers and the Q8_0 -> int8 re-quantization compute fl(x / s)
+without a division (a refined quotient, see quantize.cuh and q8_0.cuh).
+These run the exhaustive proofs of that step on the GPU: every fp32 scale
+significand against every bf16 significand over all binades the codes
+depend on (about 2.5e10 pairs), and every value a Q8_0 block can hold
+against every scale such values give (about 4.7e10 pairs); a few seconds
+each."""
 import os
 import subprocess
 import tempfile
@@ -12,17 +15,28 @@ pytestmark = pytest.mark.gpu
 HERE = os.path.dirname(os.path.abspath(__file__))
 
 
-def test_refined_quotient_is_ieee_division_for_every_bf16_input():
+def _run_check(source):
     import torch
     if not torch.cuda.is_available():
         pytest.fail("GPU tests need a CUDA device")
     from w8a8_quantized_linear_b200 import _build
     with tempfile.TemporaryDirectory() as d:
-        exe = os.path.join(d, "quotient_check")
-        subprocess.run([_build.nvcc(), *_build.ARCH, "-O3", "-o", exe, os.path.join(HERE, "quotient_check.cu")],
+        exe = os.path.join(d, "check")
+        subprocess.run([_build.nvcc(), *_build.ARCH, "-O3", "-o", exe, os.path.join(HERE, source)],
                        check=True, capture_output=True, text=True)
         res = subprocess.run([exe], capture_output=True, text=True, timeout=600)
     line = res.stdout.strip()
     assert res.returncode == 0, line + res.stderr
+    return line
+
+
+def test_refined_quotient_is_ieee_division_for_every_bf16_input():
+    line = _run_check("quotient_check.cu")
     assert "quotient mismatches 0, int8 code mismatches 0, e4m3 code mismatches 0" in line, line
     assert int(line.split()[1]) == (1 << 23) * 23 * 128
+
+
+def test_refined_quotient_is_ieee_division_for_every_q8_0_value():
+    line = _run_check("requant_quotient_check.cu")
+    assert "quotient mismatches 0, int8 code mismatches 0" in line, line
+    assert int(line.split()[1]) == 65537 * 65536 * 11
