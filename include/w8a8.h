@@ -136,7 +136,12 @@ w8a8_status q8_0_to_axis_int8(const void* blocks, int64_t N, int64_t K, int8_t* 
  *   x_bf16 [M, K] contiguous;  wq [N, K] codes of qt;  w_scale [1] (TENSOR)
  *   or [N] (AXIS);  bias_bf16 [N] or NULL;  y_bf16 [M, N] contiguous.
  *   ws: w8a8_workspace_bytes(W8A8_OP_LINEAR_FWD, M, N, K, 0) bytes; holds
- *   the activation codes and row scales of this call.
+ *   the activation codes and row scales of this call, and the int32 partial
+ *   sums when an int8 product with few output tiles is split along K (the
+ *   size depends on the shape only, never on the device).
+ * int8 with M <= 8 and K <= 16384 runs as one weight-streaming launch that
+ * quantizes the rows itself and leaves ws untouched; every path gives the
+ * same bits.
  * ---------------------------------------------------------------------- */
 w8a8_status w8a8_linear_fwd(const void* x_bf16, int64_t M, int64_t N, int64_t K,
                             w8a8_qtype qt, const void* wq, const float* w_scale, w8a8_wgran g,
@@ -153,7 +158,9 @@ w8a8_status w8a8_linear_fwd(const void* x_bf16, int64_t M, int64_t N, int64_t K,
  * contraction dimension (no transposed copy).  Tensor-wise weights only
  * (g must be W8A8_TENSOR).  N % 16 == 0.
  *   dy_bf16 [M, N];  wq [N, K];  dx_bf16 [M, K].
- *   ws: w8a8_workspace_bytes(W8A8_OP_LINEAR_DGRAD, M, N, K, 0) bytes.
+ *   ws: w8a8_workspace_bytes(W8A8_OP_LINEAR_DGRAD, M, N, K, 0) bytes (codes,
+ *   row scales and, for an int8 product with few output tiles, the int32
+ *   partial sums of the split contraction).
  * ---------------------------------------------------------------------- */
 w8a8_status w8a8_linear_dgrad(const void* dy_bf16, int64_t M, int64_t N, int64_t K,
                               w8a8_qtype qt, const void* wq, const float* w_scale, w8a8_wgran g,
@@ -164,13 +171,16 @@ w8a8_status w8a8_linear_dgrad(const void* dy_bf16, int64_t M, int64_t N, int64_t
  * 2411.05007; wiki: SVDQuant data type bfloat16):  W^T ~= L1 L2 + R^T with
  * the residual R quantized int8 tensor-wise, so
  *     T = bf16(X L1)                                   [M, r], fp32 sums
- *     y = bf16( ((acc_R * s_x[m]) * r_scale) + bias[n] + sum_j T[m,j] L2[j,n] )
- * where acc_R = Q(X) Q(R)^T on the tensor cores and the low-rank sum is an
- * fp32 accumulation in the epilogue.  1 <= r <= 64.
+ *     y = bf16( (((acc_R * s_x[m]) * r_scale) + bias[n]) + sum_j T[m,j] L2[j,n] )
+ * where acc_R = Q(X) Q(R)^T on the tensor cores, the low-rank sum is an fp32
+ * accumulation of bf16 products (on the tensor cores from zero, or in the
+ * epilogue) and each outer step is one fp32 RN operation.  r is 8, 16, 24 or
+ * 32 (W8A8_ERR_UNSUPPORTED_SHAPE otherwise).
  *   rq [N, K] int8;  r_scale [1];  l1_bf16 [K, r];  l2_bf16 [r, N];
  *   bias_bf16 [N] or NULL;  y_bf16 [M, N].
  *   ws: w8a8_workspace_bytes(W8A8_OP_SVDQ_FWD, M, N, K, r) bytes; also
- *   holds T.
+ *   holds T [M, r] bf16 (after the codes and row scales) and, when the T
+ *   product is split along K, its fp32 partial sums.
  * ---------------------------------------------------------------------- */
 w8a8_status svdq_linear_fwd(const void* x_bf16, int64_t M, int64_t N, int64_t K,
                             const void* rq, const float* r_scale, int r,
