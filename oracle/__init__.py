@@ -11,8 +11,8 @@ composes those steps in the order the pages give them:
 
 * OneTrainer wiki "Quantization", int W8A8 / float W8A8 paragraphs: weights
   quantized tensor-wise, activations token-wise, the Linear matmul in 8 bits.
-* OneTrainer wiki "Quantization", GGUF A8 int paragraph: GGUF weights
-  re-quantized to int8 axis-wise.
+* OneTrainer wiki "Quantization", GGUF A8 int / GGUF A8 float paragraphs:
+  GGUF weights re-quantized axis-wise to int8 / to float8 (e4m3).
 * bitsandbytes #1401 "LLM.int8() Refactoring: Part 1", Enhancements: the fused
   row calibrate-and-quantize op (int8_vectorwise_quant).
 * entrenar 0.7.8 ``src/quant/gguf_quant/q8_0.rs``: the Q8_0 format.
@@ -79,6 +79,7 @@ def _declare(L):
         "orc_q8_0_dequantize": [_P, _I64, _P],
         "orc_q8_0_dequantize_f32": [_P, _P, _I64, _P],
         "orc_q8_0_to_axis_int8": [_P, _I64, _I64, _P, _P],
+        "orc_q8_0_to_axis": [_P, _I64, _I64, ctypes.c_int, _P, _P],
         "orc_gemm_i8_nt": [_P, _P, _I64, _I64, _I64, _P],
         "orc_gemm_i8_nn": [_P, _P, _I64, _I64, _I64, _P],
         "orc_gemm_e4m3_nt": [_P, _P, _I64, _I64, _I64, _P, _P],
@@ -219,6 +220,16 @@ def q8_0_codes(blocks, n):
 def q8_0_scales_f16(blocks):
     b = _c(blocks, np.uint8).reshape(-1, 34)
     return np.ascontiguousarray(b[:, :2]).view(np.uint16).reshape(-1).copy()
+
+
+def q8_0_to_axis(blocks, N, K, qt):
+    """Q8_0 [N, K/32 blocks] -> axis-wise codes [N, K] (int8 for qt 0, e4m3
+    bytes for qt 1) and the row scales [N]."""
+    b = _c(blocks, np.uint8)
+    q = np.empty((N, K), np.int8 if qt == 0 else np.uint8)
+    s = np.empty((N,), np.float32)
+    lib().orc_q8_0_to_axis(_ptr(b), N, K, qt, _ptr(q), _ptr(s))
+    return q, s
 
 
 def q8_0_to_axis_int8(blocks, N, K):

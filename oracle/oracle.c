@@ -247,11 +247,14 @@ void orc_q8_0_dequantize_f32(const float* scales_f32, const int8_t* codes,
   for (int64_t i = 0; i < n; ++i) y[i] = (float)codes[i] * scales_f32[i / Q80_BLOCK];
 }
 
-/* GGUF A8 int [OT-WIKI]: "re-quantized from GGUF to int8 axis-wise".  Each
- * weight row n holds K/32 consecutive blocks; dequantize (exact), then the
- * token-wise rule with QMAX = 127 on that row. */
-void orc_q8_0_to_axis_int8(const uint8_t* blocks, int64_t N, int64_t K,
-                           int8_t* q, float* s) {
+/* GGUF A8 int / GGUF A8 float [OT-WIKI]: weights "re-quantized from GGUF to
+ * int8 axis-wise" / "to float8 (e4m3) axis-wise".  Each weight row n holds
+ * K/32 consecutive blocks; dequantize (exact), then the token-wise rule on
+ * that row: s_n = floor(absmax)/QMAX, q = code(deq / s_n), with QMAX and the
+ * code of the target type (int8: 127, RNE, clamp; e4m3: 448, RNE-satfinite).
+ * q holds N*K one-byte codes. */
+void orc_q8_0_to_axis(const uint8_t* blocks, int64_t N, int64_t K, int qt,
+                      uint8_t* q, float* s) {
   int64_t bpr = K / Q80_BLOCK;
 #pragma omp parallel for schedule(static)
   for (int64_t n = 0; n < N; ++n) {
@@ -260,11 +263,16 @@ void orc_q8_0_to_axis_int8(const uint8_t* blocks, int64_t N, int64_t K,
     float a = 0.0f;
     for (int64_t k = 0; k < K; ++k)
       if (fabsf(deq[k]) > a) a = fabsf(deq[k]);
-    float sn = absmax_scale(a, ORC_INT8);
+    float sn = absmax_scale(a, qt);
     s[n] = sn;
-    for (int64_t k = 0; k < K; ++k) q[n * K + k] = orc_f32_to_int8_sym(deq[k] / sn);
+    for (int64_t k = 0; k < K; ++k) q[n * K + k] = encode_code(deq[k] / sn, qt);
     free(deq);
   }
+}
+
+void orc_q8_0_to_axis_int8(const uint8_t* blocks, int64_t N, int64_t K,
+                           int8_t* q, float* s) {
+  orc_q8_0_to_axis(blocks, N, K, ORC_INT8, (uint8_t*)q, s);
 }
 
 /* ========================================================================== */

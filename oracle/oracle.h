@@ -10,7 +10,8 @@
  *  [OT-PR]  OneTrainer PR #1034 "New quant types, activation quantization",
  *           section "W8A8 quant types" and "SVDQuant".
  *  [OT-WIKI] OneTrainer wiki "Quantization": the float W8A8, int W8A8,
- *           GGUF A8 int and SVDQuant paragraphs ("Technical:" lines).
+ *           GGUF A8 int, GGUF A8 float and SVDQuant paragraphs
+ *           ("Technical:" lines).
  *  [BNB]    bitsandbytes #1401 "LLM.int8() Refactoring: Part 1", section
  *           "Enhancements / Improved kernels for inference" (the fused
  *           row calibrate-and-quantize op int8_vectorwise_quant).
@@ -70,7 +71,10 @@ void orc_q8_0_dequantize(const uint8_t* blocks, int64_t n, float* y);
 /* Struct dequantize: f32 scale per block times code. */
 void orc_q8_0_dequantize_f32(const float* scales_f32, const int8_t* codes,
                              int64_t n, float* y);
-/* GGUF -> axis-wise int8 re-quantization [OT-WIKI GGUF A8 int]. */
+/* GGUF -> axis-wise re-quantization [OT-WIKI GGUF A8 int (qt ORC_INT8),
+ * GGUF A8 float (qt ORC_E4M3)]: q [N,K] one-byte codes, s [N]. */
+void orc_q8_0_to_axis(const uint8_t* blocks, int64_t N, int64_t K, int qt,
+                      uint8_t* q, float* s);
 void orc_q8_0_to_axis_int8(const uint8_t* blocks, int64_t N, int64_t K,
                            int8_t* q, float* s);
 

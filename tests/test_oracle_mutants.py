@@ -33,6 +33,9 @@ PINS = [
     *[(lambda c: (lambda o: Q.test_q8_0_golden_blocks(o, c)))(c) for c in Q80_CASES],
     Q.test_q8_0_invariants, Q.test_q8_0_short_tail, Q.test_q8_0_grid_roundtrip,
     Q.test_requant_same_scale_rows_are_unchanged, Q.test_requant_invariants,
+    Q.test_requant_e4m3_closed_form, Q.test_requant_e4m3_invariants,
+    lambda o: Q.test_requant_equals_row_quantizer_on_bf16_exact_rows(o, 0),
+    lambda o: Q.test_requant_equals_row_quantizer_on_bf16_exact_rows(o, 1),
     G.test_gemm_i8_bruteforce_tiny,
     lambda o: G.test_gemm_i8_vs_numpy_int64(o, 7, 9, 33),
     G.test_gemm_i8_int32_range_check, G.test_gemm_e4m3_vs_numpy,
@@ -72,7 +75,12 @@ MUTANTS = [
      "const uint8_t* blk = blocks + (i / Q80_BLOCK) * Q80_BLOCK;"),
     ("q8_0 code offset", "y[i] = block_scale_f16(blk) * (float)(int8_t)blk[2 + i % Q80_BLOCK];",
      "y[i] = block_scale_f16(blk) * (float)(int8_t)blk[1 + i % Q80_BLOCK];"),
-    ("requant qmax 128", "float sn = absmax_scale(a, ORC_INT8);", "float sn = a / 128.0f;"),
+    ("requant qmax 128", "float sn = absmax_scale(a, qt);", "float sn = a / 128.0f;"),
+    ("requant e4m3 scale by 127", "float sn = absmax_scale(a, qt);", "float sn = absmax_scale(a, ORC_INT8);"),
+    ("requant e4m3 int8 codes", "q[n * K + k] = encode_code(deq[k] / sn, qt);",
+     "q[n * K + k] = encode_code(deq[k] / sn, ORC_INT8);"),
+    ("requant row stride", "orc_q8_0_dequantize(blocks + n * bpr * Q80_BYTES, K, deq);",
+     "orc_q8_0_dequantize(blocks + n * K, K, deq);"),
     ("gemm nt transposed B", "sum += (int64_t)A[m * K + k] * (int64_t)B[n * K + k];",
      "sum += (int64_t)A[m * K + k] * (int64_t)B[k * N + n];"),
     ("gemm nn transposed B", "sum += (int64_t)A[m * N + n] * (int64_t)B[n * K + k];",

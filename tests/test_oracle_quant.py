@@ -219,3 +219,111 @@ def test_requant_invariants(orc):
     assert np.all(np.abs(q).max(axis=1) == 127)
     err = np.abs(q.astype(np.float64) * s[:, None] - deq)
     assert np.all(err <= s[:, None] * (0.5 + 2 ** -20))
+
+
+# --------------------------------------------------------------------------- Q8_0 -> axis e4m3
+def _e4m3_grid():
+    """(value, code) of the 127 non-negative finite E4M3FN codes, built from
+    the format: 1 sign, 4 exponent bits (bias 7), 3 mantissa bits, subnormal
+    step 2^-9; S.1111.111 is NaN."""
+    out = []
+    for c in range(127):
+        e, m = c >> 3, c & 7
+        v = m * 2.0 ** -9 if e == 0 else (8 + m) * 2.0 ** (e - 10)
+        out.append((v, c))
+    return out
+
+
+def _e4m3_nearest(t):
+    """Brute force: the grid value nearest to t (exact in fp64), ties to the
+    even code, |t| >= 448 saturating to +-448."""
+    sign = 0x80 if np.signbit(t) else 0
+    a = abs(float(t))
+    if a >= 448.0:
+        return sign | 0x7E
+    best = min(_e4m3_grid(), key=lambda vc: (abs(vc[0] - a), vc[1] & 1))
+    return sign | best[1]
+
+
+def _raw_blocks(d_rows, q_rows):
+    """Q8_0 bytes from chosen f16 block scales d [N, nb] (exactly f16) and codes
+    q [N, nb, 32]."""
+    d = np.asarray(d_rows, np.float32)
+    assert np.array_equal(d.astype(np.float16).astype(np.float32), d)
+    N, nb = d.shape
+    blk = np.zeros((N, nb, 34), np.uint8)
+    blk[:, :, :2] = d.astype(np.float16).view(np.uint8).reshape(N, nb, 2)
+    blk[:, :, 2:] = np.asarray(q_rows, np.int8).view(np.uint8)
+    return blk.reshape(-1)
+
+
+def test_requant_e4m3_closed_form(orc):
+    """Rows whose largest |d q| is 112 * 2^-6 get s = 2^-8 exactly, so every
+    quotient is d q / 2^-8, a small multiple of 1/2 (4q, 2q or q/2 for block
+    scales 2^-6, 2^-7, 2^-9); its code must be the nearest E4M3 value by brute
+    force, ties to the even code, including the midpoints 68, 136, 264, ...
+    An all-zero row takes the 1e-10 floor and codes 0."""
+    rng = np.random.default_rng(11)
+    N, nb = 6, 8
+    d = np.full((N, nb), 2.0 ** -6, np.float32)
+    d[:, 1::3] = 2.0 ** -7
+    d[:, 2::3] = 2.0 ** -9
+    q = np.zeros((N, nb, 32), np.int64)
+    allq = np.arange(-112, 113)
+    q[:4].reshape(-1)[: allq.size] = allq          # every code once in the 2^-6 rows ...
+    q[:4] = q[:4].reshape(4, -1)[:, rng.permutation(nb * 32)].reshape(4, nb, 32)
+    q[4] = rng.integers(-112, 113, size=(nb, 32))
+    q[4, 1, 5] = -128                               # -128 in a 2^-7 block: quotient -256
+    q[:5, 0, 0] = 112                               # ... and the row maximum in a 2^-6 block
+    q[:5, 0, 1] = -112
+    d[:5, 0] = 2.0 ** -6
+    d[5] = 2.0 ** -6                                # row 5: all codes zero
+    blocks = _raw_blocks(d, q)
+    codes, s = orc.q8_0_to_axis(blocks, N, nb * 32, orc.E4M3)
+    assert np.all(s[:5] == np.float32(2.0 ** -8)) and s[5] == np.float32(1e-10)
+    quot = (q * (d[:, :, None].astype(np.float64) / 2.0 ** -8)).reshape(N, -1)
+    want = np.array([[_e4m3_nearest(t) for t in row] for row in quot[:5]], np.uint8)
+    assert np.array_equal(codes[:5], want)
+    assert np.all(codes[5] == 0)
+    assert _e4m3_nearest(68.0) == 0x68 and _e4m3_nearest(-68.0) == 0xE8   # tie 64 | 72 -> 64 (1.000 x 2^6)
+
+
+@pytest.mark.parametrize("qt", [0, 1])
+def test_requant_equals_row_quantizer_on_bf16_exact_rows(orc, qt):
+    """With power-of-two block scales every d q (|q| <= 127, 7 bits) is a bf16
+    value, so re-quantizing the blocks must equal quantizing the dequantized
+    weight axis-wise with the row quantizer (pinned by its own golden rows)."""
+    rng = np.random.default_rng(12 + qt)
+    N, nb = 12, 6
+    d = np.exp2(rng.integers(-14, -2, size=(N, nb))).astype(np.float32)
+    q = rng.integers(-127, 128, size=(N, nb, 32))
+    blocks = _raw_blocks(d, q)
+    deq = orc.q8_0_dequantize(blocks, N * nb * 32).reshape(N, -1)
+    wu = workloads.to_u16(torch.from_numpy(deq).to(torch.bfloat16))
+    assert np.array_equal(workloads.to_u16(torch.from_numpy(deq).to(torch.bfloat16)).view(np.uint16).astype(np.uint32) << 16,
+                          deq.view(np.uint32))
+    q1, s1 = orc.q8_0_to_axis(blocks, N, nb * 32, qt)
+    q2, s2 = orc.quantize_weight(wu, qt, orc.AXIS)
+    assert np.array_equal(s1, s2)
+    assert np.array_equal(q1.view(np.uint8), q2)
+
+
+def test_requant_e4m3_invariants(orc):
+    d = workloads.gguf_q8_0(N=64, K=512)
+    w = d["w_f32"].numpy()
+    blocks, _ = orc.q8_0_quantize(w.reshape(-1))
+    q, s = orc.q8_0_to_axis(blocks, 64, 512, orc.E4M3)
+    deq = orc.q8_0_dequantize(blocks, w.size).reshape(64, 512)
+    amax = np.abs(deq).max(axis=1)
+    assert np.array_equal(s, (amax / np.float32(448)).astype(np.float32))
+    dec = orc.decode_codes(q, orc.E4M3).astype(np.float64)
+    assert np.all(np.abs(dec).max(axis=1) == 448.0)
+    v = deq / s[:, None].astype(np.float64)
+    # half a code step: 2^-10 below 2^-6 (subnormals), 2^(E-4) in binade E above
+    e = np.floor(np.log2(np.maximum(np.abs(v), 2.0 ** -6)))
+    assert np.all(np.abs(dec - v) <= np.exp2(e - 4) * (1 + 2 ** -20))
+    assert np.all(np.sign(dec) * np.sign(deq) >= 0)
+    # the int8 re-quantization of the same blocks is the generic entry's qt 0
+    q8, s8 = orc.q8_0_to_axis_int8(blocks, 64, 512)
+    q8b, s8b = orc.q8_0_to_axis(blocks, 64, 512, orc.INT8)
+    assert np.array_equal(q8, q8b) and np.array_equal(s8, s8b)
