@@ -478,7 +478,7 @@ def run_case(args):
     import workloads
     import w8a8_quantized_linear_b200 as w8
     dev = torch.device("cuda", 0)
-    if args.case in ("requant", "gguf_m1", "gguf_m64", "svdq"):
+    if args.case in ("requant", "gguf_m1", "gguf_m64", "svdq", "requant_e4m3", "gguf_f_m1", "gguf_f_m4608"):
         return run_other_case(args, torch, workloads, w8, dev)
     wl = workloads.dit_mlp()
     if args.case in ("up", "dgrad_up"):
@@ -507,8 +507,9 @@ def run_case(args):
 
 
 def run_other_case(args, torch, workloads, w8, dev):
-    """requant: Q8_0 -> axis int8 of the 12288 x 3072 GGUF weight;
-    gguf_m1 / gguf_m64: the GGUF A8 int forward at M = 1 / 64;
+    """requant / requant_e4m3: Q8_0 -> axis int8 / e4m3 of the 12288 x 3072
+    GGUF weight; gguf_m1 / gguf_m64: the GGUF A8 int forward at M = 1 / 64;
+    gguf_f_m1 / gguf_f_m4608: the GGUF A8 float forward at M = 1 / 4608;
     svdq: the SVDQuant r = 32 forward at 4608 x 3072 x 3072."""
     if args.case == "svdq":
         d = workloads.svdquant()
@@ -516,11 +517,17 @@ def run_other_case(args, torch, workloads, w8, dev):
         x = d["x"].to(dev)
         fn = lambda: w8.svdq_linear_fwd(x, prep["rq"], prep["r_scale"], prep["l1"], prep["l2"])
     else:
-        g = workloads.gguf_q8_0(M=64)
+        g = workloads.gguf_q8_0(M=4608 if args.case == "gguf_f_m4608" else 64)
         N, K = g["w_f32"].shape
         blk = w8.q8_0_quantize(g["w_f32"].reshape(-1).to(dev))
         if args.case == "requant":
             fn = lambda: w8.q8_0_to_axis_int8(blk, N, K)
+        elif args.case == "requant_e4m3":
+            fn = lambda: w8.q8_0_to_axis_e4m3(blk, N, K)
+        elif args.case.startswith("gguf_f_m"):
+            wq, sw = w8.q8_0_to_axis_e4m3(blk, N, K)
+            x = g["x"][:int(args.case[len("gguf_f_m"):])].to(dev)
+            fn = lambda: w8.linear_fwd(x, wq, sw)
         else:
             wq, sw = w8.q8_0_to_axis_int8(blk, N, K)
             x = g["x"][:1 if args.case == "gguf_m1" else 64].to(dev)
@@ -681,6 +688,33 @@ def extras(w8, torch, workloads, dev, peaks, src):
                          "weight_GB/s": MLP * HID / (ms * 1e-3) / 1e9}
         del sets
     out["gguf_a8_int_fwd_sweep_N12288_K3072"] = sweep
+    # GGUF A8 float: Q8_0 -> axis e4m3 (same traffic as the int8 requant), then
+    # the e4m3 forward sweep with one weight scale per output column
+    wq0, sw = w8.q8_0_to_axis_e4m3(wb0, MLP, HID)
+    sets = []
+    for i in range(_nsets(nbytes(wb0, wq0))):
+        wb = wb0.clone()
+        q = torch.empty_like(wq0)
+        s = torch.empty(MLP, dtype=torch.float32, device=dev)
+        sets.append(lambda wb=wb, q=q, s=s: w8.q8_0_to_axis_e4m3(wb, MLP, HID, out=q, scale=s))
+    ms = _time_rot(sets, 30, torch, stream)
+    gbs = (wb0.numel() + MLP * HID + MLP * 4) / (ms * 1e-3) / 1e9
+    out["q8_0_to_axis_e4m3_12288x3072"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
+    del sets
+    sweep = {}
+    for M in workloads.GGUF_MS:
+        xm0 = xg[:M].contiguous()
+        sets = []
+        for i in range(_nsets(nbytes(xm0, wq0) + M * MLP * 2)):
+            xm, wq = xm0.clone(), wq0.clone()
+            y = torch.empty((M, MLP), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(w8.workspace_bytes(0, M, MLP, HID), dtype=torch.uint8, device=dev)
+            sets.append(lambda xm=xm, wq=wq, y=y, ws=ws: w8.linear_fwd(xm, wq, sw, out=y, ws=ws))
+        ms = _time_rot(sets, 30, torch, stream)
+        sweep[str(M)] = {"ms": ms, "TOPS": 2 * M * MLP * HID / ms / 1e9,
+                         "weight_GB/s": MLP * HID / (ms * 1e-3) / 1e9}
+        del sets
+    out["gguf_a8_float_fwd_sweep_N12288_K3072"] = sweep
     out["peaks"] = {"source": src, "hbm_gbs": hbm, "int8_burst_tops": tc8}
     out["method"] = ("mean over reps replayed from one CUDA graph (no host launch cost), rotating through "
                      ">= 3x L2 of input/output copies")
@@ -698,7 +732,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-extras", dest="extras", action="store_false")
-    ap.add_argument("--case", choices=["up", "down", "dgrad_down", "dgrad_up", "requant", "gguf_m1", "gguf_m64", "svdq"],
+    ap.add_argument("--case", choices=["up", "down", "dgrad_down", "dgrad_up", "requant", "gguf_m1", "gguf_m64", "svdq",
+                                       "requant_e4m3", "gguf_f_m1", "gguf_f_m4608"],
                     default=None, help="run only one of the step's four quantize+GEMM pairs, or one other kernel "
                                        "of the path (for profiling), no JSON")
     args = ap.parse_args()

@@ -126,6 +126,17 @@ w8a8_status q8_0_dequantize(const void* blocks, int64_t n, float* y, w8a8_stream
 w8a8_status q8_0_to_axis_int8(const void* blocks, int64_t N, int64_t K, int8_t* q_out,
                               float* scale, w8a8_stream_t stream);
 
+/* Re-quantize a Q8_0 weight to axis-wise float8 e4m3 (OneTrainer wiki, GGUF
+ * A8 float: weights re-quantized from GGUF to float8 axis-wise; the Linear
+ * matmuls then run in float8).  The same rows and dequantization as
+ * q8_0_to_axis_int8, with the e4m3 rule of the token-wise quantizer:
+ * s[n] = floor(max|deq|)/448, q = e4m3_rne_satfinite(deq/s[n]) (OCP E4M3FN;
+ * a -0 value keeps its sign, code 0x80).  K % 32 == 0 and K <= 131072.
+ * q_out [N, K] e4m3 bytes;  scale [N] fp32.  The result feeds
+ * w8a8_linear_fwd with W8A8_E4M3 and W8A8_AXIS. */
+w8a8_status q8_0_to_axis_e4m3(const void* blocks, int64_t N, int64_t K, uint8_t* q_out,
+                              float* scale, w8a8_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * W8A8 Linear forward (OneTrainer wiki, int/float W8A8): quantize X
  * token-wise (as w8a8_quantize_rows), multiply the codes with the weight

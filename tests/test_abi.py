@@ -27,7 +27,8 @@ def _header_functions():
 def test_header_declares_the_boundary():
     names = _header_functions()
     for want in ("w8a8_quantize_rows", "w8a8_quantize_weight", "q8_0_quantize", "q8_0_dequantize",
-                 "q8_0_to_axis_int8", "w8a8_linear_fwd", "w8a8_linear_dgrad", "svdq_linear_fwd"):
+                 "q8_0_to_axis_int8", "q8_0_to_axis_e4m3", "w8a8_linear_fwd", "w8a8_linear_dgrad",
+                 "svdq_linear_fwd"):
         assert want in names
 
 
@@ -118,6 +119,11 @@ def test_q8_0_validation(L):
     assert L.q8_0_to_axis_int8(A, 4, 48, A, A, None) == 2      # K % 32
     assert L.q8_0_to_axis_int8(A, 4, 1 << 18, A, A, None) == 2  # K too large
     assert L.q8_0_to_axis_int8(A, 0, 64, A, A, None) == 2
+    assert L.q8_0_to_axis_e4m3(A, 4, 48, A, A, None) == 2      # K % 32
+    assert L.q8_0_to_axis_e4m3(A, 4, 1 << 18, A, A, None) == 2  # K too large
+    assert L.q8_0_to_axis_e4m3(A, 0, 64, A, A, None) == 2
+    assert L.q8_0_to_axis_e4m3(A, 4, 64, None, A, None) == 1
+    assert L.q8_0_to_axis_e4m3(A, 4, 64, B, A, None) == 3       # misaligned codes
     assert L.w8a8_quantize_weight(A, 4, 64, 0, 0, A, A, None, 0, None) == 4   # tensor needs ws
     assert L.w8a8_quantize_weight(A, 4, 64, 0, 7, A, A, None, 0, None) == 1
 

@@ -111,3 +111,27 @@ def test_gguf_q8_0_requant_and_forward_sweep(w8, orc):
         rows = sample_rows(M, n=64, seed=M)
         ref = orc.linear_fwd(workloads.to_u16(x)[rows], wqr.view(np.uint8), swr)
         assert np.array_equal(u16(y)[rows], ref["y"]), M
+
+
+def test_gguf_a8_float_requant_and_forward_sweep(w8, orc):
+    """GGUF A8 float at full size: the Q8_0 weight re-quantized to axis-wise
+    e4m3 (bit for bit), then the e4m3 forward over the M sweep (sampled rows,
+    the fp8 tolerance of the parity tests)."""
+    from test_parity_gpu import _fp8_tol
+    d = workloads.gguf_q8_0(M=max(workloads.GGUF_MS))
+    w = d["w_f32"]
+    N, K = w.shape
+    blocks = w8.q8_0_quantize(w.reshape(-1).to(DEV))
+    br, _ = orc.q8_0_quantize(w.numpy().reshape(-1))
+    wq, sw = w8.q8_0_to_axis_e4m3(blocks, N, K)
+    wqr, swr = orc.q8_0_to_axis(br, N, K, 1)
+    assert np.array_equal(u8(wq), wqr) and np.array_equal(sw.cpu().numpy(), swr)
+    xall = d["x"]
+    for M in workloads.GGUF_MS:
+        x = xall[:M]
+        y = w8.linear_fwd(x.to(DEV), wq, sw)
+        rows = sample_rows(M, n=32, seed=M)
+        ref = orc.linear_fwd(workloads.to_u16(x)[rows], wqr, swr, qt=1)
+        ref["sw"] = swr[None, :]
+        err, bound = _fp8_tol(ref, u16(y)[rows])
+        assert np.all(err <= bound), (M, float((err / bound).max()))

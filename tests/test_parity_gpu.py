@@ -212,6 +212,35 @@ def test_q8_0_to_axis_int8_arbitrary_blocks(w8, orc, N, K):
     assert np.array_equal(u8(q), qr.view(np.uint8))
 
 
+# Q8_0 -> axis e4m3 (GGUF A8 float): the same kernels with the e4m3 code;
+# K = 96 and 4096 + 32 take the one-warp-per-row kernel, 12288 and 32768 the
+# team kernel, the rest the register-holding kernel
+RQ_E4M3_SHAPES = [(1, 32), (37, 96), (64, 512), (12288, 3072), (5, 4128), (7, 12288), (3, 32768), (2, 131072)]
+
+
+@pytest.mark.parametrize("N,K", RQ_E4M3_SHAPES)
+def test_q8_0_to_axis_e4m3_parity(w8, orc, N, K):
+    w = workloads.gguf_q8_0(N=N, K=K, M=1)["w_f32"].numpy().reshape(-1)
+    br, _ = orc.q8_0_quantize(w)
+    q, s = w8.q8_0_to_axis_e4m3(torch.from_numpy(br).to(DEV), N, K)
+    assert q.dtype == torch.float8_e4m3fn
+    qr, sr = orc.q8_0_to_axis(br, N, K, 1)
+    assert np.array_equal(f32(s), sr)
+    assert np.array_equal(u8(q), qr)
+
+
+@pytest.mark.parametrize("N,K", [(13, 256), (50, 3072), (11, 4096), (6, 12288), (4, 32768), (9, 96), (12, 4128)])
+def test_q8_0_to_axis_e4m3_arbitrary_blocks(w8, orc, N, K):
+    """Blocks not produced by a quantizer (see raw_q8_0_blocks): -128 codes,
+    all-zero and negative scales (so -0 values, code 0x80), f16 subnormal
+    scales (quotients in the e4m3 subnormal range)."""
+    br = workloads.raw_q8_0_blocks(N, K, seed=71 + K)
+    q, s = w8.q8_0_to_axis_e4m3(br.to(DEV), N, K)
+    qr, sr = orc.q8_0_to_axis(br.numpy(), N, K, 1)
+    assert np.array_equal(f32(s).view(np.uint32), sr.view(np.uint32))
+    assert np.array_equal(u8(q), qr)
+
+
 # --------------------------------------------------------------------------- Linear forward
 def _fp8_tol(ref, y):
     """|y - y_ref| <= 1e-3 * s_x * s_w * sum|a*b| + 1 bf16 ulp."""
@@ -262,6 +291,23 @@ def test_linear_fwd_e4m3_parity(w8, orc, M, N, K):
     assert np.array_equal(u8(wq), wqr)
     ref = orc.linear_fwd(workloads.to_u16(x), wqr, swr, qt=1, bias=workloads.to_u16(bias))
     ref["sw"] = swr[0]
+    err, bound = _fp8_tol(ref, u16(y))
+    assert np.all(err <= bound), float((err / bound).max())
+
+
+# GGUF A8 float forward: e4m3 weight codes from the Q8_0 re-quantization
+# with one scale per output column, e4m3 activations token-wise
+@pytest.mark.parametrize("M,N,K", [(1, 12288, 3072), (8, 520, 1024), (64, 1024, 3072), (300, 520, 640),
+                                   (600, 1024, 512), (129, 257, 96)])
+def test_gguf_a8_float_forward_parity(w8, orc, M, N, K):
+    d = workloads.gguf_q8_0(N=N, K=K, M=M)
+    br, _ = orc.q8_0_quantize(d["w_f32"].numpy().reshape(-1))
+    wq, sw = w8.q8_0_to_axis_e4m3(torch.from_numpy(br).to(DEV), N, K)
+    y = w8.linear_fwd(d["x"].to(DEV), wq, sw)
+    wqr, swr = orc.q8_0_to_axis(br, N, K, 1)
+    assert np.array_equal(u8(wq), wqr)
+    ref = orc.linear_fwd(workloads.to_u16(d["x"]), wqr, swr, qt=1)
+    ref["sw"] = swr[None, :]
     err, bound = _fp8_tol(ref, u16(y))
     assert np.all(err <= bound), float((err / bound).max())
 

@@ -3,8 +3,8 @@ without a division (a refined quotient, see quantize.cuh and q8_0.cuh).
 These run the exhaustive proofs of that step on the GPU: every fp32 scale
 significand against every bf16 significand over all binades the codes
 depend on (about 2.5e10 pairs), and every value a Q8_0 block can hold
-against every scale such values give (about 4.7e10 pairs); a few seconds
-each."""
+against every scale such values give, for the int8 and the e4m3 scales
+(about 4.7e10 and 8.6e10 pairs); a few seconds each."""
 import os
 import subprocess
 import tempfile
@@ -15,7 +15,7 @@ pytestmark = pytest.mark.gpu
 HERE = os.path.dirname(os.path.abspath(__file__))
 
 
-def _run_check(source):
+def _run_check(source, *args):
     import torch
     if not torch.cuda.is_available():
         pytest.fail("GPU tests need a CUDA device")
@@ -24,7 +24,7 @@ def _run_check(source):
         exe = os.path.join(d, "check")
         subprocess.run([_build.nvcc(), *_build.ARCH, "-O3", "-o", exe, os.path.join(HERE, source)],
                        check=True, capture_output=True, text=True)
-        res = subprocess.run([exe], capture_output=True, text=True, timeout=600)
+        res = subprocess.run([exe, *args], capture_output=True, text=True, timeout=600)
     line = res.stdout.strip()
     assert res.returncode == 0, line + res.stderr
     return line
@@ -37,6 +37,14 @@ def test_refined_quotient_is_ieee_division_for_every_bf16_input():
 
 
 def test_refined_quotient_is_ieee_division_for_every_q8_0_value():
-    line = _run_check("requant_quotient_check.cu")
-    assert "quotient mismatches 0, int8 code mismatches 0" in line, line
+    line = _run_check("requant_quotient_check.cu", "127")
+    assert "quotient mismatches 0, int8 code mismatches 0, e4m3 code mismatches 0" in line, line
     assert int(line.split()[1]) == 65537 * 65536 * 11
+
+
+def test_refined_quotient_is_ieee_division_for_every_q8_0_value_e4m3_scale():
+    """The e4m3 re-quantization: scales fl(a / 448), quotients down to the
+    e4m3 rounding threshold 2^-10 and up to 448."""
+    line = _run_check("requant_quotient_check.cu", "448")
+    assert "quotient mismatches 0, int8 code mismatches 0, e4m3 code mismatches 0" in line, line
+    assert int(line.split()[1]) == 65537 * 65536 * 20

@@ -31,7 +31,7 @@ STATUS = {0: "W8A8_OK", 1: "W8A8_ERR_INVALID_ARG", 2: "W8A8_ERR_UNSUPPORTED_SHAP
 
 # Every symbol include/w8a8.h declares (checked by the tests).
 EXPORTS = ("w8a8_quantize_rows", "w8a8_quantize_weight", "q8_0_bytes", "q8_0_quantize",
-           "q8_0_dequantize", "q8_0_to_axis_int8", "w8a8_linear_fwd", "w8a8_linear_dgrad",
+           "q8_0_dequantize", "q8_0_to_axis_int8", "q8_0_to_axis_e4m3", "w8a8_linear_fwd", "w8a8_linear_dgrad",
            "svdq_linear_fwd", "w8a8_qgemm_fwd", "w8a8_qgemm_dgrad", "w8a8_workspace_bytes",
            "w8a8_device_status", "w8a8_set_wait_limit_ns", "w8a8_selftest_wait",
            "w8a8_e4m3_encode", "w8a8_last_error", "w8a8_linear_fwd_noalloc")
@@ -61,6 +61,7 @@ def lib() -> ctypes.CDLL:
             "q8_0_quantize": [_P, _I64, _P, _P],
             "q8_0_dequantize": [_P, _I64, _P, _P],
             "q8_0_to_axis_int8": [_P, _I64, _I64, _P, _P, _P],
+            "q8_0_to_axis_e4m3": [_P, _I64, _I64, _P, _P, _P],
             "w8a8_linear_fwd": [_P, _I64, _I64, _I64, _I, _P, _P, _I, _P, _P, _P, _SZ, _P],
             "w8a8_linear_dgrad": [_P, _I64, _I64, _I64, _I, _P, _P, _I, _P, _P, _SZ, _P],
             "svdq_linear_fwd": [_P, _I64, _I64, _I64, _P, _P, _I, _P, _P, _P, _P, _P, _SZ, _P],
@@ -196,18 +197,32 @@ def q8_0_dequantize(blocks: torch.Tensor, n: int, out=None):
     return y
 
 
-def q8_0_to_axis_int8(blocks: torch.Tensor, N: int, K: int, out=None, scale=None):
-    """Q8_0 weight [N, K/32 blocks] -> (int8 codes [N, K], per-row scales [N])."""
+def q8_0_to_axis(blocks: torch.Tensor, N: int, K: int, qt="int8", out=None, scale=None):
+    """Q8_0 weight [N, K/32 blocks] -> (codes [N, K], per-row scales [N]):
+    int8 codes (GGUF A8 int) or float8_e4m3fn codes (GGUF A8 float)."""
+    qt = _qt(qt)
     if not (blocks.is_cuda and blocks.dtype == torch.uint8 and blocks.is_contiguous()):
         raise ValueError("blocks must be a contiguous uint8 CUDA tensor")
     if blocks.numel() < q8_0_bytes(N * K):
         raise ValueError("blocks hold fewer than N*K values")
-    q = torch.empty((N, K), dtype=torch.int8, device=blocks.device) if out is None else out
+    dt = _code_dtype(qt)
+    q = torch.empty((N, K), dtype=dt, device=blocks.device) if out is None else out
     s = torch.empty((N,), dtype=torch.float32, device=blocks.device) if scale is None else scale
-    if q.shape != (N, K) or q.dtype != torch.int8 or not q.is_contiguous() or s.numel() < N:
-        raise ValueError("out must be a contiguous int8 [N, K] tensor and scale hold N floats")
-    _check(lib().q8_0_to_axis_int8(_ptr(blocks), N, K, _ptr(q), _ptr(s), _stream(blocks.device)))
+    if q.shape != (N, K) or q.dtype != dt or not q.is_contiguous() or s.numel() < N:
+        raise ValueError("out must be a contiguous %s [N, K] tensor and scale hold N floats" % dt)
+    fn = lib().q8_0_to_axis_int8 if qt == INT8 else lib().q8_0_to_axis_e4m3
+    _check(fn(_ptr(blocks), N, K, _ptr(q), _ptr(s), _stream(blocks.device)))
     return q, s
+
+
+def q8_0_to_axis_int8(blocks: torch.Tensor, N: int, K: int, out=None, scale=None):
+    """Q8_0 weight [N, K/32 blocks] -> (int8 codes [N, K], per-row scales [N])."""
+    return q8_0_to_axis(blocks, N, K, "int8", out, scale)
+
+
+def q8_0_to_axis_e4m3(blocks: torch.Tensor, N: int, K: int, out=None, scale=None):
+    """Q8_0 weight [N, K/32 blocks] -> (e4m3 codes [N, K] as float8_e4m3fn, per-row scales [N])."""
+    return q8_0_to_axis(blocks, N, K, "e4m3", out, scale)
 
 
 # --------------------------------------------------------------------------- Linear

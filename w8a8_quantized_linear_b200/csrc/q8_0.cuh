@@ -1,6 +1,8 @@
 // q8_0.cuh - GGUF Q8_0 blocks (32 values -> f16 scale + 32 int8 codes =
 // 34 bytes; entrenar 0.7.8 q8_0.rs) on the GPU, and the re-quantization of a
-// Q8_0 weight to axis-wise int8 (OneTrainer wiki, GGUF A8 int).
+// Q8_0 weight to axis-wise int8 or e4m3 codes (OneTrainer wiki, GGUF A8 int
+// and GGUF A8 float).  QT selects the target: 0 int8 (QMAX 127), 1 e4m3
+// (QMAX 448).
 //
 // A 34-byte block is not 16-byte aligned, but 8 blocks are 272 = 17 * 16
 // bytes.  A warp handles kQ80Unroll such groups of 8 blocks per iteration
@@ -27,12 +29,6 @@ constexpr int kQ80WarpsPerBlock = 8;
 __device__ __forceinline__ uint32_t q80_code_exact(float v, float scale) {
   const float r = fminf(fmaxf(roundf(__fdiv_rn(v, scale)), -128.0f), 127.0f);
   return static_cast<uint32_t>(static_cast<int>(r)) & 0xFFu;
-}
-
-// int8 value -> float without a conversion instruction: 1.5 * 2^23 + q is
-// exact, so subtracting the magic constant leaves q.
-__device__ __forceinline__ float small_int_to_float(int q) {
-  return __fsub_rn(__int_as_float(0x4B400000 + q), kRneMagic);
 }
 
 // Quantize.  In group u of an iteration, lane l holds values [8l, 8l+8), so
@@ -144,17 +140,35 @@ __global__ void __launch_bounds__(256) q8_0_dequantize_kernel(const uint8_t* __r
   }
 }
 
-// Q8_0 [N, K/32 blocks] -> int8 [N, K] + s [N]: one warp per weight row.  The
-// row's K/32 * 34 bytes are staged in the warp's shared memory; lane l takes
-// blocks l, l+32, ...  Each value is dequantized exactly (f16 scale * code is
-// exact in fp32), the row absmax gives s, and the codes are rounded half to
-// even and clamped to +-127.
+// Code of one dequantized value x = d q for the scale s (y = fl(1/s)), with
+// the refined quotient of rq_block_codes below (exact for every value a Q8_0
+// block can hold and every scale such values give).
+template <int QT>
+__device__ __forceinline__ uint32_t rq_code(float x, float s, float y) {
+  const float q0 = __fmul_rn(x, y);
+  const float q1 = __fmaf_rn(__fmaf_rn(-q0, s, x), y, q0);
+  if constexpr (QT == 1) {
+    const float v = __uint_as_float((__float_as_uint(q1) & 0x7FFFFFFFu) | (__float_as_uint(x) & 0x80000000u));
+    return cvt_e4m3x2(v, 0.0f) & 0xFFu;
+  } else {
+    return __float_as_uint(__fadd_rn(q1, kRneMagic)) & 0xFFu;
+  }
+}
+
+// Q8_0 [N, K/32 blocks] -> codes [N, K] + s [N]: one warp per weight row, for
+// any K % 32 == 0.  The row's K/32 * 34 bytes are staged in the warp's shared
+// memory; lane l takes blocks l, l+32, ...  Each value is dequantized exactly
+// (f16 scale * code is exact in fp32), the row absmax gives s, and each value
+// gets its code from rq_code.
 constexpr int kRequantMaxWarps = 4;
-__global__ void __launch_bounds__(32 * kRequantMaxWarps) q8_0_to_axis_int8_kernel(const uint8_t* __restrict__ blocks,
+template <int QT>
+__global__ void __launch_bounds__(32 * kRequantMaxWarps) q8_0_to_axis_warp_kernel(const uint8_t* __restrict__ blocks,
                                                                                int64_t N, int64_t K,
-                                                                               int8_t* __restrict__ q,
+                                                                               uint8_t* __restrict__ q,
                                                                                float* __restrict__ scale) {
   extern __shared__ __align__(16) uint8_t rowbuf_all[];
+  griddep_launch();
+  griddep_wait();   // the blocks may be the previous kernel's output, q and scale its input
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   const int64_t nblk = K / kQ80Block;
   const int64_t row_bytes = nblk * kQ80Bytes;
@@ -186,35 +200,23 @@ __global__ void __launch_bounds__(32 * kRequantMaxWarps) q8_0_to_axis_int8_kerne
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
-    const float s = (a < 1e-10f) ? 1e-10f : __fdiv_rn(a, 127.0f);
+    const float s = absmax_scale<QT>(a);
     const float rcp = __frcp_rn(s);
     if (lane == 0) scale[n] = s;
     for (int64_t b = lane; b < nblk; b += 32) {
       const uint16_t* blk = reinterpret_cast<const uint16_t*>(rowbuf + b * kQ80Bytes);
       const float d = __half2float(__ushort_as_half(blk[0]));
-      // t = q * fl(d * rcp) lies within 4 ulp of fl(fl(d * q) / s): inside the
-      // 2^-14 margin of rne_low_byte for |t| <= 127.5
-      const float drcp = __fmul_rn(d, rcp);
-      int qv[32];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int pr = blk[1 + i];
-        qv[2 * i] = static_cast<int8_t>(pr & 0xFF);
-        qv[2 * i + 1] = static_cast<int8_t>(pr >> 8);
-      }
       uint32_t w[8];
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        bool near = false;
-        uint32_t c[8];
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t p0 = blk[1 + 2 * i], p1 = blk[2 + 2 * i];
+        uint32_t c = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) c[i] = rne_low_byte(__fmul_rn(small_int_to_float(qv[8 * g + i]), drcp), near);
-        if (near) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) c[i] = int8_code_exact(__fmul_rn(d, small_int_to_float(qv[8 * g + i])), s);
+        for (int j = 0; j < 4; ++j) {
+          const int qv = static_cast<int8_t>(((j < 2 ? p0 : p1) >> (8 * (j & 1))) & 0xFFu);
+          c |= rq_code<QT>(__fmul_rn(d, static_cast<float>(qv)), s, rcp) << (8 * j);
         }
-        w[2 * g] = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-        w[2 * g + 1] = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+        w[i] = c;
       }
       uint4* out = reinterpret_cast<uint4*>(q + n * K + b * kQ80Block);
       out[0] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -225,7 +227,7 @@ __global__ void __launch_bounds__(32 * kRequantMaxWarps) q8_0_to_axis_int8_kerne
 }
 
 // ----------------------------------------------------------------------------
-// Q8_0 -> axis int8 for rows whose blocks fill whole 16-byte units
+// Q8_0 -> axis-wise codes for rows whose blocks fill whole 16-byte units
 // (K % 256 == 0): a team of TW warps per row, thread t of the team taking
 // blocks t, t + 32 TW, ...  Each team keeps its next S - 1 rows in flight
 // into a ring of S shared-memory row buffers (cp.async) while it processes
@@ -295,47 +297,97 @@ __device__ __forceinline__ float rq_block_scale(const uint32_t (&w)[9], bool odd
   return __half2float(__ushort_as_half(static_cast<uint16_t>(prmt(w[0], 0u, odd ? 0x4432u : 0x4410u))));
 }
 
-// 32 codes of a block -> 32 axis int8 codes (8 words).  Each value
-// fl(d q) = d q is exact (an 11-bit by 8-bit product); its code is
-// fl(d q / s) rounded half to even, with the quotient refined from
-// y = fl(1/s) as in the row quantizers (encode8): q0 = fl(x y),
-// r = fl(x - q0 s), q1 = fl(q0 + r y) is the IEEE quotient for every value
-// a Q8_0 block can hold and every scale s = fl(a / 127) such values give
-// (checked exhaustively on the GPU), so no value needs a division and no
-// data-dependent branch is taken.  |x / s| <= 127 (1 + 2^-23): no clamp.
-__device__ __forceinline__ void rq_block_codes(const uint32_t (&w)[9], bool odd, float d, float s, float y,
-                                               uint32_t (&out)[8]) {
-  const uint32_t csel = odd ? 0x7654u : 0x5432u;
-  uint32_t c[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) c[k] = prmt(w[k], w[k + 1], csel);
-  const float2 d2 = make_float2(d, d), y2 = make_float2(y, y), ns2 = make_float2(-s, -s);
-  const float2 mg = make_float2(kRneMagic, kRneMagic);
+// 32 codes of a block -> 32 axis-wise codes (8 words).  Each value
+// fl(d q) = d q is exact (an 11-bit by 8-bit product); its code is that of
+// fl(d q / s), with the quotient refined from y = fl(1/s) as in the row
+// quantizers (encode8): q0 = fl(x y), r = fl(x - q0 s), q1 = fl(q0 + r y) is
+// the IEEE quotient for every value a Q8_0 block can hold and every scale
+// s = fl(a / QMAX) such values give, for QMAX 127 and 448 (checked
+// exhaustively on the GPU), so no value needs a division and no
+// data-dependent branch is taken.  |x / s| <= QMAX (1 + 2^-23): int8 needs
+// no clamp (RNE by the 1.5 * 2^23 sum), e4m3 saturates at 448 in the
+// conversion, which takes x's sign (d q = -0 has code 0x80).
+// The exact product is formed without converting the codes: with its sign
+// bit flipped, code q is the byte u = q + 128, and the fp32 pattern
+// 0x4B00uu00 is B = 2^23 + 256 u = K + 256 q with K = 2^23 + 2^15 (9
+// significant bits, so K d is exact), hence x' = fl(B d - K d) = 256 d q
+// exactly, in one fma.  The quotient is taken on x' with y / 256 and 256 s:
+// every step of the refinement scales by 2^8 exactly, so q0 and q1 are the
+// same numbers as for x, y and s.  x' keeps x's sign except for a zero value,
+// where the fma gives +0: with d > 0 that is x's sign too, and blocks with
+// d <= 0 (never written by a Q8_0 quantizer) take x = d q from its factors.
+template <int QT, bool kPosScale>
+__device__ __forceinline__ void rq_block_codes_impl(const uint32_t (&c)[8], float d, float s, float y,
+                                                    uint32_t (&out)[8]) {
+  constexpr float kK = 8421376.0f;   // 2^23 + 2^15
+  constexpr float kBias = 8388736.0f;   // 2^23 + 128
+  const float ys = y * 0.00390625f, ss = s * 256.0f;   // exact
+  const float2 d2 = make_float2(d, d), y2 = make_float2(ys, ys), ns2 = make_float2(-ss, -ss);
+  const float2 nk2 = make_float2(-kK * d, -kK * d), mg = make_float2(kRneMagic, kRneMagic);
+  const float2 nb2 = make_float2(-kBias, -kBias), d256 = make_float2(d * 256.0f, d * 256.0f);
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     uint32_t b[4];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const float2 qv = make_float2(static_cast<float>(static_cast<int8_t>(c[k] >> (16 * h))),
-                                    static_cast<float>(static_cast<int8_t>(c[k] >> (16 * h + 8))));
-      const float2 x = __fmul2_rn(qv, d2);
+      float2 x;
+      if constexpr (kPosScale) {
+        const float2 u = make_float2(__uint_as_float(prmt(c[k], 0x4B000000u, 0x7504u | ((2 * h) << 4))),
+                                     __uint_as_float(prmt(c[k], 0x4B000000u, 0x7504u | ((2 * h + 1) << 4))));
+        x = __ffma2_rn(u, d2, nk2);
+      } else {
+        const float2 u = make_float2(__uint_as_float(prmt(c[k], 0x4B000000u, 0x7540u | (2 * h))),
+                                     __uint_as_float(prmt(c[k], 0x4B000000u, 0x7540u | (2 * h + 1))));
+        x = __fmul2_rn(__fadd2_rn(u, nb2), d256);   // 256 (q d): +-0 as d q
+      }
       const float2 q0 = __fmul2_rn(x, y2);
       const float2 r = __ffma2_rn(q0, ns2, x);
-      const float2 q1 = __fadd2_rn(__ffma2_rn(r, y2, q0), mg);
-      b[2 * h] = __float_as_uint(q1.x);
-      b[2 * h + 1] = __float_as_uint(q1.y);
+      if constexpr (QT == 1) {
+        const float2 q1 = __ffma2_rn(r, y2, q0);
+        if constexpr (kPosScale) {
+          b[h] = cvt_e4m3x2(q1.x, q1.y);
+        } else {
+          const float lo = __uint_as_float((__float_as_uint(q1.x) & 0x7FFFFFFFu) | (__float_as_uint(x.x) & 0x80000000u));
+          const float hi = __uint_as_float((__float_as_uint(q1.y) & 0x7FFFFFFFu) | (__float_as_uint(x.y) & 0x80000000u));
+          b[h] = cvt_e4m3x2(lo, hi);
+        }
+      } else {
+        const float2 q1 = __fadd2_rn(__ffma2_rn(r, y2, q0), mg);
+        b[2 * h] = __float_as_uint(q1.x);
+        b[2 * h + 1] = __float_as_uint(q1.y);
+      }
     }
-    out[k] = prmt(prmt(b[0], b[1], 0x0040u), prmt(b[2], b[3], 0x0040u), 0x5410u);
+    if constexpr (QT == 1) {
+      out[k] = prmt(b[0], b[1], 0x5410u);
+    } else {
+      out[k] = prmt(prmt(b[0], b[1], 0x0040u), prmt(b[2], b[3], 0x0040u), 0x5410u);
+    }
   }
 }
 
-template <int TW, int S>
-__global__ void __launch_bounds__(kRqThreads) q8_0_to_axis_int8_team_kernel(const uint8_t* __restrict__ blocks,
-                                                                           int64_t N, int64_t K,
-                                                                           int8_t* __restrict__ q,
-                                                                           float* __restrict__ scale) {
+template <int QT>
+__device__ __forceinline__ void rq_block_codes(const uint32_t (&w)[9], bool odd, float d, float s, float y,
+                                               uint32_t (&out)[8]) {
+  const uint32_t csel = odd ? 0x7654u : 0x5432u;
+  uint32_t c[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) c[k] = prmt(w[k], w[k + 1], csel) ^ 0x80808080u;
+  if (QT == 0 || d > 0.0f) {   // int8 codes do not see the sign of a zero
+    rq_block_codes_impl<QT, true>(c, d, s, y, out);
+  } else {
+    rq_block_codes_impl<QT, false>(c, d, s, y, out);
+  }
+}
+
+template <int QT, int TW, int S>
+__global__ void __launch_bounds__(kRqThreads) q8_0_to_axis_team_kernel(const uint8_t* __restrict__ blocks,
+                                                                      int64_t N, int64_t K,
+                                                                      uint8_t* __restrict__ q,
+                                                                      float* __restrict__ scale) {
   extern __shared__ __align__(16) uint8_t rq_smem[];
   __shared__ float red[2][8];
+  griddep_launch();
+  griddep_wait();   // the blocks may be the previous kernel's output, q and scale its input
   constexpr int T = 32 * TW;
   constexpr int kTeams = kRqThreads / T;
   const int team = threadIdx.x / T, t = threadIdx.x % T;
@@ -376,7 +428,7 @@ __global__ void __launch_bounds__(kRqThreads) q8_0_to_axis_int8_team_kernel(cons
 #pragma unroll
       for (int i = 0; i < TW; ++i) a = fmaxf(a, red[it & 1][team * TW + i]);
     }
-    const float s = (a < 1e-10f) ? 1e-10f : __fdiv_rn(a, 127.0f);
+    const float s = absmax_scale<QT>(a);
     const float rcp = __frcp_rn(s);
     if (t == 0) scale[n] = s;
 #pragma unroll 1
@@ -385,7 +437,7 @@ __global__ void __launch_bounds__(kRqThreads) q8_0_to_axis_int8_team_kernel(cons
       rq_block_words(cur, b, w);
       const bool odd = b & 1;
       uint32_t o[8];
-      rq_block_codes(w, odd, rq_block_scale(w, odd), s, rcp, o);
+      rq_block_codes<QT>(w, odd, rq_block_scale(w, odd), s, rcp, o);
       uint4* dst = reinterpret_cast<uint4*>(q + n * K + 32 * static_cast<int64_t>(b));
       dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
       dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
@@ -396,35 +448,47 @@ __global__ void __launch_bounds__(kRqThreads) q8_0_to_axis_int8_team_kernel(cons
 }
 
 // The same computation for rows of at most HOLD * 32 * TW blocks: pass 1
-// keeps each thread's blocks (9 words each) in registers, so the row buffer
-// is free as soon as pass 1 has read it - the next row's copy is issued then
-// and overlaps the arithmetic of pass 2, which needs no shared memory.
-template <int TW, int HOLD, int MINB = 1>
-__global__ void __launch_bounds__(kRqThreads, MINB) q8_0_to_axis_int8_hold_kernel(const uint8_t* __restrict__ blocks,
-                                                                           int64_t N, int64_t K,
-                                                                           int8_t* __restrict__ q,
-                                                                           float* __restrict__ scale) {
+// keeps each thread's blocks (9 words each) in registers, so a row buffer is
+// free as soon as pass 1 has read it.  With S = 1 the next row's copy is
+// issued then and overlaps the arithmetic of pass 2, which needs no shared
+// memory; with S = 2 each team alternates between two row buffers and
+// issues the next row's copy before pass 1 of the current one.
+template <int QT, int TW, int HOLD, int MINB = 1, int S = 1>
+__global__ void __launch_bounds__(kRqThreads, MINB) q8_0_to_axis_hold_kernel(const uint8_t* __restrict__ blocks,
+                                                                            int64_t N, int64_t K,
+                                                                            uint8_t* __restrict__ q,
+                                                                            float* __restrict__ scale) {
+  static_assert(S == 1 || S == 2, "one or two row buffers per team");
   extern __shared__ __align__(16) uint8_t rq_smem[];
   __shared__ float red[2][8];
+  griddep_launch();
+  griddep_wait();   // the blocks may be the previous kernel's output, q and scale its input
   constexpr int T = 32 * TW;
   constexpr int kTeams = kRqThreads / T;
   const int team = threadIdx.x / T, t = threadIdx.x % T;
   const int nblk = static_cast<int>(K >> 5);
   const int row_bytes = nblk * kQ80Bytes;   // a multiple of 16
   const int nvec = row_bytes >> 4;
-  uint8_t* const buf = rq_smem + team * row_bytes;
+  uint8_t* const buf = rq_smem + S * team * row_bytes;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kTeams;
   int64_t n = blockIdx.x * static_cast<int64_t>(kTeams) + team;
-  auto fetch = [&](int64_t row) {
+  auto fetch = [&](int64_t row, int slot) {   // one commit group per call, empty past the last row
     if (row < N) {
       const uint8_t* src = blocks + row * row_bytes;
-      for (int i = t; i < nvec; i += T) cp_async16(buf + 16 * i, src + 16 * i);
+      uint8_t* dst = buf + slot * row_bytes;
+      for (int i = t; i < nvec; i += T) cp_async16(dst + 16 * i, src + 16 * i);
     }
     cp_async_commit();
   };
-  fetch(n);
+  fetch(n, 0);
   for (int it = 0; n < N; n += stride, ++it) {
-    cp_async_wait<0>();
+    const uint8_t* cur = buf + (S == 2 ? (it & 1) : 0) * row_bytes;
+    if constexpr (S == 2) {
+      fetch(n + stride, (it + 1) & 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
     team_sync<TW>(team);   // the row has landed
     uint32_t w[HOLD][9];
     float a = 0.0f;
@@ -432,13 +496,13 @@ __global__ void __launch_bounds__(kRqThreads, MINB) q8_0_to_axis_int8_hold_kerne
     for (int h = 0; h < HOLD; ++h) {
       const int b = t + h * T;
       if (b < nblk) {
-        rq_block_words(buf, b, w[h]);
+        rq_block_words(cur, b, w[h]);
         const bool odd = b & 1;
         a = fmaxf(a, __fmul_rn(fabsf(rq_block_scale(w[h], odd)), static_cast<float>(rq_block_maxabs(w[h], odd))));
       }
     }
-    team_sync<TW>(team);   // every thread has its words: refill the buffer
-    fetch(n + stride);
+    team_sync<TW>(team);   // every thread has its words: the buffer may be refilled
+    if constexpr (S == 1) fetch(n + stride, 0);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
     if constexpr (TW > 1) {
@@ -447,7 +511,7 @@ __global__ void __launch_bounds__(kRqThreads, MINB) q8_0_to_axis_int8_hold_kerne
 #pragma unroll
       for (int i = 0; i < TW; ++i) a = fmaxf(a, red[it & 1][team * TW + i]);
     }
-    const float s = (a < 1e-10f) ? 1e-10f : __fdiv_rn(a, 127.0f);
+    const float s = absmax_scale<QT>(a);
     const float rcp = __frcp_rn(s);
     if (t == 0) scale[n] = s;
 #pragma unroll
@@ -456,7 +520,7 @@ __global__ void __launch_bounds__(kRqThreads, MINB) q8_0_to_axis_int8_hold_kerne
       if (b < nblk) {
         const bool odd = b & 1;
         uint32_t o[8];
-        rq_block_codes(w[h], odd, rq_block_scale(w[h], odd), s, rcp, o);
+        rq_block_codes<QT>(w[h], odd, rq_block_scale(w[h], odd), s, rcp, o);
         uint4* dst = reinterpret_cast<uint4*>(q + n * K + 32 * static_cast<int64_t>(b));
         dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
         dst[1] = make_uint4(o[4], o[5], o[6], o[7]);

@@ -38,8 +38,8 @@ __device__ __forceinline__ float absmax_scale(float a) {
 constexpr float kRneMagic = 12582912.0f;            // 1.5 * 2^23
 constexpr float kNearHalf = 0.49993896484375f;      // 0.5 - 2^-14
 
-// Remainder form of a division-free int8 rounding, for the Q8_0 kernels
-// (whose inputs are not bf16): t = fl(v * fl(1/s)) lies within 3.0001 ulp of
+// Remainder form of a division-free int8 rounding, for the Q8_0 quantizer
+// (whose inputs are fp32, not bf16): t = fl(v * fl(1/s)) lies within 3.0001 ulp of
 // fl(v / s); d = t - rne(t) is exact, and |d| < 0.5 - 2^-14 puts no rounding
 // boundary between them, so the integer is right; otherwise `near` is set
 // and the caller takes the IEEE division.
@@ -48,11 +48,6 @@ __device__ __forceinline__ uint32_t rne_low_byte(float t, bool& near) {
   const float d = __fsub_rn(t, __fsub_rn(big, kRneMagic));
   near |= fabsf(d) > kNearHalf;
   return __float_as_uint(big) & 0xFFu;
-}
-__device__ __forceinline__ uint32_t int8_code_exact(float v, float s) {   // RNE, clamp +-127
-  int q = __float2int_rn(__fdiv_rn(v, s));
-  q = max(-127, min(127, q));
-  return static_cast<uint32_t>(q) & 0xFFu;
 }
 
 // 8 bf16 (one uint4) -> 8 codes (one uint2); y = fl(1/s).

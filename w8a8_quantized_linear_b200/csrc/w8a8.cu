@@ -124,9 +124,10 @@ cudaError_t set_smem_once(Kernel k, size_t bytes, int dev, std::atomic<uint64_t>
 
 // Launch with programmatic stream serialization: the kernel may start (and
 // run up to its griddep_wait) while the previous kernel on the stream
-// finishes.  The kernels launched this way are the row quantizers, the GEMM
-// and the split-K epilogue; each waits before touching memory that the
-// previous kernel may write or read.
+// finishes.  The kernels launched this way are the row quantizers, the GEMMs,
+// the split-K epilogue, the few-token product and the Q8_0 re-quantization;
+// each waits before touching memory that the previous kernel may write or
+// read.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                        Args&&... args) {
@@ -506,6 +507,95 @@ w8a8_status noalloc_scratch(int dev, void** out) {
 
 using namespace w8a8;
 
+// Q8_0 -> axis-wise codes of type QT (0 int8, 1 e4m3).
+template <int QT>
+static w8a8_status requant_axis(const void* blocks, int64_t N, int64_t K, uint8_t* q, float* scale,
+                                w8a8_stream_t stream, const char* name) {
+  W8A8_CHECK(N >= 1, W8A8_ERR_UNSUPPORTED_SHAPE, "N < 1");
+  W8A8_CHECK(K >= 32 && K % 32 == 0 && K <= 131072, W8A8_ERR_UNSUPPORTED_SHAPE,
+             "K must be a multiple of 32 in [32, 131072]");
+  W8A8_CHECK(blocks && q && scale, W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(blocks) && aligned16(q) && aligned16(scale), W8A8_ERR_MISALIGNED,
+             "pointers must be 16-byte aligned");
+  int dev = 0, sms = 0;
+  w8a8_status st = current_device(&dev, &sms);
+  if (st != W8A8_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const auto* bp = static_cast<const uint8_t*>(blocks);
+  const int64_t nblk = K / 32;
+  if (K % 256 == 0 && nblk <= 8 * 96) {
+    // rows of whole 16-byte units and at most 3 blocks per thread of a team
+    // of TW warps: blocks held in registers between the two passes, one row
+    // per team
+    constexpr int kBufs = 1, kCtasPerSm = 16;   // row buffers per team; grid cap per SM
+    int tw = 1;
+    while (tw * 96 < nblk) tw *= 2;
+    const size_t smem = static_cast<size_t>(kBufs * (8 / tw)) * static_cast<size_t>(nblk * 34);
+    int64_t grid = (N + (8 / tw) - 1) / (8 / tw);
+    if (grid > kCtasPerSm * static_cast<int64_t>(sms)) grid = kCtasPerSm * static_cast<int64_t>(sms);
+    static std::atomic<uint64_t> hold_smem_set[4] = {};
+    cudaError_t e = cudaSuccess;
+#define W8A8_RQ_HOLD(TW, IDX)                                                                              \
+  e = set_smem_once(q8_0_to_axis_hold_kernel<QT, TW, 3, 4, kBufs>, 64 * 1024, dev, hold_smem_set[IDX]);    \
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(requant)");                             \
+  e = launch_pdl(q8_0_to_axis_hold_kernel<QT, TW, 3, 4, kBufs>, dim3(static_cast<int>(grid)), dim3(kRqThreads), smem, cs, \
+                 bp, N, K, q, scale)
+    switch (tw) {
+      case 1: W8A8_RQ_HOLD(1, 0); break;
+      case 2: W8A8_RQ_HOLD(2, 1); break;
+      case 4: W8A8_RQ_HOLD(4, 2); break;
+      default: W8A8_RQ_HOLD(8, 3); break;
+    }
+#undef W8A8_RQ_HOLD
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return e == cudaSuccess ? W8A8_OK : cuda_fail(e, name);
+  }
+  if (K % 256 == 0) {
+    // rows of whole 16-byte units: a team of TW warps per row (at least 3
+    // blocks per thread), one row buffer per team and up to 8 blocks per SM
+    // (more warps in flight beat a deeper prefetch ring here)
+    int tw = 1;
+    while (tw < 8 && tw * 2 * 96 <= nblk) tw *= 2;
+    const size_t smem = static_cast<size_t>(8 / tw) * static_cast<size_t>(nblk * 34);
+    if (smem <= 200 * 1024) {
+      int per_sm = static_cast<int>((220 * 1024) / (smem + 1024));
+      per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
+      int64_t grid = (N + (8 / tw) - 1) / (8 / tw);
+      if (grid > static_cast<int64_t>(per_sm) * sms) grid = static_cast<int64_t>(per_sm) * sms;
+      static std::atomic<uint64_t> team_smem_set[4] = {};
+      cudaError_t e = cudaSuccess;
+#define W8A8_RQ_TEAM(TW, IDX)                                                                              \
+  e = set_smem_once(q8_0_to_axis_team_kernel<QT, TW, 1>, 200 * 1024, dev, team_smem_set[IDX]);             \
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(requant)");                             \
+  e = launch_pdl(q8_0_to_axis_team_kernel<QT, TW, 1>, dim3(static_cast<int>(grid)), dim3(kRqThreads), smem, cs, bp, N, \
+                 K, q, scale)
+      switch (tw) {
+        case 1: W8A8_RQ_TEAM(1, 0); break;
+        case 2: W8A8_RQ_TEAM(2, 1); break;
+        case 4: W8A8_RQ_TEAM(4, 2); break;
+        default: W8A8_RQ_TEAM(8, 3); break;
+      }
+#undef W8A8_RQ_TEAM
+      if (e == cudaSuccess) e = cudaGetLastError();
+      return e == cudaSuccess ? W8A8_OK : cuda_fail(e, name);
+    }
+  }
+  // other rows: one warp per row; each warp stages its row (rounded to 16 bytes) in shared memory
+  const size_t row_stride = (static_cast<size_t>(K / 32) * 34 + 15) & ~static_cast<size_t>(15);
+  int warps = static_cast<int>((200 * 1024) / row_stride);
+  warps = warps < 1 ? 1 : (warps > kRequantMaxWarps ? kRequantMaxWarps : warps);
+  const size_t smem = row_stride * warps;
+  static std::atomic<uint64_t> smem_set{0};
+  cudaError_t e = set_smem_once(q8_0_to_axis_warp_kernel<QT>, 200 * 1024, dev, smem_set);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(requant)");
+  int64_t grid = (N + warps - 1) / warps;
+  if (grid > 32 * sms) grid = 32 * sms;
+  e = launch_pdl(q8_0_to_axis_warp_kernel<QT>, dim3(static_cast<int>(grid)), dim3(32 * warps), smem, cs, bp, N, K, q,
+                 scale);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, name);
+}
+
 extern "C" {
 
 const char* w8a8_last_error(void) { return t_last_error.c_str(); }
@@ -608,87 +698,12 @@ w8a8_status q8_0_dequantize(const void* blocks, int64_t n, float* y, w8a8_stream
 
 w8a8_status q8_0_to_axis_int8(const void* blocks, int64_t N, int64_t K, int8_t* q, float* scale,
                               w8a8_stream_t stream) {
-  W8A8_CHECK(N >= 1, W8A8_ERR_UNSUPPORTED_SHAPE, "N < 1");
-  W8A8_CHECK(K >= 32 && K % 32 == 0 && K <= 131072, W8A8_ERR_UNSUPPORTED_SHAPE,
-             "K must be a multiple of 32 in [32, 131072]");
-  W8A8_CHECK(blocks && q && scale, W8A8_ERR_INVALID_ARG, "null pointer");
-  W8A8_CHECK(aligned16(blocks) && aligned16(q) && aligned16(scale), W8A8_ERR_MISALIGNED,
-             "pointers must be 16-byte aligned");
-  int dev = 0, sms = 0;
-  w8a8_status st = current_device(&dev, &sms);
-  if (st != W8A8_OK) return st;
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t nblk = K / 32;
-  if (K % 256 == 0 && nblk <= 8 * 96) {
-    // rows of whole 16-byte units and at most 3 blocks per thread of a team
-    // of TW warps: blocks held in registers between the two passes, one row
-    // per team
-    int tw = 1;
-    while (tw * 96 < nblk) tw *= 2;
-    const size_t smem = static_cast<size_t>(8 / tw) * static_cast<size_t>(nblk * 34);
-    int64_t grid = (N + (8 / tw) - 1) / (8 / tw);
-    if (grid > 16 * static_cast<int64_t>(sms)) grid = 16 * static_cast<int64_t>(sms);
-    static std::atomic<uint64_t> hold_smem_set[4] = {};
-    cudaError_t e = cudaSuccess;
-    const auto* bp = static_cast<const uint8_t*>(blocks);
-#define W8A8_RQ_HOLD(TW, IDX)                                                                              \
-  e = set_smem_once(q8_0_to_axis_int8_hold_kernel<TW, 3, 4>, 64 * 1024, dev, hold_smem_set[IDX]);          \
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(requant)");                             \
-  q8_0_to_axis_int8_hold_kernel<TW, 3, 4><<<static_cast<int>(grid), kRqThreads, smem, cs>>>(bp, N, K, q, scale)
-    switch (tw) {
-      case 1: W8A8_RQ_HOLD(1, 0); break;
-      case 2: W8A8_RQ_HOLD(2, 1); break;
-      case 4: W8A8_RQ_HOLD(4, 2); break;
-      default: W8A8_RQ_HOLD(8, 3); break;
-    }
-#undef W8A8_RQ_HOLD
-    e = cudaGetLastError();
-    return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "q8_0_to_axis_int8 launch");
-  }
-  if (K % 256 == 0) {
-    // rows of whole 16-byte units: a team of TW warps per row (at least 3
-    // blocks per thread), one row buffer per team and up to 8 blocks per SM
-    // (more warps in flight beat a deeper prefetch ring here)
-    int tw = 1;
-    while (tw < 8 && tw * 2 * 96 <= nblk) tw *= 2;
-    const size_t smem = static_cast<size_t>(8 / tw) * static_cast<size_t>(nblk * 34);
-    if (smem <= 200 * 1024) {
-      int per_sm = static_cast<int>((220 * 1024) / (smem + 1024));
-      per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
-      int64_t grid = (N + (8 / tw) - 1) / (8 / tw);
-      if (grid > static_cast<int64_t>(per_sm) * sms) grid = static_cast<int64_t>(per_sm) * sms;
-      static std::atomic<uint64_t> team_smem_set[4] = {};
-      cudaError_t e = cudaSuccess;
-      const auto* bp = static_cast<const uint8_t*>(blocks);
-#define W8A8_RQ_TEAM(TW, IDX)                                                                              \
-  e = set_smem_once(q8_0_to_axis_int8_team_kernel<TW, 1>, 200 * 1024, dev, team_smem_set[IDX]);            \
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(requant)");                             \
-  q8_0_to_axis_int8_team_kernel<TW, 1><<<static_cast<int>(grid), kRqThreads, smem, cs>>>(bp, N, K, q, scale)
-      switch (tw) {
-        case 1: W8A8_RQ_TEAM(1, 0); break;
-        case 2: W8A8_RQ_TEAM(2, 1); break;
-        case 4: W8A8_RQ_TEAM(4, 2); break;
-        default: W8A8_RQ_TEAM(8, 3); break;
-      }
-#undef W8A8_RQ_TEAM
-      e = cudaGetLastError();
-      return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "q8_0_to_axis_int8 launch");
-    }
-  }
-  // other rows: one warp per row; each warp stages its row (rounded to 16 bytes) in shared memory
-  const size_t row_stride = (static_cast<size_t>(K / 32) * 34 + 15) & ~static_cast<size_t>(15);
-  int warps = static_cast<int>((200 * 1024) / row_stride);
-  warps = warps < 1 ? 1 : (warps > kRequantMaxWarps ? kRequantMaxWarps : warps);
-  const size_t smem = row_stride * warps;
-  static std::atomic<uint64_t> smem_set{0};
-  cudaError_t e = set_smem_once(q8_0_to_axis_int8_kernel, 200 * 1024, dev, smem_set);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(requant)");
-  int64_t grid = (N + warps - 1) / warps;
-  if (grid > 32 * sms) grid = 32 * sms;
-  q8_0_to_axis_int8_kernel<<<static_cast<int>(grid), 32 * warps, smem, cs>>>(
-      static_cast<const uint8_t*>(blocks), N, K, q, scale);
-  e = cudaGetLastError();
-  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "q8_0_to_axis_int8 launch");
+  return requant_axis<0>(blocks, N, K, reinterpret_cast<uint8_t*>(q), scale, stream, "q8_0_to_axis_int8 launch");
+}
+
+w8a8_status q8_0_to_axis_e4m3(const void* blocks, int64_t N, int64_t K, uint8_t* q, float* scale,
+                              w8a8_stream_t stream) {
+  return requant_axis<1>(blocks, N, K, q, scale, stream, "q8_0_to_axis_e4m3 launch");
 }
 
 w8a8_status w8a8_qgemm_fwd(const void* xq, int64_t ldq, const float* sx, int64_t M, int64_t N, int64_t K,
