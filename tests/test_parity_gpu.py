@@ -190,8 +190,14 @@ def test_q8_0_standalone_full_size(w8, orc):
     assert np.array_equal(f32(y).view(np.uint32), orc.q8_0_dequantize(br, x.numel()).view(np.uint32))
 
 
-@pytest.mark.parametrize("N,K", [(1, 32), (37, 96), (64, 512), (12288, 3072), (5, 4096), (7, 12288),
-                                 (3, 32768), (2, 131072)])
+# K = 3072, 6144, 12288 and 24576 fill the register-holding kernel's blocks
+# exactly (its FULL form); 512 and 4096 do not; 96 and 4128 take the
+# one-warp-per-row kernel, 32768 and 131072 the team kernel
+RQ_SHAPES = [(1, 32), (37, 96), (64, 512), (12288, 3072), (5, 4096), (4, 6144), (7, 12288), (3, 24576),
+             (3, 32768), (2, 131072), (5, 4128)]
+
+
+@pytest.mark.parametrize("N,K", RQ_SHAPES)
 def test_q8_0_to_axis_int8_parity(w8, orc, N, K):
     w = workloads.gguf_q8_0(N=N, K=K, M=1)["w_f32"].numpy().reshape(-1)
     br, _ = orc.q8_0_quantize(w)
@@ -201,7 +207,8 @@ def test_q8_0_to_axis_int8_parity(w8, orc, N, K):
     assert np.array_equal(u8(q), qr.view(np.uint8))
 
 
-@pytest.mark.parametrize("N,K", [(13, 256), (50, 3072), (11, 4096), (6, 12288), (4, 32768), (9, 96)])
+@pytest.mark.parametrize("N,K", [(13, 256), (50, 3072), (11, 4096), (6, 12288), (4, 32768), (9, 96), (12, 4128),
+                                 (5, 6144), (3, 24576)])
 def test_q8_0_to_axis_int8_arbitrary_blocks(w8, orc, N, K):
     """Blocks not produced by a quantizer: -128 codes, zero, negative and
     subnormal f16 scales, rows sharing one scale (codes come back unchanged)."""
@@ -212,13 +219,8 @@ def test_q8_0_to_axis_int8_arbitrary_blocks(w8, orc, N, K):
     assert np.array_equal(u8(q), qr.view(np.uint8))
 
 
-# Q8_0 -> axis e4m3 (GGUF A8 float): the same kernels with the e4m3 code;
-# K = 96 and 4096 + 32 take the one-warp-per-row kernel, 12288 and 32768 the
-# team kernel, the rest the register-holding kernel
-RQ_E4M3_SHAPES = [(1, 32), (37, 96), (64, 512), (12288, 3072), (5, 4128), (7, 12288), (3, 32768), (2, 131072)]
-
-
-@pytest.mark.parametrize("N,K", RQ_E4M3_SHAPES)
+# Q8_0 -> axis e4m3 (GGUF A8 float): the same kernels with the e4m3 code
+@pytest.mark.parametrize("N,K", RQ_SHAPES)
 def test_q8_0_to_axis_e4m3_parity(w8, orc, N, K):
     w = workloads.gguf_q8_0(N=N, K=K, M=1)["w_f32"].numpy().reshape(-1)
     br, _ = orc.q8_0_quantize(w)
@@ -229,7 +231,8 @@ def test_q8_0_to_axis_e4m3_parity(w8, orc, N, K):
     assert np.array_equal(u8(q), qr)
 
 
-@pytest.mark.parametrize("N,K", [(13, 256), (50, 3072), (11, 4096), (6, 12288), (4, 32768), (9, 96), (12, 4128)])
+@pytest.mark.parametrize("N,K", [(13, 256), (50, 3072), (11, 4096), (6, 12288), (4, 32768), (9, 96), (12, 4128),
+                                 (5, 6144), (3, 24576)])
 def test_q8_0_to_axis_e4m3_arbitrary_blocks(w8, orc, N, K):
     """Blocks not produced by a quantizer (see raw_q8_0_blocks): -128 codes,
     all-zero and negative scales (so -0 values, code 0x80), f16 subnormal

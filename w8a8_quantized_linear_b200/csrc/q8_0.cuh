@@ -278,18 +278,25 @@ __device__ __forceinline__ void rq_block_words(const uint8_t* row, int b, uint32
   for (int i = 0; i < 9; ++i) w[i] = p[i];
 }
 
-// max |q| over the 32 codes of a block.
+// max |q| over the 32 codes of a block.  The codes fill words 1..8 of an odd
+// block; for an even block they are the last two bytes of word 0, words
+// 1..7 and the first two bytes of word 8, and one prmt joins the two halves.
+// In a word [B3 B2 B1 B0] read as two signed 16-bit lanes, lane i is
+// B(2i+1) * 256 + (B2i unsigned), so a lane's max / min carries the max / min
+// of the upper bytes in its upper byte; the word shifted left by 8 bits puts
+// B0 and B2 there.  Three-input s16x2 max / min over both forms cover all four
+// bytes, and an arithmetic shift by 8 recovers the byte.
 __device__ __forceinline__ int rq_block_maxabs(const uint32_t (&w)[9], bool odd) {
-  const uint32_t s0 = odd ? 0xD5C4u : 0xB3A2u, s1 = odd ? 0xF7E6u : 0xD5C4u;
   uint32_t mx = 0x80008000u, mn = 0x7FFF7FFFu;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint32_t p0 = prmt(w[k], w[k + 1], s0), p1 = prmt(w[k], w[k + 1], s1);
-    mx = vmax_s16x2(mx, vmax_s16x2(p0, p1));
-    mn = vmin_s16x2(mn, vmin_s16x2(p0, p1));
+  for (int k = 1; k <= 8; ++k) {
+    const uint32_t v = k < 8 ? w[k] : (odd ? w[8] : prmt(w[8], w[0], 0x7610u));
+    const uint32_t v8 = v << 8;
+    mx = vmax_s16x2(mx, vmax_s16x2(v, v8));
+    mn = vmin_s16x2(mn, vmin_s16x2(v, v8));
   }
-  const int hi = max(static_cast<int>(static_cast<int16_t>(mx & 0xFFFFu)), static_cast<int>(static_cast<int16_t>(mx >> 16)));
-  const int lo = min(static_cast<int>(static_cast<int16_t>(mn & 0xFFFFu)), static_cast<int>(static_cast<int16_t>(mn >> 16)));
+  const int hi = max(static_cast<int>(static_cast<int16_t>(mx & 0xFFFFu)), static_cast<int>(static_cast<int16_t>(mx >> 16))) >> 8;
+  const int lo = min(static_cast<int>(static_cast<int16_t>(mn & 0xFFFFu)), static_cast<int>(static_cast<int16_t>(mn >> 16))) >> 8;
   return max(hi, -lo);
 }
 
@@ -323,7 +330,10 @@ __device__ __forceinline__ void rq_block_codes_impl(const uint32_t (&c)[8], floa
   constexpr float kBias = 8388736.0f;   // 2^23 + 128
   const float ys = y * 0.00390625f, ss = s * 256.0f;   // exact
   const float2 d2 = make_float2(d, d), y2 = make_float2(ys, ys), ns2 = make_float2(-ss, -ss);
-  const float2 nk2 = make_float2(-kK * d, -kK * d), mg = make_float2(kRneMagic, kRneMagic);
+  // int8: fl(q1 + 2^23 + 128) rounds q1 to the nearest integer, ties to
+  // even (unit spacing in [2^23, 2^24), and 2^23 + 128 is even), leaving
+  // code + 128 in the low byte
+  const float2 nk2 = make_float2(-kK * d, -kK * d), mg = make_float2(kBias, kBias);
   const float2 nb2 = make_float2(-kBias, -kBias), d256 = make_float2(d * 256.0f, d * 256.0f);
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -360,7 +370,10 @@ __device__ __forceinline__ void rq_block_codes_impl(const uint32_t (&c)[8], floa
     if constexpr (QT == 1) {
       out[k] = prmt(b[0], b[1], 0x5410u);
     } else {
-      out[k] = prmt(prmt(b[0], b[1], 0x0040u), prmt(b[2], b[3], 0x0040u), 0x5410u);
+      // b = 0x4B000000 + (code + 128): integer multiply-adds put the four
+      // bytes side by side (the multiples of 256 push 0x4B out of the word),
+      // and flipping each byte's top bit gives the two's-complement codes
+      out[k] = ((b[0] & 0xFFu) + b[1] * 256u + b[2] * 65536u + b[3] * 16777216u) ^ 0x80808080u;
     }
   }
 }
@@ -452,8 +465,9 @@ __global__ void __launch_bounds__(kRqThreads) q8_0_to_axis_team_kernel(const uin
 // free as soon as pass 1 has read it.  With S = 1 the next row's copy is
 // issued then and overlaps the arithmetic of pass 2, which needs no shared
 // memory; with S = 2 each team alternates between two row buffers and
-// issues the next row's copy before pass 1 of the current one.
-template <int QT, int TW, int HOLD, int MINB = 1, int S = 1>
+// issues the next row's copy before pass 1 of the current one.  FULL: every
+// row has exactly HOLD * 32 * TW blocks (no per-block bounds test).
+template <int QT, int TW, int HOLD, int MINB = 1, int S = 1, bool FULL = false>
 __global__ void __launch_bounds__(kRqThreads, MINB) q8_0_to_axis_hold_kernel(const uint8_t* __restrict__ blocks,
                                                                             int64_t N, int64_t K,
                                                                             uint8_t* __restrict__ q,
@@ -495,7 +509,7 @@ __global__ void __launch_bounds__(kRqThreads, MINB) q8_0_to_axis_hold_kernel(con
 #pragma unroll
     for (int h = 0; h < HOLD; ++h) {
       const int b = t + h * T;
-      if (b < nblk) {
+      if (FULL || b < nblk) {
         rq_block_words(cur, b, w[h]);
         const bool odd = b & 1;
         a = fmaxf(a, __fmul_rn(fabsf(rq_block_scale(w[h], odd)), static_cast<float>(rq_block_maxabs(w[h], odd))));
@@ -517,7 +531,7 @@ __global__ void __launch_bounds__(kRqThreads, MINB) q8_0_to_axis_hold_kernel(con
 #pragma unroll
     for (int h = 0; h < HOLD; ++h) {
       const int b = t + h * T;
-      if (b < nblk) {
+      if (FULL || b < nblk) {
         const bool odd = b & 1;
         uint32_t o[8];
         rq_block_codes<QT>(w[h], odd, rq_block_scale(w[h], odd), s, rcp, o);

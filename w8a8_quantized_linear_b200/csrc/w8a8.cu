@@ -533,18 +533,19 @@ static w8a8_status requant_axis(const void* blocks, int64_t N, int64_t K, uint8_
     const size_t smem = static_cast<size_t>(kBufs * (8 / tw)) * static_cast<size_t>(nblk * 34);
     int64_t grid = (N + (8 / tw) - 1) / (8 / tw);
     if (grid > kCtasPerSm * static_cast<int64_t>(sms)) grid = kCtasPerSm * static_cast<int64_t>(sms);
-    static std::atomic<uint64_t> hold_smem_set[4] = {};
+    static std::atomic<uint64_t> hold_smem_set[8] = {};
     cudaError_t e = cudaSuccess;
-#define W8A8_RQ_HOLD(TW, IDX)                                                                              \
-  e = set_smem_once(q8_0_to_axis_hold_kernel<QT, TW, 3, 4, kBufs>, 64 * 1024, dev, hold_smem_set[IDX]);    \
+    const bool full = nblk == 96 * tw;   // every thread holds exactly 3 blocks
+#define W8A8_RQ_HOLD(TW, F, IDX)                                                                           \
+  e = set_smem_once(q8_0_to_axis_hold_kernel<QT, TW, 3, 4, kBufs, F>, 64 * 1024, dev, hold_smem_set[IDX]); \
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(requant)");                             \
-  e = launch_pdl(q8_0_to_axis_hold_kernel<QT, TW, 3, 4, kBufs>, dim3(static_cast<int>(grid)), dim3(kRqThreads), smem, cs, \
-                 bp, N, K, q, scale)
+  e = launch_pdl(q8_0_to_axis_hold_kernel<QT, TW, 3, 4, kBufs, F>, dim3(static_cast<int>(grid)), dim3(kRqThreads), smem, \
+                 cs, bp, N, K, q, scale)
     switch (tw) {
-      case 1: W8A8_RQ_HOLD(1, 0); break;
-      case 2: W8A8_RQ_HOLD(2, 1); break;
-      case 4: W8A8_RQ_HOLD(4, 2); break;
-      default: W8A8_RQ_HOLD(8, 3); break;
+      case 1: if (full) { W8A8_RQ_HOLD(1, true, 4); } else { W8A8_RQ_HOLD(1, false, 0); } break;
+      case 2: if (full) { W8A8_RQ_HOLD(2, true, 5); } else { W8A8_RQ_HOLD(2, false, 1); } break;
+      case 4: if (full) { W8A8_RQ_HOLD(4, true, 6); } else { W8A8_RQ_HOLD(4, false, 2); } break;
+      default: if (full) { W8A8_RQ_HOLD(8, true, 7); } else { W8A8_RQ_HOLD(8, false, 3); } break;
     }
 #undef W8A8_RQ_HOLD
     if (e == cudaSuccess) e = cudaGetLastError();
