@@ -466,9 +466,10 @@ __global__ void __launch_bounds__(kRqThreads) q8_0_to_axis_team_kernel(const uin
 // issued then and overlaps the arithmetic of pass 2, which needs no shared
 // memory; with S = 2 each team alternates between two row buffers and
 // issues the next row's copy before pass 1 of the current one.  FULL: every
-// row has exactly HOLD * 32 * TW blocks (no per-block bounds test).
-template <int QT, int TW, int HOLD, int MINB = 1, int S = 1, bool FULL = false>
-__global__ void __launch_bounds__(kRqThreads, MINB) q8_0_to_axis_hold_kernel(const uint8_t* __restrict__ blocks,
+// row has exactly HOLD * 32 * TW blocks (no per-block bounds test).  NT
+// threads per block.
+template <int QT, int TW, int HOLD, int MINB = 1, int S = 1, bool FULL = false, int NT = kRqThreads>
+__global__ void __launch_bounds__(NT, MINB) q8_0_to_axis_hold_kernel(const uint8_t* __restrict__ blocks,
                                                                             int64_t N, int64_t K,
                                                                             uint8_t* __restrict__ q,
                                                                             float* __restrict__ scale) {
@@ -478,7 +479,8 @@ __global__ void __launch_bounds__(kRqThreads, MINB) q8_0_to_axis_hold_kernel(con
   griddep_launch();
   griddep_wait();   // the blocks may be the previous kernel's output, q and scale its input
   constexpr int T = 32 * TW;
-  constexpr int kTeams = kRqThreads / T;
+  static_assert(NT % T == 0 && NT <= 256, "whole teams, at most 8 warps");
+  constexpr int kTeams = NT / T;
   const int team = threadIdx.x / T, t = threadIdx.x % T;
   const int nblk = static_cast<int>(K >> 5);
   const int row_bytes = nblk * kQ80Bytes;   // a multiple of 16

@@ -528,24 +528,33 @@ static w8a8_status requant_axis(const void* blocks, int64_t N, int64_t K, uint8_
     // of TW warps: blocks held in registers between the two passes, one row
     // per team
     constexpr int kBufs = 1, kCtasPerSm = 16;   // row buffers per team; grid cap per SM
+    // 128 threads per block (8 blocks per SM) for teams of 1 and 4 warps:
+    // finer blocks leave less of the last wave idle than 256-thread blocks,
+    // whose slot is held until the slowest of their rows is done (measured:
+    // 12288 x 3072 16.4 -> 15.7 us, 3072 x 12288 18.4 -> 17.8 us; teams of 2
+    // warps were slower that way, 4096 x 4096 9.8 -> 12.6 us)
+    constexpr int kNtSmall = 128;
     int tw = 1;
     while (tw * 96 < nblk) tw *= 2;
-    const size_t smem = static_cast<size_t>(kBufs * (8 / tw)) * static_cast<size_t>(nblk * 34);
-    int64_t grid = (N + (8 / tw) - 1) / (8 / tw);
-    if (grid > kCtasPerSm * static_cast<int64_t>(sms)) grid = kCtasPerSm * static_cast<int64_t>(sms);
+    const int nt = (tw == 1 || tw == 4) ? kNtSmall : kRqThreads;
+    const int teams = nt / 32 / tw;               // rows per block
+    const size_t smem = static_cast<size_t>(kBufs * teams) * static_cast<size_t>(nblk * 34);
+    int64_t grid = (N + teams - 1) / teams;
+    if (grid > kCtasPerSm * static_cast<int64_t>(sms) * (256 / nt)) grid = kCtasPerSm * static_cast<int64_t>(sms) * (256 / nt);
     static std::atomic<uint64_t> hold_smem_set[8] = {};
     cudaError_t e = cudaSuccess;
     const bool full = nblk == 96 * tw;   // every thread holds exactly 3 blocks
-#define W8A8_RQ_HOLD(TW, F, IDX)                                                                           \
-  e = set_smem_once(q8_0_to_axis_hold_kernel<QT, TW, 3, 4, kBufs, F>, 64 * 1024, dev, hold_smem_set[IDX]); \
+#define W8A8_RQ_HOLD(TW, F, IDX, NT)                                                                       \
+  e = set_smem_once(q8_0_to_axis_hold_kernel<QT, TW, 3, 1024 / NT, kBufs, F, NT>, 64 * 1024, dev,           \
+                    hold_smem_set[IDX]);                                                                   \
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(requant)");                             \
-  e = launch_pdl(q8_0_to_axis_hold_kernel<QT, TW, 3, 4, kBufs, F>, dim3(static_cast<int>(grid)), dim3(kRqThreads), smem, \
-                 cs, bp, N, K, q, scale)
+  e = launch_pdl(q8_0_to_axis_hold_kernel<QT, TW, 3, 1024 / NT, kBufs, F, NT>, dim3(static_cast<int>(grid)), dim3(NT), \
+                 smem, cs, bp, N, K, q, scale)
     switch (tw) {
-      case 1: if (full) { W8A8_RQ_HOLD(1, true, 4); } else { W8A8_RQ_HOLD(1, false, 0); } break;
-      case 2: if (full) { W8A8_RQ_HOLD(2, true, 5); } else { W8A8_RQ_HOLD(2, false, 1); } break;
-      case 4: if (full) { W8A8_RQ_HOLD(4, true, 6); } else { W8A8_RQ_HOLD(4, false, 2); } break;
-      default: if (full) { W8A8_RQ_HOLD(8, true, 7); } else { W8A8_RQ_HOLD(8, false, 3); } break;
+      case 1: if (full) { W8A8_RQ_HOLD(1, true, 4, kNtSmall); } else { W8A8_RQ_HOLD(1, false, 0, kNtSmall); } break;
+      case 2: if (full) { W8A8_RQ_HOLD(2, true, 5, kRqThreads); } else { W8A8_RQ_HOLD(2, false, 1, kRqThreads); } break;
+      case 4: if (full) { W8A8_RQ_HOLD(4, true, 6, kNtSmall); } else { W8A8_RQ_HOLD(4, false, 2, kNtSmall); } break;
+      default: if (full) { W8A8_RQ_HOLD(8, true, 7, kRqThreads); } else { W8A8_RQ_HOLD(8, false, 3, kRqThreads); } break;
     }
 #undef W8A8_RQ_HOLD
     if (e == cudaSuccess) e = cudaGetLastError();
