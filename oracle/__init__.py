@@ -369,12 +369,13 @@ def lowrank_up(t_bf16, l2_bf16):
     return lr, lr_abs
 
 
-def svdq_linear_fwd(x_bf16, rq, s_r, l1_bf16, l2_bf16, bias=None):
-    """SVDQuant forward: Y = epilogue(Q(X) Q(R)) + (X L1) L2, bf16 out.
+def svdq_linear_fwd(x_bf16, rq, s_r, l1_bf16, l2_bf16, bias=None, qt=INT8):
+    """SVDQuant forward: Y = epilogue(Q(X) Q(R)) + (X L1) L2, bf16 out, with
+    int8 (int W8A8) or e4m3 (float W8A8) codes for X and R.
 
     T = bf16(X L1) [M,r]; lr = T L2 accumulated exactly (fp64) and rounded to
-    fp32 before the add.  Returns the int part, T, lr and the bound inputs."""
-    base = linear_fwd(x_bf16, rq, s_r, INT8, bias)
+    fp32 before the add.  Returns the 8-bit part, T, lr and the bound inputs."""
+    base = linear_fwd(x_bf16, rq, s_r, qt, bias)
     t, t64 = lowrank_down(x_bf16, l1_bf16)
     lr, lr_abs = lowrank_up(t, l2_bf16)
     y32 = (base["y32"] + lr.astype(np.float32)).astype(np.float32)

@@ -11,7 +11,9 @@ out here:
     L1 = bf16(U_r diag(sqrt(sigma_r)))       [K, r]
     L2 = bf16(diag(sqrt(sigma_r)) V_r^T)     [r, N]
     R  = bf16(W - (L1 L2)^T)                 [N, K]   residual, after rounding
-    Rq, s_R = tensor-wise int8 quantization of R
+    Rq, s_R = tensor-wise quantization of R: int8 (int W8A8), or e4m3 (float
+              W8A8: the wiki says SVDQuant combines with all quantized types
+              except GGUF)
 
 so that X W^T ~= X L1 L2 + X R^T.  Activation smoothing from the paper is not
 on the pages and is not applied.
@@ -35,8 +37,9 @@ def svd_split(w_bf16, r):
     return l1, l2, resid
 
 
-def prepare(w_bf16, r):
-    """Full SVDQuant weight prep: factors plus the int8 tensor-wise residual."""
+def prepare(w_bf16, r, qt=INT8):
+    """Full SVDQuant weight prep: factors plus the tensor-wise residual codes
+    (qt: INT8 or E4M3)."""
     l1, l2, resid = svd_split(w_bf16, r)
-    rq, s_r = quantize_weight(resid, INT8, TENSOR)
+    rq, s_r = quantize_weight(resid, qt, TENSOR)
     return {"l1": l1, "l2": l2, "resid": resid, "rq": rq, "s_r": s_r}

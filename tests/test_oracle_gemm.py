@@ -212,6 +212,37 @@ def test_svdq_zero_factors_is_int_linear(orc):
     assert np.array_equal(s["y"], f["y"])
 
 
+def test_svdq_zero_factors_is_float_linear(orc):
+    """SVDQuant on float W8A8 (e4m3 residual codes): zero factors give the
+    e4m3 Linear forward exactly."""
+    x = workloads.to_u16(workloads.with_outlier_channels((16, 256), 1.0, 18))
+    w = workloads.to_u16(workloads.normal((64, 256), 0.02, 19))
+    rq, sr = orc.quantize_weight(w, orc.E4M3, orc.TENSOR)
+    z1 = np.zeros((256, 32), np.uint16)
+    z2 = np.zeros((32, 64), np.uint16)
+    s = orc.svdq_linear_fwd(x, rq, sr, z1, z2, qt=orc.E4M3)
+    f = orc.linear_fwd(x, rq, sr, qt=orc.E4M3)
+    assert np.array_equal(s["y"], f["y"])
+    rq8, sr8 = orc.quantize_weight(w, orc.INT8, orc.TENSOR)
+    assert not np.array_equal(f["y"], orc.linear_fwd(x, rq8, sr8)["y"])   # the code type is in effect
+
+
+@pytest.mark.parametrize("qt", [0, 1])
+def test_svdq_zero_residual_is_lowrank_product(orc, qt):
+    """With all residual codes zero, y is the low-rank product alone: the bf16
+    rounding of fp32(T L2), T = bf16(X L1), checked against numpy in fp64."""
+    x = workloads.normal((12, 96), 1.0, 23)
+    l1 = workloads.normal((96, 16), 0.1, 24)
+    l2 = workloads.normal((16, 40), 0.1, 25)
+    rq = np.zeros((40, 96), np.uint8)
+    sr = np.array([1e-10], np.float32)
+    s = orc.svdq_linear_fwd(workloads.to_u16(x), rq, sr, workloads.to_u16(l1), workloads.to_u16(l2), qt=qt)
+    t = torch.from_numpy((x.double() @ l1.double()).numpy().astype(np.float32)).to(torch.bfloat16)
+    lr = (t.double() @ l2.double()).numpy().astype(np.float32)
+    want = torch.from_numpy(lr).to(torch.bfloat16)
+    assert np.array_equal(s["y"], workloads.to_u16(want))
+
+
 def test_svdq_split_reduces_weight_error(orc):
     """With a rank-8 spike, the low-rank branch plus the int8 residual is a
     better approximation of W than plain tensor-wise int8."""
@@ -239,3 +270,20 @@ def test_svdq_exact_lowrank_weight(orc):
     prep = svdquant.prepare(workloads.to_u16(w), 8)
     resid = orc.bf16_to_f32(prep["resid"])
     assert np.abs(resid).max() < 0.02 * np.abs(w.float().numpy()).max()
+
+
+def test_svdq_split_reduces_weight_error_e4m3(orc):
+    """The same with an e4m3 residual (float W8A8 + SVDQuant): the factors
+    carry the spike in bf16, and the residual's e4m3 error is that of the
+    noise alone."""
+    w = workloads.rank_spike_weight(256, 320, 8, 0.5, 0.02, 20)
+    wu = workloads.to_u16(w)
+    prep = svdquant.prepare(wu, 32, orc.E4M3)
+    W = w.double().numpy()
+    lowrank = (orc.bf16_to_f32(prep["l1"]).astype(np.float64)
+               @ orc.bf16_to_f32(prep["l2"]).astype(np.float64)).T
+    deq_r = orc.decode_codes(prep["rq"], orc.E4M3).astype(np.float64) * prep["s_r"][0]
+    err_svd = np.linalg.norm(W - lowrank - deq_r)
+    wq, sw = orc.quantize_weight(wu, orc.E4M3, orc.TENSOR)
+    err_plain = np.linalg.norm(W - orc.decode_codes(wq, orc.E4M3).astype(np.float64) * sw[0])
+    assert err_svd < 0.5 * err_plain, (err_svd, err_plain)

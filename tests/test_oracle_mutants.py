@@ -41,7 +41,9 @@ PINS = [
     G.test_gemm_i8_int32_range_check, G.test_gemm_e4m3_vs_numpy,
     G.test_epilogue_closed_form, G.test_epilogue_axis_scale_indexes_columns,
     G.test_linear_fwd_reduces_to_integer_matmul, G.test_linear_dgrad_reduces_to_integer_matmul,
-    G.test_lowrank_vs_numpy,
+    G.test_lowrank_vs_numpy, G.test_svdq_zero_factors_is_float_linear,
+    lambda o: G.test_svdq_zero_residual_is_lowrank_product(o, 0),
+    lambda o: G.test_svdq_zero_residual_is_lowrank_product(o, 1),
 ]
 
 # (name, text in oracle.c, replacement)
