@@ -478,7 +478,8 @@ def run_case(args):
     import workloads
     import w8a8_quantized_linear_b200 as w8
     dev = torch.device("cuda", 0)
-    if args.case in ("requant", "gguf_m1", "gguf_m64", "svdq", "requant_e4m3", "gguf_f_m1", "gguf_f_m4608"):
+    if args.case in ("requant", "gguf_m1", "gguf_m64", "svdq", "requant_e4m3", "gguf_f_m1", "gguf_f_m4608",
+                     "svdq_e4m3"):
         return run_other_case(args, torch, workloads, w8, dev)
     wl = workloads.dit_mlp()
     if args.case in ("up", "dgrad_up"):
@@ -510,10 +511,11 @@ def run_other_case(args, torch, workloads, w8, dev):
     """requant / requant_e4m3: Q8_0 -> axis int8 / e4m3 of the 12288 x 3072
     GGUF weight; gguf_m1 / gguf_m64: the GGUF A8 int forward at M = 1 / 64;
     gguf_f_m1 / gguf_f_m4608: the GGUF A8 float forward at M = 1 / 4608;
-    svdq: the SVDQuant r = 32 forward at 4608 x 3072 x 3072."""
-    if args.case == "svdq":
+    svdq / svdq_e4m3: the SVDQuant r = 32 forward at 4608 x 3072 x 3072 with
+    an int8 / e4m3 residual."""
+    if args.case in ("svdq", "svdq_e4m3"):
         d = workloads.svdquant()
-        prep = w8.svdq_prepare(d["w"].to(dev), d["r"])
+        prep = w8.svdq_prepare(d["w"].to(dev), d["r"], "e4m3" if args.case == "svdq_e4m3" else "int8")
         x = d["x"].to(dev)
         fn = lambda: w8.svdq_linear_fwd(x, prep["rq"], prep["r_scale"], prep["l1"], prep["l2"])
     else:
@@ -630,7 +632,21 @@ def extras(w8, torch, workloads, dev, peaks, src):
     ops = 2 * M_TOK * 3072 * 3072
     out["svdquant_r32_fwd_4608x3072x3072"] = {"ms": ms, "TOPS_main": ops / ms / 1e9,
                                               "lowrank_GFLOP": 2 * 2 * M_TOK * 3072 * 32 / 1e9}
-    del sets
+    del sets, prep0
+    # the same with an e4m3 residual (float W8A8 + SVDQuant)
+    prep0 = w8.svdq_prepare(d["w"].to(dev), d["r"], "e4m3")
+    sets = []
+    for i in range(_nsets(nbytes(xx0, prep0["rq"]) + M_TOK * 3072 * 2)):
+        xx = xx0.clone()
+        rq, l1, l2 = prep0["rq"].clone(), prep0["l1"].clone(), prep0["l2"].clone()
+        y = torch.empty((M_TOK, 3072), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(w8.workspace_bytes(2, M_TOK, 3072, 3072, 32), dtype=torch.uint8, device=dev)
+        sets.append(lambda xx=xx, rq=rq, l1=l1, l2=l2, y=y, ws=ws:
+                    w8.svdq_linear_fwd(xx, rq, prep0["r_scale"], l1, l2, out=y, ws=ws))
+    ms = _time_rot(sets, 30, torch, stream)
+    out["svdquant_e4m3_r32_fwd_4608x3072x3072"] = {"ms": ms, "TOPS_main": ops / ms / 1e9,
+                                                   "lowrank_GFLOP": 2 * 2 * M_TOK * 3072 * 32 / 1e9}
+    del sets, prep0
     # GGUF Q8_0: standalone quantize / dequantize of 2^28 fp32 (each 1.3 GB of traffic)
     n = 1 << 28
     xf0 = workloads.q8_0_standalone(n).to(dev)
@@ -733,7 +749,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-extras", dest="extras", action="store_false")
     ap.add_argument("--case", choices=["up", "down", "dgrad_down", "dgrad_up", "requant", "gguf_m1", "gguf_m64", "svdq",
-                                       "requant_e4m3", "gguf_f_m1", "gguf_f_m4608"],
+                                       "requant_e4m3", "gguf_f_m1", "gguf_f_m4608", "svdq_e4m3"],
                     default=None, help="run only one of the step's four quantize+GEMM pairs, or one other kernel "
                                        "of the path (for profiling), no JSON")
     args = ap.parse_args()

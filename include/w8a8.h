@@ -198,6 +198,18 @@ w8a8_status svdq_linear_fwd(const void* x_bf16, int64_t M, int64_t N, int64_t K,
                             const void* l1_bf16, const void* l2_bf16, const void* bias_bf16,
                             void* y_bf16, void* ws, size_t ws_bytes, w8a8_stream_t stream);
 
+/* SVDQuant on float W8A8 (OneTrainer wiki, SVDQuant paragraph: it combines
+ * with all quantized data types except GGUF): svdq_linear_fwd with e4m3
+ * residual codes and e4m3 token-wise activation codes.  The residual product
+ * accumulates in fp32 on the tensor cores (kind::f8f6f4), then the same
+ * epilogue and low-rank sum.  rq [N, K] e4m3 bytes (tensor-wise, as
+ * w8a8_quantize_weight with W8A8_E4M3); every other argument as in
+ * svdq_linear_fwd, including the workspace size. */
+w8a8_status svdq_linear_fwd_e4m3(const void* x_bf16, int64_t M, int64_t N, int64_t K,
+                                 const void* rq, const float* r_scale, int r,
+                                 const void* l1_bf16, const void* l2_bf16, const void* bias_bf16,
+                                 void* y_bf16, void* ws, size_t ws_bytes, w8a8_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * The two tensor-core products on codes that are already quantized (the
  * second half of w8a8_linear_fwd / w8a8_linear_dgrad), for callers that

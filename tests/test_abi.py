@@ -28,7 +28,7 @@ def test_header_declares_the_boundary():
     names = _header_functions()
     for want in ("w8a8_quantize_rows", "w8a8_quantize_weight", "q8_0_quantize", "q8_0_dequantize",
                  "q8_0_to_axis_int8", "q8_0_to_axis_e4m3", "w8a8_linear_fwd", "w8a8_linear_dgrad",
-                 "svdq_linear_fwd"):
+                 "svdq_linear_fwd", "svdq_linear_fwd_e4m3"):
         assert want in names
 
 
@@ -108,6 +108,10 @@ def test_svdq_validation(L):
     assert L.svdq_linear_fwd(A, 8, 8, 32, A, A, 64, A, A, None, A, A, 1 << 20, None) == 2   # r > 32
     assert L.svdq_linear_fwd(A, 8, 8, 32, A, A, 32, None, A, None, A, A, 1 << 20, None) == 1
     assert L.svdq_linear_fwd(A, 8, 8, 32, A, A, 32, A, A, None, A, A, 64, None) == 4
+    assert L.svdq_linear_fwd_e4m3(A, 8, 8, 32, A, A, 12, A, A, None, A, A, 1 << 20, None) == 2   # r % 8
+    assert L.svdq_linear_fwd_e4m3(A, 8, 8, 32, A, A, 32, None, A, None, A, A, 1 << 20, None) == 1
+    assert L.svdq_linear_fwd_e4m3(A, 8, 8, 32, A, A, 32, A, A, None, A, A, 64, None) == 4
+    assert L.svdq_linear_fwd_e4m3(A, 0, 8, 32, A, A, 32, A, A, None, A, A, 0, None) == 0      # M = 0: no-op
 
 
 def test_q8_0_validation(L):

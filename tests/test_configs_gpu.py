@@ -94,6 +94,13 @@ def test_svdquant_sampled(w8, orc):
     _svdq_check(w8, orc, d["x"], d["w"], d["r"], rows=sample_rows(d["x"].shape[0], n=96))
 
 
+def test_svdquant_e4m3_sampled(w8, orc):
+    """The SVDQuant workload with an e4m3 residual (float W8A8 + SVDQuant)."""
+    from test_parity_gpu import _svdq_check
+    d = workloads.svdquant()
+    _svdq_check(w8, orc, d["x"], d["w"], d["r"], rows=sample_rows(d["x"].shape[0], n=96), qt=1)
+
+
 def test_gguf_q8_0_requant_and_forward_sweep(w8, orc):
     d = workloads.gguf_q8_0(M=max(workloads.GGUF_MS))
     w = d["w_f32"]

@@ -410,12 +410,14 @@ def test_qgemm_dgrad_equals_linear(w8):
 
 
 # --------------------------------------------------------------------------- SVDQuant
-def _svdq_check(w8, orc, x, w, r, bias=None, rows=None):
+def _svdq_check(w8, orc, x, w, r, bias=None, rows=None, qt=0):
     from oracle import svdquant
-    prep = svdquant.prepare(workloads.to_u16(w), r)
+    prep = svdquant.prepare(workloads.to_u16(w), r, qt)
     to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(DEV)
     l1, l2 = to_dev(prep["l1"]), to_dev(prep["l2"])
     rq = torch.from_numpy(prep["rq"].view(np.int8)).to(DEV)
+    if qt == 1:
+        rq = rq.view(torch.float8_e4m3fn)
     rs = torch.from_numpy(prep["s_r"]).to(DEV)
     M, K = x.shape
     N = w.shape[0]
@@ -427,18 +429,21 @@ def _svdq_check(w8, orc, x, w, r, bias=None, rows=None):
     rows = np.arange(M) if rows is None else np.asarray(rows)
     xs = workloads.to_u16(x)[rows]
     ref = orc.svdq_linear_fwd(xs, prep["rq"], prep["s_r"], prep["l1"], prep["l2"],
-                              bias=None if bias is None else workloads.to_u16(bias))
+                              bias=None if bias is None else workloads.to_u16(bias), qt=qt)
     # T: fp32 accumulation over K on the tensor cores, then one bf16 rounding
     xabs = np.abs(orc.bf16_to_f32(xs).astype(np.float64)) @ np.abs(orc.bf16_to_f32(prep["l1"]).astype(np.float64))
     gam = K * 2.0 ** -23 * xabs
     tg = bf16_bits_to_f64(u16(t_gpu)[rows])
     assert np.all(np.abs(tg - ref["t64"]) <= ulp_bf16(np.abs(ref["t64"]) + gam) + gam)
-    # y: the int part is exact; T may differ by its bound; lr sums in fp32
+    # y: the int part is exact (the e4m3 part within the fp8 bound); T may
+    # differ by its bound; lr sums in fp32
     dt = ulp_bf16(np.abs(ref["t64"]) + gam) + gam
     l2abs = np.abs(orc.bf16_to_f32(prep["l2"]).astype(np.float64))
     yr = bf16_bits_to_f64(ref["y"])
     yg = bf16_bits_to_f64(u16(y)[rows])
     bound = dt @ l2abs + 2.0 ** -16 * ref["lr_abs"] + ulp_bf16(np.maximum(np.abs(yr), np.abs(yg)))
+    if qt == 1:
+        bound = bound + 1e-3 * ref["sx"][:, None].astype(np.float64) * float(prep["s_r"][0]) * ref["absacc"]
     assert np.all(np.abs(yg - yr) <= bound), float((np.abs(yg - yr) / bound).max())
     return y, ref
 
@@ -467,6 +472,26 @@ def test_svdq_parity_pairs(w8, orc, M, N, K, r):
 def test_svdq_zero_factors_equal_int_linear(w8, M):
     x = workloads.normal((M, 256), 1.0, 61).to(DEV)
     wq, sw = w8.quantize_weight(workloads.normal((304, 256), 0.02, 62).to(DEV), "int8", "tensor")
+    l1 = torch.zeros((256, 16), dtype=torch.bfloat16, device=DEV)
+    l2 = torch.zeros((16, 304), dtype=torch.bfloat16, device=DEV)
+    assert torch.equal(w8.svdq_linear_fwd(x, wq, sw, l1, l2), w8.linear_fwd(x, wq, sw))
+
+
+# SVDQuant on float W8A8: e4m3 residual and activation codes.  Small M and
+# N % 8 != 0 take the single-SM low-rank epilogue, the rest the CTA pair.
+@pytest.mark.parametrize("M,N,K,r", [(200, 320, 256, 8), (130, 300, 256, 16), (600, 520, 512, 8),
+                                     (1024, 1024, 1024, 32), (530, 300, 256, 16), (777, 264, 384, 24)])
+def test_svdq_e4m3_parity(w8, orc, M, N, K, r):
+    x = workloads.with_outlier_channels((M, K), 1.0, seed=71 + M)
+    w = workloads.rank_spike_weight(N, K, 8, 0.5, 0.02, seed=72 + N)
+    bias = workloads.normal((N,), 0.01, seed=73)
+    _svdq_check(w8, orc, x, w, r, bias=bias, qt=1)
+
+
+@pytest.mark.parametrize("M", [130, 600])
+def test_svdq_e4m3_zero_factors_equal_float_linear(w8, M):
+    x = workloads.normal((M, 256), 1.0, 61).to(DEV)
+    wq, sw = w8.quantize_weight(workloads.normal((304, 256), 0.02, 62).to(DEV), "e4m3", "tensor")
     l1 = torch.zeros((256, 16), dtype=torch.bfloat16, device=DEV)
     l2 = torch.zeros((16, 304), dtype=torch.bfloat16, device=DEV)
     assert torch.equal(w8.svdq_linear_fwd(x, wq, sw, l1, l2), w8.linear_fwd(x, wq, sw))

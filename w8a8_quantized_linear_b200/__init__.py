@@ -32,7 +32,7 @@ STATUS = {0: "W8A8_OK", 1: "W8A8_ERR_INVALID_ARG", 2: "W8A8_ERR_UNSUPPORTED_SHAP
 # Every symbol include/w8a8.h declares (checked by the tests).
 EXPORTS = ("w8a8_quantize_rows", "w8a8_quantize_weight", "q8_0_bytes", "q8_0_quantize",
            "q8_0_dequantize", "q8_0_to_axis_int8", "q8_0_to_axis_e4m3", "w8a8_linear_fwd", "w8a8_linear_dgrad",
-           "svdq_linear_fwd", "w8a8_qgemm_fwd", "w8a8_qgemm_dgrad", "w8a8_workspace_bytes",
+           "svdq_linear_fwd", "svdq_linear_fwd_e4m3", "w8a8_qgemm_fwd", "w8a8_qgemm_dgrad", "w8a8_workspace_bytes",
            "w8a8_device_status", "w8a8_set_wait_limit_ns", "w8a8_selftest_wait",
            "w8a8_e4m3_encode", "w8a8_last_error", "w8a8_linear_fwd_noalloc")
 
@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
             "w8a8_linear_fwd": [_P, _I64, _I64, _I64, _I, _P, _P, _I, _P, _P, _P, _SZ, _P],
             "w8a8_linear_dgrad": [_P, _I64, _I64, _I64, _I, _P, _P, _I, _P, _P, _SZ, _P],
             "svdq_linear_fwd": [_P, _I64, _I64, _I64, _P, _P, _I, _P, _P, _P, _P, _P, _SZ, _P],
+            "svdq_linear_fwd_e4m3": [_P, _I64, _I64, _I64, _P, _P, _I, _P, _P, _P, _P, _P, _SZ, _P],
             "w8a8_qgemm_fwd": [_P, _I64, _P, _I64, _I64, _I64, _I, _P, _P, _I, _P, _P, _P],
             "w8a8_qgemm_dgrad": [_P, _I64, _P, _I64, _I64, _I64, _I, _P, _P, _P, _P],
             "w8a8_device_status": [_P, _I],
@@ -297,7 +298,8 @@ def qgemm_dgrad(dyq, dy_scale, wq, w_scale, out=None):
 
 def svdq_linear_fwd(x, rq, r_scale, l1, l2, bias=None, out=None, ws=None):
     """SVDQuant forward: Y = epilogue(Q(X) Rq^T) + bf16(X L1) L2.
-    x [M, K] bf16, rq [N, K] int8, r_scale [1], l1 [K, r] bf16, l2 [r, N] bf16."""
+    x [M, K] bf16, rq [N, K] int8 (int W8A8) or float8_e4m3fn (float W8A8),
+    r_scale [1], l1 [K, r] bf16, l2 [r, N] bf16."""
     _cuda_2d(x, torch.bfloat16, "x")
     M, K = x.shape
     N = rq.shape[0]
@@ -306,15 +308,22 @@ def svdq_linear_fwd(x, rq, r_scale, l1, l2, bias=None, out=None, ws=None):
         raise ValueError("l1 must be [K, r] and l2 [r, N]")
     y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else out
     ws = _workspace(OP_SVDQ_FWD, M, N, K, r, x.device, ws)
-    _check(lib().svdq_linear_fwd(_ptr(x), M, N, K, _ptr(_as_bytes(rq)), _ptr(r_scale), r, _ptr(l1), _ptr(l2),
-                                 _ptr(bias), _ptr(y), _ptr(ws), ws.numel(), _stream(x.device)))
+    if rq.dtype == torch.int8:
+        fn = lib().svdq_linear_fwd
+    elif rq.dtype == torch.float8_e4m3fn:
+        fn = lib().svdq_linear_fwd_e4m3
+    else:
+        raise ValueError("rq must hold int8 or float8_e4m3fn codes")
+    _check(fn(_ptr(x), M, N, K, _ptr(_as_bytes(rq)), _ptr(r_scale), r, _ptr(l1), _ptr(l2),
+              _ptr(bias), _ptr(y), _ptr(ws), ws.numel(), _stream(x.device)))
     return y
 
 
-def svdq_prepare(w: torch.Tensor, r: int):
+def svdq_prepare(w: torch.Tensor, r: int, qt="int8"):
     """Offline SVDQuant weight split of W [N, K] bf16 (fp64 SVD with torch):
     L1 = bf16(U_r sqrt(S_r)) [K, r], L2 = bf16(sqrt(S_r) V_r^T) [r, N],
-    R = bf16(W - (L1 L2)^T), then R quantized int8 tensor-wise by the library.
+    R = bf16(W - (L1 L2)^T), then R quantized tensor-wise (int8 or e4m3) by
+    the library.
     Returns dict(l1, l2, rq, r_scale) on w's device."""
     wt = w.detach().to(torch.float64).T            # [K, N]
     u, sig, vh = torch.linalg.svd(wt, full_matrices=False)
@@ -322,7 +331,7 @@ def svdq_prepare(w: torch.Tensor, r: int):
     l1 = (u[:, :r] * root[None, :]).to(torch.float32).to(torch.bfloat16)
     l2 = (root[:, None] * vh[:r, :]).to(torch.float32).to(torch.bfloat16)
     resid = (w.to(torch.float64) - (l1.double() @ l2.double()).T).to(torch.float32).to(torch.bfloat16)
-    rq, r_scale = quantize_weight(resid.contiguous(), "int8", "tensor")
+    rq, r_scale = quantize_weight(resid.contiguous(), qt, "tensor")
     return {"l1": l1.contiguous(), "l2": l2.contiguous(), "rq": rq, "r_scale": r_scale}
 
 

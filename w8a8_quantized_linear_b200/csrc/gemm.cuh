@@ -455,7 +455,8 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
               float d[4];
 #pragma unroll
               for (int q4 = 0; q4 < 4; ++q4) {
-                float a = __int2float_rn(static_cast<int>(rfr[mt][4 * i + q4]));
+                float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int>(rfr[mt][4 * i + q4]))
+                                            : __uint_as_float(rfr[mt][4 * i + q4]);
                 a = __fmul_rn(__fmul_rn(a, sxr[mt][q4 >> 1]), sw0);
                 if (ep.bias != nullptr) a = __fadd_rn(a, bcol[i][q4 & 1]);
                 d[q4] = __fadd_rn(a, lr[q4]);

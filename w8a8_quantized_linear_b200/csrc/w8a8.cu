@@ -606,6 +606,93 @@ static w8a8_status requant_axis(const void* blocks, int64_t N, int64_t K, uint8_
   return e == cudaSuccess ? W8A8_OK : cuda_fail(e, name);
 }
 
+// SVDQuant forward with residual codes of type QT (int8 or e4m3).
+template <int QT>
+static w8a8_status svdq_fwd_impl(const void* x, int64_t M, int64_t N, int64_t K, const void* rq, const float* r_scale,
+                                 int r, const void* l1, const void* l2, const void* bias, void* y, void* ws,
+                                 size_t ws_bytes, w8a8_stream_t stream) {
+  constexpr int kKind = (QT == W8A8_E4M3) ? kKindE4M3 : kKindI8;
+  W8A8_CHECK(M >= 0 && N >= 1 && M < (1ll << 31) && N < (1ll << 31), W8A8_ERR_UNSUPPORTED_SHAPE, "bad M/N");
+  w8a8_status st = check_k(K, "K");
+  if (st != W8A8_OK) return st;
+  W8A8_CHECK(r >= 8 && r <= 32 && r % 8 == 0, W8A8_ERR_UNSUPPORTED_SHAPE, "rank r must be 8, 16, 24 or 32");
+  if (M == 0) return W8A8_OK;
+  W8A8_CHECK(x && rq && r_scale && l1 && l2 && y, W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(x) && aligned16(rq) && aligned16(r_scale) && aligned16(l1) && aligned16(l2) && aligned16(y) &&
+                 (bias == nullptr || aligned16(bias)),
+             W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  W8A8_CHECK(ws != nullptr && ws_bytes >= ws_svdq(M, K, r), W8A8_ERR_WORKSPACE,
+             "workspace too small: need %zu bytes", ws_svdq(M, K, r));
+  W8A8_CHECK(aligned16(ws), W8A8_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+  if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Carve c(ws);
+  void* xq = c.take(static_cast<size_t>(M * K));
+  float* sx = static_cast<float*>(c.take(static_cast<size_t>(M) * 4));
+  auto* t = static_cast<__nv_bfloat16*>(c.take(static_cast<size_t>(M) * r * 2));
+  const int tsplit = t_splits(M, K);
+  SplitWs tsk;
+  if (tsplit > 1) {
+    tsk.splits = tsplit;
+    tsk.partial = static_cast<uint32_t*>(
+        c.take(static_cast<size_t>(tsplit) * static_cast<size_t>(M) * static_cast<size_t>(r) * 4));
+  }
+  if ((st = launch_quantize_rows(x, K, M, K, QT, xq, K, sx, s)) != W8A8_OK) return st;
+  // T = bf16(X L1): bf16 tensor-core GEMM, L1 [K, r] read MN-major; split
+  // along K when the rows make few tiles (fp32 partial sums, added in split
+  // order, then one bf16 rounding).
+  {
+    alignas(64) CUtensorMap ta, tb;
+    if ((st = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, K, M, K * 2, 64, kBM)) != W8A8_OK) return st;
+    if ((st = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, l1, r, K, static_cast<int64_t>(r) * 2, 64, 64)) !=
+        W8A8_OK)
+      return st;
+    EpiParams ep{};
+    ep.y = t;
+    ep.ldy = r;
+    ep.splits = tsk.splits;
+    ep.partial = tsk.partial;
+    if ((st = launch_gemm<kKindBF16, true, 64, kEpiPlain>(ta, tb, M, r, K, ep, s)) != W8A8_OK) return st;
+    if (tsk.splits > 1) {
+      int sms = 0;
+      if ((st = current_device(nullptr, &sms)) != W8A8_OK) return st;
+      int64_t grid = (M * (r / 8) + 255) / 256;
+      if (grid > 8 * static_cast<int64_t>(sms)) grid = 8 * static_cast<int64_t>(sms);
+      const uint32_t* part = tsk.partial;
+      const cudaError_t e = launch_pdl(splitk_epilogue_kernel<kKindBF16>, dim3(static_cast<unsigned>(grid)), dim3(256), 0,
+                                       s, part, tsk.splits, M, static_cast<int64_t>(r), static_cast<const float*>(nullptr),
+                                       static_cast<const float*>(nullptr), 0, static_cast<const __nv_bfloat16*>(nullptr),
+                                       t);
+      if (e != cudaSuccess) return cuda_fail(e, "split-K epilogue launch");
+    }
+  }
+  alignas(64) CUtensorMap ta, tb;
+  if ((st = make_map(&ta, code_type(), 1, xq, K, M, K, kBKBytes, kBM)) != W8A8_OK) return st;
+  const bool pair = M >= kPairMinRows && (N % 8) == 0;   // L2 rows must be 16-byte multiples for its tensor map
+  if ((st = make_map(&tb, code_type(), 1, rq, K, N, K, kBKBytes, pair ? 128 : 256)) != W8A8_OK) return st;
+  EpiParams ep{};
+  ep.s_row = sx;
+  ep.s_col = r_scale;
+  ep.s_col_axis = 0;
+  ep.bias = static_cast<const __nv_bfloat16*>(bias);
+  ep.y = static_cast<__nv_bfloat16*>(y);
+  ep.ldy = N;
+  ep.lr_t = t;
+  ep.lr_l2 = static_cast<const __nv_bfloat16*>(l2);
+  ep.r = r;
+  if (pair) {
+    // T [M, r] and L2 [r, N] tiles for the tensor-core low-rank product:
+    // 64 bf16 (128 bytes) wide, r zero-padded by the copy
+    alignas(64) CUtensorMap tt, tl2;
+    if ((st = make_map(&tt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, t, r, M, static_cast<int64_t>(r) * 2, 64, kBM)) !=
+        W8A8_OK)
+      return st;
+    if ((st = make_map(&tl2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, l2, N, r, N * 2, 64, 32)) != W8A8_OK) return st;
+    return launch_gemm_pair<kKind, false, true>(ta, tb, M, N, K, ep, s, &tt, &tl2);
+  }
+  return launch_gemm<kKind, false, 256, kEpiLowRank>(ta, tb, M, N, K, ep, s);
+}
+
 extern "C" {
 
 const char* w8a8_last_error(void) { return t_last_error.c_str(); }
@@ -833,85 +920,13 @@ w8a8_status w8a8_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, w
 w8a8_status svdq_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, const void* rq, const float* r_scale,
                             int r, const void* l1, const void* l2, const void* bias, void* y, void* ws,
                             size_t ws_bytes, w8a8_stream_t stream) {
-  W8A8_CHECK(M >= 0 && N >= 1 && M < (1ll << 31) && N < (1ll << 31), W8A8_ERR_UNSUPPORTED_SHAPE, "bad M/N");
-  w8a8_status st = check_k(K, "K");
-  if (st != W8A8_OK) return st;
-  W8A8_CHECK(r >= 8 && r <= 32 && r % 8 == 0, W8A8_ERR_UNSUPPORTED_SHAPE, "rank r must be 8, 16, 24 or 32");
-  if (M == 0) return W8A8_OK;
-  W8A8_CHECK(x && rq && r_scale && l1 && l2 && y, W8A8_ERR_INVALID_ARG, "null pointer");
-  W8A8_CHECK(aligned16(x) && aligned16(rq) && aligned16(r_scale) && aligned16(l1) && aligned16(l2) && aligned16(y) &&
-                 (bias == nullptr || aligned16(bias)),
-             W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
-  W8A8_CHECK(ws != nullptr && ws_bytes >= ws_svdq(M, K, r), W8A8_ERR_WORKSPACE,
-             "workspace too small: need %zu bytes", ws_svdq(M, K, r));
-  W8A8_CHECK(aligned16(ws), W8A8_ERR_MISALIGNED, "workspace must be 16-byte aligned");
-  if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  Carve c(ws);
-  void* xq = c.take(static_cast<size_t>(M * K));
-  float* sx = static_cast<float*>(c.take(static_cast<size_t>(M) * 4));
-  auto* t = static_cast<__nv_bfloat16*>(c.take(static_cast<size_t>(M) * r * 2));
-  const int tsplit = t_splits(M, K);
-  SplitWs tsk;
-  if (tsplit > 1) {
-    tsk.splits = tsplit;
-    tsk.partial = static_cast<uint32_t*>(
-        c.take(static_cast<size_t>(tsplit) * static_cast<size_t>(M) * static_cast<size_t>(r) * 4));
-  }
-  if ((st = launch_quantize_rows(x, K, M, K, W8A8_INT8, xq, K, sx, s)) != W8A8_OK) return st;
-  // T = bf16(X L1): bf16 tensor-core GEMM, L1 [K, r] read MN-major; split
-  // along K when the rows make few tiles (fp32 partial sums, added in split
-  // order, then one bf16 rounding).
-  {
-    alignas(64) CUtensorMap ta, tb;
-    if ((st = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, K, M, K * 2, 64, kBM)) != W8A8_OK) return st;
-    if ((st = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, l1, r, K, static_cast<int64_t>(r) * 2, 64, 64)) !=
-        W8A8_OK)
-      return st;
-    EpiParams ep{};
-    ep.y = t;
-    ep.ldy = r;
-    ep.splits = tsk.splits;
-    ep.partial = tsk.partial;
-    if ((st = launch_gemm<kKindBF16, true, 64, kEpiPlain>(ta, tb, M, r, K, ep, s)) != W8A8_OK) return st;
-    if (tsk.splits > 1) {
-      int sms = 0;
-      if ((st = current_device(nullptr, &sms)) != W8A8_OK) return st;
-      int64_t grid = (M * (r / 8) + 255) / 256;
-      if (grid > 8 * static_cast<int64_t>(sms)) grid = 8 * static_cast<int64_t>(sms);
-      const uint32_t* part = tsk.partial;
-      const cudaError_t e = launch_pdl(splitk_epilogue_kernel<kKindBF16>, dim3(static_cast<unsigned>(grid)), dim3(256), 0,
-                                       s, part, tsk.splits, M, static_cast<int64_t>(r), static_cast<const float*>(nullptr),
-                                       static_cast<const float*>(nullptr), 0, static_cast<const __nv_bfloat16*>(nullptr),
-                                       t);
-      if (e != cudaSuccess) return cuda_fail(e, "split-K epilogue launch");
-    }
-  }
-  alignas(64) CUtensorMap ta, tb;
-  if ((st = make_map(&ta, code_type(), 1, xq, K, M, K, kBKBytes, kBM)) != W8A8_OK) return st;
-  const bool pair = M >= kPairMinRows && (N % 8) == 0;   // L2 rows must be 16-byte multiples for its tensor map
-  if ((st = make_map(&tb, code_type(), 1, rq, K, N, K, kBKBytes, pair ? 128 : 256)) != W8A8_OK) return st;
-  EpiParams ep{};
-  ep.s_row = sx;
-  ep.s_col = r_scale;
-  ep.s_col_axis = 0;
-  ep.bias = static_cast<const __nv_bfloat16*>(bias);
-  ep.y = static_cast<__nv_bfloat16*>(y);
-  ep.ldy = N;
-  ep.lr_t = t;
-  ep.lr_l2 = static_cast<const __nv_bfloat16*>(l2);
-  ep.r = r;
-  if (pair) {
-    // T [M, r] and L2 [r, N] tiles for the tensor-core low-rank product:
-    // 64 bf16 (128 bytes) wide, r zero-padded by the copy
-    alignas(64) CUtensorMap tt, tl2;
-    if ((st = make_map(&tt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, t, r, M, static_cast<int64_t>(r) * 2, 64, kBM)) !=
-        W8A8_OK)
-      return st;
-    if ((st = make_map(&tl2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, l2, N, r, N * 2, 64, 32)) != W8A8_OK) return st;
-    return launch_gemm_pair<kKindI8, false, true>(ta, tb, M, N, K, ep, s, &tt, &tl2);
-  }
-  return launch_gemm<kKindI8, false, 256, kEpiLowRank>(ta, tb, M, N, K, ep, s);
+  return svdq_fwd_impl<W8A8_INT8>(x, M, N, K, rq, r_scale, r, l1, l2, bias, y, ws, ws_bytes, stream);
+}
+
+w8a8_status svdq_linear_fwd_e4m3(const void* x, int64_t M, int64_t N, int64_t K, const void* rq,
+                                 const float* r_scale, int r, const void* l1, const void* l2, const void* bias,
+                                 void* y, void* ws, size_t ws_bytes, w8a8_stream_t stream) {
+  return svdq_fwd_impl<W8A8_E4M3>(x, M, N, K, rq, r_scale, r, l1, l2, bias, y, ws, ws_bytes, stream);
 }
 
 w8a8_status w8a8_device_status(w8a8_stream_t stream, int reset) {
