@@ -11,6 +11,8 @@ composes those steps in the order the pages give them:
 
 * OneTrainer wiki "Quantization", int W8A8 / float W8A8 paragraphs: weights
   quantized tensor-wise, activations token-wise, the Linear matmul in 8 bits.
+* OneTrainer wiki "Quantization", float8 and GGUF paragraphs (weight-only):
+  the weight dequantized to the train data type (bf16), then a bf16 Linear.
 * OneTrainer wiki "Quantization", GGUF A8 int / GGUF A8 float paragraphs:
   GGUF weights re-quantized axis-wise to int8 / to float8 (e4m3).
 * bitsandbytes #1401 "LLM.int8() Refactoring: Part 1", Enhancements: the fused
@@ -80,6 +82,9 @@ def _declare(L):
         "orc_q8_0_dequantize_f32": [_P, _P, _I64, _P],
         "orc_q8_0_to_axis_int8": [_P, _I64, _I64, _P, _P],
         "orc_q8_0_to_axis": [_P, _I64, _I64, ctypes.c_int, _P, _P],
+        "orc_dequant_e4m3_bf16": [_P, _I64, ctypes.c_float, _P],
+        "orc_q8_0_dequantize_bf16": [_P, _I64, _P],
+        "orc_linear_bf16": [_P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P],
         "orc_gemm_i8_nt": [_P, _P, _I64, _I64, _I64, _P],
         "orc_gemm_i8_nn": [_P, _P, _I64, _I64, _I64, _P],
         "orc_gemm_e4m3_nt": [_P, _P, _I64, _I64, _I64, _P, _P],
@@ -382,3 +387,46 @@ def svdq_linear_fwd(x_bf16, rq, s_r, l1_bf16, l2_bf16, bias=None, qt=INT8):
     base.update({"t": t, "t64": t64, "lr": lr, "lr_abs": lr_abs,
                  "y32": y32, "y": f32_to_bf16(y32), "y32_int": base["y32"]})
     return base
+
+
+# --------------------------------------------------------------------------- weight-only types
+def dequant_e4m3_bf16(q, s):
+    """Weight-only float8: bf16 bits of dec(q) * s (fp32 RN product)."""
+    q = _c(q, np.uint8)
+    w = np.empty(q.shape, np.uint16)
+    lib().orc_dequant_e4m3_bf16(_ptr(q), q.size, float(np.float32(_c(s, np.float32).reshape(-1)[0])), _ptr(w))
+    return w
+
+
+def q8_0_dequantize_bf16(blocks, n):
+    """GGUF to the train data type: bf16 bits of f16(d) * q, n values."""
+    b = _c(blocks, np.uint8)
+    w = np.empty((n,), np.uint16)
+    lib().orc_q8_0_dequantize_bf16(_ptr(b), n, _ptr(w))
+    return w
+
+
+def linear_bf16(x_bf16, w_bf16, bias=None):
+    """bf16 Linear: returns dict(y bf16 bits, y32, acc fp64, absacc)."""
+    x = _c(x_bf16, np.uint16)
+    w = _c(w_bf16, np.uint16)
+    M, K = x.shape
+    N = w.shape[0]
+    b = None if bias is None else _c(bias, np.uint16)
+    acc = np.empty((M, N), np.float64)
+    absacc = np.empty((M, N), np.float64)
+    y32 = np.empty((M, N), np.float32)
+    y = np.empty((M, N), np.uint16)
+    lib().orc_linear_bf16(_ptr(x), _ptr(w), M, N, K, _ptr(b), _ptr(acc), _ptr(absacc), _ptr(y32), _ptr(y))
+    return {"y": y, "y32": y32, "acc": acc, "absacc": absacc}
+
+
+def float8_linear_fwd(x_bf16, wq, s_w, bias=None):
+    """Weight-only float8 forward: W = bf16(dec(Wq) s_w), then the bf16 Linear."""
+    wq = _c(wq, np.uint8)
+    return linear_bf16(x_bf16, dequant_e4m3_bf16(wq, s_w).reshape(wq.shape), bias)
+
+
+def gguf_linear_fwd(x_bf16, blocks, N, K, bias=None):
+    """GGUF (weight-only) forward: W = bf16(f16(d) q) [N, K], then the bf16 Linear."""
+    return linear_bf16(x_bf16, q8_0_dequantize_bf16(blocks, N * K).reshape(N, K), bias)

@@ -276,6 +276,51 @@ void orc_q8_0_to_axis_int8(const uint8_t* blocks, int64_t N, int64_t K,
 }
 
 /* ========================================================================== */
+/* Weight-only types [OT-WIKI float8: "Tensor-wise quantization of weights in */
+/* float8 e4m3. Dequantized to your Train Data Type"; GGUF: "dequantized to   */
+/* Train Data Type"]: the weight becomes bf16, then a bf16 Linear.            */
+/* ========================================================================== */
+
+/* w = bf16(dec(q) * s): the e4m3 value times the tensor-wise scale, one fp32
+ * RN product, then bf16 RNE. */
+void orc_dequant_e4m3_bf16(const uint8_t* q, int64_t n, float s, uint16_t* w) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) w[i] = orc_f32_to_bf16(orc_e4m3_to_f32(q[i]) * s);
+}
+
+/* w = bf16(f16(d) * q): the exact GGUF value, then bf16 RNE. */
+void orc_q8_0_dequantize_bf16(const uint8_t* blocks, int64_t n, uint16_t* w) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) {
+    const uint8_t* blk = blocks + (i / Q80_BLOCK) * Q80_BYTES;
+    w[i] = orc_f32_to_bf16(block_scale_f16(blk) * (float)(int8_t)blk[2 + i % Q80_BLOCK]);
+  }
+}
+
+/* The bf16 Linear: acc[m,n] = sum_k x[m,k] w[n,k] in fp64 (bf16 products are
+ * exact), absacc = sum |x w|; y32 = fp32(acc) (+ bias as one fp32 RN add),
+ * y = bf16(y32). */
+void orc_linear_bf16(const uint16_t* x, const uint16_t* w, int64_t M, int64_t N, int64_t K,
+                     const uint16_t* bias, double* acc, double* absacc, float* y32, uint16_t* y) {
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t n = 0; n < N; ++n) {
+      double sum = 0.0, asum = 0.0;
+      for (int64_t k = 0; k < K; ++k) {
+        double p = (double)orc_bf16_to_f32(x[m * K + k]) * (double)orc_bf16_to_f32(w[n * K + k]);
+        sum += p;
+        asum += fabs(p);
+      }
+      acc[m * N + n] = sum;
+      absacc[m * N + n] = asum;
+      float v = (float)sum;
+      if (bias) v = v + orc_bf16_to_f32(bias[n]);
+      y32[m * N + n] = v;
+      y[m * N + n] = orc_f32_to_bf16(v);
+    }
+}
+
+/* ========================================================================== */
 /* 8-bit matrix products [OT-PR "8bit matrix multiplications"; OT-WIKI        */
 /* "matrix multiplications are performed in int8 / float8"]                   */
 /* ========================================================================== */

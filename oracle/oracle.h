@@ -78,6 +78,16 @@ void orc_q8_0_to_axis(const uint8_t* blocks, int64_t N, int64_t K, int qt,
 void orc_q8_0_to_axis_int8(const uint8_t* blocks, int64_t N, int64_t K,
                            int8_t* q, float* s);
 
+/* ---- weight-only types [OT-WIKI float8, GGUF] ---------------------------- */
+/* w = bf16(e4m3_value(q) * s) for n codes (tensor-wise scale s). */
+void orc_dequant_e4m3_bf16(const uint8_t* q, int64_t n, float s, uint16_t* w);
+/* w = bf16(f16(d) * q) for the first n values of the blocks. */
+void orc_q8_0_dequantize_bf16(const uint8_t* blocks, int64_t n, uint16_t* w);
+/* bf16 Linear: acc = sum x w (fp64), absacc = sum |x w|, y32 = fp32(acc)
+ * (+ bias, fp32 RN), y = bf16(y32).  x [M,K], w [N,K], bias [N] or NULL. */
+void orc_linear_bf16(const uint16_t* x, const uint16_t* w, int64_t M, int64_t N, int64_t K,
+                     const uint16_t* bias, double* acc, double* absacc, float* y32, uint16_t* y);
+
 /* ---- 8-bit matrix products ------------------------------------------------ */
 /* acc[m,n] = sum_k A[m,k] * B[n,k] in int64; returns 0, or 1 if any sum
  * leaves the int32 range (then acc holds the truncated values). */

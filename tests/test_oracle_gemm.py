@@ -287,3 +287,73 @@ def test_svdq_split_reduces_weight_error_e4m3(orc):
     wq, sw = orc.quantize_weight(wu, orc.E4M3, orc.TENSOR)
     err_plain = np.linalg.norm(W - orc.decode_codes(wq, orc.E4M3).astype(np.float64) * sw[0])
     assert err_svd < 0.5 * err_plain, (err_svd, err_plain)
+
+
+# --------------------------------------------------------------------------- weight-only types
+@pytest.mark.parametrize("s", [1.0, 0.02 / 448, 3.1e-5, 7.77])
+def test_dequant_e4m3_bf16_vs_torch(orc, s):
+    """Every e4m3 code (NaN codes excluded) times a scale, through torch's
+    float8 -> fp32 cast, one fp32 product and torch's bf16 cast."""
+    q = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    s32 = np.float32(s)
+    got = orc.dequant_e4m3_bf16(q, np.array([s32]))
+    t = torch.from_numpy(q).view(torch.float8_e4m3fn).to(torch.float32) * torch.tensor(s32)
+    assert np.array_equal(got, workloads.to_u16(t.to(torch.bfloat16)))
+
+
+def test_q8_0_dequantize_bf16_vs_torch(orc):
+    """GGUF values f16(d) * q through torch (f16 -> fp32 cast, exact product),
+    then torch's bf16 cast; 77 values end in a short block."""
+    blocks = workloads.raw_q8_0_blocks(4, 96, seed=31).numpy()
+    n = 4 * 96 - 19
+    got = orc.q8_0_dequantize_bf16(blocks, n)
+    b = blocks.reshape(-1, 34)
+    d = torch.from_numpy(np.ascontiguousarray(b[:, :2]).view(np.float16).reshape(-1)).to(torch.float32)
+    q = torch.from_numpy(b[:, 2:].view(np.int8).astype(np.float32))
+    want = (q * d[:, None]).reshape(-1)[:n].to(torch.bfloat16)
+    assert np.array_equal(got, workloads.to_u16(want))
+
+
+def test_linear_bf16_vs_numpy_and_textbook(orc):
+    x = workloads.normal((7, 96), 1.0, 32)
+    w = workloads.normal((13, 96), 0.05, 33)
+    bias = workloads.normal((13,), 0.1, 34)
+    r = orc.linear_bf16(workloads.to_u16(x), workloads.to_u16(w), workloads.to_u16(bias))
+    ref = x.double().numpy() @ w.double().numpy().T
+    assert np.allclose(r["acc"], ref, rtol=1e-13, atol=1e-15)
+    assert np.allclose(r["absacc"], np.abs(x.double().numpy()) @ np.abs(w.double().numpy()).T, rtol=1e-13)
+    y32 = ref.astype(np.float32) + bias.float().numpy()
+    assert np.array_equal(r["y32"], y32.astype(np.float32))
+    assert np.array_equal(r["y"], workloads.to_u16(torch.from_numpy(y32).to(torch.bfloat16)))
+    # integer operands: the textbook integer matmul, exactly (non-square: a
+    # transposed operand cannot pass)
+    g = np.random.default_rng(35)
+    xi = g.integers(-8, 9, size=(5, 64)).astype(np.float32)
+    wi = g.integers(-8, 9, size=(9, 64)).astype(np.float32)
+    to = lambda a: workloads.to_u16(torch.from_numpy(a).to(torch.bfloat16))
+    ri = orc.linear_bf16(to(xi), to(wi))
+    assert np.array_equal(ri["acc"], (xi.astype(np.int64) @ wi.astype(np.int64).T).astype(np.float64))
+
+
+def test_weight_only_forwards_compose(orc):
+    """float8: quantize W tensor-wise to e4m3, dequantize to bf16, bf16 Linear;
+    GGUF: the same through Q8_0 blocks.  Both stay close to the bf16 Linear
+    on W itself (the quantization error bound of each format)."""
+    x = workloads.normal((6, 128), 1.0, 36)
+    w = workloads.normal((24, 128), 0.02, 37)
+    xu, wu = workloads.to_u16(x), workloads.to_u16(w)
+    base = orc.linear_bf16(xu, wu)["acc"]
+    wq, sw = orc.quantize_weight(wu, orc.E4M3, orc.TENSOR)
+    f8 = orc.float8_linear_fwd(xu, wq, sw)
+    assert np.array_equal(f8["y"], orc.linear_bf16(xu, orc.dequant_e4m3_bf16(wq, sw).reshape(24, 128))["y"])
+    absx = np.abs(x.double().numpy()) @ np.abs(w.double().numpy()).T
+    assert np.all(np.abs(f8["acc"] - base) <= 2 ** -4 * absx + 2 ** -9 * float(sw[0]) * np.abs(x.double().numpy()).sum(1)[:, None] + 2 ** -8 * absx)
+    blocks, s32 = orc.q8_0_quantize(w.float().numpy().reshape(-1))
+    gg = orc.gguf_linear_fwd(xu, blocks, 24, 128)
+    assert np.array_equal(gg["y"], orc.linear_bf16(xu, orc.q8_0_dequantize_bf16(blocks, 24 * 128).reshape(24, 128))["y"])
+    # per weight: half a code step of the f32 block scale, the f16 rounding of
+    # that scale (127 codes x 2^-11 relative), then one bf16 rounding
+    sb = np.repeat(s32.astype(np.float64), 32).reshape(24, 128)
+    ew = sb * (0.5 * (1 + 2 ** -20) + 127 * 2 ** -11)
+    ew = ew + 2 ** -8 * (np.abs(w.double().numpy()) + ew)
+    assert np.all(np.abs(gg["acc"] - base) <= np.abs(x.double().numpy()) @ ew.T)

@@ -44,6 +44,8 @@ PINS = [
     G.test_lowrank_vs_numpy, G.test_svdq_zero_factors_is_float_linear,
     lambda o: G.test_svdq_zero_residual_is_lowrank_product(o, 0),
     lambda o: G.test_svdq_zero_residual_is_lowrank_product(o, 1),
+    lambda o: G.test_dequant_e4m3_bf16_vs_torch(o, 3.1e-5), G.test_q8_0_dequantize_bf16_vs_torch,
+    G.test_linear_bf16_vs_numpy_and_textbook, G.test_weight_only_forwards_compose,
 ]
 
 # (name, text in oracle.c, replacement)
@@ -96,6 +98,12 @@ MUTANTS = [
      "double u = acc[m * N + n] * (double)s_row[m];"),
     ("e4m3 gemm sign", "sum += p;\n        asum += fabs(p);\n      }\n      acc[m * N + n] = sum;",
      "sum += fabs(p);\n        asum += fabs(p);\n      }\n      acc[m * N + n] = sum;"),
+    ("float8 dequant drops scale", "w[i] = orc_f32_to_bf16(orc_e4m3_to_f32(q[i]) * s);",
+     "w[i] = orc_f32_to_bf16(orc_e4m3_to_f32(q[i]));"),
+    ("gguf bf16 code offset", "w[i] = orc_f32_to_bf16(block_scale_f16(blk) * (float)(int8_t)blk[2 + i % Q80_BLOCK]);",
+     "w[i] = orc_f32_to_bf16(block_scale_f16(blk) * (float)(int8_t)blk[1 + i % Q80_BLOCK]);"),
+    ("bf16 linear transposed w", "(double)orc_bf16_to_f32(w[n * K + k]);", "(double)orc_bf16_to_f32(w[k * N + n]);"),
+    ("bf16 linear drops bias", "if (bias) v = v + orc_bf16_to_f32(bias[n]);", ""),
     ("lowrank L1 transposed", "(double)orc_bf16_to_f32(l1[k * r + j])", "(double)orc_bf16_to_f32(l1[j * K + k])"),
     ("lowrank up drops a term", "for (int64_t j = 0; j < r; ++j) {\n        double p", "for (int64_t j = 1; j < r; ++j) {\n        double p"),
 ]
