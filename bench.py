@@ -731,6 +731,41 @@ def extras(w8, torch, workloads, dev, peaks, src):
                          "weight_GB/s": MLP * HID / (ms * 1e-3) / 1e9}
         del sets
     out["gguf_a8_float_fwd_sweep_N12288_K3072"] = sweep
+    # weight-only types (float8, GGUF) on the DiT up-projection: the weight
+    # dequantized to bf16 in the workspace, then the bf16 Linear
+    tcb = peaks["bf16_tflops"]
+    xb0 = workloads.normal((M_TOK, HID), 1.0, 5).to(dev)
+    wb0 = g["w_f32"].to(torch.bfloat16).to(dev)
+    wq8, sw8 = w8.quantize_weight(wb0, "e4m3", "tensor")
+    wgg = w8.q8_0_quantize(g["w_f32"].reshape(-1).to(dev))
+    ops = 2 * M_TOK * MLP * HID
+    wsz = w8.workspace_bytes(w8.OP_WEIGHT_ONLY_FWD, M_TOK, MLP, HID)
+    res = {}
+    for name, mk in (("bf16_gemm", lambda xx, ws: (lambda: w8.bf16_linear_fwd(xx, wb0, ws=ws))),
+                     ("float8", lambda xx, ws: (lambda: w8.float8_linear_fwd(xx, wq8, sw8, ws=ws))),
+                     ("gguf", lambda xx, ws: (lambda: w8.gguf_linear_fwd(xx, wgg, MLP, ws=ws)))):
+        sets = []
+        for i in range(_nsets(nbytes(xb0) + M_TOK * MLP * 2)):
+            sets.append(mk(xb0.clone(), torch.empty(max(wsz, 16), dtype=torch.uint8, device=dev)))
+        ms = _time_rot(sets, 20, torch, stream)
+        res[name] = {"ms": ms, "TFLOPS": ops / ms / 1e9, "frac_bf16_burst": ops / ms / 1e9 / tcb}
+        del sets
+    out["weight_only_fwd_4608x12288x3072"] = res
+    # the two dequantizations alone (12288 x 3072 weight -> bf16)
+    sets_e, sets_g = [], []
+    for i in range(_nsets(MLP * HID * 3)):
+        wq, blk = wq8.clone(), wgg.clone()
+        ye = torch.empty((MLP, HID), dtype=torch.bfloat16, device=dev)
+        yg = torch.empty(MLP * HID, dtype=torch.bfloat16, device=dev)
+        sets_e.append(lambda wq=wq, ye=ye: w8.dequantize_e4m3_bf16(wq, sw8, out=ye))
+        sets_g.append(lambda blk=blk, yg=yg: w8.q8_0_dequantize_bf16(blk, MLP * HID, out=yg))
+    ms = _time_rot(sets_e, 30, torch, stream)
+    gbs = MLP * HID * 3 / (ms * 1e-3) / 1e9
+    out["dequantize_e4m3_bf16_12288x3072"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
+    ms = _time_rot(sets_g, 30, torch, stream)
+    gbs = (wgg.numel() + MLP * HID * 2) / (ms * 1e-3) / 1e9
+    out["q8_0_dequantize_bf16_12288x3072"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
+    del sets_e, sets_g, xb0, wb0
     out["peaks"] = {"source": src, "hbm_gbs": hbm, "int8_burst_tops": tc8}
     out["method"] = ("mean over reps replayed from one CUDA graph (no host launch cost), rotating through "
                      ">= 3x L2 of input/output copies")

@@ -67,7 +67,9 @@ typedef enum {
   W8A8_OP_LINEAR_FWD = 0,      /* w8a8_linear_fwd                          */
   W8A8_OP_LINEAR_DGRAD = 1,    /* w8a8_linear_dgrad                        */
   W8A8_OP_SVDQ_FWD = 2,        /* svdq_linear_fwd                          */
-  W8A8_OP_QUANTIZE_WEIGHT = 3  /* w8a8_quantize_weight (TENSOR needs 256 B) */
+  W8A8_OP_QUANTIZE_WEIGHT = 3, /* w8a8_quantize_weight (TENSOR needs 256 B) */
+  W8A8_OP_BF16_FWD = 4,        /* bf16_linear_fwd                          */
+  W8A8_OP_WEIGHT_ONLY_FWD = 5  /* float8_linear_fwd, gguf_linear_fwd        */
 } w8a8_op;
 
 /* ------------------------------------------------------------------------
@@ -116,6 +118,10 @@ w8a8_status w8a8_quantize_weight(const void* w_bf16, int64_t N, int64_t K, w8a8_
 size_t q8_0_bytes(int64_t n);
 w8a8_status q8_0_quantize(const float* x, int64_t n, void* blocks, w8a8_stream_t stream);
 w8a8_status q8_0_dequantize(const void* blocks, int64_t n, float* y, w8a8_stream_t stream);
+/* GGUF dequantized to bf16 (OneTrainer wiki, GGUF: weights dequantized to the
+ * train data type): y[i] = bf16_rne(f16(d) * q), the product exact in fp32.
+ * n >= 0 values (any n; the last block may be short).  y_bf16 [n]. */
+w8a8_status q8_0_dequantize_bf16(const void* blocks, int64_t n, void* y_bf16, w8a8_stream_t stream);
 
 /* Re-quantize a Q8_0 weight to axis-wise int8 (OneTrainer wiki, GGUF A8 int:
  * weights re-quantized from GGUF to int8 axis-wise).  Row n of W[N,K] is the
@@ -136,6 +142,39 @@ w8a8_status q8_0_to_axis_int8(const void* blocks, int64_t N, int64_t K, int8_t* 
  * w8a8_linear_fwd with W8A8_E4M3 and W8A8_AXIS. */
 w8a8_status q8_0_to_axis_e4m3(const void* blocks, int64_t N, int64_t K, uint8_t* q_out,
                               float* scale, w8a8_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Weight-only types (OneTrainer wiki, "float8": tensor-wise e4m3 weights, and
+ * "GGUF"; both dequantized to the train data type during training).  The
+ * weight stays 8-bit in memory; each forward dequantizes it to bf16 in the
+ * workspace and runs a bf16 Linear on the tensor cores:
+ *     y = bf16( fp32(sum_k x[m,k] W[n,k]) (+ bias[n]) )
+ * with fp32 sums (kind::f16 MMAs; split along K, partial sums added in split
+ * order, when the output makes few tiles) and one fp32 RN bias add.
+ * Shapes and alignment as w8a8_linear_fwd (K >= 16, K % 16 == 0, 16-byte
+ * aligned pointers); M == 0 is a no-op.
+ * ---------------------------------------------------------------------- */
+/* e4m3 codes -> bf16(value * scale[0]), n % 16 == 0.  w_bf16 [n]. */
+w8a8_status w8a8_dequantize_e4m3_bf16(const void* q, int64_t n, const float* scale, void* w_bf16,
+                                      w8a8_stream_t stream);
+/* The bf16 Linear alone: x [M, K], w [N, K], bias [N] or NULL, y [M, N], all
+ * bf16.  ws: w8a8_workspace_bytes(W8A8_OP_BF16_FWD, M, N, K, 0) bytes (0 when
+ * the product is not split; ws may then be NULL). */
+w8a8_status bf16_linear_fwd(const void* x_bf16, int64_t M, int64_t N, int64_t K, const void* w_bf16,
+                            const void* bias_bf16, void* y_bf16, void* ws, size_t ws_bytes,
+                            w8a8_stream_t stream);
+/* float8: wq [N, K] e4m3 codes with tensor-wise w_scale [1] (as
+ * w8a8_quantize_weight with W8A8_E4M3, W8A8_TENSOR).  W = bf16(dec(wq) *
+ * w_scale[0]).  ws: w8a8_workspace_bytes(W8A8_OP_WEIGHT_ONLY_FWD, M, N, K, 0)
+ * bytes; holds W [N, K] bf16, then the split partial sums. */
+w8a8_status float8_linear_fwd(const void* x_bf16, int64_t M, int64_t N, int64_t K, const void* wq,
+                              const float* w_scale, const void* bias_bf16, void* y_bf16, void* ws,
+                              size_t ws_bytes, w8a8_stream_t stream);
+/* GGUF: the weight as Q8_0 blocks over its N*K values in row-major order.
+ * W = bf16(f16(d) * q).  ws as float8_linear_fwd. */
+w8a8_status gguf_linear_fwd(const void* x_bf16, int64_t M, int64_t N, int64_t K, const void* blocks,
+                            const void* bias_bf16, void* y_bf16, void* ws, size_t ws_bytes,
+                            w8a8_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * W8A8 Linear forward (OneTrainer wiki, int/float W8A8): quantize X

@@ -69,6 +69,12 @@ def test_sizes(L):
     # output width not a multiple of 8: never split
     assert L.w8a8_workspace_bytes(0, 1, 1001, 4096, 0) == 4096 + 256
     assert L.w8a8_workspace_bytes(9, 1, 1, 16, 0) == 0
+    # bf16 Linear: nothing unless split (M = 1, N = 12288: 48 tiles -> 3 splits)
+    assert L.w8a8_workspace_bytes(4, 4608, 12288, 3072, 0) == 0
+    assert L.w8a8_workspace_bytes(4, 1, 12288, 3072, 0) == 3 * 12288 * 4
+    # weight-only: the bf16 weight, then the partial sums
+    assert L.w8a8_workspace_bytes(5, 4608, 12288, 3072, 0) == 12288 * 3072 * 2
+    assert L.w8a8_workspace_bytes(5, 1, 12288, 3072, 0) == 12288 * 3072 * 2 + 3 * 12288 * 4
 
 
 A = ctypes.c_void_p(1 << 20)        # a 16-byte aligned stand-in pointer (never dereferenced)
@@ -112,6 +118,21 @@ def test_svdq_validation(L):
     assert L.svdq_linear_fwd_e4m3(A, 8, 8, 32, A, A, 32, None, A, None, A, A, 1 << 20, None) == 1
     assert L.svdq_linear_fwd_e4m3(A, 8, 8, 32, A, A, 32, A, A, None, A, A, 64, None) == 4
     assert L.svdq_linear_fwd_e4m3(A, 0, 8, 32, A, A, 32, A, A, None, A, A, 0, None) == 0      # M = 0: no-op
+
+
+def test_weight_only_validation(L):
+    assert L.bf16_linear_fwd(A, 8, 8, 20, A, None, A, A, 1 << 20, None) == 2        # K % 16
+    assert L.bf16_linear_fwd(A, 0, 8, 32, None, None, None, None, 0, None) == 0     # M = 0: no-op
+    assert L.bf16_linear_fwd(A, 8, 8, 32, None, None, A, A, 1 << 20, None) == 1
+    assert L.bf16_linear_fwd(B, 8, 8, 32, A, None, A, A, 1 << 20, None) == 3
+    assert L.bf16_linear_fwd(A, 1, 12288, 3072, A, None, A, None, 0, None) == 4     # split needs a workspace
+    assert L.float8_linear_fwd(A, 8, 8, 32, A, A, None, A, A, 64, None) == 4        # the bf16 weight needs room
+    assert L.float8_linear_fwd(A, 8, 8, 32, A, None, None, A, A, 1 << 20, None) == 1
+    assert L.gguf_linear_fwd(A, 8, 8, 32, A, None, A, A, 64, None) == 4
+    assert L.gguf_linear_fwd(A, 8, 8, 24, A, None, A, A, 1 << 20, None) == 2
+    assert L.w8a8_dequantize_e4m3_bf16(A, 24, A, A, None) == 2                      # n % 16
+    assert L.w8a8_dequantize_e4m3_bf16(A, 32, None, A, None) == 1
+    assert L.q8_0_dequantize_bf16(A, 3, B, None) == 3
 
 
 def test_q8_0_validation(L):

@@ -142,3 +142,28 @@ def test_gguf_a8_float_requant_and_forward_sweep(w8, orc):
         ref["sw"] = swr[None, :]
         err, bound = _fp8_tol(ref, u16(y)[rows])
         assert np.all(err <= bound), (M, float((err / bound).max()))
+
+
+@pytest.mark.parametrize("kind", ["float8", "gguf"])
+def test_weight_only_dit_up_sampled(w8, orc, kind):
+    """The weight-only types on the DiT up-projection (X [4608, 3072], W
+    [12288, 3072]): the whole product on the GPU, sampled rows by the oracle."""
+    from test_parity_gpu import _bf16_tol
+    d = workloads.gguf_q8_0(M=4608)
+    w32 = d["w_f32"]
+    N, K = w32.shape
+    x = d["x"]
+    rows = sample_rows(4608, n=24, seed=5)
+    if kind == "float8":
+        wb = w32.to(torch.bfloat16)
+        wq, sw = w8.quantize_weight(wb.to(DEV), "e4m3", "tensor")
+        y = w8.float8_linear_fwd(x.to(DEV), wq, sw)
+        wqr, swr = orc.quantize_weight(workloads.to_u16(wb), 1, 0)
+        assert np.array_equal(u8(wq), wqr)
+        ref = orc.float8_linear_fwd(workloads.to_u16(x)[rows], wqr, swr)
+    else:
+        br, _ = orc.q8_0_quantize(w32.numpy().reshape(-1))
+        y = w8.gguf_linear_fwd(x.to(DEV), torch.from_numpy(br).to(DEV), N)
+        ref = orc.gguf_linear_fwd(workloads.to_u16(x)[rows], br, N, K)
+    err, bound = _bf16_tol(ref, u16(y)[rows], K)
+    assert np.all(err <= bound), float((err / bound).max())

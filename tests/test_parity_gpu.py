@@ -497,6 +497,88 @@ def test_svdq_e4m3_zero_factors_equal_float_linear(w8, M):
     assert torch.equal(w8.svdq_linear_fwd(x, wq, sw, l1, l2), w8.linear_fwd(x, wq, sw))
 
 
+# --------------------------------------------------------------------------- weight-only types
+@pytest.mark.parametrize("n,s", [(256, 1.0), (4096 * 16, 0.02 / 448), ((1 << 20) + 48, 3.1e-5)])
+def test_dequantize_e4m3_bf16_parity(w8, orc, n, s):
+    codes = torch.arange(n, dtype=torch.int64).remainder(256).to(torch.uint8)
+    codes[codes == 0x7F] = 0x7E          # no NaN codes: a quantizer never writes them
+    codes[codes == 0xFF] = 0xFE
+    codes = codes[torch.randperm(n, generator=torch.Generator().manual_seed(n))]
+    sc = torch.tensor([s], dtype=torch.float32)
+    w = w8.dequantize_e4m3_bf16(codes.to(DEV).view(torch.float8_e4m3fn), sc.to(DEV))
+    assert np.array_equal(u16(w), orc.dequant_e4m3_bf16(codes.numpy(), sc.numpy()))
+
+
+@pytest.mark.parametrize("n", [77, 4096, (1 << 20) + 3])
+def test_q8_0_dequantize_bf16_parity(w8, orc, n):
+    x = workloads.q8_0_standalone(n, seed=n).numpy()
+    br, _ = orc.q8_0_quantize(x)
+    y = w8.q8_0_dequantize_bf16(torch.from_numpy(br).to(DEV), n)
+    assert np.array_equal(u16(y), orc.q8_0_dequantize_bf16(br, n))
+
+
+def _bf16_tol(ref, y, K):
+    """fp32 sums on the tensor cores: |y - y_ref| <= K 2^-23 sum|x w| + 1 bf16 ulp."""
+    yr = bf16_bits_to_f64(ref["y"])
+    yg = bf16_bits_to_f64(y)
+    bound = K * 2.0 ** -23 * ref["absacc"] + ulp_bf16(np.maximum(np.abs(yr), np.abs(yg)))
+    return np.abs(yg - yr), bound
+
+
+# (600, 520, 512) and (1024, 1024, 1024): the CTA pair; (1, 3072, 4096) and
+# (64, 1024, 3072): split along K; the rest single-SM tiles, ragged edges
+BF16_SHAPES = [(600, 520, 512), (1024, 1024, 1024), (1, 3072, 4096), (64, 1024, 3072), (129, 257, 96),
+               (300, 520, 640), (1, 16, 16), (530, 300, 256)]
+
+
+@pytest.mark.parametrize("M,N,K", BF16_SHAPES)
+def test_bf16_linear_parity(w8, orc, M, N, K):
+    x = workloads.with_outlier_channels((M, K), 1.0, seed=81 + M)
+    w = workloads.normal((N, K), 0.02, seed=82 + N)
+    bias = workloads.normal((N,), 0.01, seed=83)
+    y = w8.bf16_linear_fwd(x.to(DEV), w.to(DEV), bias=bias.to(DEV))
+    ref = orc.linear_bf16(workloads.to_u16(x), workloads.to_u16(w), workloads.to_u16(bias))
+    err, bound = _bf16_tol(ref, u16(y), K)
+    assert np.all(err <= bound), float((err / bound).max())
+
+
+@pytest.mark.parametrize("M,N,K", [(600, 520, 512), (1, 3072, 4096), (129, 257, 96), (64, 1024, 3072)])
+def test_float8_weight_only_parity(w8, orc, M, N, K):
+    x = workloads.normal((M, K), 1.0, seed=84 + M)
+    w = workloads.normal((N, K), 0.02, seed=85 + N)
+    bias = workloads.normal((N,), 0.01, seed=86)
+    wq, sw = w8.quantize_weight(w.to(DEV), "e4m3", "tensor")
+    y = w8.float8_linear_fwd(x.to(DEV), wq, sw, bias=bias.to(DEV))
+    wqr, swr = orc.quantize_weight(workloads.to_u16(w), 1, 0)
+    assert np.array_equal(u8(wq), wqr)
+    ref = orc.float8_linear_fwd(workloads.to_u16(x), wqr, swr, workloads.to_u16(bias))
+    err, bound = _bf16_tol(ref, u16(y), K)
+    assert np.all(err <= bound), float((err / bound).max())
+
+
+@pytest.mark.parametrize("M,N,K", [(600, 520, 512), (1, 3072, 4096), (129, 264, 96), (64, 1024, 3072)])
+def test_gguf_weight_only_parity(w8, orc, M, N, K):
+    d = workloads.gguf_q8_0(N=N, K=K, M=M)
+    br, _ = orc.q8_0_quantize(d["w_f32"].numpy().reshape(-1))
+    bias = workloads.normal((N,), 0.01, seed=87)
+    y = w8.gguf_linear_fwd(d["x"].to(DEV), torch.from_numpy(br).to(DEV), N, bias=bias.to(DEV))
+    ref = orc.gguf_linear_fwd(workloads.to_u16(d["x"]), br, N, K, workloads.to_u16(bias))
+    err, bound = _bf16_tol(ref, u16(y), K)
+    assert np.all(err <= bound), float((err / bound).max())
+
+
+def test_weight_only_m0_and_unsplit_equal_split(w8):
+    x = workloads.normal((64, 3072), 1.0, 88).to(DEV)
+    w = workloads.normal((1024, 3072), 0.02, 89).to(DEV)
+    assert w8.bf16_linear_fwd(x[:0], w).shape == (0, 1024)
+    # one row through the split path equals itself computed within a
+    # larger, unsplit product up to the fp32 summation order
+    y_all = w8.bf16_linear_fwd(torch.cat([x] * 10), w)[:64]
+    y_small = w8.bf16_linear_fwd(x, w)
+    d = (y_all.float() - y_small.float()).abs()
+    assert float(d.max()) <= 2 ** -6 * float(y_all.float().abs().max())
+
+
 # --------------------------------------------------------------------------- diagnostics
 def test_device_status_clean_then_bounded_wait_times_out(w8):
     assert w8.device_status(reset=True) == 0

@@ -24,6 +24,7 @@ LIB_PATH = os.path.join(_PKG, "libw8a8.so")
 INT8, E4M3 = 0, 1
 TENSOR, AXIS = 0, 1
 OP_LINEAR_FWD, OP_LINEAR_DGRAD, OP_SVDQ_FWD, OP_QUANTIZE_WEIGHT = 0, 1, 2, 3
+OP_BF16_FWD, OP_WEIGHT_ONLY_FWD = 4, 5
 
 STATUS = {0: "W8A8_OK", 1: "W8A8_ERR_INVALID_ARG", 2: "W8A8_ERR_UNSUPPORTED_SHAPE",
           3: "W8A8_ERR_MISALIGNED", 4: "W8A8_ERR_WORKSPACE", 5: "W8A8_ERR_CUDA",
@@ -34,7 +35,8 @@ EXPORTS = ("w8a8_quantize_rows", "w8a8_quantize_weight", "q8_0_bytes", "q8_0_qua
            "q8_0_dequantize", "q8_0_to_axis_int8", "q8_0_to_axis_e4m3", "w8a8_linear_fwd", "w8a8_linear_dgrad",
            "svdq_linear_fwd", "svdq_linear_fwd_e4m3", "w8a8_qgemm_fwd", "w8a8_qgemm_dgrad", "w8a8_workspace_bytes",
            "w8a8_device_status", "w8a8_set_wait_limit_ns", "w8a8_selftest_wait",
-           "w8a8_e4m3_encode", "w8a8_last_error", "w8a8_linear_fwd_noalloc")
+           "w8a8_e4m3_encode", "w8a8_last_error", "w8a8_linear_fwd_noalloc", "q8_0_dequantize_bf16",
+           "w8a8_dequantize_e4m3_bf16", "bf16_linear_fwd", "float8_linear_fwd", "gguf_linear_fwd")
 
 
 class W8A8Error(RuntimeError):
@@ -73,6 +75,11 @@ def lib() -> ctypes.CDLL:
             "w8a8_selftest_wait": [_U64, _P],
             "w8a8_e4m3_encode": [_P, _I64, _P, _P],
             "w8a8_linear_fwd_noalloc": [_P, _I64, _I64, _I64, _I, _P, _P, _I, _P, _P, _P],
+            "q8_0_dequantize_bf16": [_P, _I64, _P, _P],
+            "w8a8_dequantize_e4m3_bf16": [_P, _I64, _P, _P, _P],
+            "bf16_linear_fwd": [_P, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P],
+            "float8_linear_fwd": [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _SZ, _P],
+            "gguf_linear_fwd": [_P, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -198,6 +205,27 @@ def q8_0_dequantize(blocks: torch.Tensor, n: int, out=None):
     return y
 
 
+def q8_0_dequantize_bf16(blocks: torch.Tensor, n: int, out=None):
+    """GGUF Q8_0 blocks -> bf16 [n] (f16 scale x code, rounded to bf16)."""
+    if not (blocks.is_cuda and blocks.dtype == torch.uint8 and blocks.is_contiguous()):
+        raise ValueError("blocks must be a contiguous uint8 CUDA tensor")
+    if blocks.numel() < q8_0_bytes(n):
+        raise ValueError("blocks hold fewer than n values")
+    y = torch.empty(n, dtype=torch.bfloat16, device=blocks.device) if out is None else out
+    _check(lib().q8_0_dequantize_bf16(_ptr(blocks), n, _ptr(y), _stream(blocks.device)))
+    return y
+
+
+def dequantize_e4m3_bf16(wq: torch.Tensor, scale: torch.Tensor, out=None):
+    """e4m3 codes (float8_e4m3fn) -> bf16(value * scale[0]), same shape."""
+    if not (wq.is_cuda and wq.dtype == torch.float8_e4m3fn and wq.is_contiguous()):
+        raise ValueError("wq must be a contiguous float8_e4m3fn CUDA tensor")
+    y = torch.empty(wq.shape, dtype=torch.bfloat16, device=wq.device) if out is None else out
+    _check(lib().w8a8_dequantize_e4m3_bf16(_ptr(_as_bytes(wq)), wq.numel(), _ptr(scale), _ptr(y),
+                                           _stream(wq.device)))
+    return y
+
+
 def q8_0_to_axis(blocks: torch.Tensor, N: int, K: int, qt="int8", out=None, scale=None):
     """Q8_0 weight [N, K/32 blocks] -> (codes [N, K], per-row scales [N]):
     int8 codes (GGUF A8 int) or float8_e4m3fn codes (GGUF A8 float)."""
@@ -241,6 +269,52 @@ def linear_fwd(x, wq, w_scale, bias=None, out=None, ws=None):
     ws = _workspace(OP_LINEAR_FWD, M, N, K, 0, x.device, ws)
     _check(lib().w8a8_linear_fwd(_ptr(x), M, N, K, qt, _ptr(_as_bytes(wq)), _ptr(w_scale), g, _ptr(bias),
                                  _ptr(y), _ptr(ws), ws.numel(), _stream(x.device)))
+    return y
+
+
+def bf16_linear_fwd(x, w, bias=None, out=None, ws=None):
+    """Y = bf16(X W^T + bias) on the tensor cores: x [M, K], w [N, K] bf16."""
+    _cuda_2d(x, torch.bfloat16, "x")
+    _cuda_2d(w, torch.bfloat16, "w")
+    M, K = x.shape
+    N = w.shape[0]
+    if w.shape[1] != K:
+        raise ValueError("w must be [N, K]")
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else out
+    ws = _workspace(OP_BF16_FWD, M, N, K, 0, x.device, ws)
+    _check(lib().bf16_linear_fwd(_ptr(x), M, N, K, _ptr(w), _ptr(bias), _ptr(y), _ptr(ws), ws.numel(),
+                                 _stream(x.device)))
+    return y
+
+
+def float8_linear_fwd(x, wq, w_scale, bias=None, out=None, ws=None):
+    """Weight-only float8: W = bf16(dec(wq) * w_scale[0]) [N, K], then the bf16
+    Linear.  wq float8_e4m3fn [N, K] (tensor-wise), w_scale [1]."""
+    _cuda_2d(x, torch.bfloat16, "x")
+    if wq.dtype != torch.float8_e4m3fn or wq.dim() != 2 or wq.shape[1] != x.shape[1]:
+        raise ValueError("wq must be float8_e4m3fn [N, K]")
+    M, K = x.shape
+    N = wq.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else out
+    ws = _workspace(OP_WEIGHT_ONLY_FWD, M, N, K, 0, x.device, ws)
+    _check(lib().float8_linear_fwd(_ptr(x), M, N, K, _ptr(_as_bytes(wq)), _ptr(w_scale), _ptr(bias), _ptr(y),
+                                   _ptr(ws), ws.numel(), _stream(x.device)))
+    return y
+
+
+def gguf_linear_fwd(x, blocks, N, bias=None, out=None, ws=None):
+    """GGUF (weight-only): W = bf16(f16(d) q) from the Q8_0 blocks of the
+    row-major [N, K] weight, then the bf16 Linear."""
+    _cuda_2d(x, torch.bfloat16, "x")
+    M, K = x.shape
+    if not (blocks.is_cuda and blocks.dtype == torch.uint8 and blocks.is_contiguous()):
+        raise ValueError("blocks must be a contiguous uint8 CUDA tensor")
+    if blocks.numel() < q8_0_bytes(N * K):
+        raise ValueError("blocks hold fewer than N*K values")
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else out
+    ws = _workspace(OP_WEIGHT_ONLY_FWD, M, N, K, 0, x.device, ws)
+    _check(lib().gguf_linear_fwd(_ptr(x), M, N, K, _ptr(blocks), _ptr(bias), _ptr(y), _ptr(ws), ws.numel(),
+                                 _stream(x.device)))
     return y
 
 

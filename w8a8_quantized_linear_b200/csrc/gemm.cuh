@@ -115,6 +115,8 @@ __device__ __forceinline__ void epilogue_scale_chunks(const EpiParams& ep, const
           for (int j = 0; j < 32; ++j) sw[j] = (nc + j < N) ? __ldg(ep.s_col + nc + j) : 0.0f;
         }
       }
+    }
+    {
       if (ep.bias != nullptr) {
         if (full_chunk) {
   #pragma unroll
@@ -138,10 +140,8 @@ __device__ __forceinline__ void epilogue_scale_chunks(const EpiParams& ep, const
   #pragma unroll
     for (int j = 0; j < 32; ++j) {
       float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int>(r[j])) : __uint_as_float(r[j]);
-      if constexpr (EPI != kEpiPlain) {
-        a = __fmul_rn(__fmul_rn(a, sx), (kAxisOk && ep.s_col_axis) ? sw[j] : sw0);
-        if (ep.bias != nullptr) a = __fadd_rn(a, bs[j]);
-      }
+      if constexpr (EPI != kEpiPlain) a = __fmul_rn(__fmul_rn(a, sx), (kAxisOk && ep.s_col_axis) ? sw[j] : sw0);
+      if (ep.bias != nullptr) a = __fadd_rn(a, bs[j]);
       if constexpr (LR) a = __fadd_rn(a, __uint_as_float(lr[j]));
       v[j] = a;
     }
@@ -547,8 +547,8 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
 // the partial sums added in split order and every other step the fp32 RN
 // operation of the fused epilogue, so the result equals the unsplit one
 // (int8) or is reproducible (e4m3).  KIND = kKindBF16 is the plain form:
-// y = bf16(sum_s partial), fp32 sums in split order, no scales.  8 columns
-// per thread: N % 8 == 0, y contiguous [M, N].
+// y = bf16(sum_s partial (+ bias[n])), fp32 sums in split order, no scales.
+// 8 columns per thread: N % 8 == 0, y contiguous [M, N].
 template <int KIND>
 __global__ void __launch_bounds__(256) splitk_epilogue_kernel(const uint32_t* __restrict__ partial, int splits,
                                                               int64_t M, int64_t N, const float* __restrict__ s_row,
@@ -576,11 +576,18 @@ __global__ void __launch_bounds__(256) splitk_epilogue_kernel(const uint32_t* __
         r[j] = (KIND == kKindI8) ? r[j] + t[j] : __float_as_uint(__fadd_rn(__uint_as_float(r[j]), __uint_as_float(t[j])));
     }
     if constexpr (KIND == kKindBF16) {
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(r[j]);
+      if (bias != nullptr) {
+        const uint4 b = __ldg(reinterpret_cast<const uint4*>(bias + n));
+        v[0] = __fadd_rn(v[0], bf16_lo(b.x)); v[1] = __fadd_rn(v[1], bf16_hi(b.x));
+        v[2] = __fadd_rn(v[2], bf16_lo(b.y)); v[3] = __fadd_rn(v[3], bf16_hi(b.y));
+        v[4] = __fadd_rn(v[4], bf16_lo(b.z)); v[5] = __fadd_rn(v[5], bf16_hi(b.z));
+        v[6] = __fadd_rn(v[6], bf16_lo(b.w)); v[7] = __fadd_rn(v[7], bf16_hi(b.w));
+      }
       *reinterpret_cast<uint4*>(y + m * N + n) =
-          make_uint4(pack_bf16x2(__uint_as_float(r[0]), __uint_as_float(r[1])),
-                     pack_bf16x2(__uint_as_float(r[2]), __uint_as_float(r[3])),
-                     pack_bf16x2(__uint_as_float(r[4]), __uint_as_float(r[5])),
-                     pack_bf16x2(__uint_as_float(r[6]), __uint_as_float(r[7])));
+          make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
       continue;
     }
     const float sx = s_row[m];

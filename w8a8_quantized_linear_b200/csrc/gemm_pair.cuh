@@ -40,7 +40,7 @@ template <int KIND, bool LR>
 struct PairCfg {
   static constexpr int kBN = 256;                  // pair tile N (each CTA holds 128 rows or columns of B)
   static constexpr int kBHalf = kBN / 2;
-  static constexpr int kBK = kBKBytes;             // 128 codes per stage
+  static constexpr int kBK = kBKBytes / (KIND == kKindBF16 ? 2 : 1);   // K elements per 128-byte stage row
   static constexpr int kABytes = kBM * kBKBytes;   // 16 KB: this CTA's 128 rows of A
   static constexpr int kBBytes = kBHalf * kBKBytes;   // 16 KB: this CTA's half of B
   static constexpr int kStageBytes = kABytes + kBBytes;
@@ -64,6 +64,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KIND, LR>::k
                      const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmT,
                      const __grid_constant__ CUtensorMap tmL2, int M, int N, int Kc, EpiParams ep) {
   using C = PairCfg<KIND, LR>;
+  static_assert(KIND != kKindBF16 || (!B_MN && !LR), "bf16 operands: K-major B, no low-rank branch");
+  // bf16 operands (the weight-only Linear): y = bf16(acc (+ bias)), no scales
+  constexpr int kEpi = (KIND == kKindBF16) ? kEpiPlain : kEpiScale;
   constexpr int BN = C::kBN;
   constexpr uint32_t kIdesc = idesc<KIND>(2 * kBM, BN, B_MN);
   constexpr uint32_t kIdescLr = idesc<kKindBF16>(2 * kBM, BN, true);   // T K-major, L2 MN-major
@@ -242,10 +245,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KIND, LR>::k
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[acc], acc_phase, abort_flag, 0x400u | acc, limit))) break;
       tc_fence_after();
       const int row = m0 + quarter * 32 + lane;
-      const float sx = row < M ? ep.s_row[row] : 0.0f;
-      const float sw0 = ep.s_col_axis ? 1.0f : ep.s_col[0];
+      float sx = 1.0f, sw0 = 1.0f;
+      if constexpr (kEpi != kEpiPlain) {
+        sx = row < M ? ep.s_row[row] : 0.0f;
+        sw0 = ep.s_col_axis ? 1.0f : ep.s_col[0];
+      }
       const uint32_t tacc = tmem + lane_base + static_cast<uint32_t>(acc * 256);
-      epilogue_scale_chunks<KIND, kEpiScale, BN, kGroups, !LR, LR>(ep, &tmY, tacc, m0, n0, M, N, quarter, group, lane,
+      epilogue_scale_chunks<KIND, kEpi, BN, kGroups, !LR, LR>(ep, &tmY, tacc, m0, n0, M, N, quarter, group, lane,
                                                                     sx, sw0, sOut + e * 2 * C::kOutBufBytes, out_iter,
                                                                     tacc + BN);
       tc_fence_before();

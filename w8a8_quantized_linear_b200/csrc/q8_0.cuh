@@ -94,9 +94,14 @@ __global__ void __launch_bounds__(256) q8_0_quantize_kernel(const float* __restr
 }
 
 // Dequantize: kQ80Unroll groups copied to shared memory with 16-byte loads,
-// then in group u lane l writes values [8l, 8l+8) = f16 scale * code.
+// then in group u lane l writes values [8l, 8l+8) = f16 scale * code (exact
+// in fp32).  BF16: the values rounded to bf16 (RNE), for the GGUF weight
+// dequantized to the train data type (OneTrainer wiki, GGUF).
+template <bool BF16>
 __global__ void __launch_bounds__(256) q8_0_dequantize_kernel(const uint8_t* __restrict__ blocks, int64_t n,
-                                                              float* __restrict__ y) {
+                                                              void* __restrict__ yv) {
+  griddep_launch();
+  griddep_wait();   // the blocks may be the previous kernel's output, y its input
   __shared__ __align__(16) uint8_t stage[kQ80WarpsPerBlock][kQ80Chunk];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* st = stage[warp];
@@ -126,14 +131,27 @@ __global__ void __launch_bounds__(256) q8_0_dequantize_kernel(const uint8_t* __r
         v[i + 1] = d * static_cast<float>(static_cast<int8_t>(pair >> 8));
       }
       const int64_t base = (c * kQ80Unroll + u) * 256 + lane * 8;
-      if (base + 8 <= n) {
-        float4* o = reinterpret_cast<float4*>(y + base);
-        o[0] = make_float4(v[0], v[1], v[2], v[3]);
-        o[1] = make_float4(v[4], v[5], v[6], v[7]);
-      } else {
+      if constexpr (BF16) {
+        __nv_bfloat16* y = static_cast<__nv_bfloat16*>(yv);
+        if (base + 8 <= n) {
+          *reinterpret_cast<uint4*>(y + base) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                                           pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+        } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (base + i < n) y[base + i] = v[i];
+          for (int i = 0; i < 8; ++i)
+            if (base + i < n) y[base + i] = __float2bfloat16_rn(v[i]);
+        }
+      } else {
+        float* y = static_cast<float*>(yv);
+        if (base + 8 <= n) {
+          float4* o = reinterpret_cast<float4*>(y + base);
+          o[0] = make_float4(v[0], v[1], v[2], v[3]);
+          o[1] = make_float4(v[4], v[5], v[6], v[7]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (base + i < n) y[base + i] = v[i];
+        }
       }
     }
     __syncwarp();

@@ -17,6 +17,7 @@
 #include "quantize.cuh"
 #include "q8_0.cuh"
 #include "gemv.cuh"
+#include "weight_only.cuh"
 
 namespace w8a8 {
 namespace {
@@ -468,6 +469,98 @@ w8a8_status gemm_dgrad(const void* dyq, int64_t lda, const float* sdy, int64_t M
   return launch_splitk_epilogue(qt, *sk, M, K, sdy, sw, 0, nullptr, dx, st);
 }
 
+// ---------------------------------------------------------------------------
+// The bf16 Linear of the weight-only types (OneTrainer wiki, float8 and GGUF:
+// the weight dequantized to the train data type): y = bf16(X W^T (+ bias)),
+// fp32 sums on the tensor cores (kind::f16), split along K (fp32 partial sums
+// added in split order) when the output makes few tiles.
+int bf16_splits(int64_t M, int64_t N, int64_t K) {
+  const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + 255) / 256);
+  const int64_t num_kb = (K + 63) / 64;
+  if (tiles <= 0 || tiles * 2 > kSplitSms || (N % 8) != 0) return 1;
+  int64_t s = kSplitSms / tiles;
+  if (s > num_kb / 4) s = num_kb / 4;
+  if (s > 16) s = 16;
+  return s < 2 ? 1 : static_cast<int>(s);
+}
+size_t split_bytes(int s, int64_t M, int64_t N) {
+  return s > 1 ? static_cast<size_t>(s) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4 : 0;
+}
+// Workspace of bf16_linear_fwd (partial sums only) and of the weight-only
+// forwards (the dequantized weight [N, K] bf16, then the partial sums).
+size_t ws_bf16(int64_t M, int64_t N, int64_t K) {
+  Carve c(nullptr);
+  const size_t p = split_bytes(bf16_splits(M, N, K), M, N);
+  if (p) c.take(p);
+  return c.off;
+}
+size_t ws_weight_only(int64_t M, int64_t N, int64_t K) {
+  Carve c(nullptr);
+  c.take(static_cast<size_t>(N) * static_cast<size_t>(K) * 2);
+  const size_t p = split_bytes(bf16_splits(M, N, K), M, N);
+  if (p) c.take(p);
+  return c.off;
+}
+
+w8a8_status gemm_bf16(const void* x, int64_t M, int64_t N, int64_t K, const void* w, const void* bias, void* y,
+                      Carve& c, cudaStream_t st) {
+  const int splits = bf16_splits(M, N, K);
+  alignas(64) CUtensorMap ta, tb;
+  w8a8_status s = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, K, M, K * 2, 64, kBM);
+  if (s != W8A8_OK) return s;
+  EpiParams ep{};
+  ep.bias = static_cast<const __nv_bfloat16*>(bias);
+  ep.y = static_cast<__nv_bfloat16*>(y);
+  ep.ldy = N;
+  ep.splits = 1;
+  if (splits == 1 && M >= kPairMinRows) {
+    if ((s = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w, K, N, K * 2, 64, 128)) != W8A8_OK) return s;
+    return launch_gemm_pair<kKindBF16, false>(ta, tb, M, N, K, ep, st);
+  }
+  if ((s = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w, K, N, K * 2, 64, 256)) != W8A8_OK) return s;
+  if (splits > 1) {
+    ep.splits = splits;
+    ep.partial = static_cast<uint32_t*>(c.take(split_bytes(splits, M, N)));
+  }
+  if ((s = launch_gemm<kKindBF16, false, 256, kEpiPlain>(ta, tb, M, N, K, ep, st)) != W8A8_OK || splits == 1) return s;
+  int sms = 0;
+  if ((s = current_device(nullptr, &sms)) != W8A8_OK) return s;
+  int64_t grid = (M * (N / 8) + 255) / 256;
+  if (grid > 8 * static_cast<int64_t>(sms)) grid = 8 * static_cast<int64_t>(sms);
+  const uint32_t* part = ep.partial;
+  const cudaError_t e =
+      launch_pdl(splitk_epilogue_kernel<kKindBF16>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, part, splits, M,
+                 N, static_cast<const float*>(nullptr), static_cast<const float*>(nullptr), 0, ep.bias, ep.y);
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "split-K epilogue launch");
+}
+
+// Q8_0 -> fp32 (BF16 = false) or bf16 values.
+template <bool BF16>
+w8a8_status launch_q8_0_dequant(const void* blocks, int64_t n, void* y, cudaStream_t st) {
+  int sms = 0;
+  w8a8_status s = current_device(nullptr, &sms);
+  if (s != W8A8_OK) return s;
+  const int64_t chunks = (n + 256 * kQ80Unroll - 1) / (256 * kQ80Unroll);
+  int64_t grid = (chunks + kQ80WarpsPerBlock - 1) / kQ80WarpsPerBlock;
+  if (grid > 16 * sms) grid = 16 * sms;
+  const cudaError_t e = launch_pdl(q8_0_dequantize_kernel<BF16>, dim3(static_cast<int>(grid)), dim3(256), 0, st,
+                                   static_cast<const uint8_t*>(blocks), n, y);
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "q8_0 dequantize launch");
+}
+
+// e4m3 codes -> bf16(value * scale), n % 16 == 0.
+w8a8_status launch_dequant_e4m3(const void* q, int64_t n, const float* scale, void* w, cudaStream_t st) {
+  int sms = 0;
+  w8a8_status s = current_device(nullptr, &sms);
+  if (s != W8A8_OK) return s;
+  const int64_t n8 = n / 8;
+  int64_t grid = (n8 + 255) / 256;
+  if (grid > 8 * static_cast<int64_t>(sms)) grid = 8 * static_cast<int64_t>(sms);
+  const cudaError_t e = launch_pdl(dequant_e4m3_bf16_kernel, dim3(static_cast<int>(grid)), dim3(256), 0, st,
+                                   static_cast<const uint2*>(q), n8, scale, static_cast<uint4*>(w));
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "e4m3 dequantize launch");
+}
+
 #define W8A8_CHECK(cond, status, ...) \
   do {                                \
     if (!(cond)) return fail(status, __VA_ARGS__); \
@@ -706,6 +799,8 @@ size_t w8a8_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
     case W8A8_OP_LINEAR_DGRAD: return ws_linear(M, round_up(N, 16), K);
     case W8A8_OP_SVDQ_FWD: return ws_svdq(M, K, r);
     case W8A8_OP_QUANTIZE_WEIGHT: return 256;
+    case W8A8_OP_BF16_FWD: return ws_bf16(M, N, K);
+    case W8A8_OP_WEIGHT_ONLY_FWD: return ws_weight_only(M, N, K);
     default: return 0;
   }
 }
@@ -781,16 +876,74 @@ w8a8_status q8_0_dequantize(const void* blocks, int64_t n, float* y, w8a8_stream
   if (n == 0) return W8A8_OK;
   W8A8_CHECK(y && blocks, W8A8_ERR_INVALID_ARG, "null pointer");
   W8A8_CHECK(aligned16(y) && aligned16(blocks), W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
-  int sms = 0;
-  w8a8_status st = current_device(nullptr, &sms);
+  return launch_q8_0_dequant<false>(blocks, n, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+w8a8_status q8_0_dequantize_bf16(const void* blocks, int64_t n, void* y, w8a8_stream_t stream) {
+  W8A8_CHECK(n >= 0, W8A8_ERR_UNSUPPORTED_SHAPE, "n < 0");
+  if (n == 0) return W8A8_OK;
+  W8A8_CHECK(y && blocks, W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(y) && aligned16(blocks), W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  return launch_q8_0_dequant<true>(blocks, n, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+w8a8_status w8a8_dequantize_e4m3_bf16(const void* q, int64_t n, const float* scale, void* w,
+                                      w8a8_stream_t stream) {
+  W8A8_CHECK(n >= 0 && n % 16 == 0, W8A8_ERR_UNSUPPORTED_SHAPE, "n must be a non-negative multiple of 16");
+  if (n == 0) return W8A8_OK;
+  W8A8_CHECK(q && scale && w, W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(q) && aligned16(scale) && aligned16(w), W8A8_ERR_MISALIGNED,
+             "pointers must be 16-byte aligned");
+  return launch_dequant_e4m3(q, n, scale, w, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// Shared argument checks of the bf16-Linear entry points.
+static w8a8_status check_bf16_linear(const void* x, int64_t M, int64_t N, int64_t K, const void* w, const void* bias,
+                                     const void* y, const void* ws, size_t ws_bytes, size_t need,
+                                     bool need_scale = false, const void* scale = nullptr) {
+  W8A8_CHECK(M >= 0 && N >= 1 && M < (1ll << 31) && N < (1ll << 31), W8A8_ERR_UNSUPPORTED_SHAPE, "bad M/N");
+  w8a8_status st = check_k(K, "K");
   if (st != W8A8_OK) return st;
-  const int64_t chunks = (n + 256 * kQ80Unroll - 1) / (256 * kQ80Unroll);
-  int64_t grid = (chunks + kQ80WarpsPerBlock - 1) / kQ80WarpsPerBlock;
-  if (grid > 16 * sms) grid = 16 * sms;
-  q8_0_dequantize_kernel<<<static_cast<int>(grid), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint8_t*>(blocks), n, y);
-  cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "q8_0_dequantize launch");
+  if (M == 0) return W8A8_OK;
+  W8A8_CHECK(x && w && y && (!need_scale || scale), W8A8_ERR_INVALID_ARG, "null pointer");
+  W8A8_CHECK(aligned16(x) && aligned16(w) && aligned16(y) && (bias == nullptr || aligned16(bias)) &&
+                 (!need_scale || aligned16(scale)),
+             W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  W8A8_CHECK(need == 0 || (ws != nullptr && ws_bytes >= need), W8A8_ERR_WORKSPACE, "workspace too small: need %zu bytes",
+             need);
+  W8A8_CHECK(ws == nullptr || aligned16(ws), W8A8_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+  return current_device(nullptr, nullptr);
+}
+
+w8a8_status bf16_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, const void* w, const void* bias, void* y,
+                            void* ws, size_t ws_bytes, w8a8_stream_t stream) {
+  w8a8_status st = check_bf16_linear(x, M, N, K, w, bias, y, ws, ws_bytes, M > 0 ? ws_bf16(M, N, K) : 0);
+  if (st != W8A8_OK || M == 0) return st;
+  Carve c(ws);
+  return gemm_bf16(x, M, N, K, w, bias, y, c, reinterpret_cast<cudaStream_t>(stream));
+}
+
+w8a8_status float8_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, const void* wq, const float* w_scale,
+                              const void* bias, void* y, void* ws, size_t ws_bytes, w8a8_stream_t stream) {
+  w8a8_status st = check_bf16_linear(x, M, N, K, wq, bias, y, ws, ws_bytes, M > 0 ? ws_weight_only(M, N, K) : 0,
+                                     true, w_scale);
+  if (st != W8A8_OK || M == 0) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Carve c(ws);
+  void* wb = c.take(static_cast<size_t>(N) * static_cast<size_t>(K) * 2);
+  if ((st = launch_dequant_e4m3(wq, N * K, w_scale, wb, s)) != W8A8_OK) return st;
+  return gemm_bf16(x, M, N, K, wb, bias, y, c, s);
+}
+
+w8a8_status gguf_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, const void* blocks, const void* bias,
+                            void* y, void* ws, size_t ws_bytes, w8a8_stream_t stream) {
+  w8a8_status st = check_bf16_linear(x, M, N, K, blocks, bias, y, ws, ws_bytes, M > 0 ? ws_weight_only(M, N, K) : 0);
+  if (st != W8A8_OK || M == 0) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Carve c(ws);
+  void* wb = c.take(static_cast<size_t>(N) * static_cast<size_t>(K) * 2);
+  if ((st = launch_q8_0_dequant<true>(blocks, N * K, wb, s)) != W8A8_OK) return st;
+  return gemm_bf16(x, M, N, K, wb, bias, y, c, s);
 }
 
 w8a8_status q8_0_to_axis_int8(const void* blocks, int64_t N, int64_t K, int8_t* q, float* scale,
