@@ -479,7 +479,7 @@ def run_case(args):
     import w8a8_quantized_linear_b200 as w8
     dev = torch.device("cuda", 0)
     if args.case in ("requant", "gguf_m1", "gguf_m64", "svdq", "requant_e4m3", "gguf_f_m1", "gguf_f_m4608",
-                     "svdq_e4m3"):
+                     "svdq_e4m3", "wo_float8", "wo_gguf"):
         return run_other_case(args, torch, workloads, w8, dev)
     wl = workloads.dit_mlp()
     if args.case in ("up", "dgrad_up"):
@@ -512,8 +512,18 @@ def run_other_case(args, torch, workloads, w8, dev):
     GGUF weight; gguf_m1 / gguf_m64: the GGUF A8 int forward at M = 1 / 64;
     gguf_f_m1 / gguf_f_m4608: the GGUF A8 float forward at M = 1 / 4608;
     svdq / svdq_e4m3: the SVDQuant r = 32 forward at 4608 x 3072 x 3072 with
-    an int8 / e4m3 residual."""
-    if args.case in ("svdq", "svdq_e4m3"):
+    an int8 / e4m3 residual; wo_float8 / wo_gguf: the weight-only forwards
+    on the DiT up-projection (dequantize to bf16, then the bf16 Linear)."""
+    if args.case in ("wo_float8", "wo_gguf"):
+        g = workloads.gguf_q8_0(M=M_TOK)
+        x = g["x"].to(dev)
+        if args.case == "wo_float8":
+            wq, sw = w8.quantize_weight(g["w_f32"].to(torch.bfloat16).to(dev), "e4m3", "tensor")
+            fn = lambda: w8.float8_linear_fwd(x, wq, sw)
+        else:
+            blk = w8.q8_0_quantize(g["w_f32"].reshape(-1).to(dev))
+            fn = lambda: w8.gguf_linear_fwd(x, blk, MLP)
+    elif args.case in ("svdq", "svdq_e4m3"):
         d = workloads.svdquant()
         prep = w8.svdq_prepare(d["w"].to(dev), d["r"], "e4m3" if args.case == "svdq_e4m3" else "int8")
         x = d["x"].to(dev)
@@ -784,7 +794,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-extras", dest="extras", action="store_false")
     ap.add_argument("--case", choices=["up", "down", "dgrad_down", "dgrad_up", "requant", "gguf_m1", "gguf_m64", "svdq",
-                                       "requant_e4m3", "gguf_f_m1", "gguf_f_m4608", "svdq_e4m3"],
+                                       "requant_e4m3", "gguf_f_m1", "gguf_f_m4608", "svdq_e4m3", "wo_float8",
+                                       "wo_gguf"],
                     default=None, help="run only one of the step's four quantize+GEMM pairs, or one other kernel "
                                        "of the path (for profiling), no JSON")
     args = ap.parse_args()
