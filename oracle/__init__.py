@@ -83,6 +83,8 @@ def _declare(L):
         "orc_q8_0_to_axis_int8": [_P, _I64, _I64, _P, _P],
         "orc_q8_0_to_axis": [_P, _I64, _I64, ctypes.c_int, _P, _P],
         "orc_dequant_e4m3_bf16": [_P, _I64, ctypes.c_float, _P],
+        "orc_act": [_P, _I64, ctypes.c_int, _P],
+        "orc_row_absmax_bf16": [_P, _I64, _I64, _P],
         "orc_q8_0_dequantize_bf16": [_P, _I64, _P],
         "orc_linear_bf16": [_P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P],
         "orc_gemm_i8_nt": [_P, _P, _I64, _I64, _I64, _P],
@@ -317,11 +319,33 @@ def epilogue(acc, s_row, s_w, bias=None):
 
 
 # --------------------------------------------------------------------------- composed ops
-def linear_fwd(x_bf16, wq, s_w, qt=INT8, bias=None):
-    """W8A8 Linear forward: Q(X) token-wise, 8-bit matmul with Q(W), epilogue.
+ACT_NONE, ACT_GELU, ACT_GELU_TANH = 0, 1, 2
+
+
+def act_f32(v, act):
+    """The activation of fp32 values (double math, one rounding to fp32)."""
+    v = _c(v, np.float32)
+    out = np.empty(v.shape, np.float32)
+    lib().orc_act(_ptr(v), v.size, act, _ptr(out))
+    return out
+
+
+def row_absmax_bf16(y_bf16):
+    """max_n |y[m, n]| of bf16 values, fp32 [M]."""
+    y = _c(y_bf16, np.uint16)
+    M, N = y.shape
+    a = np.empty((M,), np.float32)
+    lib().orc_row_absmax_bf16(_ptr(y), M, N, _ptr(a))
+    return a
+
+
+def linear_fwd(x_bf16, wq, s_w, qt=INT8, bias=None, act=ACT_NONE):
+    """W8A8 Linear forward: Q(X) token-wise, 8-bit matmul with Q(W), epilogue,
+    then the optional activation on the fp32 epilogue value.
 
     Returns a dict: y (bf16 bits), y32, xq, sx, acc and, for e4m3, absacc
-    (sum |a*b| per output, for the fp8 tolerance)."""
+    (sum |a*b| per output, for the fp8 tolerance); with an activation also
+    pre (the fp32 value it was applied to); amax = the rows' max |y|."""
     xq, sx = quantize_rows(x_bf16, qt)
     out = {"xq": xq, "sx": sx}
     if qt == INT8:
@@ -331,6 +355,11 @@ def linear_fwd(x_bf16, wq, s_w, qt=INT8, bias=None):
         out["absacc"] = absacc
     out["acc"] = acc
     out["y"], out["y32"] = epilogue(acc, sx, s_w, bias)
+    if act != ACT_NONE:
+        out["pre"] = out["y32"]
+        out["y32"] = act_f32(out["pre"], act)
+        out["y"] = f32_to_bf16(out["y32"])
+    out["amax"] = row_absmax_bf16(out["y"])
     return out
 
 

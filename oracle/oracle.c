@@ -16,6 +16,9 @@
 #include "oracle.h"
 
 #include <math.h>
+#ifndef M_PI
+#define M_PI 3.14159265358979323846
+#endif
 #include <stdlib.h>
 #include <string.h>
 
@@ -273,6 +276,35 @@ void orc_q8_0_to_axis(const uint8_t* blocks, int64_t N, int64_t K, int qt,
 void orc_q8_0_to_axis_int8(const uint8_t* blocks, int64_t N, int64_t K,
                            int8_t* q, float* s) {
   orc_q8_0_to_axis(blocks, N, K, ORC_INT8, (uint8_t*)q, s);
+}
+
+/* ========================================================================== */
+/* The activation between two projections and the row absmax of an output     */
+/* [SURVEY reading: the DiT MLP's GELU, optional; the fused absmax is a       */
+/* property of the output, max_n |y[m,n]|].                                   */
+/* ========================================================================== */
+
+/* GELU, exact form: 0.5 v (1 + erf(v / sqrt 2)); tanh form: 0.5 v (1 +
+ * tanh(sqrt(2/pi) (v + 0.044715 v^3))).  In double, rounded once to fp32. */
+void orc_act(const float* v, int64_t n, int act, float* out) {
+  for (int64_t i = 0; i < n; ++i) {
+    double x = (double)v[i], r = x;
+    if (act == 1) r = 0.5 * x * (1.0 + erf(x / sqrt(2.0)));
+    if (act == 2) r = 0.5 * x * (1.0 + tanh(sqrt(2.0 / M_PI) * (x + 0.044715 * x * x * x)));
+    out[i] = (float)r;
+  }
+}
+
+/* amax[m] = max_n |bf16 y[m, n]| as fp32. */
+void orc_row_absmax_bf16(const uint16_t* y, int64_t M, int64_t N, float* amax) {
+  for (int64_t m = 0; m < M; ++m) {
+    float a = 0.0f;
+    for (int64_t n = 0; n < N; ++n) {
+      float v = fabsf(orc_bf16_to_f32(y[m * N + n]));
+      if (v > a) a = v;
+    }
+    amax[m] = a;
+  }
 }
 
 /* ========================================================================== */

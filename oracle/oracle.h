@@ -78,6 +78,13 @@ void orc_q8_0_to_axis(const uint8_t* blocks, int64_t N, int64_t K, int qt,
 void orc_q8_0_to_axis_int8(const uint8_t* blocks, int64_t N, int64_t K,
                            int8_t* q, float* s);
 
+/* ---- activation and row absmax (the MLP chain) --------------------------- */
+/* act 1: GELU 0.5 v (1 + erf(v / sqrt 2)); act 2: the tanh form; in double,
+ * rounded once to fp32.  act 0 copies. */
+void orc_act(const float* v, int64_t n, int act, float* out);
+/* amax[m] = max_n |y[m, n]| of bf16 values. */
+void orc_row_absmax_bf16(const uint16_t* y, int64_t M, int64_t N, float* amax);
+
 /* ---- weight-only types [OT-WIKI float8, GGUF] ---------------------------- */
 /* w = bf16(e4m3_value(q) * s) for n codes (tensor-wise scale s). */
 void orc_dequant_e4m3_bf16(const uint8_t* q, int64_t n, float s, uint16_t* w);

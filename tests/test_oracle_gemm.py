@@ -357,3 +357,42 @@ def test_weight_only_forwards_compose(orc):
     ew = sb * (0.5 * (1 + 2 ** -20) + 127 * 2 ** -11)
     ew = ew + 2 ** -8 * (np.abs(w.double().numpy()) + ew)
     assert np.all(np.abs(gg["acc"] - base) <= np.abs(x.double().numpy()) @ ew.T)
+
+
+# --------------------------------------------------------------------------- activation and row absmax
+def test_gelu_closed_forms_and_library(orc):
+    """GELU(1) = Phi(1) and GELU(-1) = -Phi(-1) (the normal CDF at 1); the odd
+    identity GELU(v) - GELU(-v) = v of both forms; the exact form equals
+    scipy's erf composed in double, rounded once; the tanh form stays within
+    1e-3 of it."""
+    from scipy.special import erf
+    g = orc.act_f32(np.array([1.0, -1.0, 0.0], np.float32), orc.ACT_GELU)
+    assert g[0] == np.float32(0.8413447460685429) and g[1] == np.float32(-0.15865525393145707) and g[2] == 0.0
+    v = np.linspace(-6, 6, 4001).astype(np.float32)
+    for act in (orc.ACT_GELU, orc.ACT_GELU_TANH):
+        a, b = orc.act_f32(v, act).astype(np.float64), orc.act_f32(-v, act).astype(np.float64)
+        assert np.all(np.abs(a - b - v) <= 4 * np.spacing(np.maximum(np.abs(v), 1e-30).astype(np.float32)))
+    vd = v.astype(np.float64)
+    ref = (0.5 * vd * (1.0 + erf(vd / np.sqrt(2.0)))).astype(np.float32)
+    assert np.array_equal(orc.act_f32(v, orc.ACT_GELU), ref)
+    assert np.all(np.abs(orc.act_f32(v, orc.ACT_GELU_TANH) - ref) <= 1e-3)
+    assert np.array_equal(orc.act_f32(v, orc.ACT_NONE), v)
+
+
+def test_row_absmax_and_activated_forward(orc):
+    x = workloads.to_u16(workloads.with_outlier_channels((9, 128), 1.0, 40))
+    w = workloads.to_u16(workloads.normal((40, 128), 0.02, 41))
+    bias = workloads.to_u16(workloads.normal((40,), 0.01, 42))
+    wq, sw = orc.quantize_weight(w, orc.INT8, orc.TENSOR)
+    base = orc.linear_fwd(x, wq, sw, bias=bias)
+    yb = orc.bf16_to_f32(base["y"])
+    assert np.array_equal(base["amax"], np.abs(yb).max(axis=1))
+    g = orc.linear_fwd(x, wq, sw, bias=bias, act=orc.ACT_GELU)
+    assert np.array_equal(g["pre"], base["y32"])
+    assert np.array_equal(g["y"], orc.f32_to_bf16(orc.act_f32(base["y32"], orc.ACT_GELU)))
+    assert np.array_equal(g["amax"], np.abs(orc.bf16_to_f32(g["y"])).max(axis=1))
+    assert np.all(orc.bf16_to_f32(g["y"]) >= -0.17)     # GELU's minimum is about -0.17
+    # maxima placed by hand: last column, first column, negative, all zero
+    yh = np.zeros((4, 9), np.float32)
+    yh[0, 8], yh[1, 0], yh[2, 4], yh[2, 5] = -3.0, 2.5, 1.0, -0.5
+    assert orc.row_absmax_bf16(orc.f32_to_bf16(yh)).tolist() == [3.0, 2.5, 1.0, 0.0]

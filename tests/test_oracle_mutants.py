@@ -46,6 +46,7 @@ PINS = [
     lambda o: G.test_svdq_zero_residual_is_lowrank_product(o, 1),
     lambda o: G.test_dequant_e4m3_bf16_vs_torch(o, 3.1e-5), G.test_q8_0_dequantize_bf16_vs_torch,
     G.test_linear_bf16_vs_numpy_and_textbook, G.test_weight_only_forwards_compose,
+    G.test_gelu_closed_forms_and_library, G.test_row_absmax_and_activated_forward,
 ]
 
 # (name, text in oracle.c, replacement)
@@ -104,6 +105,10 @@ MUTANTS = [
      "w[i] = orc_f32_to_bf16(block_scale_f16(blk) * (float)(int8_t)blk[1 + i % Q80_BLOCK]);"),
     ("bf16 linear transposed w", "(double)orc_bf16_to_f32(w[n * K + k]);", "(double)orc_bf16_to_f32(w[k * N + n]);"),
     ("bf16 linear drops bias", "if (bias) v = v + orc_bf16_to_f32(bias[n]);", ""),
+    ("gelu scaled argument", "r = 0.5 * x * (1.0 + erf(x / sqrt(2.0)));", "r = 0.5 * x * (1.0 + erf(x / 2.0));"),
+    ("gelu tanh cubic dropped", "(x + 0.044715 * x * x * x)", "(x)"),
+    ("row absmax skips the last column", "for (int64_t n = 0; n < N; ++n) {\n      float v = fabsf(orc_bf16_to_f32(y[m * N + n]));",
+     "for (int64_t n = 0; n + 1 < N; ++n) {\n      float v = fabsf(orc_bf16_to_f32(y[m * N + n]));"),
     ("lowrank L1 transposed", "(double)orc_bf16_to_f32(l1[k * r + j])", "(double)orc_bf16_to_f32(l1[j * K + k])"),
     ("lowrank up drops a term", "for (int64_t j = 0; j < r; ++j) {\n        double p", "for (int64_t j = 1; j < r; ++j) {\n        double p"),
 ]
