@@ -41,9 +41,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic of one launch of the dominant kernel from an ncu capture, keyed
 # by the hash of the kernel source it was taken on (null when they differ).
-GEMM_TRAFFIC = {"source_sha": "8f7b3f8153ef2a77", "bytes_per_launch": 124070400,
+GEMM_TRAFFIC = {"source_sha": "755bca19a5dc6ae3", "bytes_per_launch": 122816000,
                 "note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one up-proj launch "
-                        "(bench.py --case up): 52.00 MB read + 72.07 MB written"}
+                        "(bench.py --case up): 52.11 MB read + 70.71 MB written"}
 
 
 def gemm_source_sha() -> str:
@@ -608,6 +608,37 @@ def extras(w8, torch, workloads, dev, peaks, src):
     gbs = (x0.numel() * 3 + M_TOK * 4) / (ms * 1e-3) / 1e9
     out["quantize_rows_4608x12288"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
     del x0, sets
+    # DiT MLP forward with GELU between the projections: the down-projection's
+    # quantizer reduces each row itself, or takes the row absmax that the
+    # up-projection's epilogue gathered (same codes, same output)
+    wl = workloads.dit_mlp()
+    w1q, s1 = w8.quantize_weight(wl["w1"].to(dev), "int8", "tensor")
+    w2q, s2 = w8.quantize_weight(wl["w2"].to(dev), "int8", "tensor")
+    xm0 = wl["x"].to(dev)
+    res = {}
+    for name, fused in (("unfused", False), ("fused_absmax", True)):
+        sets = []
+        for i in range(_nsets(nbytes(xm0) + M_TOK * MLP * 3 + M_TOK * HID * 2)):
+            xm = xm0.clone()
+            y1 = torch.empty((M_TOK, MLP), dtype=torch.bfloat16, device=dev)
+            y2 = torch.empty((M_TOK, HID), dtype=torch.bfloat16, device=dev)
+            a1 = torch.empty(M_TOK, dtype=torch.int32, device=dev)
+            ws1 = torch.empty(w8.workspace_bytes(0, M_TOK, MLP, HID), dtype=torch.uint8, device=dev)
+            ws2 = torch.empty(w8.workspace_bytes(0, M_TOK, HID, MLP), dtype=torch.uint8, device=dev)
+            if fused:
+                def fn(xm=xm, y1=y1, y2=y2, a1=a1, ws1=ws1, ws2=ws2):
+                    w8.linear_fwd_ex(xm, w1q, s1, act="gelu", y_amax=a1, out=y1, ws=ws1)
+                    w8.linear_fwd_ex(y1, w2q, s2, x_amax=a1, out=y2, ws=ws2)
+            else:
+                def fn(xm=xm, y1=y1, y2=y2, ws1=ws1, ws2=ws2):
+                    w8.linear_fwd_ex(xm, w1q, s1, act="gelu", out=y1, ws=ws1)
+                    w8.linear_fwd(y1, w2q, s2, out=y2, ws=ws2)
+            sets.append(fn)
+        ms = _time_rot(sets, 10, torch, stream)
+        res[name] = {"ms": ms, "TOPS": 2 * 2 * M_TOK * MLP * HID / ms / 1e9}
+        del sets
+    out["dit_mlp_fwd_gelu_4608x3072x12288"] = res
+    del xm0, w1q, w2q
     # float W8A8 forward (e4m3, bias) 4096 x 3072 x 3072
     d = workloads.float_w8a8()
     wq0, sw = w8.quantize_weight(d["w"].to(dev), "e4m3", "tensor")

@@ -63,6 +63,7 @@ typedef enum {
 
 typedef enum { W8A8_INT8 = 0, W8A8_E4M3 = 1 } w8a8_qtype;
 typedef enum { W8A8_TENSOR = 0, W8A8_AXIS = 1 } w8a8_wgran;
+typedef enum { W8A8_ACT_NONE = 0, W8A8_ACT_GELU = 1, W8A8_ACT_GELU_TANH = 2 } w8a8_act;
 typedef enum {
   W8A8_OP_LINEAR_FWD = 0,      /* w8a8_linear_fwd                          */
   W8A8_OP_LINEAR_DGRAD = 1,    /* w8a8_linear_dgrad                        */
@@ -197,6 +198,30 @@ w8a8_status w8a8_linear_fwd(const void* x_bf16, int64_t M, int64_t N, int64_t K,
                             w8a8_qtype qt, const void* wq, const float* w_scale, w8a8_wgran g,
                             const void* bias_bf16, void* y_bf16,
                             void* ws, size_t ws_bytes, w8a8_stream_t stream);
+
+/* w8a8_linear_fwd for a chain of projections (an MLP block): the same
+ * product, with
+ *   act     W8A8_ACT_GELU (0.5 v (1 + erf(v / sqrt 2))) or W8A8_ACT_GELU_TANH
+ *           (0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3)))) applied to the
+ *           fp32 epilogue value before the bf16 rounding (fp32 math
+ *           functions: within a few fp32 ulp of the exact function);
+ *   y_amax  [M] uint32 or NULL: receives max_n |y[m, n]| of the bf16 outputs
+ *           as fp32 bits (the GEMM epilogue folds each tile's rows in with
+ *           atomicMax; the call clears the buffer first);
+ *   x_amax  [M] uint32 or NULL: max_k |x[m, k]| as fp32 bits, e.g. the
+ *           y_amax of the call that produced x.  The token-wise quantizer
+ *           then skips its reduction; the codes are the same as without it
+ *           when x_amax is the true row absmax.
+ * x_amax and y_amax must not be the same buffer.  With act, x_amax or y_amax
+ * set, the few-token weight-streaming kernel is not used.  Workspace as
+ * w8a8_linear_fwd.  (The pages blame the unfused quantization for W8A8's
+ * need of a compiler, OneTrainer wiki: A8 is faster only with compiled
+ * transformer blocks.) */
+w8a8_status w8a8_linear_fwd_ex(const void* x_bf16, int64_t M, int64_t N, int64_t K,
+                               w8a8_qtype qt, const void* wq, const float* w_scale, w8a8_wgran g,
+                               const void* bias_bf16, w8a8_act act, const uint32_t* x_amax,
+                               uint32_t* y_amax, void* y_bf16, void* ws, size_t ws_bytes,
+                               w8a8_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * W8A8 Linear input gradient for LoRA training with frozen quantized weights

@@ -120,6 +120,14 @@ def test_svdq_validation(L):
     assert L.svdq_linear_fwd_e4m3(A, 0, 8, 32, A, A, 32, A, A, None, A, A, 0, None) == 0      # M = 0: no-op
 
 
+def test_linear_fwd_ex_validation(L):
+    args = lambda act, xa, ya: (A, 8, 8, 32, 0, A, A, 0, None, act, xa, ya, A, A, 1 << 20, None)
+    assert L.w8a8_linear_fwd_ex(*args(3, None, None)) == 1        # unknown activation
+    assert L.w8a8_linear_fwd_ex(*args(1, A, A)) == 1              # x_amax aliases y_amax
+    assert L.w8a8_linear_fwd_ex(*args(1, B, None)) == 3           # misaligned x_amax
+    assert L.w8a8_linear_fwd_ex(A, 0, 8, 32, 0, A, A, 0, None, 1, None, None, A, A, 0, None) == 0   # M = 0
+
+
 def test_weight_only_validation(L):
     assert L.bf16_linear_fwd(A, 8, 8, 20, A, None, A, A, 1 << 20, None) == 2        # K % 16
     assert L.bf16_linear_fwd(A, 0, 8, 32, None, None, None, None, 0, None) == 0     # M = 0: no-op

@@ -497,6 +497,76 @@ def test_svdq_e4m3_zero_factors_equal_float_linear(w8, M):
     assert torch.equal(w8.svdq_linear_fwd(x, wq, sw, l1, l2), w8.linear_fwd(x, wq, sw))
 
 
+# --------------------------------------------------------------------------- fused MLP chain
+def _amax_of(y):
+    """Row max |y| of a bf16 CUDA tensor, as fp32 bit patterns (int32)."""
+    return y.float().abs().amax(dim=1).view(torch.int32)
+
+
+# pair kernel (600 rows), single-SM (130), split-K (7 x 1000 x 4096, 1 x 2048 x 3072), e4m3
+CHAIN_SHAPES = [(600, 520, 512, "int8"), (130, 264, 256, "int8"), (7, 1000, 4096, "int8"), (1, 2048, 3072, "int8"),
+                (600, 520, 512, "e4m3"), (33, 256, 1024, "e4m3")]
+
+
+@pytest.mark.parametrize("M,N,K,qt", CHAIN_SHAPES)
+def test_linear_fwd_ex_row_absmax(w8, orc, M, N, K, qt):
+    """Without an activation the output is linear_fwd's bit for bit, and
+    y_amax holds each row's max |y| exactly (every epilogue form: pair,
+    single-SM, split-K)."""
+    x = workloads.with_outlier_channels((M, K), 1.0, seed=91 + M).to(DEV)
+    wq, sw = w8.quantize_weight(workloads.normal((N, K), 0.02, seed=92).to(DEV), qt, "tensor")
+    bias = workloads.normal((N,), 0.01, seed=93).to(DEV)
+    amax = torch.full((M,), 12345, dtype=torch.int32, device=DEV)   # the call clears it
+    y = w8.linear_fwd_ex(x, wq, sw, bias=bias, y_amax=amax)
+    assert torch.equal(y, w8.linear_fwd(x, wq, sw, bias=bias))
+    assert torch.equal(amax, _amax_of(y))
+
+
+@pytest.mark.parametrize("act", ["gelu", "gelu_tanh"])
+@pytest.mark.parametrize("M,N,K,qt", CHAIN_SHAPES)
+def test_linear_fwd_ex_gelu_parity(w8, orc, M, N, K, qt, act):
+    """GELU on the fp32 epilogue value.  Bound: 1 bf16 ulp plus the fp32
+    evaluation error of the activation (the erf / tanh of CUDA's math library
+    within a few units of 2^-23 absolute, scaled by |v|); for e4m3 also the
+    GEMM bound, through GELU's slope (|GELU'| < 1.13)."""
+    x = workloads.with_outlier_channels((M, K), 1.0, seed=94 + M)
+    w = workloads.normal((N, K), 0.02, seed=95)
+    bias = workloads.normal((N,), 0.01, seed=96)
+    q = QT[qt]
+    wq, sw = w8.quantize_weight(w.to(DEV), qt, "tensor")
+    amax = torch.zeros((M,), dtype=torch.int32, device=DEV)
+    y = w8.linear_fwd_ex(x.to(DEV), wq, sw, bias=bias.to(DEV), act=act, y_amax=amax)
+    assert torch.equal(amax, _amax_of(y))
+    wqr, swr = orc.quantize_weight(workloads.to_u16(w), q, 0)
+    a = orc.ACT_GELU if act == "gelu" else orc.ACT_GELU_TANH
+    ref = orc.linear_fwd(workloads.to_u16(x), wqr, swr, qt=q, bias=workloads.to_u16(bias), act=a)
+    v = np.abs(ref["pre"].astype(np.float64))
+    yr = bf16_bits_to_f64(ref["y"])
+    yg = bf16_bits_to_f64(u16(y))
+    bound = ulp_bf16(np.maximum(np.abs(yr), np.abs(yg))) + 2.0 ** -19 * (v + 0.05 * v ** 3)
+    if q == 1:
+        bound = bound + 1.13 * 1e-3 * ref["sx"][:, None].astype(np.float64) * float(swr[0]) * ref["absacc"]
+    err = np.abs(yg - yr)
+    assert np.all(err <= bound), float((err / bound).max())
+
+
+@pytest.mark.parametrize("M", [1, 64, 600])
+def test_mlp_chain_given_absmax_equals_unfused(w8, M):
+    """Up-projection with GELU hands its row absmax to the down-projection,
+    whose quantizer then skips the reduction: the result is the unfused
+    chain's bit for bit."""
+    x = workloads.normal((M, 512), 1.0, 97).to(DEV)
+    w1q, s1 = w8.quantize_weight(workloads.normal((1024, 512), 0.02, 98).to(DEV), "int8", "tensor")
+    w2q, s2 = w8.quantize_weight(workloads.normal((512, 1024), 0.02, 99).to(DEV), "int8", "tensor")
+    a1 = torch.zeros((M,), dtype=torch.int32, device=DEV)
+    y1 = w8.linear_fwd_ex(x, w1q, s1, act="gelu", y_amax=a1)
+    y2 = w8.linear_fwd_ex(y1, w2q, s2, x_amax=a1)
+    assert torch.equal(y2, w8.linear_fwd(y1, w2q, s2))
+    # and with a wrong absmax the codes change: the given value is used
+    y2w = w8.linear_fwd_ex(y1, w2q, s2, x_amax=(a1.view(torch.float32) * 2).view(torch.int32).contiguous())
+    assert not torch.equal(y2w, y2)
+
+
 # --------------------------------------------------------------------------- weight-only types
 @pytest.mark.parametrize("n,s", [(256, 1.0), (4096 * 16, 0.02 / 448), ((1 << 20) + 48, 3.1e-5)])
 def test_dequantize_e4m3_bf16_parity(w8, orc, n, s):

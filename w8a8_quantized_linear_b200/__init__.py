@@ -25,6 +25,7 @@ INT8, E4M3 = 0, 1
 TENSOR, AXIS = 0, 1
 OP_LINEAR_FWD, OP_LINEAR_DGRAD, OP_SVDQ_FWD, OP_QUANTIZE_WEIGHT = 0, 1, 2, 3
 OP_BF16_FWD, OP_WEIGHT_ONLY_FWD = 4, 5
+ACTS = {"none": 0, "gelu": 1, "gelu_tanh": 2}
 
 STATUS = {0: "W8A8_OK", 1: "W8A8_ERR_INVALID_ARG", 2: "W8A8_ERR_UNSUPPORTED_SHAPE",
           3: "W8A8_ERR_MISALIGNED", 4: "W8A8_ERR_WORKSPACE", 5: "W8A8_ERR_CUDA",
@@ -36,7 +37,8 @@ EXPORTS = ("w8a8_quantize_rows", "w8a8_quantize_weight", "q8_0_bytes", "q8_0_qua
            "svdq_linear_fwd", "svdq_linear_fwd_e4m3", "w8a8_qgemm_fwd", "w8a8_qgemm_dgrad", "w8a8_workspace_bytes",
            "w8a8_device_status", "w8a8_set_wait_limit_ns", "w8a8_selftest_wait",
            "w8a8_e4m3_encode", "w8a8_last_error", "w8a8_linear_fwd_noalloc", "q8_0_dequantize_bf16",
-           "w8a8_dequantize_e4m3_bf16", "bf16_linear_fwd", "float8_linear_fwd", "gguf_linear_fwd")
+           "w8a8_dequantize_e4m3_bf16", "bf16_linear_fwd", "float8_linear_fwd", "gguf_linear_fwd",
+           "w8a8_linear_fwd_ex")
 
 
 class W8A8Error(RuntimeError):
@@ -76,6 +78,7 @@ def lib() -> ctypes.CDLL:
             "w8a8_e4m3_encode": [_P, _I64, _P, _P],
             "w8a8_linear_fwd_noalloc": [_P, _I64, _I64, _I64, _I, _P, _P, _I, _P, _P, _P],
             "q8_0_dequantize_bf16": [_P, _I64, _P, _P],
+            "w8a8_linear_fwd_ex": [_P, _I64, _I64, _I64, _I, _P, _P, _I, _P, _I, _P, _P, _P, _P, _SZ, _P],
             "w8a8_dequantize_e4m3_bf16": [_P, _I64, _P, _P, _P],
             "bf16_linear_fwd": [_P, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P],
             "float8_linear_fwd": [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _SZ, _P],
@@ -315,6 +318,29 @@ def gguf_linear_fwd(x, blocks, N, bias=None, out=None, ws=None):
     ws = _workspace(OP_WEIGHT_ONLY_FWD, M, N, K, 0, x.device, ws)
     _check(lib().gguf_linear_fwd(_ptr(x), M, N, K, _ptr(blocks), _ptr(bias), _ptr(y), _ptr(ws), ws.numel(),
                                  _stream(x.device)))
+    return y
+
+
+def linear_fwd_ex(x, wq, w_scale, bias=None, act="none", x_amax=None, y_amax=None, out=None, ws=None):
+    """linear_fwd for a chain of projections: optional activation ("gelu",
+    "gelu_tanh") on the fp32 epilogue value; y_amax (int32 [M] CUDA tensor)
+    receives the rows' max |y| as fp32 bits; x_amax supplies the rows' max |x|
+    (e.g. the previous call's y_amax) so the quantizer skips its reduction."""
+    _cuda_2d(x, torch.bfloat16, "x")
+    qt = _qt(wq.dtype)
+    M, K = x.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError("wq must be [N, K]")
+    for name, a in (("x_amax", x_amax), ("y_amax", y_amax)):
+        if a is not None and not (a.is_cuda and a.dtype == torch.int32 and a.is_contiguous() and a.numel() >= M):
+            raise ValueError("%s must be a contiguous int32 CUDA tensor of at least M entries" % name)
+    g = AXIS if w_scale.numel() > 1 else TENSOR
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device) if out is None else out
+    ws = _workspace(OP_LINEAR_FWD, M, N, K, 0, x.device, ws)
+    _check(lib().w8a8_linear_fwd_ex(_ptr(x), M, N, K, qt, _ptr(_as_bytes(wq)), _ptr(w_scale), g, _ptr(bias),
+                                    ACTS[act], _ptr(x_amax), _ptr(y_amax), _ptr(y), _ptr(ws), ws.numel(),
+                                    _stream(x.device)))
     return y
 
 

@@ -48,7 +48,32 @@ struct EpiParams {
   int r;
   int splits;                    // K splits per tile (>= 1; > 1 not with kEpiLowRank)
   uint32_t* partial;             // [splits, M, N] raw sums (splits > 1)
+  int act;                       // kActNone / kActGelu / kActGeluTanh, applied last (kEpiScale)
+  uint32_t* y_amax;              // [M] or null: atomicMax of max |y| per row (fp32 bits of the bf16 values)
 };
+
+// Optional activation between two projections (the MLP's GELU): the exact
+// form 0.5 v (1 + erf(v / sqrt 2)) or the tanh form 0.5 v (1 + tanh(sqrt(2/pi)
+// (v + 0.044715 v^3))), on the fp32 epilogue value, before the bf16 rounding.
+enum { kActNone = 0, kActGelu = 1, kActGeluTanh = 2 };
+__device__ __forceinline__ float apply_act(float v, int act) {
+  if (act == kActGelu) return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
+  if (act == kActGeluTanh) return 0.5f * v * (1.0f + tanhf(0.79788456080286536f * (v + 0.044715f * v * v * v)));
+  return v;
+}
+
+// Row absmax of bf16 outputs: max over |bf16| as 16-bit lanes (the magnitude
+// bits order like the values), then one atomicMax on the fp32 bits (a
+// non-negative float orders like its bit pattern).
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t m, uint32_t packed) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(m), "r"(packed & 0x7FFF7FFFu));
+  return d;
+}
+__device__ __forceinline__ void row_amax_commit(uint32_t* y_amax, int64_t row, uint32_t m) {
+  const uint32_t h = (m & 0xFFFFu) > (m >> 16) ? (m & 0xFFFFu) : (m >> 16);
+  if (h != 0) atomicMax(y_amax + row, h << 16);
+}
 
 template <int KIND, int BN, int EPI>
 struct GemmCfg {
@@ -93,6 +118,7 @@ __device__ __forceinline__ void epilogue_scale_chunks(const EpiParams& ep, const
                                                       uint32_t tlr = 0) {
   const int row = m0 + quarter * 32 + lane;
   const bool row_ok = row < M;
+  uint32_t amx = 0;   // this lane's row: max |y| over the tile's columns, as two bf16 lanes
   #pragma unroll 1
   for (int c = group; c < BN / 32; c += kGroups) {
     const int nc = n0 + c * 32;
@@ -145,6 +171,19 @@ __device__ __forceinline__ void epilogue_scale_chunks(const EpiParams& ep, const
       if constexpr (LR) a = __fadd_rn(a, __uint_as_float(lr[j]));
       v[j] = a;
     }
+    if constexpr (EPI == kEpiScale && !LR) {
+      if (ep.act != kActNone) {
+  #pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = apply_act(v[j], ep.act);
+      }
+      if (ep.y_amax != nullptr) {
+  #pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          // columns past N hold 0 (zero-filled operands, no bias there): no effect
+          amx = bf16x2_absmax(amx, pack_bf16x2(v[j], v[j + 1]));
+        }
+      }
+    }
     if (ep.tma_store) {
       // Stage the warp's 32 x 32 bf16 block in shared memory with the 64-byte
       // swizzle (16-byte unit j of row l at unit j ^ ((l >> 1) & 3)), then
@@ -185,6 +224,9 @@ __device__ __forceinline__ void epilogue_scale_chunks(const EpiParams& ep, const
           if (nc + j < N) out[j] = __float2bfloat16_rn(v[j]);
       }
     }
+  }
+  if constexpr (EPI == kEpiScale && !LR) {
+    if (ep.y_amax != nullptr && row_ok) row_amax_commit(ep.y_amax, row, amx);
   }
 }
 
@@ -554,7 +596,8 @@ __global__ void __launch_bounds__(256) splitk_epilogue_kernel(const uint32_t* __
                                                               int64_t M, int64_t N, const float* __restrict__ s_row,
                                                               const float* __restrict__ s_col, int axis,
                                                               const __nv_bfloat16* __restrict__ bias,
-                                                              __nv_bfloat16* __restrict__ y) {
+                                                              __nv_bfloat16* __restrict__ y, int act = kActNone,
+                                                              uint32_t* __restrict__ y_amax = nullptr) {
   griddep_launch();
   griddep_wait();   // the partial sums come from the GEMM just before
   const int64_t n8 = N >> 3;
@@ -611,10 +654,13 @@ __global__ void __launch_bounds__(256) splitk_epilogue_kernel(const uint32_t* __
       float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int>(r[j])) : __uint_as_float(r[j]);
       a = __fmul_rn(__fmul_rn(a, sx), sw[j]);
       if (bias != nullptr) a = __fadd_rn(a, bs[j]);
-      v[j] = a;
+      v[j] = (act != kActNone) ? apply_act(a, act) : a;
     }
-    *reinterpret_cast<uint4*>(y + m * N + n) =
-        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    const uint4 out = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                 pack_bf16x2(v[6], v[7]));
+    *reinterpret_cast<uint4*>(y + m * N + n) = out;
+    if (y_amax != nullptr)
+      row_amax_commit(y_amax, m, bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(bf16x2_absmax(0u, out.x), out.y), out.z), out.w));
   }
 }
 

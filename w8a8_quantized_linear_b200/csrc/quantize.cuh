@@ -100,6 +100,18 @@ __device__ __forceinline__ float bf2_absmax_final(uint32_t m) {
   return fmaxf(fabsf(bf16_lo(m)), fabsf(bf16_hi(m)));
 }
 
+// Optional side jobs of the row quantizers in a fused chain of Linears (the
+// CHAIN instantiations; the others carry no code for them):
+// zero_out [zero_n] is cleared (the next projection's row-absmax buffer, which
+// its GEMM epilogue fills with atomicMax after this kernel has completed), and
+// amax_in, when given, holds each row's absmax as fp32 bits (written by the
+// producing GEMM's epilogue), so the row needs no reduction.
+__device__ __forceinline__ void clear_words(uint32_t* zero_out, int64_t zero_n) {
+  if (zero_out == nullptr) return;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < zero_n; i += stride) zero_out[i] = 0u;
+}
+
 // Block-wide max; every thread gets the result.  red: >= 32 floats of smem.
 __device__ __forceinline__ float block_max(float v, float* red) {
 #pragma unroll
@@ -118,13 +130,17 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 // One block per row (grid-stride over rows).  The row's 16-byte vectors
 // v = tid + j*blockDim are held in registers for j < kRowVecs; longer rows
 // re-read the remainder (an L2 hit) in the second pass.
-template <int QT>
+template <int QT, bool CHAIN = false>
 __global__ void __launch_bounds__(1024) quantize_rows_kernel(const __nv_bfloat16* __restrict__ x, int64_t ldx,
                                                              int64_t M, int64_t K, uint8_t* __restrict__ q,
-                                                             int64_t ldq, float* __restrict__ scale) {
+                                                             int64_t ldq, float* __restrict__ scale,
+                                                             const uint32_t* __restrict__ amax_in = nullptr,
+                                                             uint32_t* __restrict__ zero_out = nullptr,
+                                                             int64_t zero_n = 0) {
   __shared__ float red[32];
   griddep_launch();
   griddep_wait();   // x may be the previous kernel's output
+  if constexpr (CHAIN) clear_words(zero_out, zero_n);
   const int64_t nv = K >> 3;
   for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
     const uint4* row = reinterpret_cast<const uint4*>(x + m * ldx);
@@ -140,7 +156,7 @@ __global__ void __launch_bounds__(1024) quantize_rows_kernel(const __nv_bfloat16
     }
     for (int64_t v = threadIdx.x + static_cast<int64_t>(kRowVecs) * blockDim.x; v < nv; v += blockDim.x)
       mb = absmax8(__ldg(row + v), mb);
-    const float a = block_max(bf2_absmax_final(mb), red);
+    const float a = (CHAIN && amax_in != nullptr) ? __uint_as_float(amax_in[m]) : block_max(bf2_absmax_final(mb), red);
     const float s = absmax_scale<QT>(a);
     const float rcp = __frcp_rn(s);
     if (threadIdx.x == 0) scale[m] = s;
@@ -160,13 +176,17 @@ __global__ void __launch_bounds__(1024) quantize_rows_kernel(const __nv_bfloat16
 // (one pass over HBM).  Teams reduce the absmax with warp shuffles and, for
 // TW > 1, a per-team named barrier over double-buffered shared slots.
 constexpr int kTeamVecs = 8;
-template <int QT, int TW>
+template <int QT, int TW, bool CHAIN = false>
 __global__ void __launch_bounds__(256, 4) quantize_rows_team_kernel(const __nv_bfloat16* __restrict__ x, int64_t ldx,
                                                                  int64_t M, int64_t K, uint8_t* __restrict__ q,
-                                                                 int64_t ldq, float* __restrict__ scale) {
+                                                                 int64_t ldq, float* __restrict__ scale,
+                                                                 const uint32_t* __restrict__ amax_in = nullptr,
+                                                                 uint32_t* __restrict__ zero_out = nullptr,
+                                                                 int64_t zero_n = 0) {
   __shared__ float red[2][8];
   griddep_launch();
   griddep_wait();   // x may be the previous kernel's output
+  if constexpr (CHAIN) clear_words(zero_out, zero_n);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int team = warp / TW, tw = warp % TW;
   const int teams = (blockDim.x >> 5) / TW;
@@ -182,18 +202,23 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_team_kernel(const __nv_b
       const int v = tl + j * (32 * TW);
       if (v < nv) keep[j] = __ldg(row + v);
     }
-    uint32_t mb = 0;
+    float a;
+    if (CHAIN && amax_in != nullptr) {   // uniform over the kernel
+      a = __uint_as_float(amax_in[m]);
+    } else {
+      uint32_t mb = 0;
 #pragma unroll
-    for (int j = 0; j < kTeamVecs; ++j)
-      if (tl + j * (32 * TW) < nv) mb = absmax8(keep[j], mb);
-    float a = bf2_absmax_final(mb);
+      for (int j = 0; j < kTeamVecs; ++j)
+        if (tl + j * (32 * TW) < nv) mb = absmax8(keep[j], mb);
+      a = bf2_absmax_final(mb);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
-    if constexpr (TW > 1) {
-      if (lane == 0) red[iter & 1][warp] = a;
-      asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(32 * TW) : "memory");
+      for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+      if constexpr (TW > 1) {
+        if (lane == 0) red[iter & 1][warp] = a;
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(32 * TW) : "memory");
 #pragma unroll
-      for (int i = 0; i < TW; ++i) a = fmaxf(a, red[iter & 1][team * TW + i]);
+        for (int i = 0; i < TW; ++i) a = fmaxf(a, red[iter & 1][team * TW + i]);
+      }
     }
     const float s = absmax_scale<QT>(a);
     const float rcp = __frcp_rn(s);

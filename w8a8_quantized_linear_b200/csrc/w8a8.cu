@@ -248,10 +248,12 @@ w8a8_status launch_gemv(const void* x, int64_t M, int64_t N, int64_t K, const vo
 constexpr int64_t kPairMinRows = 512;
 
 w8a8_status launch_quantize_rows(const void* x, int64_t ldx, int64_t M, int64_t K, int qt, void* q, int64_t ldq,
-                                 float* s, cudaStream_t st) {
+                                 float* s, cudaStream_t st, const uint32_t* amax_in = nullptr,
+                                 uint32_t* zero_out = nullptr, int64_t zero_n = 0) {
   const auto* xp = static_cast<const __nv_bfloat16*>(x);
   auto* qp = static_cast<uint8_t*>(q);
   const int64_t nv = K / 8;
+  const bool chain = amax_in != nullptr || zero_out != nullptr;
   const int64_t tw = (nv + 32 * kTeamVecs - 1) / (32 * kTeamVecs);   // warps per row
   if (tw <= 8) {
     int team_w = 1;
@@ -259,8 +261,11 @@ w8a8_status launch_quantize_rows(const void* x, int64_t ldx, int64_t M, int64_t 
     const int64_t teams = 8 / team_w;
     const int grid = static_cast<int>((M + teams - 1) / teams < (1 << 20) ? (M + teams - 1) / teams : (1 << 20));
     cudaError_t e = cudaSuccess;
-#define W8A8_TEAM_LAUNCH(QT, TW) \
-  e = launch_pdl(quantize_rows_team_kernel<QT, TW>, dim3(grid), dim3(256), 0, st, xp, ldx, M, K, qp, ldq, s)
+#define W8A8_TEAM_LAUNCH(QT, TW)                                                                                    \
+  e = chain ? launch_pdl(quantize_rows_team_kernel<QT, TW, true>, dim3(grid), dim3(256), 0, st, xp, ldx, M, K, qp, ldq, \
+                         s, amax_in, zero_out, zero_n)                                                                \
+            : launch_pdl(quantize_rows_team_kernel<QT, TW, false>, dim3(grid), dim3(256), 0, st, xp, ldx, M, K, qp,     \
+                         ldq, s, amax_in, zero_out, zero_n)
     if (qt == W8A8_E4M3) {
       switch (team_w) {
         case 1: W8A8_TEAM_LAUNCH(1, 1); break;
@@ -284,12 +289,17 @@ w8a8_status launch_quantize_rows(const void* x, int64_t ldx, int64_t M, int64_t 
     if (t < 32) t = 32;
     if (t > 1024) t = 1024;
     const int grid = static_cast<int>(M < (1 << 20) ? M : (1 << 20));
+    const dim3 gd(grid), bd(static_cast<unsigned>(t));
     const cudaError_t e =
         (qt == W8A8_E4M3)
-            ? launch_pdl(quantize_rows_kernel<1>, dim3(grid), dim3(static_cast<unsigned>(t)), 0, st, xp, ldx, M, K,
-                         qp, ldq, s)
-            : launch_pdl(quantize_rows_kernel<0>, dim3(grid), dim3(static_cast<unsigned>(t)), 0, st, xp, ldx, M, K,
-                         qp, ldq, s);
+            ? (chain ? launch_pdl(quantize_rows_kernel<1, true>, gd, bd, 0, st, xp, ldx, M, K, qp, ldq, s, amax_in,
+                                  zero_out, zero_n)
+                     : launch_pdl(quantize_rows_kernel<1, false>, gd, bd, 0, st, xp, ldx, M, K, qp, ldq, s, amax_in,
+                                  zero_out, zero_n))
+            : (chain ? launch_pdl(quantize_rows_kernel<0, true>, gd, bd, 0, st, xp, ldx, M, K, qp, ldq, s, amax_in,
+                                  zero_out, zero_n)
+                     : launch_pdl(quantize_rows_kernel<0, false>, gd, bd, 0, st, xp, ldx, M, K, qp, ldq, s, amax_in,
+                                  zero_out, zero_n));
     return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "quantize_rows launch");
   }
 }
@@ -360,7 +370,8 @@ SplitWs carve_split(Carve& c, int64_t M, int64_t Nout, const LinearWs& w, int qt
 
 // The finishing kernel of a split product (after the GEMM on the stream).
 w8a8_status launch_splitk_epilogue(int qt, const SplitWs& sk, int64_t M, int64_t Nout, const float* sx,
-                                   const float* sw, int axis, const void* bias, void* y, cudaStream_t st) {
+                                   const float* sw, int axis, const void* bias, void* y, cudaStream_t st,
+                                   int act = kActNone, uint32_t* y_amax = nullptr) {
   int sms = 0;
   w8a8_status s = current_device(nullptr, &sms);
   if (s != W8A8_OK) return s;
@@ -372,9 +383,9 @@ w8a8_status launch_splitk_epilogue(int qt, const SplitWs& sk, int64_t M, int64_t
   const cudaError_t e =
       (qt == W8A8_E4M3)
           ? launch_pdl(splitk_epilogue_kernel<kKindE4M3>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, part,
-                       sk.splits, M, Nout, sx, sw, axis, b, yp)
+                       sk.splits, M, Nout, sx, sw, axis, b, yp, act, y_amax)
           : launch_pdl(splitk_epilogue_kernel<kKindI8>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, part,
-                       sk.splits, M, Nout, sx, sw, axis, b, yp);
+                       sk.splits, M, Nout, sx, sw, axis, b, yp, act, y_amax);
   return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "split-K epilogue launch");
 }
 
@@ -411,7 +422,7 @@ CUtensorMapDataType code_type() { return CU_TENSOR_MAP_DATA_TYPE_UINT8; }
 // sk: split-K workspace (partial sums), or null for an unsplit product.
 w8a8_status gemm_fwd(const void* xq, int64_t lda, const float* sx, int64_t M, int64_t N, int64_t K, int qt,
                      const void* wq, const float* sw, int g, const void* bias, void* y, cudaStream_t st,
-                     const SplitWs* sk = nullptr) {
+                     const SplitWs* sk = nullptr, int act = kActNone, uint32_t* y_amax = nullptr) {
   alignas(64) CUtensorMap ta, tb;
   w8a8_status s = make_map(&ta, code_type(), 1, xq, K, M, lda, kBKBytes, kBM);
   if (s != W8A8_OK) return s;
@@ -425,6 +436,8 @@ w8a8_status gemm_fwd(const void* xq, int64_t lda, const float* sx, int64_t M, in
   ep.y = static_cast<__nv_bfloat16*>(y);
   ep.ldy = N;
   ep.splits = 1;
+  ep.act = act;
+  ep.y_amax = y_amax;
   if (sk != nullptr && sk->splits > 1) {
     ep.splits = sk->splits;
     ep.partial = sk->partial;
@@ -438,7 +451,7 @@ w8a8_status gemm_fwd(const void* xq, int64_t lda, const float* sx, int64_t M, in
   s = (qt == W8A8_E4M3) ? launch_gemm<kKindE4M3, false, 256, kEpiScale>(ta, tb, M, N, K, ep, st)
                         : launch_gemm<kKindI8, false, 256, kEpiScale>(ta, tb, M, N, K, ep, st);
   if (s != W8A8_OK || ep.splits == 1) return s;
-  return launch_splitk_epilogue(qt, *sk, M, N, sx, sw, g == W8A8_AXIS, bias, y, st);
+  return launch_splitk_epilogue(qt, *sk, M, N, sx, sw, g == W8A8_AXIS, bias, y, st, act, y_amax);
 }
 
 // dgrad: A = dyq [M, lda] (contraction N), B = wq [N, K] read MN-major.
@@ -530,7 +543,8 @@ w8a8_status gemm_bf16(const void* x, int64_t M, int64_t N, int64_t K, const void
   const uint32_t* part = ep.partial;
   const cudaError_t e =
       launch_pdl(splitk_epilogue_kernel<kKindBF16>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, part, splits, M,
-                 N, static_cast<const float*>(nullptr), static_cast<const float*>(nullptr), 0, ep.bias, ep.y);
+                 N, static_cast<const float*>(nullptr), static_cast<const float*>(nullptr), 0, ep.bias, ep.y,
+                 static_cast<int>(kActNone), static_cast<uint32_t*>(nullptr));
   return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "split-K epilogue launch");
 }
 
@@ -755,7 +769,7 @@ static w8a8_status svdq_fwd_impl(const void* x, int64_t M, int64_t N, int64_t K,
       const cudaError_t e = launch_pdl(splitk_epilogue_kernel<kKindBF16>, dim3(static_cast<unsigned>(grid)), dim3(256), 0,
                                        s, part, tsk.splits, M, static_cast<int64_t>(r), static_cast<const float*>(nullptr),
                                        static_cast<const float*>(nullptr), 0, static_cast<const __nv_bfloat16*>(nullptr),
-                                       t);
+                                       t, static_cast<int>(kActNone), static_cast<uint32_t*>(nullptr));
       if (e != cudaSuccess) return cuda_fail(e, "split-K epilogue launch");
     }
   }
@@ -992,28 +1006,41 @@ w8a8_status w8a8_qgemm_dgrad(const void* dyq, int64_t ldq, const float* sdy, int
 w8a8_status w8a8_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, w8a8_qtype qt, const void* wq,
                             const float* sw, w8a8_wgran g, const void* bias, void* y, void* ws, size_t ws_bytes,
                             w8a8_stream_t stream) {
+  return w8a8_linear_fwd_ex(x, M, N, K, qt, wq, sw, g, bias, W8A8_ACT_NONE, nullptr, nullptr, y, ws, ws_bytes, stream);
+}
+
+w8a8_status w8a8_linear_fwd_ex(const void* x, int64_t M, int64_t N, int64_t K, w8a8_qtype qt, const void* wq,
+                               const float* sw, w8a8_wgran g, const void* bias, w8a8_act act, const uint32_t* x_amax,
+                               uint32_t* y_amax, void* y, void* ws, size_t ws_bytes, w8a8_stream_t stream) {
   W8A8_CHECK(valid_qt(qt) && valid_g(g), W8A8_ERR_INVALID_ARG, "invalid qtype/granularity");
+  W8A8_CHECK(act == W8A8_ACT_NONE || act == W8A8_ACT_GELU || act == W8A8_ACT_GELU_TANH, W8A8_ERR_INVALID_ARG,
+             "invalid activation %d", static_cast<int>(act));
   W8A8_CHECK(M >= 0 && N >= 1 && M < (1ll << 31) && N < (1ll << 31), W8A8_ERR_UNSUPPORTED_SHAPE, "bad M/N");
   w8a8_status st = check_k(K, "K");
   if (st != W8A8_OK) return st;
   if (M == 0) return W8A8_OK;   // empty tensors may carry null pointers
   W8A8_CHECK(x && wq && sw && y, W8A8_ERR_INVALID_ARG, "null pointer");
-  W8A8_CHECK(aligned16(x) && aligned16(wq) && aligned16(sw) && aligned16(y) && (bias == nullptr || aligned16(bias)),
+  W8A8_CHECK(aligned16(x) && aligned16(wq) && aligned16(sw) && aligned16(y) && (bias == nullptr || aligned16(bias)) &&
+                 (x_amax == nullptr || aligned16(x_amax)) && (y_amax == nullptr || aligned16(y_amax)),
              W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
+  W8A8_CHECK(x_amax == nullptr || y_amax == nullptr || x_amax != y_amax, W8A8_ERR_INVALID_ARG,
+             "x_amax and y_amax must be different buffers");
   const LinearWs lw = linear_ws(M, K, N);
   W8A8_CHECK(ws != nullptr && ws_bytes >= lw.bytes, W8A8_ERR_WORKSPACE, "workspace too small: need %zu bytes",
              lw.bytes);
   W8A8_CHECK(aligned16(ws), W8A8_ERR_MISALIGNED, "workspace must be 16-byte aligned");
   if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (qt == W8A8_INT8 && M <= kGemvMaxRows && K <= kGemvMaxK)   // a few tokens: one weight-streaming launch
+  const bool plain = act == W8A8_ACT_NONE && x_amax == nullptr && y_amax == nullptr;
+  if (plain && qt == W8A8_INT8 && M <= kGemvMaxRows && K <= kGemvMaxK)   // a few tokens: one weight-streaming launch
     return launch_gemv(x, M, N, K, wq, sw, g == W8A8_AXIS, bias, y, s);
   Carve c(ws);
   void* xq = c.take(static_cast<size_t>(M * K));
   float* sx = static_cast<float*>(c.take(static_cast<size_t>(M) * 4));
   const SplitWs sk = carve_split(c, M, N, lw, qt);
-  if ((st = launch_quantize_rows(x, K, M, K, qt, xq, K, sx, s)) != W8A8_OK) return st;
-  return gemm_fwd(xq, K, sx, M, N, K, qt, wq, sw, g, bias, y, s, &sk);
+  // the quantizer clears y_amax; the GEMM's epilogue runs after it completes
+  if ((st = launch_quantize_rows(x, K, M, K, qt, xq, K, sx, s, x_amax, y_amax, y_amax ? M : 0)) != W8A8_OK) return st;
+  return gemm_fwd(xq, K, sx, M, N, K, qt, wq, sw, g, bias, y, s, &sk, static_cast<int>(act), y_amax);
 }
 
 w8a8_status w8a8_linear_fwd_noalloc(const void* x, int64_t M, int64_t N, int64_t K, w8a8_qtype qt, const void* wq,
