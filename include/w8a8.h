@@ -190,9 +190,11 @@ w8a8_status gguf_linear_fwd(const void* x_bf16, int64_t M, int64_t N, int64_t K,
  *   the activation codes and row scales of this call, and the int32 partial
  *   sums when an int8 product with few output tiles is split along K (the
  *   size depends on the shape only, never on the device).
- * int8 with M <= 8 and K <= 16384 runs as one weight-streaming launch that
- * quantizes the rows itself and leaves ws untouched; every path gives the
- * same bits.
+ * A few tokens run as one weight-streaming launch on the CUDA cores that
+ * quantizes the rows itself and leaves ws untouched: int8 with M <= 4 and
+ * K <= 16384 (dp4a; the same bits as every other path), e4m3 with M == 1
+ * and K <= 32768 (codes decoded to fp32, exact products, fp32 sums in
+ * another order: within the e4m3 bound).
  * ---------------------------------------------------------------------- */
 w8a8_status w8a8_linear_fwd(const void* x_bf16, int64_t M, int64_t N, int64_t K,
                             w8a8_qtype qt, const void* wq, const float* w_scale, w8a8_wgran g,

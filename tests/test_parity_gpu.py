@@ -344,13 +344,14 @@ def test_linear_fwd_m0_noop(w8):
     assert w8.linear_fwd(x, wq, sw).shape == (0, 32)
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 7, 16), (2, 300, 48), (5, 1000, 3072), (8, 513, 16384), (3, 64, 16400)])
+@pytest.mark.parametrize("M,N,K", [(1, 7, 16), (2, 300, 48), (4, 1000, 3072), (4, 513, 16384), (3, 64, 16400),
+                                   (5, 1000, 3072)])
 @pytest.mark.parametrize("gran", ["tensor", "axis"])
 def test_linear_fwd_few_tokens(w8, orc, M, N, K, gran):
-    """M <= 8 int8 forwards run as one weight-streaming launch (dp4a on the
-    CUDA cores, the rows quantized inside it; K <= 16384, else the GEMM):
-    bit-exact with the oracle and with the tensor-core product on the same
-    codes."""
+    """M <= 4 int8 forwards run as one weight-streaming launch (dp4a on the
+    CUDA cores, the rows quantized inside it; K <= 16384, else the GEMM; M = 5
+    takes the GEMM): bit-exact with the oracle and with the tensor-core
+    product on the same codes."""
     x = workloads.with_outlier_channels((M, K), 1.0, seed=M * 31 + K)
     w = workloads.normal((N, K), 0.02, seed=N + 17)
     bias = workloads.normal((N,), 0.01, seed=N + 18)
@@ -361,6 +362,31 @@ def test_linear_fwd_few_tokens(w8, orc, M, N, K, gran):
     assert np.array_equal(u16(y), ref["y"])
     xq, sx = w8.quantize_rows(x.to(DEV), "int8")
     assert torch.equal(y, w8.qgemm_fwd(xq, sx, wq, sw, bias=bias.to(DEV)))
+
+
+# the e4m3 few-token kernel (M <= 4): ragged N, K = 16 and K not a multiple
+# of 512, the largest K that fits (M = 1: 32768, M = 4: 8192), both weight
+# granularities
+@pytest.mark.parametrize("M,N,K,gran", [(1, 16, 16, "tensor"), (1, 3000, 4112, "axis"), (2, 257, 1024, "tensor"),
+                                        (3, 1000, 3072, "axis"), (4, 520, 8192, "tensor"), (1, 264, 32768, "axis"),
+                                        (4, 12288, 3072, "axis")])
+def test_linear_fwd_e4m3_few_tokens(w8, orc, M, N, K, gran):
+    x = workloads.with_outlier_channels((M, K), 1.0, seed=101 + M + K)
+    w = workloads.normal((N, K), 0.02, seed=102 + N)
+    bias = workloads.normal((N,), 0.01, seed=103)
+    wq, sw = w8.quantize_weight(w.to(DEV), "e4m3", gran)
+    y = w8.linear_fwd(x.to(DEV), wq, sw, bias=bias.to(DEV))
+    wqr, swr = orc.quantize_weight(workloads.to_u16(w), 1, 1 if gran == "axis" else 0)
+    assert np.array_equal(u8(wq), wqr)
+    ref = orc.linear_fwd(workloads.to_u16(x), wqr, swr, qt=1, bias=workloads.to_u16(bias))
+    ref["sw"] = swr[None, :] if gran == "axis" else swr[0]
+    err, bound = _fp8_tol(ref, u16(y))
+    assert np.all(err <= bound), float((err / bound).max())
+    # the same product through the tensor-core path (the chained entry point
+    # does not take the few-token kernel): both within the bound of the oracle
+    y2 = w8.linear_fwd_ex(x.to(DEV), wq, sw, bias=bias.to(DEV), y_amax=torch.zeros(M, dtype=torch.int32, device=DEV))
+    err2, bound2 = _fp8_tol(ref, u16(y2))
+    assert np.all(err2 <= bound2)
 
 
 def test_linear_fwd_split_equals_unsplit(w8):

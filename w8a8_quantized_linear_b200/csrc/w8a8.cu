@@ -209,7 +209,7 @@ w8a8_status launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, int64
   return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "gemm pair launch");
 }
 
-// The few-token int8 forward in one launch (gemv.cuh): M <= kGemvMaxRows,
+// The few-token int8 forward in one launch (gemv.cuh): M <= kGemvUseRows,
 // K <= kGemvMaxK; each block quantizes the M rows itself.
 w8a8_status launch_gemv(const void* x, int64_t M, int64_t N, int64_t K, const void* wq, const float* sw, int axis,
                         const void* bias, void* y, cudaStream_t st) {
@@ -237,7 +237,7 @@ w8a8_status launch_gemv(const void* x, int64_t M, int64_t N, int64_t K, const vo
                      static_cast<int>(N), static_cast<int>(K), wp, sw, axis, bp, yp);                            \
     break;
   switch (M) {
-    W8A8_GEMV(1) W8A8_GEMV(2) W8A8_GEMV(3) W8A8_GEMV(4) W8A8_GEMV(5) W8A8_GEMV(6) W8A8_GEMV(7) W8A8_GEMV(8)
+    W8A8_GEMV(1) W8A8_GEMV(2) W8A8_GEMV(3) W8A8_GEMV(4)
     default: return fail(W8A8_ERR_UNSUPPORTED_SHAPE, "gemv rows");
   }
 #undef W8A8_GEMV
@@ -613,6 +613,43 @@ w8a8_status noalloc_scratch(int dev, void** out) {
 }  // namespace w8a8
 
 using namespace w8a8;
+
+// The few-token e4m3 forward (gemv.cuh): M <= kGemvE4m3MaxRows and the M
+// activation rows (fp32, K rounded up to 512) within kGemvE4m3SmemBytes.
+static bool gemv_e4m3_fits(int64_t M, int64_t K) {
+  return M >= 1 && M <= kGemvE4m3MaxRows && M * ((K + 511) / 512) * 512 * 4 <= kGemvE4m3SmemBytes;
+}
+static w8a8_status launch_gemv_e4m3(const void* x, int64_t M, int64_t N, int64_t K, const void* wq, const float* sw,
+                                    int axis, const void* bias, void* y, cudaStream_t st) {
+  int dev = 0, sms = 0;
+  w8a8_status s = current_device(&dev, &sms);
+  if (s != W8A8_OK) return s;
+  static std::atomic<uint64_t> smem_set[kGemvE4m3MaxRows] = {};
+  const size_t smem = static_cast<size_t>(M * ((K + 511) / 512) * 512 * 4);
+  const int64_t reg_cap = M == 1 ? 4 : (M == 2 ? 3 : 2);   // gemv_e4m3_min_blocks
+  int64_t per_sm = static_cast<int64_t>(200 * 1024) / static_cast<int64_t>(smem + 1024);
+  per_sm = per_sm < 1 ? 1 : (per_sm > reg_cap ? reg_cap : per_sm);
+  int64_t grid = (N + kGemvThreads / 32 - 1) / (kGemvThreads / 32);
+  if (grid > per_sm * sms) grid = per_sm * sms;
+  const auto* xp = static_cast<const __nv_bfloat16*>(x);
+  const auto* wp = static_cast<const uint8_t*>(wq);
+  const auto* bp = static_cast<const __nv_bfloat16*>(bias);
+  auto* yp = static_cast<__nv_bfloat16*>(y);
+  cudaError_t e = cudaSuccess;
+#define W8A8_GEMV_E4(MM)                                                                                          \
+  case MM:                                                                                                        \
+    e = set_smem_once(gemv_e4m3_kernel<MM>, kGemvE4m3SmemBytes, dev, smem_set[MM - 1]);                           \
+    if (e == cudaSuccess)                                                                                         \
+      e = launch_pdl(gemv_e4m3_kernel<MM>, dim3(static_cast<unsigned>(grid)), dim3(kGemvThreads), smem, st, xp, K, \
+                     static_cast<int>(N), static_cast<int>(K), wp, sw, axis, bp, yp);                             \
+    break;
+  switch (M) {
+    W8A8_GEMV_E4(1)
+    default: return fail(W8A8_ERR_UNSUPPORTED_SHAPE, "gemv rows");
+  }
+#undef W8A8_GEMV_E4
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "gemv launch");
+}
 
 // Q8_0 -> axis-wise codes of type QT (0 int8, 1 e4m3).
 template <int QT>
@@ -1032,8 +1069,14 @@ w8a8_status w8a8_linear_fwd_ex(const void* x, int64_t M, int64_t N, int64_t K, w
   if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool plain = act == W8A8_ACT_NONE && x_amax == nullptr && y_amax == nullptr;
-  if (plain && qt == W8A8_INT8 && M <= kGemvMaxRows && K <= kGemvMaxK)   // a few tokens: one weight-streaming launch
+  // A few tokens: one weight-streaming launch on the CUDA cores.  Measured
+  // at N = 12288, K = 3072 against quantize + tensor-core GEMM: int8 wins up
+  // to 4 rows (9.5 / 11.5 / 13.9 / 16.8 us against 14.5 / 15.9 / 17.1 / 18.5),
+  // e4m3 (decoded in fp32) only for one row (13.5 against 17.6 us).
+  if (plain && qt == W8A8_INT8 && M <= kGemvUseRows && K <= kGemvMaxK)
     return launch_gemv(x, M, N, K, wq, sw, g == W8A8_AXIS, bias, y, s);
+  if (plain && qt == W8A8_E4M3 && M == 1 && gemv_e4m3_fits(M, K))
+    return launch_gemv_e4m3(x, M, N, K, wq, sw, g == W8A8_AXIS, bias, y, s);
   Carve c(ws);
   void* xq = c.take(static_cast<size_t>(M * K));
   float* sx = static_cast<float*>(c.take(static_cast<size_t>(M) * 4));
