@@ -792,6 +792,21 @@ def extras(w8, torch, workloads, dev, peaks, src):
         res[name] = {"ms": ms, "TFLOPS": ops / ms / 1e9, "frac_bf16_burst": ops / ms / 1e9 / tcb}
         del sets
     out["weight_only_fwd_4608x12288x3072"] = res
+    # their input gradients through the same weight: dY [4608, 12288] -> dX [4608, 3072]
+    dy0 = workloads.normal((M_TOK, MLP), 1e-3, 7).to(dev)
+    wsd = w8.workspace_bytes(w8.OP_WEIGHT_ONLY_DGRAD, M_TOK, MLP, HID)
+    res = {}
+    for name, mk in (("bf16_gemm", lambda dd, ws: (lambda: w8.bf16_linear_dgrad(dd, wb0, ws=ws))),
+                     ("float8", lambda dd, ws: (lambda: w8.float8_linear_dgrad(dd, wq8, sw8, ws=ws))),
+                     ("gguf", lambda dd, ws: (lambda: w8.gguf_linear_dgrad(dd, wgg, HID, ws=ws)))):
+        sets = []
+        for i in range(_nsets(nbytes(dy0) + M_TOK * HID * 2)):
+            sets.append(mk(dy0.clone(), torch.empty(max(wsd, 16), dtype=torch.uint8, device=dev)))
+        ms = _time_rot(sets, 20, torch, stream)
+        res[name] = {"ms": ms, "TFLOPS": ops / ms / 1e9, "frac_bf16_burst": ops / ms / 1e9 / tcb}
+        del sets
+    out["weight_only_dgrad_4608x12288x3072"] = res
+    del dy0
     # the two dequantizations alone (12288 x 3072 weight -> bf16)
     sets_e, sets_g = [], []
     for i in range(_nsets(MLP * HID * 3)):

@@ -70,7 +70,9 @@ typedef enum {
   W8A8_OP_SVDQ_FWD = 2,        /* svdq_linear_fwd                          */
   W8A8_OP_QUANTIZE_WEIGHT = 3, /* w8a8_quantize_weight (TENSOR needs 256 B) */
   W8A8_OP_BF16_FWD = 4,        /* bf16_linear_fwd                          */
-  W8A8_OP_WEIGHT_ONLY_FWD = 5  /* float8_linear_fwd, gguf_linear_fwd        */
+  W8A8_OP_WEIGHT_ONLY_FWD = 5, /* float8_linear_fwd, gguf_linear_fwd        */
+  W8A8_OP_BF16_DGRAD = 6,      /* bf16_linear_dgrad                        */
+  W8A8_OP_WEIGHT_ONLY_DGRAD = 7 /* float8_linear_dgrad, gguf_linear_dgrad  */
 } w8a8_op;
 
 /* ------------------------------------------------------------------------
@@ -176,6 +178,21 @@ w8a8_status float8_linear_fwd(const void* x_bf16, int64_t M, int64_t N, int64_t 
 w8a8_status gguf_linear_fwd(const void* x_bf16, int64_t M, int64_t N, int64_t K, const void* blocks,
                             const void* bias_bf16, void* y_bf16, void* ws, size_t ws_bytes,
                             w8a8_stream_t stream);
+
+/* The input gradients of the weight-only types (the LoRA training through
+ * the frozen, dequantized weight):  dX = bf16( fp32(sum_n dY[m,n] W[n,k]) ),
+ * the bf16 weight read with its rows as the contraction (no transposed
+ * copy).  dy [M, N] bf16 with N % 8 == 0, dx [M, K] bf16, K % 16 == 0.
+ * ws: w8a8_workspace_bytes(W8A8_OP_BF16_DGRAD, ...) for the bf16 weight,
+ * W8A8_OP_WEIGHT_ONLY_DGRAD for the float8 / GGUF weights (the dequantized
+ * weight first, then the split partial sums). */
+w8a8_status bf16_linear_dgrad(const void* dy_bf16, int64_t M, int64_t N, int64_t K, const void* w_bf16,
+                              void* dx_bf16, void* ws, size_t ws_bytes, w8a8_stream_t stream);
+w8a8_status float8_linear_dgrad(const void* dy_bf16, int64_t M, int64_t N, int64_t K, const void* wq,
+                                const float* w_scale, void* dx_bf16, void* ws, size_t ws_bytes,
+                                w8a8_stream_t stream);
+w8a8_status gguf_linear_dgrad(const void* dy_bf16, int64_t M, int64_t N, int64_t K, const void* blocks,
+                              void* dx_bf16, void* ws, size_t ws_bytes, w8a8_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * W8A8 Linear forward (OneTrainer wiki, int/float W8A8): quantize X

@@ -459,3 +459,10 @@ def float8_linear_fwd(x_bf16, wq, s_w, bias=None):
 def gguf_linear_fwd(x_bf16, blocks, N, K, bias=None):
     """GGUF (weight-only) forward: W = bf16(f16(d) q) [N, K], then the bf16 Linear."""
     return linear_bf16(x_bf16, q8_0_dequantize_bf16(blocks, N * K).reshape(N, K), bias)
+
+
+def linear_bf16_dgrad(dy_bf16, w_bf16):
+    """dX = bf16(fp32(dY W)): the bf16 Linear with the explicit transposed
+    weight W^T [K, N] (the contraction runs over W's rows)."""
+    w = _c(w_bf16, np.uint16)
+    return linear_bf16(dy_bf16, np.ascontiguousarray(w.T))

@@ -141,6 +141,11 @@ def test_weight_only_validation(L):
     assert L.w8a8_dequantize_e4m3_bf16(A, 24, A, A, None) == 2                      # n % 16
     assert L.w8a8_dequantize_e4m3_bf16(A, 32, None, A, None) == 1
     assert L.q8_0_dequantize_bf16(A, 3, B, None) == 3
+    assert L.bf16_linear_dgrad(A, 8, 12, 32, A, A, A, 1 << 20, None) == 2      # N % 8
+    assert L.bf16_linear_dgrad(A, 8, 16, 24, A, A, A, 1 << 20, None) == 2      # K % 16
+    assert L.float8_linear_dgrad(A, 8, 16, 32, A, None, A, A, 1 << 20, None) == 1
+    assert L.gguf_linear_dgrad(A, 8, 16, 32, A, A, A, 64, None) == 4
+    assert L.bf16_linear_dgrad(A, 0, 16, 32, None, None, None, 0, None) == 0     # M = 0
 
 
 def test_q8_0_validation(L):

@@ -396,3 +396,15 @@ def test_row_absmax_and_activated_forward(orc):
     yh = np.zeros((4, 9), np.float32)
     yh[0, 8], yh[1, 0], yh[2, 4], yh[2, 5] = -3.0, 2.5, 1.0, -0.5
     assert orc.row_absmax_bf16(orc.f32_to_bf16(yh)).tolist() == [3.0, 2.5, 1.0, 0.0]
+
+
+def test_linear_bf16_dgrad_is_the_textbook_product(orc):
+    """dX = dY W with integer operands: exact, and non-square so that a
+    transposed operand cannot pass."""
+    g = np.random.default_rng(43)
+    dy = g.integers(-8, 9, size=(5, 24)).astype(np.float32)
+    w = g.integers(-8, 9, size=(24, 40)).astype(np.float32)
+    to = lambda a: workloads.to_u16(torch.from_numpy(a).to(torch.bfloat16))
+    r = orc.linear_bf16_dgrad(to(dy), to(w))
+    assert r["acc"].shape == (5, 40)
+    assert np.array_equal(r["acc"], (dy.astype(np.int64) @ w.astype(np.int64)).astype(np.float64))

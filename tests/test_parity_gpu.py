@@ -663,6 +663,43 @@ def test_gguf_weight_only_parity(w8, orc, M, N, K):
     assert np.all(err <= bound), float((err / bound).max())
 
 
+# input gradients: (600, 520, 512) and (1024, 1024, 3072) the CTA pair (the
+# weight read MN-major, two 64-column atoms per CTA), (1, 3072, 4096) and
+# (64, 1024, 3072) split along the contraction, the rest single-SM tiles
+BF16_DGRAD_SHAPES = [(600, 520, 512), (1024, 1024, 3072), (1, 3072, 4096), (64, 1024, 3072), (130, 264, 96),
+                     (300, 520, 640)]
+
+
+@pytest.mark.parametrize("M,N,K", BF16_DGRAD_SHAPES)
+def test_bf16_linear_dgrad_parity(w8, orc, M, N, K):
+    dy = workloads.normal((M, N), 1e-3, seed=111 + M)
+    w = workloads.normal((N, K), 0.02, seed=112 + N)
+    dx = w8.bf16_linear_dgrad(dy.to(DEV), w.to(DEV))
+    ref = orc.linear_bf16_dgrad(workloads.to_u16(dy), workloads.to_u16(w))
+    err, bound = _bf16_tol(ref, u16(dx), N)
+    assert np.all(err <= bound), float((err / bound).max())
+
+
+@pytest.mark.parametrize("M,N,K", [(600, 520, 512), (64, 1024, 3072), (130, 264, 96)])
+@pytest.mark.parametrize("kind", ["float8", "gguf"])
+def test_weight_only_dgrad_parity(w8, orc, M, N, K, kind):
+    dy = workloads.normal((M, N), 1e-3, seed=113 + M)
+    w32 = workloads.normal((N, K), 0.02, seed=114 + N).float()
+    if kind == "float8":
+        wb = w32.to(torch.bfloat16)
+        wq, sw = w8.quantize_weight(wb.to(DEV), "e4m3", "tensor")
+        dx = w8.float8_linear_dgrad(dy.to(DEV), wq, sw)
+        wqr, swr = orc.quantize_weight(workloads.to_u16(wb), 1, 0)
+        wd = orc.dequant_e4m3_bf16(wqr, swr).reshape(N, K)
+    else:
+        br, _ = orc.q8_0_quantize(w32.numpy().reshape(-1))
+        dx = w8.gguf_linear_dgrad(dy.to(DEV), torch.from_numpy(br).to(DEV), K)
+        wd = orc.q8_0_dequantize_bf16(br, N * K).reshape(N, K)
+    ref = orc.linear_bf16_dgrad(workloads.to_u16(dy), wd)
+    err, bound = _bf16_tol(ref, u16(dx), N)
+    assert np.all(err <= bound), float((err / bound).max())
+
+
 def test_weight_only_m0_and_unsplit_equal_split(w8):
     x = workloads.normal((64, 3072), 1.0, 88).to(DEV)
     w = workloads.normal((1024, 3072), 0.02, 89).to(DEV)

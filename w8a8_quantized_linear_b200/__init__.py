@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_PKG, "libw8a8.so")
 INT8, E4M3 = 0, 1
 TENSOR, AXIS = 0, 1
 OP_LINEAR_FWD, OP_LINEAR_DGRAD, OP_SVDQ_FWD, OP_QUANTIZE_WEIGHT = 0, 1, 2, 3
-OP_BF16_FWD, OP_WEIGHT_ONLY_FWD = 4, 5
+OP_BF16_FWD, OP_WEIGHT_ONLY_FWD, OP_BF16_DGRAD, OP_WEIGHT_ONLY_DGRAD = 4, 5, 6, 7
 ACTS = {"none": 0, "gelu": 1, "gelu_tanh": 2}
 
 STATUS = {0: "W8A8_OK", 1: "W8A8_ERR_INVALID_ARG", 2: "W8A8_ERR_UNSUPPORTED_SHAPE",
@@ -38,7 +38,7 @@ EXPORTS = ("w8a8_quantize_rows", "w8a8_quantize_weight", "q8_0_bytes", "q8_0_qua
            "w8a8_device_status", "w8a8_set_wait_limit_ns", "w8a8_selftest_wait",
            "w8a8_e4m3_encode", "w8a8_last_error", "w8a8_linear_fwd_noalloc", "q8_0_dequantize_bf16",
            "w8a8_dequantize_e4m3_bf16", "bf16_linear_fwd", "float8_linear_fwd", "gguf_linear_fwd",
-           "w8a8_linear_fwd_ex")
+           "w8a8_linear_fwd_ex", "bf16_linear_dgrad", "float8_linear_dgrad", "gguf_linear_dgrad")
 
 
 class W8A8Error(RuntimeError):
@@ -83,6 +83,9 @@ def lib() -> ctypes.CDLL:
             "bf16_linear_fwd": [_P, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P],
             "float8_linear_fwd": [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _SZ, _P],
             "gguf_linear_fwd": [_P, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P],
+            "bf16_linear_dgrad": [_P, _I64, _I64, _I64, _P, _P, _P, _SZ, _P],
+            "float8_linear_dgrad": [_P, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P],
+            "gguf_linear_dgrad": [_P, _I64, _I64, _I64, _P, _P, _P, _SZ, _P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -342,6 +345,49 @@ def linear_fwd_ex(x, wq, w_scale, bias=None, act="none", x_amax=None, y_amax=Non
                                     ACTS[act], _ptr(x_amax), _ptr(y_amax), _ptr(y), _ptr(ws), ws.numel(),
                                     _stream(x.device)))
     return y
+
+
+def _dgrad_out(dy, K, out):
+    _cuda_2d(dy, torch.bfloat16, "dy")
+    M, N = dy.shape
+    return M, N, (torch.empty((M, K), dtype=torch.bfloat16, device=dy.device) if out is None else out)
+
+
+def bf16_linear_dgrad(dy, w, out=None, ws=None):
+    """dX = bf16(dY W): dy [M, N], w [N, K] bf16."""
+    _cuda_2d(w, torch.bfloat16, "w")
+    N, K = w.shape
+    M, N2, dx = _dgrad_out(dy, K, out)
+    if N2 != N:
+        raise ValueError("dy must be [M, N] with w [N, K]")
+    ws = _workspace(OP_BF16_DGRAD, M, N, K, 0, dy.device, ws)
+    _check(lib().bf16_linear_dgrad(_ptr(dy), M, N, K, _ptr(w), _ptr(dx), _ptr(ws), ws.numel(), _stream(dy.device)))
+    return dx
+
+
+def float8_linear_dgrad(dy, wq, w_scale, out=None, ws=None):
+    """Weight-only float8 input gradient: dX = bf16(dY W), W = bf16(dec(wq) w_scale[0])."""
+    if wq.dtype != torch.float8_e4m3fn or wq.dim() != 2:
+        raise ValueError("wq must be float8_e4m3fn [N, K]")
+    N, K = wq.shape
+    M, N2, dx = _dgrad_out(dy, K, out)
+    if N2 != N:
+        raise ValueError("dy must be [M, N] with wq [N, K]")
+    ws = _workspace(OP_WEIGHT_ONLY_DGRAD, M, N, K, 0, dy.device, ws)
+    _check(lib().float8_linear_dgrad(_ptr(dy), M, N, K, _ptr(_as_bytes(wq)), _ptr(w_scale), _ptr(dx), _ptr(ws),
+                                     ws.numel(), _stream(dy.device)))
+    return dx
+
+
+def gguf_linear_dgrad(dy, blocks, K, out=None, ws=None):
+    """GGUF input gradient: dX = bf16(dY W), W = bf16(f16(d) q) [N, K] from the Q8_0 blocks."""
+    M, N, dx = _dgrad_out(dy, K, out)
+    if blocks.numel() < q8_0_bytes(N * K):
+        raise ValueError("blocks hold fewer than N*K values")
+    ws = _workspace(OP_WEIGHT_ONLY_DGRAD, M, N, K, 0, dy.device, ws)
+    _check(lib().gguf_linear_dgrad(_ptr(dy), M, N, K, _ptr(blocks), _ptr(dx), _ptr(ws), ws.numel(),
+                                   _stream(dy.device)))
+    return dx
 
 
 def linear_fwd_noalloc(x, wq, w_scale, out, bias=None):

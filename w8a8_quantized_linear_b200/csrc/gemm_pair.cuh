@@ -64,7 +64,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KIND, LR>::k
                      const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmT,
                      const __grid_constant__ CUtensorMap tmL2, int M, int N, int Kc, EpiParams ep) {
   using C = PairCfg<KIND, LR>;
-  static_assert(KIND != kKindBF16 || (!B_MN && !LR), "bf16 operands: K-major B, no low-rank branch");
+  static_assert(KIND != kKindBF16 || !LR, "bf16 operands: no low-rank branch");
   // bf16 operands (the weight-only Linear): y = bf16(acc (+ bias)), no scales
   constexpr int kEpi = (KIND == kKindBF16) ? kEpiPlain : kEpiScale;
   constexpr int BN = C::kBN;
@@ -153,10 +153,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KIND, LR>::k
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
           const uint32_t fb = mapa_shared(&full[stage], 0);   // the even CTA's full[stage]
           tma_load_2d_pair(sA + stage * C::kABytes, &tmA, fb, kb * C::kBK, m0);
-          if constexpr (!B_MN)
+          if constexpr (!B_MN) {
             tma_load_2d_pair(sB + stage * C::kBBytes, &tmB, fb, kb * C::kBK, nh);
-          else
+          } else if constexpr (KIND != kKindBF16) {
             tma_load_2d_pair(sB + stage * C::kBBytes, &tmB, fb, nh, kb * C::kBK);
+          } else {
+            // bf16 MN-major: this CTA's 128 columns are two 128-byte atoms of
+            // 64 columns, each [64 K rows][128 B]
+            tma_load_2d_pair(sB + stage * C::kBBytes, &tmB, fb, nh, kb * C::kBK);
+            tma_load_2d_pair(sB + stage * C::kBBytes + C::kBK * 128, &tmB, fb, nh + 64, kb * C::kBK);
+          }
           issued |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -204,7 +210,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KIND, LR>::k
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint64_t ad = sdesc_sw128(a_base + k * 32, 16, 1024);
-            const uint64_t bd = B_MN ? sdesc_sw128(b_base + k * (32 * 128), 16, 1024) : sdesc_sw128(b_base + k * 32, 16, 1024);
+            // MN-major B: an MMA's K rows (32 codes or 16 bf16) are rows of
+            // 128 bytes; bf16 atoms of 64 columns lie kBK rows apart (LBO)
+            const uint64_t bd = !B_MN ? sdesc_sw128(b_base + k * 32, 16, 1024)
+                                : (KIND == kKindBF16 ? sdesc_sw128(b_base + k * (16 * 128), C::kBK * 128, 1024)
+                                                     : sdesc_sw128(b_base + k * (32 * 128), 16, 1024));
             tc_mma_pair<KIND>(d, ad, bd, kIdesc, (kb > 0 || k > 0) ? 1u : 0u);
           }
           tc_commit_pair_mc(&empty[stage], 0x3);

@@ -507,6 +507,19 @@ size_t ws_bf16(int64_t M, int64_t N, int64_t K) {
   if (p) c.take(p);
   return c.off;
 }
+size_t ws_bf16_dgrad(int64_t M, int64_t N, int64_t K) {
+  Carve c(nullptr);
+  const size_t p = split_bytes(bf16_splits(M, K, N), M, K);
+  if (p) c.take(p);
+  return c.off;
+}
+size_t ws_weight_only_dgrad(int64_t M, int64_t N, int64_t K) {
+  Carve c(nullptr);
+  c.take(static_cast<size_t>(N) * static_cast<size_t>(K) * 2);
+  const size_t p = split_bytes(bf16_splits(M, K, N), M, K);
+  if (p) c.take(p);
+  return c.off;
+}
 size_t ws_weight_only(int64_t M, int64_t N, int64_t K) {
   Carve c(nullptr);
   c.take(static_cast<size_t>(N) * static_cast<size_t>(K) * 2);
@@ -515,37 +528,55 @@ size_t ws_weight_only(int64_t M, int64_t N, int64_t K) {
   return c.off;
 }
 
-w8a8_status gemm_bf16(const void* x, int64_t M, int64_t N, int64_t K, const void* w, const void* bias, void* y,
-                      Carve& c, cudaStream_t st) {
-  const int splits = bf16_splits(M, N, K);
+// fwd: y [M, N] = x [M, K] w[N, K]^T (+ bias).  dgrad (B_MN): y [M, K] =
+// x [M, N] w [N, K], the weight read MN-major (its rows are the
+// contraction); Nout = K, Kc = N.
+template <bool DGRAD>
+w8a8_status gemm_bf16_t(const void* x, int64_t M, int64_t N, int64_t K, const void* w, const void* bias, void* y,
+                        Carve& c, cudaStream_t st) {
+  const int64_t nout = DGRAD ? K : N, kc = DGRAD ? N : K;
+  const int splits = bf16_splits(M, nout, kc);
   alignas(64) CUtensorMap ta, tb;
-  w8a8_status s = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, K, M, K * 2, 64, kBM);
+  w8a8_status s = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, kc, M, kc * 2, 64, kBM);
   if (s != W8A8_OK) return s;
   EpiParams ep{};
   ep.bias = static_cast<const __nv_bfloat16*>(bias);
   ep.y = static_cast<__nv_bfloat16*>(y);
-  ep.ldy = N;
+  ep.ldy = nout;
   ep.splits = 1;
   if (splits == 1 && M >= kPairMinRows) {
-    if ((s = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w, K, N, K * 2, 64, 128)) != W8A8_OK) return s;
-    return launch_gemm_pair<kKindBF16, false>(ta, tb, M, N, K, ep, st);
+    if (DGRAD)
+      s = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w, K, N, K * 2, 64, 64);
+    else
+      s = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w, K, N, K * 2, 64, 128);
+    if (s != W8A8_OK) return s;
+    return launch_gemm_pair<kKindBF16, DGRAD>(ta, tb, M, nout, kc, ep, st);
   }
-  if ((s = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w, K, N, K * 2, 64, 256)) != W8A8_OK) return s;
+  if (DGRAD)
+    s = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w, K, N, K * 2, 64, 64);
+  else
+    s = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w, K, N, K * 2, 64, 256);
+  if (s != W8A8_OK) return s;
   if (splits > 1) {
     ep.splits = splits;
-    ep.partial = static_cast<uint32_t*>(c.take(split_bytes(splits, M, N)));
+    ep.partial = static_cast<uint32_t*>(c.take(split_bytes(splits, M, nout)));
   }
-  if ((s = launch_gemm<kKindBF16, false, 256, kEpiPlain>(ta, tb, M, N, K, ep, st)) != W8A8_OK || splits == 1) return s;
+  if ((s = launch_gemm<kKindBF16, DGRAD, 256, kEpiPlain>(ta, tb, M, nout, kc, ep, st)) != W8A8_OK || splits == 1)
+    return s;
   int sms = 0;
   if ((s = current_device(nullptr, &sms)) != W8A8_OK) return s;
-  int64_t grid = (M * (N / 8) + 255) / 256;
+  int64_t grid = (M * (nout / 8) + 255) / 256;
   if (grid > 8 * static_cast<int64_t>(sms)) grid = 8 * static_cast<int64_t>(sms);
   const uint32_t* part = ep.partial;
   const cudaError_t e =
       launch_pdl(splitk_epilogue_kernel<kKindBF16>, dim3(static_cast<unsigned>(grid)), dim3(256), 0, st, part, splits, M,
-                 N, static_cast<const float*>(nullptr), static_cast<const float*>(nullptr), 0, ep.bias, ep.y,
+                 nout, static_cast<const float*>(nullptr), static_cast<const float*>(nullptr), 0, ep.bias, ep.y,
                  static_cast<int>(kActNone), static_cast<uint32_t*>(nullptr));
   return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "split-K epilogue launch");
+}
+w8a8_status gemm_bf16(const void* x, int64_t M, int64_t N, int64_t K, const void* w, const void* bias, void* y,
+                      Carve& c, cudaStream_t st) {
+  return gemm_bf16_t<false>(x, M, N, K, w, bias, y, c, st);
 }
 
 // Q8_0 -> fp32 (BF16 = false) or bf16 values.
@@ -852,6 +883,8 @@ size_t w8a8_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
     case W8A8_OP_QUANTIZE_WEIGHT: return 256;
     case W8A8_OP_BF16_FWD: return ws_bf16(M, N, K);
     case W8A8_OP_WEIGHT_ONLY_FWD: return ws_weight_only(M, N, K);
+    case W8A8_OP_BF16_DGRAD: return ws_bf16_dgrad(M, N, K);
+    case W8A8_OP_WEIGHT_ONLY_DGRAD: return ws_weight_only_dgrad(M, N, K);
     default: return 0;
   }
 }
@@ -984,6 +1017,45 @@ w8a8_status float8_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, co
   void* wb = c.take(static_cast<size_t>(N) * static_cast<size_t>(K) * 2);
   if ((st = launch_dequant_e4m3(wq, N * K, w_scale, wb, s)) != W8A8_OK) return st;
   return gemm_bf16(x, M, N, K, wb, bias, y, c, s);
+}
+
+// dgrad argument checks: dy [M, N] (N % 8 == 0: 16-byte rows), dx [M, K].
+static w8a8_status check_bf16_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, const void* w, const void* dx,
+                                    const void* ws, size_t ws_bytes, size_t need, bool need_scale = false,
+                                    const void* scale = nullptr) {
+  W8A8_CHECK(N >= 8 && N % 8 == 0, W8A8_ERR_UNSUPPORTED_SHAPE, "N must be a multiple of 8 (16-byte dY rows)");
+  return check_bf16_linear(dy, M, N, K, w, nullptr, dx, ws, ws_bytes, need, need_scale, scale);
+}
+
+w8a8_status bf16_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, const void* w, void* dx, void* ws,
+                              size_t ws_bytes, w8a8_stream_t stream) {
+  w8a8_status st = check_bf16_dgrad(dy, M, N, K, w, dx, ws, ws_bytes, M > 0 ? ws_bf16_dgrad(M, N, K) : 0);
+  if (st != W8A8_OK || M == 0) return st;
+  Carve c(ws);
+  return gemm_bf16_t<true>(dy, M, N, K, w, nullptr, dx, c, reinterpret_cast<cudaStream_t>(stream));
+}
+
+w8a8_status float8_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, const void* wq,
+                                const float* w_scale, void* dx, void* ws, size_t ws_bytes, w8a8_stream_t stream) {
+  w8a8_status st = check_bf16_dgrad(dy, M, N, K, wq, dx, ws, ws_bytes, M > 0 ? ws_weight_only_dgrad(M, N, K) : 0,
+                                    true, w_scale);
+  if (st != W8A8_OK || M == 0) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Carve c(ws);
+  void* wb = c.take(static_cast<size_t>(N) * static_cast<size_t>(K) * 2);
+  if ((st = launch_dequant_e4m3(wq, N * K, w_scale, wb, s)) != W8A8_OK) return st;
+  return gemm_bf16_t<true>(dy, M, N, K, wb, nullptr, dx, c, s);
+}
+
+w8a8_status gguf_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, const void* blocks, void* dx, void* ws,
+                              size_t ws_bytes, w8a8_stream_t stream) {
+  w8a8_status st = check_bf16_dgrad(dy, M, N, K, blocks, dx, ws, ws_bytes, M > 0 ? ws_weight_only_dgrad(M, N, K) : 0);
+  if (st != W8A8_OK || M == 0) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Carve c(ws);
+  void* wb = c.take(static_cast<size_t>(N) * static_cast<size_t>(K) * 2);
+  if ((st = launch_q8_0_dequant<true>(blocks, N * K, wb, s)) != W8A8_OK) return st;
+  return gemm_bf16_t<true>(dy, M, N, K, wb, nullptr, dx, c, s);
 }
 
 w8a8_status gguf_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, const void* blocks, const void* bias,
