@@ -483,7 +483,7 @@ def test_svdq_parity_small(w8, orc, r):
 
 
 @pytest.mark.parametrize("M,N,K,r", [(600, 520, 512, 8), (777, 264, 384, 24), (1024, 1024, 1024, 32),
-                                     (520, 136, 256, 16), (530, 300, 256, 16)])
+                                     (520, 136, 256, 16), (530, 300, 256, 16), (601, 264, 272, 16)])
 def test_svdq_parity_pairs(w8, orc, M, N, K, r):
     """M >= 512 with N % 8 == 0 runs the CTA-pair kernel, whose low-rank sum
     is a second tensor-core product (256 x 128 tiles, ragged edges, r padded
