@@ -479,7 +479,7 @@ def run_case(args):
     import w8a8_quantized_linear_b200 as w8
     dev = torch.device("cuda", 0)
     if args.case in ("requant", "gguf_m1", "gguf_m64", "svdq", "requant_e4m3", "gguf_f_m1", "gguf_f_m4608",
-                     "svdq_e4m3", "wo_float8", "wo_gguf"):
+                     "svdq_e4m3", "wo_float8", "wo_gguf", "gguf_m512"):
         return run_other_case(args, torch, workloads, w8, dev)
     wl = workloads.dit_mlp()
     if args.case in ("up", "dgrad_up"):
@@ -509,7 +509,7 @@ def run_case(args):
 
 def run_other_case(args, torch, workloads, w8, dev):
     """requant / requant_e4m3: Q8_0 -> axis int8 / e4m3 of the 12288 x 3072
-    GGUF weight; gguf_m1 / gguf_m64: the GGUF A8 int forward at M = 1 / 64;
+    GGUF weight; gguf_m1 / gguf_m64 / gguf_m512: the GGUF A8 int forward at M = 1 / 64 / 512;
     gguf_f_m1 / gguf_f_m4608: the GGUF A8 float forward at M = 1 / 4608;
     svdq / svdq_e4m3: the SVDQuant r = 32 forward at 4608 x 3072 x 3072 with
     an int8 / e4m3 residual; wo_float8 / wo_gguf: the weight-only forwards
@@ -529,7 +529,7 @@ def run_other_case(args, torch, workloads, w8, dev):
         x = d["x"].to(dev)
         fn = lambda: w8.svdq_linear_fwd(x, prep["rq"], prep["r_scale"], prep["l1"], prep["l2"])
     else:
-        g = workloads.gguf_q8_0(M=4608 if args.case == "gguf_f_m4608" else 64)
+        g = workloads.gguf_q8_0(M=4608 if args.case == "gguf_f_m4608" else 512)
         N, K = g["w_f32"].shape
         blk = w8.q8_0_quantize(g["w_f32"].reshape(-1).to(dev))
         if args.case == "requant":
@@ -542,7 +542,7 @@ def run_other_case(args, torch, workloads, w8, dev):
             fn = lambda: w8.linear_fwd(x, wq, sw)
         else:
             wq, sw = w8.q8_0_to_axis_int8(blk, N, K)
-            x = g["x"][:1 if args.case == "gguf_m1" else 64].to(dev)
+            x = g["x"][:{"gguf_m1": 1, "gguf_m64": 64, "gguf_m512": 512}[args.case]].to(dev)
             fn = lambda: w8.linear_fwd(x, wq, sw)
     for _ in range(args.warmup + args.steps):
         fn()
@@ -841,7 +841,7 @@ def main():
     ap.add_argument("--no-extras", dest="extras", action="store_false")
     ap.add_argument("--case", choices=["up", "down", "dgrad_down", "dgrad_up", "requant", "gguf_m1", "gguf_m64", "svdq",
                                        "requant_e4m3", "gguf_f_m1", "gguf_f_m4608", "svdq_e4m3", "wo_float8",
-                                       "wo_gguf"],
+                                       "wo_gguf", "gguf_m512"],
                     default=None, help="run only one of the step's four quantize+GEMM pairs, or one other kernel "
                                        "of the path (for profiling), no JSON")
     args = ap.parse_args()

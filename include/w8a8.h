@@ -208,10 +208,11 @@ w8a8_status gguf_linear_dgrad(const void* dy_bf16, int64_t M, int64_t N, int64_t
  *   sums when an int8 product with few output tiles is split along K (the
  *   size depends on the shape only, never on the device).
  * A few tokens run as one weight-streaming launch on the CUDA cores that
- * quantizes the rows itself and leaves ws untouched: int8 with M <= 4 and
+ * quantizes the rows itself and leaves ws untouched: int8 with M <= 2 and
  * K <= 16384 (dp4a; the same bits as every other path), e4m3 with M == 1
  * and K <= 32768 (codes decoded to fp32, exact products, fp32 sums in
- * another order: within the e4m3 bound).
+ * another order: within the e4m3 bound).  Up to 128 tokens otherwise run the
+ * transposed tensor-core product (the weight as the 128-row operand).
  * ---------------------------------------------------------------------- */
 w8a8_status w8a8_linear_fwd(const void* x_bf16, int64_t M, int64_t N, int64_t K,
                             w8a8_qtype qt, const void* wq, const float* w_scale, w8a8_wgran g,

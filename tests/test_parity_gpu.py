@@ -344,14 +344,15 @@ def test_linear_fwd_m0_noop(w8):
     assert w8.linear_fwd(x, wq, sw).shape == (0, 32)
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 7, 16), (2, 300, 48), (4, 1000, 3072), (4, 513, 16384), (3, 64, 16400),
-                                   (5, 1000, 3072)])
+@pytest.mark.parametrize("M,N,K", [(1, 7, 16), (2, 300, 48), (2, 513, 16384), (2, 64, 16400), (4, 1000, 3072),
+                                   (64, 1000, 3072), (128, 264, 4096), (33, 12288, 3072)])
 @pytest.mark.parametrize("gran", ["tensor", "axis"])
 def test_linear_fwd_few_tokens(w8, orc, M, N, K, gran):
-    """M <= 4 int8 forwards run as one weight-streaming launch (dp4a on the
-    CUDA cores, the rows quantized inside it; K <= 16384, else the GEMM; M = 5
-    takes the GEMM): bit-exact with the oracle and with the tensor-core
-    product on the same codes."""
+    """M <= 2 int8 forwards run as one weight-streaming launch (dp4a on the
+    CUDA cores, the rows quantized inside it; K <= 16384, else the GEMM);
+    up to 128 tokens the transposed tensor-core product (weight rows as the
+    MMA's M, split along K for few weight tiles): bit-exact with the oracle
+    and with the tensor-core product on the same codes."""
     x = workloads.with_outlier_channels((M, K), 1.0, seed=M * 31 + K)
     w = workloads.normal((N, K), 0.02, seed=N + 17)
     bias = workloads.normal((N,), 0.01, seed=N + 18)
@@ -364,9 +365,9 @@ def test_linear_fwd_few_tokens(w8, orc, M, N, K, gran):
     assert torch.equal(y, w8.qgemm_fwd(xq, sx, wq, sw, bias=bias.to(DEV)))
 
 
-# the e4m3 few-token kernel (M <= 4): ragged N, K = 16 and K not a multiple
-# of 512, the largest K that fits (M = 1: 32768, M = 4: 8192), both weight
-# granularities
+# e4m3 few-token forwards: M = 1 runs the CUDA-core kernel (K up to 32768),
+# 2..4 the transposed tensor-core product; ragged N, K = 16 and K not a
+# multiple of 512, both weight granularities
 @pytest.mark.parametrize("M,N,K,gran", [(1, 16, 16, "tensor"), (1, 3000, 4112, "axis"), (2, 257, 1024, "tensor"),
                                         (3, 1000, 3072, "axis"), (4, 520, 8192, "tensor"), (1, 264, 32768, "axis"),
                                         (4, 12288, 3072, "axis")])

@@ -33,7 +33,7 @@ constexpr int kBM = 128;
 constexpr int kBKBytes = 128;
 
 enum { kKindI8 = 0, kKindE4M3 = 1, kKindBF16 = 2 };
-enum { kEpiScale = 0, kEpiLowRank = 1, kEpiPlain = 2 };
+enum { kEpiScale = 0, kEpiLowRank = 1, kEpiPlain = 2, kEpiScaleT = 3 };
 
 struct EpiParams {
   const float* s_row;            // [M] row (token) scales          (kEpiScale/LowRank)
@@ -315,9 +315,11 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
             tma_load_2d(b + j * (C::kBK * 128), &tmB, &full[st], n0 + j * (128 / C::kElem), kb * C::kBK);
         }
       };
-      // The weight (B) tiles of the first unit's first stages are requested
+      // The weight tiles of the first unit's first stages are requested
       // before waiting for the previous kernel, which never writes them; the
-      // activation codes (A) it may be producing are read after the wait.
+      // activation codes it may be producing are read after the wait.  The
+      // weight is B, or A in the transposed form (kEpiScaleT).
+      constexpr bool kWeightA = (EPI == kEpiScaleT);
       int pre = 0;
       if (static_cast<int>(blockIdx.x) < num_units) {
         const int tile = blockIdx.x / splits, split = blockIdx.x - tile * splits;
@@ -325,7 +327,10 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
         pre = (kb1 - kb0) < kStages ? (kb1 - kb0) : kStages;
         for (int i = 0; i < pre; ++i) {
           mbar_arrive_expect_tx(&full[i], C::kStageBytes);
-          load_b(i, kb0 + i, (tile / tiles_m) * BN);
+          if constexpr (kWeightA)
+            tma_load_2d(sA + i * C::kABytes, &tmA, &full[i], (kb0 + i) * C::kBK, (tile % tiles_m) * kBM);
+          else
+            load_b(i, kb0 + i, (tile / tiles_m) * BN);
           issued |= 1u << i;
         }
       }
@@ -337,12 +342,18 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, 0x100u | stage, limit)) { ok = false; break; }
           if (pre > 0) {
-            --pre;   // this stage's B tile and byte count are in flight already
+            --pre;   // this stage's weight tile and byte count are in flight already
           } else {
             mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-            load_b(stage, kb, n0);
+            if constexpr (kWeightA)
+              tma_load_2d(sA + stage * C::kABytes, &tmA, &full[stage], kb * C::kBK, m0);
+            else
+              load_b(stage, kb, n0);
           }
-          tma_load_2d(sA + stage * C::kABytes, &tmA, &full[stage], kb * C::kBK, m0);
+          if constexpr (kWeightA)
+            load_b(stage, kb, n0);
+          else
+            tma_load_2d(sA + stage * C::kABytes, &tmA, &full[stage], kb * C::kBK, m0);
           issued |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -528,6 +539,44 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
               bulk_commit();
             }
             ++out_iter;
+          }
+        }
+      } else if constexpr (EPI == kEpiScaleT) {
+        // Transposed product (few tokens): the kernel's rows are weight rows n
+        // (A = the weight codes) and its columns tokens m (B = the activation
+        // codes), so a lane holds y[m, n] for one n and the chunk's 32 m.
+        // y[m, n] = bf16(((acc * s_x[m]) * s_w[n or 0]) + bias[n]) - the fp32
+        // steps of the other epilogues - is stored for each m, 32 lanes
+        // writing 32 consecutive n; split partial sums go to partial[split][m][n].
+        const int row = m0 + quarter * 32 + lane;   // n
+        const bool row_ok = row < M;
+        const float swr = row_ok ? (ep.s_col_axis ? ep.s_col[row] : ep.s_col[0]) : 0.0f;
+        const float br = (ep.bias != nullptr && row_ok) ? __bfloat162float(ep.bias[row]) : 0.0f;
+  #pragma unroll 1
+        for (int c = group; c < BN / 32; c += kGroups) {
+          const int nc = n0 + c * 32;               // first token of the chunk
+          if (nc >= N) break;                       // warp-uniform
+          float sxc[32];
+  #pragma unroll
+          for (int j = 0; j < 32; ++j) sxc[j] = (nc + j < N) ? __ldg(ep.s_row + nc + j) : 0.0f;
+          uint32_t r[32];
+          tmem_ld_x32(tmem + lane_base + static_cast<uint32_t>(acc * BN + c * 32), r);
+          tmem_ld_wait();
+          if (row_ok) {
+            if (splits > 1) {
+              uint32_t* pcol = ep.partial + static_cast<int64_t>(split) * N * M + row;
+              for (int j = 0; j < 32; ++j)
+                if (nc + j < N) pcol[static_cast<int64_t>(nc + j) * M] = r[j];
+            } else {
+              for (int j = 0; j < 32; ++j) {
+                if (nc + j < N) {
+                  float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int>(r[j])) : __uint_as_float(r[j]);
+                  a = __fmul_rn(__fmul_rn(a, sxc[j]), swr);
+                  if (ep.bias != nullptr) a = __fadd_rn(a, br);
+                  ep.y[static_cast<int64_t>(nc + j) * ep.ldy + row] = __float2bfloat16_rn(a);
+                }
+              }
+            }
           }
         }
       } else {

@@ -16,7 +16,7 @@
 namespace w8a8 {
 
 constexpr int kGemvMaxRows = 8;    // rows the kernel supports
-constexpr int kGemvUseRows = 4;    // rows for which it beats quantize + GEMM (the library's choice)
+constexpr int kGemvUseRows = 2;    // rows for which it beats quantize + GEMM (the library's choice)
 constexpr int kGemvThreads = 256;
 constexpr int kGemvMaxK = 16384;   // M * K codes in shared memory: at most 128 KB
 

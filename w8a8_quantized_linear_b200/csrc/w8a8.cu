@@ -162,8 +162,13 @@ template <int KIND, bool B_MN, int BN, int EPI>
 w8a8_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t M, int64_t N, int64_t Kc,
                         EpiParams ep, cudaStream_t st) {
   alignas(64) CUtensorMap ty;
-  w8a8_status ms = make_out_map(&ty, &ep, M, N);
-  if (ms != W8A8_OK) return ms;
+  if constexpr (EPI == kEpiScaleT) {   // direct transposed stores, no output map
+    std::memset(&ty, 0, sizeof(ty));
+    ep.tma_store = 0;
+  } else {
+    w8a8_status ms = make_out_map(&ty, &ep, M, N);
+    if (ms != W8A8_OK) return ms;
+  }
   using C = GemmCfg<KIND, BN, EPI>;
   static std::atomic<uint64_t> smem_set{0};
   int dev = 0, sms = 0;
@@ -237,7 +242,7 @@ w8a8_status launch_gemv(const void* x, int64_t M, int64_t N, int64_t K, const vo
                      static_cast<int>(N), static_cast<int>(K), wp, sw, axis, bp, yp);                            \
     break;
   switch (M) {
-    W8A8_GEMV(1) W8A8_GEMV(2) W8A8_GEMV(3) W8A8_GEMV(4)
+    W8A8_GEMV(1) W8A8_GEMV(2)
     default: return fail(W8A8_ERR_UNSUPPORTED_SHAPE, "gemv rows");
   }
 #undef W8A8_GEMV
@@ -336,14 +341,33 @@ int choose_splits(int64_t M, int64_t Nout, int64_t Kc) {
   return s < 2 ? 1 : static_cast<int>(s);
 }
 
+// The transposed forward for few tokens (M <= kSwapMaxRows): the weight is
+// the 128-row MMA operand A and the tokens the N side (64 or 128 columns), so
+// no MMA rows are padding and each stage is mostly weight bytes.
+constexpr int64_t kSwapMaxRows = 128;
+bool use_swap(int64_t M) { return M >= 1 && M <= kSwapMaxRows; }
+int swap_bn(int64_t M) { return M <= 64 ? 64 : 128; }
+int choose_splits_t(int64_t M, int64_t Nout, int64_t Kc) {
+  const int64_t tiles = ((Nout + kBM - 1) / kBM) * ((M + swap_bn(M) - 1) / swap_bn(M));
+  const int64_t num_kb = (Kc + kBKBytes - 1) / kBKBytes;
+  if (tiles <= 0 || tiles * 2 > kSplitSms || (Nout % 8) != 0) return 1;
+  int64_t s = kSplitSms / tiles;
+  if (s > num_kb / 4) s = num_kb / 4;
+  if (s > 16) s = 16;
+  return s < 2 ? 1 : static_cast<int>(s);
+}
+
 // Workspace of a linear call: codes [M, ld] and row scales [M], then, when
-// the GEMM is split, the partial sums [S, M, Nout].
+// the GEMM is split, the partial sums [S, M, Nout] (for a forward with few
+// tokens, room for either layout's split count).
 struct LinearWs {
   size_t bytes;
   int splits;
 };
-LinearWs linear_ws(int64_t M, int64_t ld, int64_t Nout) {
-  LinearWs w{0, choose_splits(M, Nout, ld)};
+LinearWs linear_ws(int64_t M, int64_t ld, int64_t Nout, bool fwd = false) {
+  int sp = choose_splits(M, Nout, ld);
+  if (fwd && use_swap(M) && choose_splits_t(M, Nout, ld) > sp) sp = choose_splits_t(M, Nout, ld);
+  LinearWs w{0, sp};
   Carve c(nullptr);
   c.take(static_cast<size_t>(M * ld));
   c.take(static_cast<size_t>(M) * 4);
@@ -351,7 +375,7 @@ LinearWs linear_ws(int64_t M, int64_t ld, int64_t Nout) {
   w.bytes = c.off;
   return w;
 }
-size_t ws_linear(int64_t M, int64_t ld, int64_t Nout) { return linear_ws(M, ld, Nout).bytes; }
+size_t ws_linear(int64_t M, int64_t ld, int64_t Nout, bool fwd = false) { return linear_ws(M, ld, Nout, fwd).bytes; }
 
 // The split-K part of a carved workspace.
 struct SplitWs {
@@ -441,6 +465,25 @@ w8a8_status gemm_fwd(const void* xq, int64_t lda, const float* sx, int64_t M, in
   if (sk != nullptr && sk->splits > 1) {
     ep.splits = sk->splits;
     ep.partial = sk->partial;
+  }
+  if (use_swap(M) && act == kActNone && y_amax == nullptr) {
+    // transposed: A = the weight [N, K], B = the codes [M, K]; the kernel's
+    // rows are n and its columns m; split count chosen for this layout (the
+    // workspace has room for it)
+    if (ep.splits > 1) ep.splits = choose_splits_t(M, N, K);
+    const int bn = swap_bn(M);
+    if ((s = make_map(&ta, code_type(), 1, wq, K, N, K, kBKBytes, kBM)) != W8A8_OK) return s;
+    if ((s = make_map(&tb, code_type(), 1, xq, K, M, lda, kBKBytes, bn)) != W8A8_OK) return s;
+    if (bn == 64)
+      s = (qt == W8A8_E4M3) ? launch_gemm<kKindE4M3, false, 64, kEpiScaleT>(ta, tb, N, M, K, ep, st)
+                            : launch_gemm<kKindI8, false, 64, kEpiScaleT>(ta, tb, N, M, K, ep, st);
+    else
+      s = (qt == W8A8_E4M3) ? launch_gemm<kKindE4M3, false, 128, kEpiScaleT>(ta, tb, N, M, K, ep, st)
+                            : launch_gemm<kKindI8, false, 128, kEpiScaleT>(ta, tb, N, M, K, ep, st);
+    if (s != W8A8_OK || ep.splits == 1) return s;
+    SplitWs skt = *sk;
+    skt.splits = ep.splits;
+    return launch_splitk_epilogue(qt, skt, M, N, sx, sw, g == W8A8_AXIS, bias, y, st);
   }
   if (ep.splits == 1 && M >= kPairMinRows) {
     // B in halves of 128 rows, one per CTA of the pair
@@ -877,7 +920,7 @@ size_t q8_0_bytes(int64_t n) { return n <= 0 ? 0 : static_cast<size_t>((n + 31) 
 size_t w8a8_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
   if (M < 0 || N < 0 || K < 0) return 0;
   switch (op) {
-    case W8A8_OP_LINEAR_FWD: return ws_linear(M, K, N);
+    case W8A8_OP_LINEAR_FWD: return ws_linear(M, K, N, true);
     case W8A8_OP_LINEAR_DGRAD: return ws_linear(M, round_up(N, 16), K);
     case W8A8_OP_SVDQ_FWD: return ws_svdq(M, K, r);
     case W8A8_OP_QUANTIZE_WEIGHT: return 256;
@@ -1134,7 +1177,7 @@ w8a8_status w8a8_linear_fwd_ex(const void* x, int64_t M, int64_t N, int64_t K, w
              W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
   W8A8_CHECK(x_amax == nullptr || y_amax == nullptr || x_amax != y_amax, W8A8_ERR_INVALID_ARG,
              "x_amax and y_amax must be different buffers");
-  const LinearWs lw = linear_ws(M, K, N);
+  const LinearWs lw = linear_ws(M, K, N, true);
   W8A8_CHECK(ws != nullptr && ws_bytes >= lw.bytes, W8A8_ERR_WORKSPACE, "workspace too small: need %zu bytes",
              lw.bytes);
   W8A8_CHECK(aligned16(ws), W8A8_ERR_MISALIGNED, "workspace must be 16-byte aligned");
@@ -1142,9 +1185,10 @@ w8a8_status w8a8_linear_fwd_ex(const void* x, int64_t M, int64_t N, int64_t K, w
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool plain = act == W8A8_ACT_NONE && x_amax == nullptr && y_amax == nullptr;
   // A few tokens: one weight-streaming launch on the CUDA cores.  Measured
-  // at N = 12288, K = 3072 against quantize + tensor-core GEMM: int8 wins up
-  // to 4 rows (9.5 / 11.5 / 13.9 / 16.8 us against 14.5 / 15.9 / 17.1 / 18.5),
-  // e4m3 (decoded in fp32) only for one row (13.5 against 17.6 us).
+  // at N = 12288, K = 3072 against quantize + the transposed tensor-core
+  // GEMM (about 13.5-14 us from 3 to 64 rows): int8 wins for 1 and 2 rows
+  // (9.5 / 11.5 us; 13.9 at 3, 16.8 at 4), e4m3 (decoded in fp32) for one
+  // row only (13.5 us).
   if (plain && qt == W8A8_INT8 && M <= kGemvUseRows && K <= kGemvMaxK)
     return launch_gemv(x, M, N, K, wq, sw, g == W8A8_AXIS, bias, y, s);
   if (plain && qt == W8A8_E4M3 && M == 1 && gemv_e4m3_fits(M, K))
