@@ -639,6 +639,20 @@ def extras(w8, torch, workloads, dev, peaks, src):
         del sets
     out["dit_mlp_fwd_gelu_4608x3072x12288"] = res
     del xm0, w1q, w2q
+    # the tiny int W8A8 forward (256 x 512 x 512): latency-bound, reported
+    # without a bar
+    d = workloads.int_tiny()
+    wqt, swt = w8.quantize_weight(d["w"].to(dev), "int8", "tensor")
+    sets = []
+    for i in range(4):
+        xt = d["x"].to(dev).clone()
+        yt = torch.empty((256, 512), dtype=torch.bfloat16, device=dev)
+        wst = torch.empty(w8.workspace_bytes(0, 256, 512, 512), dtype=torch.uint8, device=dev)
+        sets.append(lambda xt=xt, yt=yt, wst=wst: w8.linear_fwd(xt, wqt, swt, out=yt, ws=wst))
+    ms = _time_rot(sets, 50, torch, stream)
+    out["int_w8a8_fwd_tiny_256x512x512"] = {"ms": ms, "TOPS": 2 * 256 * 512 * 512 / ms / 1e9,
+                                            "note": "inputs L2-resident (1 MB); launch- and latency-bound"}
+    del sets
     # float W8A8 forward (e4m3, bias) 4096 x 3072 x 3072
     d = workloads.float_w8a8()
     wq0, sw = w8.quantize_weight(d["w"].to(dev), "e4m3", "tensor")
