@@ -280,8 +280,8 @@ void orc_q8_0_to_axis_int8(const uint8_t* blocks, int64_t N, int64_t K,
 
 /* ========================================================================== */
 /* The activation between two projections and the row absmax of an output     */
-/* [SURVEY reading: the DiT MLP's GELU, optional; the fused absmax is a       */
-/* property of the output, max_n |y[m,n]|].                                   */
+/* (not on the pages: the optional GELU of a DiT MLP block, read plainly; the */
+/* row absmax is a property of the output, max_n |y[m,n]|).                   */
 /* ========================================================================== */
 
 /* GELU, exact form: 0.5 v (1 + erf(v / sqrt 2)); tanh form: 0.5 v (1 +
