@@ -566,7 +566,7 @@ def _time_rot(fns, reps, torch, stream):
     its own buffers), are captured once in a CUDA graph, and the graph is
     replayed between two events on the launching stream: host-side launch
     cost is left out, as in a captured model step (every call of the library
-    is stream-ordered and capturable)."""
+    is stream-ordered and capturable).  The fastest of three replays."""
     for f in fns:
         f()
     torch.cuda.synchronize()
@@ -578,13 +578,17 @@ def _time_rot(fns, reps, torch, stream):
     g.replay()
     torch.cuda.synchronize()
     E = lambda: torch.cuda.Event(enable_timing=True)
-    a, b = E(), E()
-    a.record(stream)
-    g.replay()
-    b.record(stream)
-    torch.cuda.synchronize()
+    best = None
+    for _ in range(3):   # the fastest of three replays (clock and scheduling noise)
+        a, b = E(), E()
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        t = a.elapsed_time(b) / n
+        best = t if best is None or t < best else best
     del g
-    return a.elapsed_time(b) / n
+    return best
 
 
 def extras(w8, torch, workloads, dev, peaks, src):
@@ -837,8 +841,8 @@ def extras(w8, torch, workloads, dev, peaks, src):
     out["q8_0_dequantize_bf16_12288x3072"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
     del sets_e, sets_g, xb0, wb0
     out["peaks"] = {"source": src, "hbm_gbs": hbm, "int8_burst_tops": tc8}
-    out["method"] = ("mean over reps replayed from one CUDA graph (no host launch cost), rotating through "
-                     ">= 3x L2 of input/output copies")
+    out["method"] = ("mean over the reps of one CUDA-graph replay (no host launch cost), rotating through "
+                     ">= 3x L2 of input/output copies; the fastest of three replays")
     assert w8.device_status() == 0
     return out
 
