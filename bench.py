@@ -591,6 +591,14 @@ def _time_rot(fns, reps, torch, stream):
     return best
 
 
+def _gemm_roof_ms(M, N, K, hbm_gbs, tops):
+    """Roofline time of a W8A8 forward in ms: the slower of streaming its
+    bytes (8-bit weight, bf16 activations in and out, 8-bit codes written and
+    read) at the copy bandwidth and its 2MNK operations at the 8-bit peak."""
+    nbytes = N * K + M * K * 2 + M * K * 2 + M * N * 2
+    return max(nbytes / (hbm_gbs * 1e9), 2.0 * M * N * K / (tops * 1e12)) * 1e3
+
+
 def extras(w8, torch, workloads, dev, peaks, src):
     """The other rows of the hot path, each timed on its own: mean over reps
     launched back to back, rotating through copies of the inputs and outputs
@@ -690,6 +698,7 @@ def extras(w8, torch, workloads, dev, peaks, src):
     ms = _time_rot(sets, 30, torch, stream)
     ops = 2 * M_TOK * 3072 * 3072
     out["svdquant_r32_fwd_4608x3072x3072"] = {"ms": ms, "TOPS_main": ops / ms / 1e9,
+                                              "frac_int8_burst": ops / ms / 1e9 / tc8,
                                               "lowrank_GFLOP": 2 * 2 * M_TOK * 3072 * 32 / 1e9}
     del sets, prep0
     # the same with an e4m3 residual (float W8A8 + SVDQuant)
@@ -704,6 +713,7 @@ def extras(w8, torch, workloads, dev, peaks, src):
                     w8.svdq_linear_fwd(xx, rq, prep0["r_scale"], l1, l2, out=y, ws=ws))
     ms = _time_rot(sets, 30, torch, stream)
     out["svdquant_e4m3_r32_fwd_4608x3072x3072"] = {"ms": ms, "TOPS_main": ops / ms / 1e9,
+                                                   "frac_fp8_burst": ops / ms / 1e9 / tc8,
                                                    "lowrank_GFLOP": 2 * 2 * M_TOK * 3072 * 32 / 1e9}
     del sets, prep0
     # GGUF Q8_0: standalone quantize / dequantize of 2^28 fp32 (each 1.3 GB of traffic)
@@ -760,7 +770,8 @@ def extras(w8, torch, workloads, dev, peaks, src):
             sets.append(lambda xm=xm, wq=wq, y=y, ws=ws: w8.linear_fwd(xm, wq, sw, out=y, ws=ws))
         ms = _time_rot(sets, 30, torch, stream)
         sweep[str(M)] = {"ms": ms, "TOPS": 2 * M * MLP * HID / ms / 1e9,
-                         "weight_GB/s": MLP * HID / (ms * 1e-3) / 1e9}
+                         "weight_GB/s": MLP * HID / (ms * 1e-3) / 1e9,
+                         "roofline_frac": _gemm_roof_ms(M, MLP, HID, hbm, tc8) / ms}
         del sets
     out["gguf_a8_int_fwd_sweep_N12288_K3072"] = sweep
     # GGUF A8 float: Q8_0 -> axis e4m3 (same traffic as the int8 requant), then
@@ -787,7 +798,8 @@ def extras(w8, torch, workloads, dev, peaks, src):
             sets.append(lambda xm=xm, wq=wq, y=y, ws=ws: w8.linear_fwd(xm, wq, sw, out=y, ws=ws))
         ms = _time_rot(sets, 30, torch, stream)
         sweep[str(M)] = {"ms": ms, "TOPS": 2 * M * MLP * HID / ms / 1e9,
-                         "weight_GB/s": MLP * HID / (ms * 1e-3) / 1e9}
+                         "weight_GB/s": MLP * HID / (ms * 1e-3) / 1e9,
+                         "roofline_frac": _gemm_roof_ms(M, MLP, HID, hbm, tc8) / ms}
         del sets
     out["gguf_a8_float_fwd_sweep_N12288_K3072"] = sweep
     # weight-only types (float8, GGUF) on the DiT up-projection: the weight
