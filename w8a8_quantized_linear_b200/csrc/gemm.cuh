@@ -89,14 +89,17 @@ struct GemmCfg {
   static constexpr int kLrBytes = (EPI == kEpiLowRank) ? BN * kLrStride * 2 : 0;
   static constexpr int kEpiWarps = 8;   // two per TMEM lane quarter, splitting the column chunks
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
-  // as many pipeline stages as the shared memory holds (4 for 128x256 tiles,
-  // 8 for 128x64 tiles, whose CTAs must keep more bytes in flight), at most 8
-  static constexpr int kFixedBytes = 1024 + ((kLrBytes + 1023) & ~1023) + kEpiWarps * 2 * 32 * 32 * 2 + 256;
-  static constexpr int kStagesFit = (232448 - kFixedBytes) / kStageBytes;
-  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   // per epilogue warp, two 32 x 32 bf16 staging buffers for the TMA store
+  // (none in the transposed form, which stores directly)
   static constexpr int kOutBufBytes = 32 * 32 * 2;
-  static constexpr int kOutBytes = kEpiWarps * 2 * kOutBufBytes;
+  static constexpr int kOutBytes = (EPI == kEpiScaleT) ? 0 : kEpiWarps * 2 * kOutBufBytes;
+  static constexpr int kFixedBytes = 1024 + ((kLrBytes + 1023) & ~1023) + kOutBytes + 256;
+  static constexpr int kStagesFit = (232448 - kFixedBytes) / kStageBytes;
+  // as many pipeline stages as the shared memory holds (4 for 128x256 tiles,
+  // 8 for 128x64 tiles, whose CTAs must keep more bytes in flight), at most
+  // 8, or 10 in the transposed form (a weight stream on few SMs)
+  static constexpr int kMaxStages = (EPI == kEpiScaleT) ? 10 : 8;
+  static constexpr int kStages = kStagesFit > kMaxStages ? kMaxStages : kStagesFit;
   static constexpr size_t kSmem = 1024 /*alignment slack*/ + static_cast<size_t>(kStages) * kStageBytes +
                                   ((kLrBytes + 1023) & ~1023) + kOutBytes + 256 /*barriers*/;
   static constexpr int kCtasPerSm = 1;
