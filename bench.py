@@ -41,9 +41,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic of one launch of the dominant kernel from an ncu capture, keyed
 # by the hash of the kernel source it was taken on (null when they differ).
-GEMM_TRAFFIC = {"source_sha": "755bca19a5dc6ae3", "bytes_per_launch": 122816000,
+GEMM_TRAFFIC = {"source_sha": "1d21b284b654280d", "bytes_per_launch": 123021056,
                 "note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one up-proj launch "
-                        "(bench.py --case up): 52.11 MB read + 70.71 MB written"}
+                        "(bench.py --case up): 52.05 MB read + 70.97 MB written"}
 
 
 def gemm_source_sha() -> str:
@@ -124,7 +124,7 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
         load = [v for v in sm if v >= 0.3 * max(mx or sm)] or sm
-        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(mx) if mx else None,
+        return {"sm_mhz": statistics.median(load), "sm_mhz_min": min(load), "sm_max_mhz": max(mx) if mx else None,
                 "power_w_max": max(pw) if pw else None, "reasons": reasons, "samples": len(mine)}
 
     def summary(self):
@@ -466,7 +466,9 @@ def run_ours(args, rank, world, local_rank):
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": oracle_cores(), "kind": "oracle",
                                 "sample": "%d of %d token rows of the same step (row-local), %.1f s" % (n, M_TOK, dt)}
     if args.extras and world == 1:
-        line["extras"] = extras(w8, torch, workloads, dev, peaks, src)
+        with ClockSampler(*gpu_identity(torch, dev)) as clk_x:
+            line["extras"] = extras(w8, torch, workloads, dev, peaks, src)
+        line["extras"]["clocks"] = clk_x.summary()   # over all extras: a dip shows in sm_mhz_min
     print(json.dumps(line), flush=True)
     return 0
 
