@@ -751,6 +751,19 @@ def extras(w8, torch, workloads, dev, peaks, src):
     gbs = (wb0.numel() + MLP * HID + MLP * 4) / (ms * 1e-3) / 1e9
     out["q8_0_to_axis_int8_12288x3072"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
     del sets
+    # GGUF A8 float: Q8_0 -> axis e4m3 (same traffic as the int8 requant); the
+    # e4m3 forward sweep, one weight scale per output column, runs below
+    wq0e, swe = w8.q8_0_to_axis_e4m3(wb0, MLP, HID)
+    sets = []
+    for i in range(_nsets(nbytes(wb0, wq0))):
+        wb = wb0.clone()
+        q = torch.empty_like(wq0e)
+        s = torch.empty(MLP, dtype=torch.float32, device=dev)
+        sets.append(lambda wb=wb, q=q, s=s: w8.q8_0_to_axis_e4m3(wb, MLP, HID, out=q, scale=s))
+    ms = _time_rot(sets, 30, torch, stream)
+    gbs = (wb0.numel() + MLP * HID + MLP * 4) / (ms * 1e-3) / 1e9
+    out["q8_0_to_axis_e4m3_12288x3072"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
+    del sets
     # tensor-wise weight quantization (load time), 12288 x 3072
     wt0 = workloads.normal((MLP, HID), 0.02, 9).to(dev)
     sets = [lambda wt=(wt0 if i == 0 else wt0.clone()): w8.quantize_weight(wt, "int8", "tensor")
@@ -758,60 +771,52 @@ def extras(w8, torch, workloads, dev, peaks, src):
     ms = _time_rot(sets, 30, torch, stream)
     out["quantize_weight_tensor_12288x3072"] = {"ms": ms, "GB/s": wt0.numel() * 3 / (ms * 1e-3) / 1e9}
     del sets, wt0
-    # GGUF A8 int forward sweep over M: the weight is rotated too, so that
-    # small M streams it from HBM as it would in a model
-    sweep = {}
+    # the weight-only types' two dequantizations alone (12288 x 3072 weight -> bf16)
+    wq8, sw8 = w8.quantize_weight(g["w_f32"].to(torch.bfloat16).to(dev), "e4m3", "tensor")
+    wgg = w8.q8_0_quantize(g["w_f32"].reshape(-1).to(dev))
+    sets_e, sets_g = [], []
+    for i in range(_nsets(MLP * HID * 3)):
+        wq, blk = wq8.clone(), wgg.clone()
+        ye = torch.empty((MLP, HID), dtype=torch.bfloat16, device=dev)
+        yg = torch.empty(MLP * HID, dtype=torch.bfloat16, device=dev)
+        sets_e.append(lambda wq=wq, ye=ye: w8.dequantize_e4m3_bf16(wq, sw8, out=ye))
+        sets_g.append(lambda blk=blk, yg=yg: w8.q8_0_dequantize_bf16(blk, MLP * HID, out=yg))
+    ms = _time_rot(sets_e, 30, torch, stream)
+    gbs = MLP * HID * 3 / (ms * 1e-3) / 1e9
+    out["dequantize_e4m3_bf16_12288x3072"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
+    ms = _time_rot(sets_g, 30, torch, stream)
+    gbs = (wgg.numel() + MLP * HID * 2) / (ms * 1e-3) / 1e9
+    out["q8_0_dequantize_bf16_12288x3072"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
+    del sets_e, sets_g
+    # GGUF A8 int and float forward sweeps over M, interleaved so that the
+    # few-token points (latency-bound) run before the large products: kernels
+    # timed after several long power-capped GEMMs ran up to 25-40 % slower for
+    # seconds, so the bandwidth- and latency-bound lines above come first too.
+    # The weight is rotated, so that small M streams it from HBM as in a model.
+    sweeps = {"int8": {}, "e4m3": {}}
     xg = g["x"].to(dev)
     for M in workloads.GGUF_MS:
         xm0 = xg[:M].contiguous()
-        sets = []
-        for i in range(_nsets(nbytes(xm0, wq0) + M * MLP * 2)):
-            xm, wq = xm0.clone(), wq0.clone()
-            y = torch.empty((M, MLP), dtype=torch.bfloat16, device=dev)
-            ws = torch.empty(w8.workspace_bytes(0, M, MLP, HID), dtype=torch.uint8, device=dev)
-            sets.append(lambda xm=xm, wq=wq, y=y, ws=ws: w8.linear_fwd(xm, wq, sw, out=y, ws=ws))
-        ms = _time_rot(sets, 30, torch, stream)
-        sweep[str(M)] = {"ms": ms, "TOPS": 2 * M * MLP * HID / ms / 1e9,
-                         "weight_GB/s": MLP * HID / (ms * 1e-3) / 1e9,
-                         "roofline_frac": _gemm_roof_ms(M, MLP, HID, hbm, tc8) / ms}
-        del sets
-    out["gguf_a8_int_fwd_sweep_N12288_K3072"] = sweep
-    # GGUF A8 float: Q8_0 -> axis e4m3 (same traffic as the int8 requant), then
-    # the e4m3 forward sweep with one weight scale per output column
-    wq0, sw = w8.q8_0_to_axis_e4m3(wb0, MLP, HID)
-    sets = []
-    for i in range(_nsets(nbytes(wb0, wq0))):
-        wb = wb0.clone()
-        q = torch.empty_like(wq0)
-        s = torch.empty(MLP, dtype=torch.float32, device=dev)
-        sets.append(lambda wb=wb, q=q, s=s: w8.q8_0_to_axis_e4m3(wb, MLP, HID, out=q, scale=s))
-    ms = _time_rot(sets, 30, torch, stream)
-    gbs = (wb0.numel() + MLP * HID + MLP * 4) / (ms * 1e-3) / 1e9
-    out["q8_0_to_axis_e4m3_12288x3072"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
-    del sets
-    sweep = {}
-    for M in workloads.GGUF_MS:
-        xm0 = xg[:M].contiguous()
-        sets = []
-        for i in range(_nsets(nbytes(xm0, wq0) + M * MLP * 2)):
-            xm, wq = xm0.clone(), wq0.clone()
-            y = torch.empty((M, MLP), dtype=torch.bfloat16, device=dev)
-            ws = torch.empty(w8.workspace_bytes(0, M, MLP, HID), dtype=torch.uint8, device=dev)
-            sets.append(lambda xm=xm, wq=wq, y=y, ws=ws: w8.linear_fwd(xm, wq, sw, out=y, ws=ws))
-        ms = _time_rot(sets, 30, torch, stream)
-        sweep[str(M)] = {"ms": ms, "TOPS": 2 * M * MLP * HID / ms / 1e9,
-                         "weight_GB/s": MLP * HID / (ms * 1e-3) / 1e9,
-                         "roofline_frac": _gemm_roof_ms(M, MLP, HID, hbm, tc8) / ms}
-        del sets
-    out["gguf_a8_float_fwd_sweep_N12288_K3072"] = sweep
+        for qt, wqq, sww in (("int8", wq0, sw), ("e4m3", wq0e, swe)):
+            sets = []
+            for i in range(_nsets(nbytes(xm0, wqq) + M * MLP * 2)):
+                xm, wq = xm0.clone(), wqq.clone()
+                y = torch.empty((M, MLP), dtype=torch.bfloat16, device=dev)
+                ws = torch.empty(w8.workspace_bytes(0, M, MLP, HID), dtype=torch.uint8, device=dev)
+                sets.append(lambda xm=xm, wq=wq, y=y, ws=ws, sww=sww: w8.linear_fwd(xm, wq, sww, out=y, ws=ws))
+            ms = _time_rot(sets, 30, torch, stream)
+            sweeps[qt][str(M)] = {"ms": ms, "TOPS": 2 * M * MLP * HID / ms / 1e9,
+                                  "weight_GB/s": MLP * HID / (ms * 1e-3) / 1e9,
+                                  "roofline_frac": _gemm_roof_ms(M, MLP, HID, hbm, tc8) / ms}
+            del sets
+    out["gguf_a8_int_fwd_sweep_N12288_K3072"] = sweeps["int8"]
+    out["gguf_a8_float_fwd_sweep_N12288_K3072"] = sweeps["e4m3"]
     # weight-only types (float8, GGUF) on the DiT up-projection: the weight
     # dequantized to bf16 in the workspace, then the bf16 Linear
     tcb = peaks["bf16_tflops"]
     xb0 = workloads.normal((M_TOK, HID), 1.0, 5).to(dev)
     wb0 = g["w_f32"].to(torch.bfloat16).to(dev)
-    wq8, sw8 = w8.quantize_weight(wb0, "e4m3", "tensor")
-    wgg = w8.q8_0_quantize(g["w_f32"].reshape(-1).to(dev))
-    ops = 2 * M_TOK * MLP * HID
+    ops = 2 * M_TOK * MLP * HID   # wq8, sw8, wgg: quantized above from the same weight
     wsz = w8.workspace_bytes(w8.OP_WEIGHT_ONLY_FWD, M_TOK, MLP, HID)
     res = {}
     for name, mk in (("bf16_gemm", lambda xx, ws: (lambda: w8.bf16_linear_fwd(xx, wb0, ws=ws))),
@@ -839,21 +844,7 @@ def extras(w8, torch, workloads, dev, peaks, src):
         del sets
     out["weight_only_dgrad_4608x12288x3072"] = res
     del dy0
-    # the two dequantizations alone (12288 x 3072 weight -> bf16)
-    sets_e, sets_g = [], []
-    for i in range(_nsets(MLP * HID * 3)):
-        wq, blk = wq8.clone(), wgg.clone()
-        ye = torch.empty((MLP, HID), dtype=torch.bfloat16, device=dev)
-        yg = torch.empty(MLP * HID, dtype=torch.bfloat16, device=dev)
-        sets_e.append(lambda wq=wq, ye=ye: w8.dequantize_e4m3_bf16(wq, sw8, out=ye))
-        sets_g.append(lambda blk=blk, yg=yg: w8.q8_0_dequantize_bf16(blk, MLP * HID, out=yg))
-    ms = _time_rot(sets_e, 30, torch, stream)
-    gbs = MLP * HID * 3 / (ms * 1e-3) / 1e9
-    out["dequantize_e4m3_bf16_12288x3072"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
-    ms = _time_rot(sets_g, 30, torch, stream)
-    gbs = (wgg.numel() + MLP * HID * 2) / (ms * 1e-3) / 1e9
-    out["q8_0_dequantize_bf16_12288x3072"] = {"ms": ms, "GB/s": gbs, "hbm_frac": gbs / hbm}
-    del sets_e, sets_g, xb0, wb0
+    del xb0, wb0
     out["peaks"] = {"source": src, "hbm_gbs": hbm, "int8_burst_tops": tc8}
     out["method"] = ("mean over the reps of one CUDA-graph replay (no host launch cost), rotating through "
                      ">= 3x L2 of input/output copies; the fastest of three replays")
