@@ -28,6 +28,10 @@
  *    Other shapes return W8A8_ERR_UNSUPPORTED_SHAPE before any launch.
  *  - Inputs are finite (no NaN/Inf); results for non-finite inputs are
  *    unspecified.
+ *  - Tracing: every compute call is one NVTX range named after the call
+ *    (nested when one call is built on another), so a profiler's timeline
+ *    groups each call's launches; without a profiling tool the ranges cost
+ *    nothing measurable.
  *  - Errors: argument errors return before any launch.  A failed launch
  *    returns W8A8_ERR_CUDA.  A device that is not compute capability 10.0
  *    returns W8A8_ERR_UNSUPPORTED_DEVICE; there is no CPU fallback.  Kernels

@@ -10,6 +10,8 @@
 #include <string>
 #include <utility>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "w8a8.h"
 #include "device.cuh"
 #include "gemm.cuh"
@@ -911,6 +913,18 @@ static w8a8_status svdq_fwd_impl(const void* x, int64_t M, int64_t N, int64_t K,
   return launch_gemm<kKind, false, 256, kEpiLowRank>(ta, tb, M, N, K, ep, s);
 }
 
+// Tracing: every compute call of the C ABI is one NVTX range named after the
+// call (its launches nest inside it in a profiler's timeline).  The NVTX
+// header is inert until a profiling tool injects itself, so an untraced run
+// pays one predictable branch per call.
+struct TraceRange {
+  explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+  ~TraceRange() { nvtxRangePop(); }
+  TraceRange(const TraceRange&) = delete;
+  TraceRange& operator=(const TraceRange&) = delete;
+};
+#define W8A8_TRACE() const TraceRange w8a8_trace_range_(__func__)
+
 extern "C" {
 
 const char* w8a8_last_error(void) { return t_last_error.c_str(); }
@@ -934,6 +948,7 @@ size_t w8a8_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r) {
 
 w8a8_status w8a8_quantize_rows(const void* x, int64_t M, int64_t K, int64_t ldx, w8a8_qtype qt, void* q,
                                int64_t ldq, float* s, w8a8_stream_t stream) {
+  W8A8_TRACE();
   W8A8_CHECK(valid_qt(qt), W8A8_ERR_INVALID_ARG, "invalid qtype %d", static_cast<int>(qt));
   W8A8_CHECK(M >= 0, W8A8_ERR_UNSUPPORTED_SHAPE, "M < 0");
   w8a8_status st = check_k(K, "K");
@@ -949,6 +964,7 @@ w8a8_status w8a8_quantize_rows(const void* x, int64_t M, int64_t K, int64_t ldx,
 
 w8a8_status w8a8_quantize_weight(const void* w, int64_t N, int64_t K, w8a8_qtype qt, w8a8_wgran g, void* q,
                                  float* scale, void* ws, size_t ws_bytes, w8a8_stream_t stream) {
+  W8A8_TRACE();
   W8A8_CHECK(valid_qt(qt) && valid_g(g), W8A8_ERR_INVALID_ARG, "invalid qtype/granularity");
   W8A8_CHECK(N >= 1, W8A8_ERR_UNSUPPORTED_SHAPE, "N < 1");
   w8a8_status st = check_k(K, "K");
@@ -982,6 +998,7 @@ w8a8_status w8a8_quantize_weight(const void* w, int64_t N, int64_t K, w8a8_qtype
 }
 
 w8a8_status q8_0_quantize(const float* x, int64_t n, void* blocks, w8a8_stream_t stream) {
+  W8A8_TRACE();
   W8A8_CHECK(n >= 0, W8A8_ERR_UNSUPPORTED_SHAPE, "n < 0");
   if (n == 0) return W8A8_OK;
   W8A8_CHECK(x && blocks, W8A8_ERR_INVALID_ARG, "null pointer");
@@ -999,6 +1016,7 @@ w8a8_status q8_0_quantize(const float* x, int64_t n, void* blocks, w8a8_stream_t
 }
 
 w8a8_status q8_0_dequantize(const void* blocks, int64_t n, float* y, w8a8_stream_t stream) {
+  W8A8_TRACE();
   W8A8_CHECK(n >= 0, W8A8_ERR_UNSUPPORTED_SHAPE, "n < 0");
   if (n == 0) return W8A8_OK;
   W8A8_CHECK(y && blocks, W8A8_ERR_INVALID_ARG, "null pointer");
@@ -1007,6 +1025,7 @@ w8a8_status q8_0_dequantize(const void* blocks, int64_t n, float* y, w8a8_stream
 }
 
 w8a8_status q8_0_dequantize_bf16(const void* blocks, int64_t n, void* y, w8a8_stream_t stream) {
+  W8A8_TRACE();
   W8A8_CHECK(n >= 0, W8A8_ERR_UNSUPPORTED_SHAPE, "n < 0");
   if (n == 0) return W8A8_OK;
   W8A8_CHECK(y && blocks, W8A8_ERR_INVALID_ARG, "null pointer");
@@ -1016,6 +1035,7 @@ w8a8_status q8_0_dequantize_bf16(const void* blocks, int64_t n, void* y, w8a8_st
 
 w8a8_status w8a8_dequantize_e4m3_bf16(const void* q, int64_t n, const float* scale, void* w,
                                       w8a8_stream_t stream) {
+  W8A8_TRACE();
   W8A8_CHECK(n >= 0 && n % 16 == 0, W8A8_ERR_UNSUPPORTED_SHAPE, "n must be a non-negative multiple of 16");
   if (n == 0) return W8A8_OK;
   W8A8_CHECK(q && scale && w, W8A8_ERR_INVALID_ARG, "null pointer");
@@ -1044,6 +1064,7 @@ static w8a8_status check_bf16_linear(const void* x, int64_t M, int64_t N, int64_
 
 w8a8_status bf16_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, const void* w, const void* bias, void* y,
                             void* ws, size_t ws_bytes, w8a8_stream_t stream) {
+  W8A8_TRACE();
   w8a8_status st = check_bf16_linear(x, M, N, K, w, bias, y, ws, ws_bytes, M > 0 ? ws_bf16(M, N, K) : 0);
   if (st != W8A8_OK || M == 0) return st;
   Carve c(ws);
@@ -1052,6 +1073,7 @@ w8a8_status bf16_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, cons
 
 w8a8_status float8_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, const void* wq, const float* w_scale,
                               const void* bias, void* y, void* ws, size_t ws_bytes, w8a8_stream_t stream) {
+  W8A8_TRACE();
   w8a8_status st = check_bf16_linear(x, M, N, K, wq, bias, y, ws, ws_bytes, M > 0 ? ws_weight_only(M, N, K) : 0,
                                      true, w_scale);
   if (st != W8A8_OK || M == 0) return st;
@@ -1072,6 +1094,7 @@ static w8a8_status check_bf16_dgrad(const void* dy, int64_t M, int64_t N, int64_
 
 w8a8_status bf16_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, const void* w, void* dx, void* ws,
                               size_t ws_bytes, w8a8_stream_t stream) {
+  W8A8_TRACE();
   w8a8_status st = check_bf16_dgrad(dy, M, N, K, w, dx, ws, ws_bytes, M > 0 ? ws_bf16_dgrad(M, N, K) : 0);
   if (st != W8A8_OK || M == 0) return st;
   Carve c(ws);
@@ -1080,6 +1103,7 @@ w8a8_status bf16_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, c
 
 w8a8_status float8_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, const void* wq,
                                 const float* w_scale, void* dx, void* ws, size_t ws_bytes, w8a8_stream_t stream) {
+  W8A8_TRACE();
   w8a8_status st = check_bf16_dgrad(dy, M, N, K, wq, dx, ws, ws_bytes, M > 0 ? ws_weight_only_dgrad(M, N, K) : 0,
                                     true, w_scale);
   if (st != W8A8_OK || M == 0) return st;
@@ -1092,6 +1116,7 @@ w8a8_status float8_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K,
 
 w8a8_status gguf_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, const void* blocks, void* dx, void* ws,
                               size_t ws_bytes, w8a8_stream_t stream) {
+  W8A8_TRACE();
   w8a8_status st = check_bf16_dgrad(dy, M, N, K, blocks, dx, ws, ws_bytes, M > 0 ? ws_weight_only_dgrad(M, N, K) : 0);
   if (st != W8A8_OK || M == 0) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -1103,6 +1128,7 @@ w8a8_status gguf_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, c
 
 w8a8_status gguf_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, const void* blocks, const void* bias,
                             void* y, void* ws, size_t ws_bytes, w8a8_stream_t stream) {
+  W8A8_TRACE();
   w8a8_status st = check_bf16_linear(x, M, N, K, blocks, bias, y, ws, ws_bytes, M > 0 ? ws_weight_only(M, N, K) : 0);
   if (st != W8A8_OK || M == 0) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -1114,17 +1140,20 @@ w8a8_status gguf_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, cons
 
 w8a8_status q8_0_to_axis_int8(const void* blocks, int64_t N, int64_t K, int8_t* q, float* scale,
                               w8a8_stream_t stream) {
+  W8A8_TRACE();
   return requant_axis<0>(blocks, N, K, reinterpret_cast<uint8_t*>(q), scale, stream, "q8_0_to_axis_int8 launch");
 }
 
 w8a8_status q8_0_to_axis_e4m3(const void* blocks, int64_t N, int64_t K, uint8_t* q, float* scale,
                               w8a8_stream_t stream) {
+  W8A8_TRACE();
   return requant_axis<1>(blocks, N, K, q, scale, stream, "q8_0_to_axis_e4m3 launch");
 }
 
 w8a8_status w8a8_qgemm_fwd(const void* xq, int64_t ldq, const float* sx, int64_t M, int64_t N, int64_t K,
                            w8a8_qtype qt, const void* wq, const float* sw, w8a8_wgran g, const void* bias, void* y,
                            w8a8_stream_t stream) {
+  W8A8_TRACE();
   W8A8_CHECK(valid_qt(qt) && valid_g(g), W8A8_ERR_INVALID_ARG, "invalid qtype/granularity");
   W8A8_CHECK(M >= 0 && N >= 1 && M < (1ll << 31) && N < (1ll << 31), W8A8_ERR_UNSUPPORTED_SHAPE, "bad M/N");
   w8a8_status st = check_k(K, "K");
@@ -1141,6 +1170,7 @@ w8a8_status w8a8_qgemm_fwd(const void* xq, int64_t ldq, const float* sx, int64_t
 
 w8a8_status w8a8_qgemm_dgrad(const void* dyq, int64_t ldq, const float* sdy, int64_t M, int64_t N, int64_t K,
                              w8a8_qtype qt, const void* wq, const float* sw, void* dx, w8a8_stream_t stream) {
+  W8A8_TRACE();
   W8A8_CHECK(valid_qt(qt), W8A8_ERR_INVALID_ARG, "invalid qtype");
   W8A8_CHECK(M >= 0 && M < (1ll << 31), W8A8_ERR_UNSUPPORTED_SHAPE, "bad M");
   w8a8_status st = check_k(K, "K");
@@ -1158,12 +1188,14 @@ w8a8_status w8a8_qgemm_dgrad(const void* dyq, int64_t ldq, const float* sdy, int
 w8a8_status w8a8_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, w8a8_qtype qt, const void* wq,
                             const float* sw, w8a8_wgran g, const void* bias, void* y, void* ws, size_t ws_bytes,
                             w8a8_stream_t stream) {
+  W8A8_TRACE();
   return w8a8_linear_fwd_ex(x, M, N, K, qt, wq, sw, g, bias, W8A8_ACT_NONE, nullptr, nullptr, y, ws, ws_bytes, stream);
 }
 
 w8a8_status w8a8_linear_fwd_ex(const void* x, int64_t M, int64_t N, int64_t K, w8a8_qtype qt, const void* wq,
                                const float* sw, w8a8_wgran g, const void* bias, w8a8_act act, const uint32_t* x_amax,
                                uint32_t* y_amax, void* y, void* ws, size_t ws_bytes, w8a8_stream_t stream) {
+  W8A8_TRACE();
   W8A8_CHECK(valid_qt(qt) && valid_g(g), W8A8_ERR_INVALID_ARG, "invalid qtype/granularity");
   W8A8_CHECK(act == W8A8_ACT_NONE || act == W8A8_ACT_GELU || act == W8A8_ACT_GELU_TANH, W8A8_ERR_INVALID_ARG,
              "invalid activation %d", static_cast<int>(act));
@@ -1204,6 +1236,7 @@ w8a8_status w8a8_linear_fwd_ex(const void* x, int64_t M, int64_t N, int64_t K, w
 
 w8a8_status w8a8_linear_fwd_noalloc(const void* x, int64_t M, int64_t N, int64_t K, w8a8_qtype qt, const void* wq,
                                     const float* sw, w8a8_wgran g, const void* bias, void* y, w8a8_stream_t stream) {
+  W8A8_TRACE();
   W8A8_CHECK(valid_qt(qt) && valid_g(g), W8A8_ERR_INVALID_ARG, "invalid qtype/granularity");
   W8A8_CHECK(M >= 0 && N >= 1 && M < (1ll << 31) && N < (1ll << 31), W8A8_ERR_UNSUPPORTED_SHAPE, "bad M/N");
   w8a8_status st = check_k(K, "K");
@@ -1232,6 +1265,7 @@ w8a8_status w8a8_linear_fwd_noalloc(const void* x, int64_t M, int64_t N, int64_t
 w8a8_status w8a8_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, w8a8_qtype qt, const void* wq,
                               const float* sw, w8a8_wgran g, void* dx, void* ws, size_t ws_bytes,
                               w8a8_stream_t stream) {
+  W8A8_TRACE();
   W8A8_CHECK(valid_qt(qt) && valid_g(g), W8A8_ERR_INVALID_ARG, "invalid qtype/granularity");
   W8A8_CHECK(g == W8A8_TENSOR, W8A8_ERR_INVALID_ARG, "dgrad reads a tensor-wise weight scale");
   W8A8_CHECK(M >= 0 && M < (1ll << 31), W8A8_ERR_UNSUPPORTED_SHAPE, "bad M");
@@ -1259,12 +1293,14 @@ w8a8_status w8a8_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, w
 w8a8_status svdq_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, const void* rq, const float* r_scale,
                             int r, const void* l1, const void* l2, const void* bias, void* y, void* ws,
                             size_t ws_bytes, w8a8_stream_t stream) {
+  W8A8_TRACE();
   return svdq_fwd_impl<W8A8_INT8>(x, M, N, K, rq, r_scale, r, l1, l2, bias, y, ws, ws_bytes, stream);
 }
 
 w8a8_status svdq_linear_fwd_e4m3(const void* x, int64_t M, int64_t N, int64_t K, const void* rq,
                                  const float* r_scale, int r, const void* l1, const void* l2, const void* bias,
                                  void* y, void* ws, size_t ws_bytes, w8a8_stream_t stream) {
+  W8A8_TRACE();
   return svdq_fwd_impl<W8A8_E4M3>(x, M, N, K, rq, r_scale, r, l1, l2, bias, y, ws, ws_bytes, stream);
 }
 
@@ -1296,6 +1332,7 @@ w8a8_status w8a8_set_wait_limit_ns(uint64_t limit_ns) {
 }
 
 w8a8_status w8a8_selftest_wait(uint64_t limit_ns, w8a8_stream_t stream) {
+  W8A8_TRACE();
   W8A8_CHECK(limit_ns > 0 && limit_ns <= 10000000000ull, W8A8_ERR_INVALID_ARG, "limit must be in (0, 10 s]");
   w8a8_status st = current_device(nullptr, nullptr);
   if (st != W8A8_OK) return st;
@@ -1305,6 +1342,7 @@ w8a8_status w8a8_selftest_wait(uint64_t limit_ns, w8a8_stream_t stream) {
 }
 
 w8a8_status w8a8_e4m3_encode(const float* x, int64_t n, uint8_t* y, w8a8_stream_t stream) {
+  W8A8_TRACE();
   W8A8_CHECK(n >= 0, W8A8_ERR_UNSUPPORTED_SHAPE, "n < 0");
   if (n == 0) return W8A8_OK;
   W8A8_CHECK(x && y, W8A8_ERR_INVALID_ARG, "null pointer");
