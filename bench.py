@@ -469,8 +469,60 @@ def run_ours(args, rank, world, local_rank):
         with ClockSampler(*gpu_identity(torch, dev)) as clk_x:
             line["extras"] = extras(w8, torch, workloads, dev, peaks, src)
         line["extras"]["clocks"] = clk_x.summary()   # over all extras: a dip shows in sm_mhz_min
+    # the compact per-row summary goes last, so that a reader keeping only the
+    # end of the line still sees every row's number
+    line["rows"] = summary_rows(line)
     print(json.dumps(line), flush=True)
     return 0
+
+
+def _g3(v):
+    """A number rounded to 3 significant digits (None passes through)."""
+    return None if v is None else float("%.3g" % v)
+
+
+def summary_rows(line):
+    """One short entry per row of the hot path: microseconds, and the
+    fraction of the roofline the row is bound by (HBM copy bandwidth, or the
+    8-bit / bf16 tensor peak), taken from the headline and the extras."""
+    rf = line["roofline"]
+    rows = {"headline_dit_mlp_fwd_dgrad": {"TOPS": _g3(line["value"]), "ms": _g3(line["ms_per_step"]),
+                                           "gemm_frac": _g3(rf["frac"]), "e2e_TOPS": _g3((line.get("e2e") or {}).get("value"))}}
+    x = line.get("extras")
+    if not x:
+        return rows
+    us = lambda d: _g3(d["ms"] * 1e3)
+    bw = lambda d: {"us": us(d), "hbm_frac": _g3(d["hbm_frac"])}
+    rows["a1_quantize_rows_4608x12288"] = bw(x["quantize_rows_4608x12288"])
+    rows["a2_quantize_weight_tensor_12288x3072"] = {"us": us(x["quantize_weight_tensor_12288x3072"]),
+                                                    "GBps": _g3(x["quantize_weight_tensor_12288x3072"]["GB/s"])}
+    rows["a3_q8_0_quantize_2^28"] = bw(x["q8_0_quantize_2^28"])
+    rows["a3_q8_0_dequantize_2^28"] = bw(x["q8_0_dequantize_2^28"])
+    rows["a4_q8_0_to_axis_int8_12288x3072"] = bw(x["q8_0_to_axis_int8_12288x3072"])
+    rows["f2_q8_0_to_axis_e4m3_12288x3072"] = bw(x["q8_0_to_axis_e4m3_12288x3072"])
+    d = x["int_w8a8_fwd_tiny_256x512x512"]
+    rows["cfg1_int_tiny_256x512x512"] = {"us": us(d)}
+    d = x["float_w8a8_fwd_4096x3072x3072"]
+    rows["cfg2_float_w8a8_4096x3072x3072"] = {"us": us(d), "TOPS": _g3(d["TOPS"]), "gemm_us": _g3(d["gemm_ms"] * 1e3),
+                                              "gemm_frac_fp8": _g3(d["gemm_frac_fp8_burst"])}
+    d = x["svdquant_r32_fwd_4608x3072x3072"]
+    rows["cfg4_svdquant_int8_r32"] = {"us": us(d), "frac_int8": _g3(d["frac_int8_burst"])}
+    d = x["svdquant_e4m3_r32_fwd_4608x3072x3072"]
+    rows["f4_svdquant_e4m3_r32"] = {"us": us(d), "frac_fp8": _g3(d["frac_fp8_burst"])}
+    for key, name in (("gguf_a8_int_fwd_sweep_N12288_K3072", "cfg5_gguf_a8_int"),
+                      ("gguf_a8_float_fwd_sweep_N12288_K3072", "f2_gguf_a8_float")):
+        rows[name] = {m: [us(v), _g3(v["roofline_frac"])] for m, v in x[key].items()}
+    rows["cfg5_format"] = "M: [us, roofline_frac]"
+    wo = x["weight_only_fwd_4608x12288x3072"]
+    wd = x["weight_only_dgrad_4608x12288x3072"]
+    rows["f3_weight_only_frac_bf16"] = {k: [_g3(wo[k]["frac_bf16_burst"]), _g3(wd[k]["frac_bf16_burst"])]
+                                        for k in ("bf16_gemm", "float8", "gguf")}
+    rows["f3_format"] = "[fwd, dgrad] at 4608x12288x3072"
+    rows["a3_dequant_bf16_12288x3072_hbm_frac"] = {"e4m3": _g3(x["dequantize_e4m3_bf16_12288x3072"]["hbm_frac"]),
+                                                   "q8_0": _g3(x["q8_0_dequantize_bf16_12288x3072"]["hbm_frac"])}
+    f1 = x["dit_mlp_fwd_gelu_4608x3072x12288"]
+    rows["f1_mlp_fwd_gelu_us"] = {k: us(v) for k, v in f1.items()}
+    return rows
 
 
 def run_case(args):

@@ -19,6 +19,15 @@
  *    (size from w8a8_workspace_bytes).
  *  - Streams: all work is enqueued on `stream` (a cudaStream_t; NULL is the
  *    legacy default stream).  Calls return as soon as the work is enqueued.
+ *    Calls on one stream take effect in stream order, whatever produced
+ *    their inputs (a previous call, e.g. a weight preparation, or any other
+ *    kernel): a call's kernels may be launched while the kernel before them
+ *    finishes (programmatic dependent launch) and set themselves up, but
+ *    read nothing before it has completed.  The one early read - the weight
+ *    tiles of a few-row or split product in w8a8_linear_fwd(_ex),
+ *    w8a8_linear_fwd_noalloc, w8a8_linear_dgrad and svdq_linear_fwd(_e4m3) -
+ *    comes after that call's own row quantizer, which waits for every
+ *    earlier kernel on the stream first.
  *  - Alignment: every device pointer must be 16-byte aligned
  *    (W8A8_ERR_MISALIGNED otherwise) - the alignment to 16 that fixed the
  *    misaligned-address offloading bug in OneTrainer PR #1034, Known issues.
@@ -325,7 +334,8 @@ w8a8_status w8a8_qgemm_dgrad(const void* dyq, int64_t ldq, const float* dy_scale
  * or plugin host that owns all device memory and exposes no allocator, a
  * latency-critical path that must not call cudaMalloc because it can
  * synchronize the device, a language binding with no CUDA allocator).  This
- * entry point computes exactly what w8a8_linear_fwd computes, but keeps the
+ * entry point computes exactly what w8a8_linear_fwd computes (the same
+ * kernels for the same shapes, so the same bits), but keeps the
  * activation codes and row scales in a fixed scratch array that is part of
  * the library itself (a file-scope __device__ array of
  * W8A8_NOALLOC_SCRATCH_BYTES; every GPU that loads the library holds it
@@ -336,9 +346,12 @@ w8a8_status w8a8_qgemm_dgrad(const void* dyq, int64_t ldq, const float* dy_scale
  * Limits: M * K <= W8A8_NOALLOC_MAX_CODES and M <= W8A8_NOALLOC_MAX_ROWS;
  * larger problems return W8A8_ERR_WORKSPACE before any launch (use
  * w8a8_linear_fwd with a workspace instead).
- * Set-up: the first call on each device looks up the scratch array's device
- * address (cudaGetSymbolAddress) with that device current; make that first
- * call before any stream capture.
+ * Set-up: the first call in each CUDA context (normally one per device: its
+ * primary context) looks up the scratch array's device address
+ * (cudaGetSymbolAddress) with that device current, and keeps it for that
+ * context; make that first call before any stream capture.  A new context
+ * (after cudaDeviceReset, or a second context on a device) gets its own
+ * lookup on its first call.
  * Sharing: all calls on a device use the same scratch, which keeps the last
  * call's contents (every byte a call reads was written earlier by the same
  * call, so nothing needs clearing).  Calls whose kernels overlap on the GPU

@@ -1,7 +1,14 @@
 """Parity at the workloads' full sizes, in the launch configuration the bench
 times.  Each step is row-local (token scales are per row, weights fixed), so
 the oracle recomputes a seeded sample of whole output rows - plus the last
-128-row tile - from the same inputs; the GPU computes everything."""
+128-row tile - from the same inputs; the GPU computes everything.
+
+With W8A8_FULL_PARITY=1 in the environment every row is compared instead of
+a sample: all outputs of every workload here, e.g. the four outputs of the
+DiT MLP block and the 16384-token GGUF forward, against the oracle on all
+host cores (a few minutes)."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -32,7 +39,14 @@ def u8(t):
     return t.detach().cpu().contiguous().view(torch.uint8).numpy()
 
 
+FULL = os.environ.get("W8A8_FULL_PARITY", "") not in ("", "0")
+
+
 def sample_rows(M, n=192, seed=0):
+    """A seeded sample of n rows plus row 0 and the last 128-row tile; every
+    row in full-parity mode."""
+    if FULL:
+        return np.arange(M)
     rng = np.random.default_rng(seed)
     rows = set(rng.choice(M, size=min(n, M), replace=False).tolist())
     rows |= set(range(max(0, M - 128), M)) | {0}

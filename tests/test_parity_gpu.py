@@ -438,14 +438,12 @@ def test_qgemm_dgrad_equals_linear(w8):
 
 # --------------------------------------------------------------------------- SVDQuant
 def _svdq_check(w8, orc, x, w, r, bias=None, rows=None, qt=0):
-    from oracle import svdquant
-    prep = svdquant.prepare(workloads.to_u16(w), r, qt)
-    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(DEV)
-    l1, l2 = to_dev(prep["l1"]), to_dev(prep["l2"])
-    rq = torch.from_numpy(prep["rq"].view(np.int8)).to(DEV)
-    if qt == 1:
-        rq = rq.view(torch.float8_e4m3fn)
-    rs = torch.from_numpy(prep["s_r"]).to(DEV)
+    """The library's own weight preparation (svdq_prepare) feeds both sides:
+    the forward on the GPU and the oracle's forward on the same factors and
+    residual codes."""
+    dp = w8.svdq_prepare(w.to(DEV), r, "int8" if qt == 0 else "e4m3")
+    l1, l2, rq, rs = dp["l1"], dp["l2"], dp["rq"], dp["r_scale"]
+    prep = {"l1": u16(l1), "l2": u16(l2), "rq": u8(rq), "s_r": f32(rs)}
     M, K = x.shape
     N = w.shape[0]
     ws = torch.empty(w8.workspace_bytes(w8.OP_SVDQ_FWD, M, N, K, r), dtype=torch.uint8, device=DEV)

@@ -44,6 +44,9 @@ CASES = [  # (M, N, K, qtype, granularity, bias) - two calls in a row per case
     [(300, 520, 640, "int8", "tensor", False), (1, 16, 16, "int8", "tensor", False)],
     [(4608, 3072, 3072, "int8", "tensor", False), (129, 257, 96, "int8", "axis", True)],
     [(256, 512, 512, "e4m3", "tensor", True), (2048, 1024, 4096, "e4m3", "tensor", False)],
+    # few rows: the one-launch CUDA-core kernels, axis scales and bias
+    [(2, 3072, 3072, "int8", "axis", True), (1, 520, 640, "e4m3", "axis", True)],
+    [(64, 12288, 3072, "int8", "axis", True), (3, 3072, 3072, "e4m3", "tensor", True)],
 ]
 
 

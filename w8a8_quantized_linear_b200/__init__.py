@@ -465,20 +465,9 @@ def svdq_linear_fwd(x, rq, r_scale, l1, l2, bias=None, out=None, ws=None):
     return y
 
 
-def svdq_prepare(w: torch.Tensor, r: int, qt="int8"):
-    """Offline SVDQuant weight split of W [N, K] bf16 (fp64 SVD with torch):
-    L1 = bf16(U_r sqrt(S_r)) [K, r], L2 = bf16(sqrt(S_r) V_r^T) [r, N],
-    R = bf16(W - (L1 L2)^T), then R quantized tensor-wise (int8 or e4m3) by
-    the library.
-    Returns dict(l1, l2, rq, r_scale) on w's device."""
-    wt = w.detach().to(torch.float64).T            # [K, N]
-    u, sig, vh = torch.linalg.svd(wt, full_matrices=False)
-    root = sig[:r].sqrt()
-    l1 = (u[:, :r] * root[None, :]).to(torch.float32).to(torch.bfloat16)
-    l2 = (root[:, None] * vh[:r, :]).to(torch.float32).to(torch.bfloat16)
-    resid = (w.to(torch.float64) - (l1.double() @ l2.double()).T).to(torch.float32).to(torch.bfloat16)
-    rq, r_scale = quantize_weight(resid.contiguous(), qt, "tensor")
-    return {"l1": l1.contiguous(), "l2": l2.contiguous(), "rq": rq, "r_scale": r_scale}
+# The SVDQuant weight split is offline preparation, kept out of this binding:
+# see weight_prep.py (svd_split, svdq_prepare).
+from .weight_prep import svd_split, svdq_prepare  # noqa: E402,F401
 
 
 # --------------------------------------------------------------------------- diagnostics

@@ -42,8 +42,11 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 // griddep_wait() returns when the previous kernel has completed and its
 // memory writes are visible (at once when there is no such kernel); a
 // kernel touches no global memory that the previous one may write or read
-// before it.  Weights are the exception the GEMM relies on: no kernel that
-// runs directly before it with an early trigger writes them.
+// before it.  The one exception is the single-SM GEMM's weight prefetch
+// (EpiParams::early_weights), allowed only right after the row quantizer of
+// the same call: that quantizer calls griddep_wait before griddep_launch, so
+// when the GEMM starts, every kernel before the quantizer has completed, and
+// the quantizer itself writes only activation codes and scales.
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }

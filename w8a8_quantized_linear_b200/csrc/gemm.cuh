@@ -50,6 +50,13 @@ struct EpiParams {
   uint32_t* partial;             // [splits, M, N] raw sums (splits > 1)
   int act;                       // kActNone / kActGelu / kActGeluTanh, applied last (kEpiScale)
   uint32_t* y_amax;              // [M] or null: atomicMax of max |y| per row (fp32 bits of the bf16 values)
+  // 1: the weight (B, or A in the transposed form) may be read before
+  // griddepcontrol.wait.  The host sets it only when the kernel just before
+  // this GEMM on the stream is the row quantizer of the same call, which
+  // waits for every earlier kernel before it lets this one launch and never
+  // writes the weight; a weight that an earlier kernel wrote is then
+  // complete.  0 (every other caller): nothing is read before the wait.
+  int early_weights;
 };
 
 // Optional activation between two projections (the MLP's GELU): the exact
@@ -318,13 +325,14 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
             tma_load_2d(b + j * (C::kBK * 128), &tmB, &full[st], n0 + j * (128 / C::kElem), kb * C::kBK);
         }
       };
-      // The weight tiles of the first unit's first stages are requested
-      // before waiting for the previous kernel, which never writes them; the
-      // activation codes it may be producing are read after the wait.  The
-      // weight is B, or A in the transposed form (kEpiScaleT).
+      // With ep.early_weights the weight tiles of the first unit's first
+      // stages are requested before waiting for the previous kernel (the
+      // same call's row quantizer, which never writes them); the activation
+      // codes it may be producing are read after the wait.  The weight is B,
+      // or A in the transposed form (kEpiScaleT).
       constexpr bool kWeightA = (EPI == kEpiScaleT);
       int pre = 0;
-      if (static_cast<int>(blockIdx.x) < num_units) {
+      if (ep.early_weights && static_cast<int>(blockIdx.x) < num_units) {
         const int tile = blockIdx.x / splits, split = blockIdx.x - tile * splits;
         const int kb0 = split * num_kb / splits, kb1 = (split + 1) * num_kb / splits;
         pre = (kb1 - kb0) < kStages ? (kb1 - kb0) : kStages;

@@ -138,8 +138,12 @@ __global__ void __launch_bounds__(1024) quantize_rows_kernel(const __nv_bfloat16
                                                              uint32_t* __restrict__ zero_out = nullptr,
                                                              int64_t zero_n = 0) {
   __shared__ float red[32];
-  griddep_launch();
+  // Wait first, then let the next kernel launch: a GEMM launched after this
+  // quantizer may read its weight before its own wait, and that is safe only
+  // once every kernel before this one (a weight producer among them) has
+  // completed.
   griddep_wait();   // x may be the previous kernel's output
+  griddep_launch();
   if constexpr (CHAIN) clear_words(zero_out, zero_n);
   const int64_t nv = K >> 3;
   for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
@@ -184,8 +188,12 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_team_kernel(const __nv_b
                                                                  uint32_t* __restrict__ zero_out = nullptr,
                                                                  int64_t zero_n = 0) {
   __shared__ float red[2][8];
-  griddep_launch();
+  // Wait first, then let the next kernel launch: a GEMM launched after this
+  // quantizer may read its weight before its own wait, and that is safe only
+  // once every kernel before this one (a weight producer among them) has
+  // completed.
   griddep_wait();   // x may be the previous kernel's output
+  griddep_launch();
   if constexpr (CHAIN) clear_words(zero_out, zero_n);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int team = warp / TW, tw = warp % TW;

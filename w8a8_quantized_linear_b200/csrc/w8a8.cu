@@ -128,9 +128,12 @@ cudaError_t set_smem_once(Kernel k, size_t bytes, int dev, std::atomic<uint64_t>
 // Launch with programmatic stream serialization: the kernel may start (and
 // run up to its griddep_wait) while the previous kernel on the stream
 // finishes.  The kernels launched this way are the row quantizers, the GEMMs,
-// the split-K epilogue, the few-token product and the Q8_0 re-quantization;
-// each waits before touching memory that the previous kernel may write or
-// read.
+// the split-K epilogue, the few-token product, the Q8_0 re-quantization and
+// the dequantizers; each waits before touching memory that the previous
+// kernel may write or read.  The single exception, the single-SM GEMM's
+// weight prefetch, is enabled only where the kernel before it is the same
+// call's row quantizer (EpiParams::early_weights), which waits for all
+// earlier work before it lets the GEMM launch.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                        Args&&... args) {
@@ -446,9 +449,13 @@ CUtensorMapDataType code_type() { return CU_TENSOR_MAP_DATA_TYPE_UINT8; }
 
 // GEMM on codes.  fwd: A = xq [M, lda] K-major, B = wq [N, K] K-major.
 // sk: split-K workspace (partial sums), or null for an unsplit product.
+// early_weights: the kernel just before on the stream is this call's row
+// quantizer, so the single-SM GEMM may fetch weight tiles before its wait
+// (EpiParams::early_weights); false when the caller launched nothing before.
 w8a8_status gemm_fwd(const void* xq, int64_t lda, const float* sx, int64_t M, int64_t N, int64_t K, int qt,
                      const void* wq, const float* sw, int g, const void* bias, void* y, cudaStream_t st,
-                     const SplitWs* sk = nullptr, int act = kActNone, uint32_t* y_amax = nullptr) {
+                     const SplitWs* sk = nullptr, int act = kActNone, uint32_t* y_amax = nullptr,
+                     bool early_weights = false) {
   alignas(64) CUtensorMap ta, tb;
   w8a8_status s = make_map(&ta, code_type(), 1, xq, K, M, lda, kBKBytes, kBM);
   if (s != W8A8_OK) return s;
@@ -464,6 +471,7 @@ w8a8_status gemm_fwd(const void* xq, int64_t lda, const float* sx, int64_t M, in
   ep.splits = 1;
   ep.act = act;
   ep.y_amax = y_amax;
+  ep.early_weights = early_weights ? 1 : 0;
   if (sk != nullptr && sk->splits > 1) {
     ep.splits = sk->splits;
     ep.partial = sk->partial;
@@ -500,8 +508,10 @@ w8a8_status gemm_fwd(const void* xq, int64_t lda, const float* sx, int64_t M, in
 }
 
 // dgrad: A = dyq [M, lda] (contraction N), B = wq [N, K] read MN-major.
+// early_weights as for gemm_fwd.
 w8a8_status gemm_dgrad(const void* dyq, int64_t lda, const float* sdy, int64_t M, int64_t N, int64_t K, int qt,
-                       const void* wq, const float* sw, void* dx, cudaStream_t st, const SplitWs* sk = nullptr) {
+                       const void* wq, const float* sw, void* dx, cudaStream_t st, const SplitWs* sk = nullptr,
+                       bool early_weights = false) {
   alignas(64) CUtensorMap ta, tb;
   w8a8_status s = make_map(&ta, code_type(), 1, dyq, N, M, lda, kBKBytes, kBM);
   if (s != W8A8_OK) return s;
@@ -514,6 +524,7 @@ w8a8_status gemm_dgrad(const void* dyq, int64_t lda, const float* sdy, int64_t M
   ep.y = static_cast<__nv_bfloat16*>(dx);
   ep.ldy = K;
   ep.splits = 1;
+  ep.early_weights = early_weights ? 1 : 0;
   if (sk != nullptr && sk->splits > 1) {
     ep.splits = sk->splits;
     ep.partial = sk->partial;
@@ -667,21 +678,68 @@ w8a8_status check_k(int64_t K, const char* name) {
 // Scratch of w8a8_linear_fwd_noalloc: activation codes at offset 0, row
 // scales at offset W8A8_NOALLOC_MAX_CODES (both 256-byte aligned).  Host code
 // only sees a stand-in for this symbol; its device address comes from
-// cudaGetSymbolAddress, once per device, with that device current.
+// cudaGetSymbolAddress with the device current.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[W8A8_NOALLOC_SCRATCH_BYTES];
 
+// The address belongs to the module instance of one CUDA context, so it is
+// cached per context: keyed on the context's process-unique id
+// (cuCtxGetId), which no later context reuses - after cudaDeviceReset, or
+// under another context on the same device, the first call looks the
+// address up again.  The lookup allocates nothing.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+struct NoallocSlot {
+  unsigned long long ctx_id = 0;   // 0: empty (context ids start at 1)
+  void* addr = nullptr;
+};
+constexpr int kNoallocSlots = 16;
 std::mutex g_noalloc_mu;
-void* g_noalloc_addr[kMaxDevices] = {};
+NoallocSlot g_noalloc_slot[kNoallocSlots];
+int g_noalloc_next = 0;
 
-w8a8_status noalloc_scratch(int dev, void** out) {
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion(name, &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
+
+w8a8_status current_ctx_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_ctx = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (!get_ctx || !get_id) return fail(W8A8_ERR_CUDA, "cuCtxGetCurrent / cuCtxGetId unavailable");
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return fail(W8A8_ERR_CUDA, "no current CUDA context");
+  if (get_id(ctx, id) != CUDA_SUCCESS) return fail(W8A8_ERR_CUDA, "cuCtxGetId failed");
+  return W8A8_OK;
+}
+
+w8a8_status noalloc_scratch(void** out) {
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
+  unsigned long long id = 0;
+  if (current_ctx_id(&id) != W8A8_OK) {
+    // no context is current yet: the symbol lookup below makes the device's
+    // primary context current, then the id is taken again
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
-    g_noalloc_addr[dev] = p;
+    w8a8_status st = current_ctx_id(&id);
+    if (st != W8A8_OK) return st;
   }
-  *out = g_noalloc_addr[dev];
+  for (const NoallocSlot& sl : g_noalloc_slot)
+    if (sl.ctx_id == id) {
+      *out = sl.addr;
+      return W8A8_OK;
+    }
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+  g_noalloc_slot[g_noalloc_next] = NoallocSlot{id, p};
+  g_noalloc_next = (g_noalloc_next + 1) % kNoallocSlots;
+  *out = p;
   return W8A8_OK;
 }
 
@@ -872,6 +930,7 @@ static w8a8_status svdq_fwd_impl(const void* x, int64_t M, int64_t N, int64_t K,
     ep.ldy = r;
     ep.splits = tsk.splits;
     ep.partial = tsk.partial;
+    ep.early_weights = 1;   // L1 is read early: the kernel just before is this call's row quantizer
     if ((st = launch_gemm<kKindBF16, true, 64, kEpiPlain>(ta, tb, M, r, K, ep, s)) != W8A8_OK) return st;
     if (tsk.splits > 1) {
       int sms = 0;
@@ -900,6 +959,9 @@ static w8a8_status svdq_fwd_impl(const void* x, int64_t M, int64_t N, int64_t K,
   ep.lr_t = t;
   ep.lr_l2 = static_cast<const __nv_bfloat16*>(l2);
   ep.r = r;
+  // Rq is read early: the kernels since this call's row quantizer (the T
+  // product and its split-K finish) write only T and its partial sums
+  ep.early_weights = 1;
   if (pair) {
     // T [M, r] and L2 [r, N] tiles for the tensor-core low-rank product:
     // 64 bf16 (128 bytes) wide, r zero-padded by the copy
@@ -1231,7 +1293,8 @@ w8a8_status w8a8_linear_fwd_ex(const void* x, int64_t M, int64_t N, int64_t K, w
   const SplitWs sk = carve_split(c, M, N, lw, qt);
   // the quantizer clears y_amax; the GEMM's epilogue runs after it completes
   if ((st = launch_quantize_rows(x, K, M, K, qt, xq, K, sx, s, x_amax, y_amax, y_amax ? M : 0)) != W8A8_OK) return st;
-  return gemm_fwd(xq, K, sx, M, N, K, qt, wq, sw, g, bias, y, s, &sk, static_cast<int>(act), y_amax);
+  return gemm_fwd(xq, K, sx, M, N, K, qt, wq, sw, g, bias, y, s, &sk, static_cast<int>(act), y_amax,
+                  /*early_weights=*/true);
 }
 
 w8a8_status w8a8_linear_fwd_noalloc(const void* x, int64_t M, int64_t N, int64_t K, w8a8_qtype qt, const void* wq,
@@ -1251,15 +1314,20 @@ w8a8_status w8a8_linear_fwd_noalloc(const void* x, int64_t M, int64_t N, int64_t
   W8A8_CHECK(x && wq && sw && y, W8A8_ERR_INVALID_ARG, "null pointer");
   W8A8_CHECK(aligned16(x) && aligned16(wq) && aligned16(sw) && aligned16(y) && (bias == nullptr || aligned16(bias)),
              W8A8_ERR_MISALIGNED, "pointers must be 16-byte aligned");
-  int dev = 0;
-  if ((st = current_device(&dev, nullptr)) != W8A8_OK) return st;
-  void* scratch = nullptr;
-  if ((st = noalloc_scratch(dev, &scratch)) != W8A8_OK) return st;
+  if ((st = current_device(nullptr, nullptr)) != W8A8_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // The few-token kernels need no scratch: the same dispatch as
+  // w8a8_linear_fwd, so that both compute the same bits.
+  if (qt == W8A8_INT8 && M <= kGemvUseRows && K <= kGemvMaxK)
+    return launch_gemv(x, M, N, K, wq, sw, g == W8A8_AXIS, bias, y, s);
+  if (qt == W8A8_E4M3 && M == 1 && gemv_e4m3_fits(M, K))
+    return launch_gemv_e4m3(x, M, N, K, wq, sw, g == W8A8_AXIS, bias, y, s);
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != W8A8_OK) return st;
   void* xq = scratch;
   float* sx = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + W8A8_NOALLOC_MAX_CODES);
   if ((st = launch_quantize_rows(x, K, M, K, qt, xq, K, sx, s)) != W8A8_OK) return st;
-  return gemm_fwd(xq, K, sx, M, N, K, qt, wq, sw, g, bias, y, s);
+  return gemm_fwd(xq, K, sx, M, N, K, qt, wq, sw, g, bias, y, s, nullptr, kActNone, nullptr, /*early_weights=*/true);
 }
 
 w8a8_status w8a8_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, w8a8_qtype qt, const void* wq,
@@ -1287,7 +1355,7 @@ w8a8_status w8a8_linear_dgrad(const void* dy, int64_t M, int64_t N, int64_t K, w
   float* sdy = static_cast<float*>(c.take(static_cast<size_t>(M) * 4));
   const SplitWs sk = carve_split(c, M, K, lw, qt);
   if ((st = launch_quantize_rows(dy, N, M, N, qt, dyq, N, sdy, s)) != W8A8_OK) return st;
-  return gemm_dgrad(dyq, N, sdy, M, N, K, qt, wq, sw, dx, s, &sk);
+  return gemm_dgrad(dyq, N, sdy, M, N, K, qt, wq, sw, dx, s, &sk, /*early_weights=*/true);
 }
 
 w8a8_status svdq_linear_fwd(const void* x, int64_t M, int64_t N, int64_t K, const void* rq, const float* r_scale,
