@@ -448,13 +448,19 @@ def _svdq_check(w8, orc, x, w, r, bias=None, rows=None, qt=0):
     N = w.shape[0]
     ws = torch.empty(w8.workspace_bytes(w8.OP_SVDQ_FWD, M, N, K, r), dtype=torch.uint8, device=DEV)
     y = w8.svdq_linear_fwd(x.to(DEV), rq, rs, l1, l2, bias=None if bias is None else bias.to(DEV), ws=ws)
-    # T = bf16(X L1) as the kernel left it in the workspace
-    off = -(-(M * K) // 256) * 256 + -(-(M * 4) // 256) * 256
+    # the activation codes, row scales and T = bf16(X L1) as the kernels left
+    # them in the workspace (codes [M, K] at 0, scales [M] and T [M, r] each
+    # on the next 256-byte boundary)
+    off_s = -(-(M * K) // 256) * 256
+    off = off_s + -(-(M * 4) // 256) * 256
     t_gpu = ws[off:off + M * r * 2].view(torch.bfloat16).view(M, r)
     rows = np.arange(M) if rows is None else np.asarray(rows)
     xs = workloads.to_u16(x)[rows]
     ref = orc.svdq_linear_fwd(xs, prep["rq"], prep["s_r"], prep["l1"], prep["l2"],
                               bias=None if bias is None else workloads.to_u16(bias), qt=qt)
+    assert np.array_equal(u8(ws[:M * K]).reshape(M, K)[rows], ref["xq"])
+    assert np.array_equal(f32(ws[off_s:off_s + M * 4].view(torch.float32))[rows].view(np.uint32),
+                          ref["sx"].view(np.uint32))
     # T: fp32 accumulation over K on the tensor cores, then one bf16 rounding
     xabs = np.abs(orc.bf16_to_f32(xs).astype(np.float64)) @ np.abs(orc.bf16_to_f32(prep["l1"]).astype(np.float64))
     gam = K * 2.0 ** -23 * xabs
@@ -485,12 +491,22 @@ def test_svdq_parity_small(w8, orc, r):
                                      (520, 136, 256, 16), (530, 300, 256, 16), (601, 264, 272, 16)])
 def test_svdq_parity_pairs(w8, orc, M, N, K, r):
     """M >= 512 with N % 8 == 0 runs the CTA-pair kernel, whose low-rank sum
-    is a second tensor-core product (256 x 128 tiles, ragged edges, r padded
-    to the MMA's K steps); (530, 300) keeps the single-SM form."""
+    is a tensor-core product of the pair written, in two halves of the tile's
+    columns, into the TMEM the tile's int32 sums occupied (ragged edges, r
+    padded to the MMA's K steps); (530, 300) keeps the single-SM form."""
     x = workloads.with_outlier_channels((M, K), 1.0, seed=M + r)
     w = workloads.rank_spike_weight(N, K, 8, 0.5, 0.02, seed=N + K)
     bias = workloads.normal((N,), 0.01, seed=N + 7)
     _svdq_check(w8, orc, x, w, r, bias=bias)
+
+
+@pytest.mark.parametrize("qt", [0, 1])
+def test_svdq_parity_long_rows(w8, orc, qt):
+    """Long rows (K = 6400): the T product's split along K and the row
+    quantizer's multi-warp teams."""
+    x = workloads.with_outlier_channels((130, 6400), 1.0, seed=74)
+    w = workloads.rank_spike_weight(264, 6400, 8, 0.5, 0.02, seed=75)
+    _svdq_check(w8, orc, x, w, 16, bias=workloads.normal((264,), 0.01, seed=76), qt=qt)
 
 
 @pytest.mark.parametrize("M", [130, 600])

@@ -82,6 +82,11 @@ __device__ __forceinline__ void row_amax_commit(uint32_t* y_amax, int64_t row, u
   if (h != 0) atomicMax(y_amax + row, h << 16);
 }
 
+// Low-rank (SVDQuant) epilogue: ranks up to 32; the staged L2^T rows are
+// kLowRankStride bf16 apart.
+constexpr int kLowRankMaxRank = 32;
+constexpr int kLowRankStride = 40;
+
 template <int KIND, int BN, int EPI>
 struct GemmCfg {
   static constexpr int kElem = (KIND == kKindBF16) ? 2 : 1;
@@ -91,9 +96,7 @@ struct GemmCfg {
   static constexpr int kBBytes = BN * kBKBytes;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;
-  static constexpr int kMaxRank = 32;
-  static constexpr int kLrStride = 40;   // bf16 per row of the transposed L2 tile (32 ranks + 8 pad: no bank conflicts)
-  static constexpr int kLrBytes = (EPI == kEpiLowRank) ? BN * kLrStride * 2 : 0;
+  static constexpr int kLrBytes = (EPI == kEpiLowRank) ? BN * kLowRankStride * 2 : 0;   // L2^T tile (stage_l2t)
   static constexpr int kEpiWarps = 8;   // two per TMEM lane quarter, splitting the column chunks
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
   // per epilogue warp, two 32 x 32 bf16 staging buffers for the TMA store
@@ -240,6 +243,166 @@ __device__ __forceinline__ void epilogue_scale_chunks(const EpiParams& ep, const
   }
 }
 
+// The SVDQuant low-rank epilogue.  L2^T of the tile's columns is staged in
+// shared memory: sLr[n][k] = L2[k][n0 + n] (bf16), zero for k >= r or
+// n0 + n >= N, rows kLowRankStride bf16 apart (32 ranks + 8 pad: no bank
+// conflicts for the fragment loads).  The copy moves units of 8 columns of
+// one rank: lane k of a warp takes rank k, so the transposing 2-byte stores
+// of a warp hit 32 consecutive ranks (no bank conflicts); every load of a
+// thread is issued before its first store (one round trip to L2, not one
+// per unit).  `et` is the thread's index among the kEpiThreads epilogue
+// threads.
+template <int BN, int kEpiThreads>
+__device__ __forceinline__ void stage_l2t(const EpiParams& ep, uint16_t* sLr, int n0, int N, int et) {
+  static_assert(kEpiThreads % 32 == 0 && BN % 8 == 0, "whole warps, whole units");
+  constexpr int kUnits = kLowRankMaxRank * BN / 8;
+  constexpr int kPer = (kUnits + kEpiThreads - 1) / kEpiThreads;
+  const bool vec = (N & 7) == 0;             // 16-byte aligned rows of L2
+  uint4 v[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int i = et + u * kEpiThreads;
+    const int k = i & 31, n = (i >> 5) * 8;
+    v[u] = make_uint4(0u, 0u, 0u, 0u);
+    if (i < kUnits && k < ep.r) {
+      const __nv_bfloat16* src = ep.lr_l2 + static_cast<int64_t>(k) * N + n0 + n;
+      if (vec && n0 + n + 8 <= N) {
+        v[u] = __ldg(reinterpret_cast<const uint4*>(src));
+      } else {
+        uint32_t h[4] = {0u, 0u, 0u, 0u};
+        for (int j = 0; j < 8; ++j)
+          if (n0 + n + j < N) h[j >> 1] |= static_cast<uint32_t>(__bfloat16_as_ushort(src[j])) << (16 * (j & 1));
+        v[u] = make_uint4(h[0], h[1], h[2], h[3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int i = et + u * kEpiThreads;
+    if (i < kUnits) {
+      const int k = i & 31, n = (i >> 5) * 8;
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        sLr[(n + j) * kLowRankStride + k] = static_cast<uint16_t>(w[j >> 1] >> (16 * (j & 1)));
+    }
+  }
+}
+
+// One epilogue warp's part of a 128-row x BN tile with the low-rank term:
+// y = bf16((((acc * s_x) * s_w) + bias) + lr), each step an fp32 RN
+// operation, lr = T L2 for the element, computed on the tensor cores by
+// warp-level bf16 MMAs from a zero accumulator (the MMA does not add an fp32
+// C operand at full precision).  The accumulator is read with 16x256b loads,
+// whose register layout is the m16n8 fragment layout of those MMAs, so each
+// thread holds the int32 / fp32 sums of exactly the elements its lr
+// fragments cover.  tacc: TMEM address of the accumulator buffer (column
+// offset, lane 0); T rows come from ep.lr_t (global, [M, r]); sLr holds L2^T
+// (stage_l2t); the warp's 32 x 32 blocks go out through its two staging
+// buffers sOutWarp with TMA stores, or directly when ldy % 8 != 0.
+template <int KIND, int BN, int kGroups>
+__device__ __forceinline__ void epilogue_lowrank_tile(const EpiParams& ep, const CUtensorMap* tmY, uint32_t tacc, int m0,
+                                                      int n0, int M, int N, int quarter, int group, int lane,
+                                                      const uint16_t* sLr, uint8_t* sOutWarp, uint32_t& out_iter) {
+  const int g = lane >> 2, tq = lane & 3;
+  const int rbase = m0 + quarter * 32;
+  const float sw0 = ep.s_col[0];    // the residual's tensor-wise scale
+  uint32_t afr[2][2][4];            // T fragments [m16 tile][k16 step][4]
+  float sxr[2][2];                  // s_x of rows g and g + 8 in each m16 tile
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int rr = rbase + mt * 16 + g + hh * 8;
+      sxr[mt][hh] = rr < M ? ep.s_row[rr] : 0.0f;
+    }
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const int rr = rbase + mt * 16 + g + (q4 & 1) * 8;
+        const int kk = ks * 16 + 2 * tq + (q4 >> 1) * 8;
+        afr[mt][ks][q4] = (rr < M && kk < ep.r)
+                              ? *reinterpret_cast<const uint32_t*>(ep.lr_t + static_cast<int64_t>(rr) * ep.r + kk)
+                              : 0u;
+      }
+    }
+  }
+  const int nks = (ep.r + 15) / 16;
+#pragma unroll 1
+  for (int c = group; c < BN / 32; c += kGroups) {
+    const int nc = n0 + c * 32;
+    if (nc >= N) break;                       // warp-uniform
+    float bcol[4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int n = nc + 8 * i + 2 * tq + u;
+        bcol[i][u] = (ep.bias != nullptr && n < N) ? __bfloat162float(ep.bias[n]) : 0.0f;
+      }
+    }
+    uint32_t rfr[2][16];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+      tmem_ld_16x256b_x4(tacc + (static_cast<uint32_t>(quarter * 32 + mt * 16) << 16) + static_cast<uint32_t>(c * 32),
+                         rfr[mt]);
+    tmem_ld_wait();
+    uint8_t* buf = sOutWarp + (out_iter & 1) * (32 * 32 * 2);
+    if (ep.tma_store) {
+      if (lane == 0) bulk_wait_read<1>();
+      __syncwarp();
+    }
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float lr[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        const uint16_t* brow = sLr + (c * 32 + 8 * i + g) * kLowRankStride + 2 * tq;
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+          if (ks < nks)
+            mma_bf16_m16n8k16(lr, afr[mt][ks], *reinterpret_cast<const uint32_t*>(brow + ks * 16),
+                              *reinterpret_cast<const uint32_t*>(brow + ks * 16 + 8));
+        }
+        float d[4];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int>(rfr[mt][4 * i + q4]))
+                                      : __uint_as_float(rfr[mt][4 * i + q4]);
+          a = __fmul_rn(__fmul_rn(a, sxr[mt][q4 >> 1]), sw0);
+          if (ep.bias != nullptr) a = __fadd_rn(a, bcol[i][q4 & 1]);
+          d[q4] = __fadd_rn(a, lr[q4]);
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int rl = mt * 16 + g + hh * 8;            // row within the warp's 32-row block
+          if (ep.tma_store) {
+            *reinterpret_cast<uint32_t*>(buf + rl * 64 + ((i ^ ((rl >> 1) & 3)) << 4) + 4 * tq) =
+                pack_bf16x2(d[2 * hh], d[2 * hh + 1]);
+          } else {   // row stride not a 16-byte multiple: guarded 2-byte stores
+            const int rr = rbase + rl, n = nc + 8 * i + 2 * tq;
+            if (rr < M) {
+              __nv_bfloat16* out = ep.y + static_cast<int64_t>(rr) * ep.ldy;
+              if (n < N) out[n] = __float2bfloat16_rn(d[2 * hh]);
+              if (n + 1 < N) out[n + 1] = __float2bfloat16_rn(d[2 * hh + 1]);
+            }
+          }
+        }
+      }
+    }
+    if (ep.tma_store) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && rbase < M) {
+        tma_store_2d(tmY, buf, nc, rbase);
+        bulk_commit();
+      }
+      ++out_iter;
+    }
+  }
+}
+
 template <int KIND, bool B_MN, int BN, int EPI>
 __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -256,7 +419,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
   constexpr int kStages = C::kStages;
   uint8_t* sA = smem;                                        // kStages x kABytes
   uint8_t* sB = smem + kStages * C::kABytes;                 // kStages x kBBytes
-  uint16_t* sLr = reinterpret_cast<uint16_t*>(smem + kStages * C::kStageBytes);   // L2^T [BN][kLrStride] bf16
+  uint16_t* sLr = reinterpret_cast<uint16_t*>(smem + kStages * C::kStageBytes);   // L2^T [BN][kLowRankStride] bf16
   uint8_t* sOut = smem + kStages * C::kStageBytes + ((C::kLrBytes + 1023) & ~1023);   // epilogue staging
   uint8_t* tail = sOut + C::kOutBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(tail);
@@ -430,16 +593,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
         // is overwritten.
         if (local > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(lr_done, (local - 1) & 1, abort_flag, 0x500u, limit)))
           break;
-        // L2^T for the tile: sLr[n][k] = L2[k][n0 + n] (bf16), zero for k >= r
-        // or n0 + n >= N.  Consecutive threads read consecutive n (coalesced).
-        const int et = threadIdx.x - 64;
-        for (int i = et; i < C::kMaxRank * BN; i += kEpiThreads) {
-          const int k = i / BN, n = i % BN;
-          uint16_t v = 0;
-          if (k < ep.r && n0 + n < N)
-            v = __bfloat16_as_ushort(ep.lr_l2[static_cast<int64_t>(k) * N + n0 + n]);
-          sLr[n * C::kLrStride + k] = v;
-        }
+        stage_l2t<BN, kEpiThreads>(ep, sLr, n0, N, threadIdx.x - 64);
         mbar_arrive(lr_ready);
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(lr_ready, local & 1, abort_flag, 0x600u, limit))) break;
       }
@@ -448,110 +602,8 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[acc], acc_phase, abort_flag, 0x400u | acc, limit))) break;
       tc_fence_after();
       if constexpr (EPI == kEpiLowRank) {
-        // Accumulator read in the m16n8 fragment layout (16x256b loads), the
-        // layout of warp-level bf16 MMAs that compute T * L2 on the tensor
-        // cores for the same elements.
-        const int g = lane >> 2, tq = lane & 3;
-        const int rbase = m0 + quarter * 32;
-        const float sw0 = ep.s_col[0];    // the residual's tensor-wise scale
-        uint32_t afr[2][2][4];            // T fragments [m16 tile][k16 step][4]
-        float sxr[2][2];                  // s_x of rows g and g + 8 in each m16 tile
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int rr = rbase + mt * 16 + g + hh * 8;
-            sxr[mt][hh] = rr < M ? ep.s_row[rr] : 0.0f;
-          }
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const int rr = rbase + mt * 16 + g + (q4 & 1) * 8;
-              const int kk = ks * 16 + 2 * tq + (q4 >> 1) * 8;
-              afr[mt][ks][q4] = (rr < M && kk < ep.r)
-                                    ? *reinterpret_cast<const uint32_t*>(ep.lr_t + static_cast<int64_t>(rr) * ep.r + kk)
-                                    : 0u;
-            }
-          }
-        }
-        const int nks = (ep.r + 15) / 16;
-#pragma unroll 1
-        for (int c = group; c < BN / 32; c += kGroups) {
-          const int nc = n0 + c * 32;
-          if (nc >= N) break;                       // warp-uniform
-          float bcol[4][2];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int n = nc + 8 * i + 2 * tq + u;
-              bcol[i][u] = (ep.bias != nullptr && n < N) ? __bfloat162float(ep.bias[n]) : 0.0f;
-            }
-          }
-          uint32_t rfr[2][16];
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt)
-            tmem_ld_16x256b_x4(tmem + (static_cast<uint32_t>(quarter * 32 + mt * 16) << 16) +
-                                   static_cast<uint32_t>(acc * BN + c * 32),
-                               rfr[mt]);
-          tmem_ld_wait();
-          uint8_t* buf = sOut + ((e * 2 + (out_iter & 1)) * C::kOutBufBytes);
-          if (ep.tma_store) {
-            if (lane == 0) bulk_wait_read<1>();
-            __syncwarp();
-          }
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              // lr = T * L2 on the tensor cores from a zero accumulator (the
-              // MMA does not add an fp32 C operand at full precision), then
-              // y = (((acc * s_x) * s_w) + bias) + lr, each an fp32 RN operation.
-              float lr[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-              const uint16_t* brow = sLr + (c * 32 + 8 * i + g) * C::kLrStride + 2 * tq;
-#pragma unroll
-              for (int ks = 0; ks < 2; ++ks) {
-                if (ks < nks)
-                  mma_bf16_m16n8k16(lr, afr[mt][ks], *reinterpret_cast<const uint32_t*>(brow + ks * 16),
-                                    *reinterpret_cast<const uint32_t*>(brow + ks * 16 + 8));
-              }
-              float d[4];
-#pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4) {
-                float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int>(rfr[mt][4 * i + q4]))
-                                            : __uint_as_float(rfr[mt][4 * i + q4]);
-                a = __fmul_rn(__fmul_rn(a, sxr[mt][q4 >> 1]), sw0);
-                if (ep.bias != nullptr) a = __fadd_rn(a, bcol[i][q4 & 1]);
-                d[q4] = __fadd_rn(a, lr[q4]);
-              }
-#pragma unroll
-              for (int hh = 0; hh < 2; ++hh) {
-                const int rl = mt * 16 + g + hh * 8;            // row within the warp's 32-row block
-                if (ep.tma_store) {
-                  *reinterpret_cast<uint32_t*>(buf + rl * 64 + ((i ^ ((rl >> 1) & 3)) << 4) + 4 * tq) =
-                      pack_bf16x2(d[2 * hh], d[2 * hh + 1]);
-                } else {   // row stride not a 16-byte multiple: guarded 2-byte stores
-                  const int rr = rbase + rl, n = nc + 8 * i + 2 * tq;
-                  if (rr < M) {
-                    __nv_bfloat16* out = ep.y + static_cast<int64_t>(rr) * ep.ldy;
-                    if (n < N) out[n] = __float2bfloat16_rn(d[2 * hh]);
-                    if (n + 1 < N) out[n + 1] = __float2bfloat16_rn(d[2 * hh + 1]);
-                  }
-                }
-              }
-            }
-          }
-          if (ep.tma_store) {
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0 && rbase < M) {
-              tma_store_2d(&tmY, buf, nc, rbase);
-              bulk_commit();
-            }
-            ++out_iter;
-          }
-        }
+        epilogue_lowrank_tile<KIND, BN, kGroups>(ep, &tmY, tmem + static_cast<uint32_t>(acc * BN), m0, n0, M, N,
+                                                 quarter, group, lane, sLr, sOut + e * 2 * C::kOutBufBytes, out_iter);
       } else if constexpr (EPI == kEpiScaleT) {
         // Transposed product (few tokens): the kernel's rows are weight rows n
         // (A = the weight codes) and its columns tokens m (B = the activation

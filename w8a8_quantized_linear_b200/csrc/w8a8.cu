@@ -915,11 +915,11 @@ static w8a8_status svdq_fwd_impl(const void* x, int64_t M, int64_t N, int64_t K,
     tsk.partial = static_cast<uint32_t*>(
         c.take(static_cast<size_t>(tsplit) * static_cast<size_t>(M) * static_cast<size_t>(r) * 4));
   }
-  if ((st = launch_quantize_rows(x, K, M, K, QT, xq, K, sx, s)) != W8A8_OK) return st;
-  // T = bf16(X L1): bf16 tensor-core GEMM, L1 [K, r] read MN-major; split
-  // along K when the rows make few tiles (fp32 partial sums, added in split
-  // order, then one bf16 rounding).
   {
+    // the row quantizer, then T = bf16(X L1) as a bf16 tensor-core GEMM, L1
+    // [K, r] read MN-major, split along K when the rows make few tiles (fp32
+    // partial sums, added in split order, then one bf16 rounding)
+    if ((st = launch_quantize_rows(x, K, M, K, QT, xq, K, sx, s)) != W8A8_OK) return st;
     alignas(64) CUtensorMap ta, tb;
     if ((st = make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, K, M, K * 2, 64, kBM)) != W8A8_OK) return st;
     if ((st = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, l1, r, K, static_cast<int64_t>(r) * 2, 64, 64)) !=
@@ -959,8 +959,9 @@ static w8a8_status svdq_fwd_impl(const void* x, int64_t M, int64_t N, int64_t K,
   ep.lr_t = t;
   ep.lr_l2 = static_cast<const __nv_bfloat16*>(l2);
   ep.r = r;
-  // Rq is read early: the kernels since this call's row quantizer (the T
-  // product and its split-K finish) write only T and its partial sums
+  // Rq is read early by the single-SM kernel: the kernels since this call's
+  // first kernel (which waits for all earlier work before it lets the next
+  // one launch) write only the codes, scales, T and T's partial sums
   ep.early_weights = 1;
   if (pair) {
     // T [M, r] and L2 [r, N] tiles for the tensor-core low-rank product:
