@@ -283,6 +283,37 @@ def test_linear_fwd_int8_axis_bias_parity(w8, orc, M, N, K):
     assert np.array_equal(u16(y), ref["y"])
 
 
+# CTA-pair forwards (M >= 512) with both formats, both weight scale
+# granularities and a bias: fewer tiles than pairs at (600, 520, 512),
+# (1024, 1024, 1024) and the ragged (777, 264, 384); two full rounds over the
+# 74 pairs and a partial third at (4096, 3072, 256)
+PAIR_SHAPES = [(600, 520, 512), (1024, 1024, 1024), (777, 264, 384), (4096, 3072, 256)]
+
+
+@pytest.mark.parametrize("qt", ["int8", "e4m3"])
+@pytest.mark.parametrize("gran", ["tensor", "axis"])
+@pytest.mark.parametrize("M,N,K", PAIR_SHAPES)
+def test_linear_fwd_pair_parity(w8, orc, qt, gran, M, N, K):
+    x = workloads.with_outlier_channels((M, K), 1.0, seed=M + 2 * N + K)
+    w = workloads.normal((N, K), 0.02, seed=N + 9)
+    bias = workloads.normal((N,), 0.01, seed=N + 10)
+    q, g = QT[qt], (0 if gran == "tensor" else 1)
+    wq, sw = w8.quantize_weight(w.to(DEV), qt, gran)
+    xd, bd = x.to(DEV), bias.to(DEV)
+    y = w8.linear_fwd(xd, wq, sw, bias=bd)
+    assert torch.equal(y, w8.linear_fwd(xd, wq, sw, bias=bd))        # deterministic
+    wqr, swr = orc.quantize_weight(workloads.to_u16(w), q, g)
+    assert np.array_equal(u8(wq), wqr)
+    rows = np.unique(np.concatenate([np.arange(0, M, 7), np.arange(max(0, M - 256), M)]))
+    ref = orc.linear_fwd(workloads.to_u16(x)[rows], wqr, swr, qt=q, bias=workloads.to_u16(bias))
+    if q == 0:
+        assert np.array_equal(u16(y)[rows], ref["y"])
+    else:
+        ref["sw"] = swr[0] if g == 0 else swr[None, :]
+        err, bound = _fp8_tol(ref, u16(y)[rows])
+        assert np.all(err <= bound), float((err / bound).max())
+
+
 @pytest.mark.parametrize("M,N,K", [(256, 512, 512), (300, 520, 640), (1, 16, 16), (129, 257, 96), (5, 264, 4096)])
 def test_linear_fwd_e4m3_parity(w8, orc, M, N, K):
     x = workloads.with_outlier_channels((M, K), 1.0, seed=M + N)
