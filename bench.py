@@ -533,7 +533,7 @@ def run_case(args):
     import w8a8_quantized_linear_b200 as w8
     dev = torch.device("cuda", 0)
     if args.case in ("requant", "gguf_m1", "gguf_m64", "svdq", "requant_e4m3", "gguf_f_m1", "gguf_f_m4608",
-                     "svdq_e4m3", "wo_float8", "wo_gguf", "gguf_m512"):
+                     "svdq_e4m3", "wo_float8", "wo_gguf", "gguf_m512", "q8_0_quant", "q8_0_dequant"):
         return run_other_case(args, torch, workloads, w8, dev)
     wl = workloads.dit_mlp()
     if args.case in ("up", "dgrad_up"):
@@ -568,7 +568,16 @@ def run_other_case(args, torch, workloads, w8, dev):
     svdq / svdq_e4m3: the SVDQuant r = 32 forward at 4608 x 3072 x 3072 with
     an int8 / e4m3 residual; wo_float8 / wo_gguf: the weight-only forwards
     on the DiT up-projection (dequantize to bf16, then the bf16 Linear)."""
-    if args.case in ("wo_float8", "wo_gguf"):
+    if args.case in ("q8_0_quant", "q8_0_dequant"):
+        # the standalone Q8_0 quantize / dequantize, 2^26 fp32 values (256 MiB,
+        # twice the L2; the bench extras time 2^28)
+        n = 1 << 26
+        xf = workloads.q8_0_standalone(n).to(dev)
+        blk = w8.q8_0_quantize(xf)
+        yf = torch.empty_like(xf)
+        fn = (lambda: w8.q8_0_quantize(xf, out=blk)) if args.case == "q8_0_quant" else \
+            (lambda: w8.q8_0_dequantize(blk, n, out=yf))
+    elif args.case in ("wo_float8", "wo_gguf"):
         g = workloads.gguf_q8_0(M=M_TOK)
         x = g["x"].to(dev)
         if args.case == "wo_float8":
@@ -916,7 +925,7 @@ def main():
     ap.add_argument("--no-extras", dest="extras", action="store_false")
     ap.add_argument("--case", choices=["up", "down", "dgrad_down", "dgrad_up", "requant", "gguf_m1", "gguf_m64", "svdq",
                                        "requant_e4m3", "gguf_f_m1", "gguf_f_m4608", "svdq_e4m3", "wo_float8",
-                                       "wo_gguf", "gguf_m512"],
+                                       "wo_gguf", "gguf_m512", "q8_0_quant", "q8_0_dequant"],
                     default=None, help="run only one of the step's four quantize+GEMM pairs, or one other kernel "
                                        "of the path (for profiling), no JSON")
     args = ap.parse_args()
