@@ -71,7 +71,8 @@ typedef enum {
   W8A8_ERR_WORKSPACE = 4,
   W8A8_ERR_CUDA = 5,
   W8A8_ERR_DEVICE_TIMEOUT = 6,
-  W8A8_ERR_UNSUPPORTED_DEVICE = 7
+  W8A8_ERR_UNSUPPORTED_DEVICE = 7,
+  W8A8_ERR_DEVICE_BOUNDS = 8   /* debug build only: a device-side index check failed */
 } w8a8_status;
 
 typedef enum { W8A8_INT8 = 0, W8A8_E4M3 = 1 } w8a8_qtype;
@@ -387,6 +388,23 @@ size_t w8a8_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, int r);
 w8a8_status w8a8_device_status(w8a8_stream_t stream, int reset);
 w8a8_status w8a8_set_wait_limit_ns(uint64_t limit_ns);
 w8a8_status w8a8_selftest_wait(uint64_t limit_ns, w8a8_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Debug build (the same sources compiled with W8A8_DEBUG_CHECKS=1 into
+ * libw8a8_debug.so; not on the pages).  Every plain (non-TMA) global-memory
+ * access of a kernel first checks the index it derived against the extent
+ * the call's shape implies; an index outside that extent records
+ * W8A8_ERR_DEVICE_BOUNDS and the check's site in the status word read by
+ * w8a8_device_status, and the access is skipped - nothing faults.  TMA copies
+ * need no check (the hardware clips stores and zero-fills loads at the
+ * tensor map's bounds).  The release build, libw8a8.so, has no checks.
+ *  w8a8_selftest_bounds: one kernel evaluates a check one past the end of
+ *    an extent (it touches no memory): the debug build then records
+ *    W8A8_ERR_DEVICE_BOUNDS (site 0xBFFF); the release build records nothing.
+ *  w8a8_debug_checks: 1 in the debug build, 0 in the release build.
+ * ---------------------------------------------------------------------- */
+w8a8_status w8a8_selftest_bounds(w8a8_stream_t stream);
+int w8a8_debug_checks(void);
 w8a8_status w8a8_e4m3_encode(const float* x, int64_t n, uint8_t* y, w8a8_stream_t stream);
 const char* w8a8_last_error(void);
 

@@ -172,3 +172,16 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(w8, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         w8.lib()
+
+
+def test_debug_build_exports_and_reports_its_checks(L):
+    """libw8a8_debug.so (device-side index checks that record an error code
+    instead of faulting) builds from the same sources, exports the same
+    functions, and says it is the checked build; the release build says not."""
+    from w8a8_quantized_linear_b200 import _build
+    D = ctypes.CDLL(_build.build(debug=True))
+    for n in _header_functions():
+        assert hasattr(D, n), n
+    D.w8a8_debug_checks.restype = ctypes.c_int
+    assert D.w8a8_debug_checks() == 1
+    assert L.w8a8_debug_checks() == 0

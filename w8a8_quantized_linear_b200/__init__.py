@@ -19,7 +19,9 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libw8a8.so")
+# W8A8_LIBRARY=debug selects the build with device-side index checks
+# (libw8a8_debug.so, see include/w8a8.h); the default is the release build.
+LIB_PATH = os.path.join(_PKG, "libw8a8_debug.so" if os.environ.get("W8A8_LIBRARY") == "debug" else "libw8a8.so")
 
 INT8, E4M3 = 0, 1
 TENSOR, AXIS = 0, 1
@@ -29,7 +31,7 @@ ACTS = {"none": 0, "gelu": 1, "gelu_tanh": 2}
 
 STATUS = {0: "W8A8_OK", 1: "W8A8_ERR_INVALID_ARG", 2: "W8A8_ERR_UNSUPPORTED_SHAPE",
           3: "W8A8_ERR_MISALIGNED", 4: "W8A8_ERR_WORKSPACE", 5: "W8A8_ERR_CUDA",
-          6: "W8A8_ERR_DEVICE_TIMEOUT", 7: "W8A8_ERR_UNSUPPORTED_DEVICE"}
+          6: "W8A8_ERR_DEVICE_TIMEOUT", 7: "W8A8_ERR_UNSUPPORTED_DEVICE", 8: "W8A8_ERR_DEVICE_BOUNDS"}
 
 # Every symbol include/w8a8.h declares (checked by the tests).
 EXPORTS = ("w8a8_quantize_rows", "w8a8_quantize_weight", "q8_0_bytes", "q8_0_quantize",
@@ -38,7 +40,8 @@ EXPORTS = ("w8a8_quantize_rows", "w8a8_quantize_weight", "q8_0_bytes", "q8_0_qua
            "w8a8_device_status", "w8a8_set_wait_limit_ns", "w8a8_selftest_wait",
            "w8a8_e4m3_encode", "w8a8_last_error", "w8a8_linear_fwd_noalloc", "q8_0_dequantize_bf16",
            "w8a8_dequantize_e4m3_bf16", "bf16_linear_fwd", "float8_linear_fwd", "gguf_linear_fwd",
-           "w8a8_linear_fwd_ex", "bf16_linear_dgrad", "float8_linear_dgrad", "gguf_linear_dgrad")
+           "w8a8_linear_fwd_ex", "bf16_linear_dgrad", "float8_linear_dgrad", "gguf_linear_dgrad",
+           "w8a8_selftest_bounds", "w8a8_debug_checks")
 
 
 class W8A8Error(RuntimeError):
@@ -56,8 +59,8 @@ def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise RuntimeError("libw8a8.so is not built (run `python -m w8a8_quantized_linear_b200._build`); "
-                               "there is no fallback path")
+            raise RuntimeError("%s is not built (run `python -m w8a8_quantized_linear_b200._build`); "
+                               "there is no fallback path" % os.path.basename(LIB_PATH))
         L = ctypes.CDLL(LIB_PATH)
         sig = {
             "w8a8_quantize_rows": [_P, _I64, _I64, _I64, _I, _P, _I64, _P, _P],
@@ -75,6 +78,7 @@ def lib() -> ctypes.CDLL:
             "w8a8_device_status": [_P, _I],
             "w8a8_set_wait_limit_ns": [_U64],
             "w8a8_selftest_wait": [_U64, _P],
+            "w8a8_selftest_bounds": [_P],
             "w8a8_e4m3_encode": [_P, _I64, _P, _P],
             "w8a8_linear_fwd_noalloc": [_P, _I64, _I64, _I64, _I, _P, _P, _I, _P, _P, _P],
             "q8_0_dequantize_bf16": [_P, _I64, _P, _P],
@@ -97,6 +101,8 @@ def lib() -> ctypes.CDLL:
         L.w8a8_workspace_bytes.restype = _SZ
         L.w8a8_last_error.argtypes = []
         L.w8a8_last_error.restype = ctypes.c_char_p
+        L.w8a8_debug_checks.argtypes = []
+        L.w8a8_debug_checks.restype = _I
         _lib = L
     return _lib
 
@@ -483,6 +489,17 @@ def set_wait_limit_ns(limit_ns: int):
 
 def selftest_wait(limit_ns: int):
     _check(lib().w8a8_selftest_wait(int(limit_ns), _stream()))
+
+
+def selftest_bounds():
+    """One failing device-side index check (no memory touched): the debug
+    build records W8A8_ERR_DEVICE_BOUNDS, the release build nothing."""
+    _check(lib().w8a8_selftest_bounds(_stream()))
+
+
+def debug_checks() -> bool:
+    """True when the loaded library is the debug build with index checks."""
+    return bool(lib().w8a8_debug_checks())
 
 
 def e4m3_encode(x: torch.Tensor):

@@ -12,6 +12,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libw8a8.so")
+# the same sources with the device-side index checks (W8A8_DEBUG_CHECKS=1)
+LIB_DEBUG = os.path.join(PKG, "libw8a8_debug.so")
 MAIN = os.path.join(CSRC, "w8a8.cu")
 HEADERS = [os.path.join(ROOT, "include", "w8a8.h")] + [
     os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith((".cuh", ".cu"))]
@@ -31,28 +33,31 @@ def command(out: str = LIB, extra=()) -> list:
             "-I", os.path.join(ROOT, "include"), "-o", out, MAIN, *extra]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(h) <= t for h in HEADERS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + ".tmp.%d" % os.getpid()
-    cmd = command(tmp, ["-Xptxas", "-v"] if verbose else [])
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Build libw8a8.so, or with debug=True libw8a8_debug.so (device-side
+    index checks that record an error code instead of faulting)."""
+    lib = LIB_DEBUG if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    tmp = lib + ".tmp.%d" % os.getpid()
+    extra = (["-Xptxas", "-v"] if verbose else []) + (["-DW8A8_DEBUG_CHECKS=1"] if debug else [])
+    cmd = command(tmp, extra)
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError("nvcc failed building libw8a8.so")
+        raise RuntimeError("nvcc failed building %s" % os.path.basename(lib))
     if verbose:
         sys.stderr.write(res.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug="--debug" in sys.argv))

@@ -15,7 +15,7 @@ namespace w8a8 {
 // Per-device status word.  The first device-side error wins; the host reads
 // it with w8a8_device_status().  Kernels never trap.
 // ----------------------------------------------------------------------------
-enum DeviceError : unsigned { kDevOk = 0, kDevTimeout = 6 };
+enum DeviceError : unsigned { kDevOk = 0, kDevTimeout = 6, kDevBounds = 8 };
 
 __device__ unsigned g_status = 0;
 __device__ unsigned g_status_site = 0;        // which wait gave up (debugging)
@@ -23,6 +23,28 @@ __device__ unsigned long long g_wait_limit_ns = 2000000000ull;
 
 __device__ __forceinline__ void record_error(unsigned code, unsigned site) {
   if (atomicCAS(&g_status, 0u, code) == 0u) atomicExch(&g_status_site, site);
+}
+
+// Index checks of the debug build (libw8a8_debug.so, compiled with
+// W8A8_DEBUG_CHECKS=1): before a plain global-memory access, the index the
+// kernel derived is checked against the extent that the shape implies; an
+// index outside [0, extent) records kDevBounds and the site in the status
+// word, and the caller skips the access instead of touching the memory.
+// In the release build the check is the constant true and compiles away.
+// (TMA copies need no check: the hardware clips stores and zero-fills loads
+// at the tensor map's bounds.)
+#ifndef W8A8_DEBUG_CHECKS
+#define W8A8_DEBUG_CHECKS 0
+#endif
+__device__ __forceinline__ bool in_bounds(int64_t i, int64_t extent, unsigned site) {
+#if W8A8_DEBUG_CHECKS
+  if (i >= 0 && i < extent) return true;
+  record_error(kDevBounds, site);
+  return false;
+#else
+  (void)i; (void)extent; (void)site;
+  return true;
+#endif
 }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {

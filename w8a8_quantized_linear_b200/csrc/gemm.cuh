@@ -220,7 +220,7 @@ __device__ __forceinline__ void epilogue_scale_chunks(const EpiParams& ep, const
         bulk_commit();
       }
       ++out_iter;
-    } else if (row_ok) {
+    } else if (row_ok && in_bounds(row, M, 0xB101) && in_bounds(nc, N, 0xB102)) {
       __nv_bfloat16* out = ep.y + static_cast<int64_t>(row) * ep.ldy + nc;
       if (nc + 32 <= N && (ep.ldy & 7) == 0) {
   #pragma unroll
@@ -267,11 +267,13 @@ __device__ __forceinline__ void stage_l2t(const EpiParams& ep, uint16_t* sLr, in
     if (i < kUnits && k < ep.r) {
       const __nv_bfloat16* src = ep.lr_l2 + static_cast<int64_t>(k) * N + n0 + n;
       if (vec && n0 + n + 8 <= N) {
-        v[u] = __ldg(reinterpret_cast<const uint4*>(src));
+        if (in_bounds(static_cast<int64_t>(k) * N + n0 + n + 7, static_cast<int64_t>(ep.r) * N, 0xB105))
+          v[u] = __ldg(reinterpret_cast<const uint4*>(src));
       } else {
         uint32_t h[4] = {0u, 0u, 0u, 0u};
         for (int j = 0; j < 8; ++j)
-          if (n0 + n + j < N) h[j >> 1] |= static_cast<uint32_t>(__bfloat16_as_ushort(src[j])) << (16 * (j & 1));
+          if (n0 + n + j < N && in_bounds(static_cast<int64_t>(k) * N + n0 + n + j, static_cast<int64_t>(ep.r) * N, 0xB105))
+            h[j >> 1] |= static_cast<uint32_t>(__bfloat16_as_ushort(src[j])) << (16 * (j & 1));
         v[u] = make_uint4(h[0], h[1], h[2], h[3]);
       }
     }
@@ -322,7 +324,8 @@ __device__ __forceinline__ void epilogue_lowrank_tile(const EpiParams& ep, const
       for (int q4 = 0; q4 < 4; ++q4) {
         const int rr = rbase + mt * 16 + g + (q4 & 1) * 8;
         const int kk = ks * 16 + 2 * tq + (q4 >> 1) * 8;
-        afr[mt][ks][q4] = (rr < M && kk < ep.r)
+        afr[mt][ks][q4] = (rr < M && kk < ep.r && in_bounds(static_cast<int64_t>(rr) * ep.r + kk,
+                                                            static_cast<int64_t>(M) * ep.r, 0xB104))
                               ? *reinterpret_cast<const uint32_t*>(ep.lr_t + static_cast<int64_t>(rr) * ep.r + kk)
                               : 0u;
       }
@@ -382,7 +385,7 @@ __device__ __forceinline__ void epilogue_lowrank_tile(const EpiParams& ep, const
                 pack_bf16x2(d[2 * hh], d[2 * hh + 1]);
           } else {   // row stride not a 16-byte multiple: guarded 2-byte stores
             const int rr = rbase + rl, n = nc + 8 * i + 2 * tq;
-            if (rr < M) {
+            if (rr < M && in_bounds(rr, M, 0xB101)) {
               __nv_bfloat16* out = ep.y + static_cast<int64_t>(rr) * ep.ldy;
               if (n < N) out[n] = __float2bfloat16_rn(d[2 * hh]);
               if (n + 1 < N) out[n + 1] = __float2bfloat16_rn(d[2 * hh + 1]);
@@ -629,10 +632,13 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
             if (splits > 1) {
               uint32_t* pcol = ep.partial + static_cast<int64_t>(split) * N * M + row;
               for (int j = 0; j < 32; ++j)
-                if (nc + j < N) pcol[static_cast<int64_t>(nc + j) * M] = r[j];
+                if (nc + j < N && in_bounds((static_cast<int64_t>(split) * N + nc + j) * M + row,
+                                            static_cast<int64_t>(splits) * N * M, 0xB103))
+                  pcol[static_cast<int64_t>(nc + j) * M] = r[j];
             } else {
               for (int j = 0; j < 32; ++j) {
-                if (nc + j < N) {
+                if (nc + j < N && in_bounds(static_cast<int64_t>(nc + j) * ep.ldy + row,
+                                            static_cast<int64_t>(N) * ep.ldy, 0xB106)) {
                   float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int>(r[j])) : __uint_as_float(r[j]);
                   a = __fmul_rn(__fmul_rn(a, sxc[j]), swr);
                   if (ep.bias != nullptr) a = __fadd_rn(a, br);
@@ -660,7 +666,8 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
             uint32_t r[32];
             tmem_ld_x32(tmem + lane_base + static_cast<uint32_t>(acc * BN + c * 32), r);
             tmem_ld_wait();
-            if (row_ok) {
+            if (row_ok && in_bounds((static_cast<int64_t>(split) * M + row) * N + nc, static_cast<int64_t>(splits) * M * N,
+                                    0xB103)) {
               if (vec_partial && nc + 32 <= N) {
   #pragma unroll
                 for (int j = 0; j < 32; j += 4)
@@ -717,6 +724,7 @@ __global__ void __launch_bounds__(256) splitk_epilogue_kernel(const uint32_t* __
   const int64_t plane = M * N;
   for (int64_t i = blockIdx.x * 256ll + threadIdx.x; i < total; i += static_cast<int64_t>(gridDim.x) * 256) {
     const int64_t m = i / n8, n = (i - m * n8) * 8;
+    if (!in_bounds(m, M, 0xB107) || !in_bounds(n + 7, N, 0xB107)) continue;
     const uint4* p = reinterpret_cast<const uint4*>(partial + m * N + n);
     uint4 lo = __ldcg(p), hi = __ldcg(p + 1);
     uint32_t r[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};

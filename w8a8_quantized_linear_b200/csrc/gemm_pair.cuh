@@ -99,7 +99,7 @@ __device__ __forceinline__ void store_block_bf16(const EpiParams& ep, const CUte
       bulk_commit();
     }
     ++out_iter;
-  } else if (rbase + lane < M) {
+  } else if (rbase + lane < M && in_bounds(rbase + lane, M, 0xB201) && in_bounds(nc, N, 0xB201)) {
     __nv_bfloat16* out = ep.y + static_cast<int64_t>(rbase + lane) * ep.ldy + nc;
     for (int j = 0; j < 32; ++j)
       if (nc + j < N) out[j] = __float2bfloat16_rn(v[j]);

@@ -29,13 +29,15 @@ __device__ __forceinline__ void gemv_quantize_rows(const __nv_bfloat16* __restri
   for (int m = 0; m < M; ++m) {
     const uint4* row = reinterpret_cast<const uint4*>(x + m * ldx);
     uint32_t mb = 0;
-    for (int v = threadIdx.x; v < nv; v += kGemvThreads) mb = absmax8(__ldg(row + v), mb);
+    for (int v = threadIdx.x; v < nv; v += kGemvThreads)
+      if (in_bounds(v, nv, 0xB303)) mb = absmax8(__ldg(row + v), mb);
     const float a = block_max(bf2_absmax_final(mb), red);
     const float s = absmax_scale<0>(a);
     const float y = __frcp_rn(s);
     if (threadIdx.x == 0) s_out[m] = s;
     uint2* out = reinterpret_cast<uint2*>(codes + m * K);
-    for (int v = threadIdx.x; v < nv; v += kGemvThreads) out[v] = encode8<0>(__ldg(row + v), s, y);
+    for (int v = threadIdx.x; v < nv; v += kGemvThreads)
+      if (in_bounds(v, nv, 0xB303)) out[v] = encode8<0>(__ldg(row + v), s, y);
   }
   __syncthreads();
 }
@@ -58,6 +60,7 @@ __global__ void __launch_bounds__(kGemvThreads, 4) gemv_int8_kernel(const __nv_b
   const int nv = K >> 4;   // 16-byte units per row
   const float sw0 = axis ? 0.0f : s_col[0];
   for (int n = blockIdx.x * (kGemvThreads / 32) + warp; n < N; n += gridDim.x * (kGemvThreads / 32)) {
+    if (!in_bounds(n, N, 0xB301)) break;   // warp-uniform
     const uint4* wrow = reinterpret_cast<const uint4*>(wq + static_cast<int64_t>(n) * K);
     int acc[M];
 #pragma unroll
@@ -68,7 +71,7 @@ __global__ void __launch_bounds__(kGemvThreads, 4) gemv_int8_kernel(const __nv_b
       uint4 w8[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u)
-        if (base + 32 * u < nv) w8[u] = __ldg(wrow + base + 32 * u);
+        if (base + 32 * u < nv && in_bounds(base + 32 * u, nv, 0xB301)) w8[u] = __ldg(wrow + base + 32 * u);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         if (base + 32 * u < nv) {
@@ -96,7 +99,8 @@ __global__ void __launch_bounds__(kGemvThreads, 4) gemv_int8_kernel(const __nv_b
       float f = __int2float_rn(a);
       f = __fmul_rn(__fmul_rn(f, sx[lane]), axis ? __ldg(s_col + n) : sw0);
       if (bias != nullptr) f = __fadd_rn(f, __bfloat162float(bias[n]));
-      y[static_cast<int64_t>(lane) * N + n] = __float2bfloat16_rn(f);
+      if (in_bounds(static_cast<int64_t>(lane) * N + n, static_cast<int64_t>(M) * N, 0xB302))
+        y[static_cast<int64_t>(lane) * N + n] = __float2bfloat16_rn(f);
     }
   }
 }
@@ -147,7 +151,8 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_e4m3_min_blocks<M>()) gemv_
   for (int m = 0; m < M; ++m) {
     const uint4* row = reinterpret_cast<const uint4*>(x + m * ldx);
     uint32_t mb = 0;
-    for (int v = threadIdx.x; v < nv; v += kGemvThreads) mb = absmax8(__ldg(row + v), mb);
+    for (int v = threadIdx.x; v < nv; v += kGemvThreads)
+      if (in_bounds(v, nv, 0xB303)) mb = absmax8(__ldg(row + v), mb);
     const float a = block_max(bf2_absmax_final(mb), red);
     const float s = absmax_scale<1>(a);
     const float yr = __frcp_rn(s);
@@ -181,6 +186,7 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_e4m3_min_blocks<M>()) gemv_
   const int nu = K >> 4;   // 16-code units per weight row
   const float sw0 = axis ? 0.0f : s_col[0];
   for (int n = blockIdx.x * (kGemvThreads / 32) + warp; n < N; n += gridDim.x * (kGemvThreads / 32)) {
+    if (!in_bounds(n, N, 0xB301)) break;   // warp-uniform
     const uint4* wrow = reinterpret_cast<const uint4*>(wq + static_cast<int64_t>(n) * K);
     float acc[M];
 #pragma unroll
@@ -189,7 +195,7 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_e4m3_min_blocks<M>()) gemv_
       uint4 w8[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u)
-        if (base + 32 * u < nu) w8[u] = __ldg(wrow + base + 32 * u);
+        if (base + 32 * u < nu && in_bounds(base + 32 * u, nu, 0xB301)) w8[u] = __ldg(wrow + base + 32 * u);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int U = base + 32 * u;
@@ -232,7 +238,8 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_e4m3_min_blocks<M>()) gemv_
       float f = __fmul_rn(a, 256.0f);   // the products carried 2^-8
       f = __fmul_rn(__fmul_rn(f, sx[lane]), axis ? __ldg(s_col + n) : sw0);
       if (bias != nullptr) f = __fadd_rn(f, __bfloat162float(bias[n]));
-      y[static_cast<int64_t>(lane) * N + n] = __float2bfloat16_rn(f);
+      if (in_bounds(static_cast<int64_t>(lane) * N + n, static_cast<int64_t>(M) * N, 0xB302))
+        y[static_cast<int64_t>(lane) * N + n] = __float2bfloat16_rn(f);
     }
   }
 }

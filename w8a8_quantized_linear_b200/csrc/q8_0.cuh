@@ -46,7 +46,7 @@ __global__ void __launch_bounds__(256) q8_0_quantize_kernel(const float* __restr
 #pragma unroll
     for (int u = 0; u < kQ80Unroll; ++u) {
       const int64_t base = (c * kQ80Unroll + u) * 256 + lane * 8;
-      if (base + 8 <= n) {
+      if (base + 8 <= n && in_bounds(base + 7, n, 0xB401)) {
         const float4 p0 = __ldg(reinterpret_cast<const float4*>(x + base));
         const float4 p1 = __ldg(reinterpret_cast<const float4*>(x + base) + 1);
         v[u][0] = p0.x; v[u][1] = p0.y; v[u][2] = p0.z; v[u][3] = p0.w;
@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(256) q8_0_quantize_kernel(const float* __restr
     __syncwarp();
     for (int i = lane; i < kQ80Chunk / 16; i += 32) {
       const int64_t off = c * kQ80Chunk + i * 16;
-      if (off + 16 <= nbytes) {
+      if (off + 16 <= nbytes && in_bounds(off + 15, nbytes, 0xB401)) {
         *reinterpret_cast<uint4*>(blocks + off) = *reinterpret_cast<const uint4*>(st + i * 16);
       } else {
         for (int b = 0; b < 16; ++b)
@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(256) q8_0_dequantize_kernel(const uint8_t* __r
        c += static_cast<int64_t>(gridDim.x) * kQ80WarpsPerBlock) {
     for (int i = lane; i < kQ80Chunk / 16; i += 32) {
       const int64_t off = c * kQ80Chunk + i * 16;
-      if (off + 16 <= nbytes) {
+      if (off + 16 <= nbytes && in_bounds(off + 15, nbytes, 0xB402)) {
         *reinterpret_cast<uint4*>(st + i * 16) = __ldg(reinterpret_cast<const uint4*>(blocks + off));
       } else {
         for (int b = 0; b < 16; ++b) st[i * 16 + b] = (off + b < nbytes) ? blocks[off + b] : 0;
@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(256) q8_0_dequantize_kernel(const uint8_t* __r
       const int64_t base = (c * kQ80Unroll + u) * 256 + lane * 8;
       if constexpr (BF16) {
         __nv_bfloat16* y = static_cast<__nv_bfloat16*>(yv);
-        if (base + 8 <= n) {
+        if (base + 8 <= n && in_bounds(base + 7, n, 0xB402)) {
           *reinterpret_cast<uint4*>(y + base) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
                                                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
         } else {
@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(256) q8_0_dequantize_kernel(const uint8_t* __r
         }
       } else {
         float* y = static_cast<float*>(yv);
-        if (base + 8 <= n) {
+        if (base + 8 <= n && in_bounds(base + 7, n, 0xB402)) {
           float4* o = reinterpret_cast<float4*>(y + base);
           o[0] = make_float4(v[0], v[1], v[2], v[3]);
           o[1] = make_float4(v[4], v[5], v[6], v[7]);
@@ -194,6 +194,7 @@ __global__ void __launch_bounds__(32 * kRequantMaxWarps) q8_0_to_axis_warp_kerne
   uint8_t* rowbuf = rowbuf_all + warp * row_stride;
   for (int64_t n = blockIdx.x * static_cast<int64_t>(nwarps) + warp; n < N;
        n += static_cast<int64_t>(gridDim.x) * nwarps) {
+    if (!in_bounds(n, N, 0xB403)) break;   // warp-uniform
     const uint8_t* src = blocks + n * row_bytes;
     if (((reinterpret_cast<uintptr_t>(src) | static_cast<uintptr_t>(row_bytes)) & 15) == 0) {
       for (int64_t i = lane; i < row_bytes / 16; i += 32)
@@ -237,6 +238,7 @@ __global__ void __launch_bounds__(32 * kRequantMaxWarps) q8_0_to_axis_warp_kerne
         w[i] = c;
       }
       uint4* out = reinterpret_cast<uint4*>(q + n * K + b * kQ80Block);
+      if (!in_bounds(n * K + b * kQ80Block + 31, N * K, 0xB404)) continue;
       out[0] = make_uint4(w[0], w[1], w[2], w[3]);
       out[1] = make_uint4(w[4], w[5], w[6], w[7]);
     }
@@ -470,6 +472,7 @@ __global__ void __launch_bounds__(kRqThreads) q8_0_to_axis_team_kernel(const uin
       uint32_t o[8];
       rq_block_codes<QT>(w, odd, rq_block_scale(w, odd), s, rcp, o);
       uint4* dst = reinterpret_cast<uint4*>(q + n * K + 32 * static_cast<int64_t>(b));
+      if (!in_bounds(n * K + 32 * static_cast<int64_t>(b) + 31, N * K, 0xB404)) continue;
       dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
       dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
     }
@@ -556,6 +559,7 @@ __global__ void __launch_bounds__(NT, MINB) q8_0_to_axis_hold_kernel(const uint8
         uint32_t o[8];
         rq_block_codes<QT>(w[h], odd, rq_block_scale(w[h], odd), s, rcp, o);
         uint4* dst = reinterpret_cast<uint4*>(q + n * K + 32 * static_cast<int64_t>(b));
+        if (!in_bounds(n * K + 32 * static_cast<int64_t>(b) + 31, N * K, 0xB404)) continue;
         dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
         dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
       }

@@ -109,7 +109,8 @@ __device__ __forceinline__ float bf2_absmax_final(uint32_t m) {
 __device__ __forceinline__ void clear_words(uint32_t* zero_out, int64_t zero_n) {
   if (zero_out == nullptr) return;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < zero_n; i += stride) zero_out[i] = 0u;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < zero_n; i += stride)
+    if (in_bounds(i, zero_n, 0xB006)) zero_out[i] = 0u;
 }
 
 // Block-wide max; every thread gets the result.  red: >= 32 floats of smem.
@@ -147,19 +148,20 @@ __global__ void __launch_bounds__(1024) quantize_rows_kernel(const __nv_bfloat16
   if constexpr (CHAIN) clear_words(zero_out, zero_n);
   const int64_t nv = K >> 3;
   for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+    if (!in_bounds(m, M, 0xB001)) break;
     const uint4* row = reinterpret_cast<const uint4*>(x + m * ldx);
     uint4 keep[kRowVecs];
     uint32_t mb = 0;
 #pragma unroll
     for (int j = 0; j < kRowVecs; ++j) {
       const int64_t v = threadIdx.x + static_cast<int64_t>(j) * blockDim.x;
-      if (v < nv) {
+      if (v < nv && in_bounds(v, nv, 0xB002)) {
         keep[j] = __ldg(row + v);
         mb = absmax8(keep[j], mb);
       }
     }
     for (int64_t v = threadIdx.x + static_cast<int64_t>(kRowVecs) * blockDim.x; v < nv; v += blockDim.x)
-      mb = absmax8(__ldg(row + v), mb);
+      if (in_bounds(v, nv, 0xB002)) mb = absmax8(__ldg(row + v), mb);
     const float a = (CHAIN && amax_in != nullptr) ? __uint_as_float(amax_in[m]) : block_max(bf2_absmax_final(mb), red);
     const float s = absmax_scale<QT>(a);
     const float rcp = __frcp_rn(s);
@@ -168,10 +170,10 @@ __global__ void __launch_bounds__(1024) quantize_rows_kernel(const __nv_bfloat16
 #pragma unroll
     for (int j = 0; j < kRowVecs; ++j) {
       const int64_t v = threadIdx.x + static_cast<int64_t>(j) * blockDim.x;
-      if (v < nv) out[v] = encode8<QT>(keep[j], s, rcp);
+      if (v < nv && in_bounds(v, nv, 0xB002)) out[v] = encode8<QT>(keep[j], s, rcp);
     }
     for (int64_t v = threadIdx.x + static_cast<int64_t>(kRowVecs) * blockDim.x; v < nv; v += blockDim.x)
-      out[v] = encode8<QT>(__ldg(row + v), s, rcp);
+      if (in_bounds(v, nv, 0xB002)) out[v] = encode8<QT>(__ldg(row + v), s, rcp);
   }
 }
 
@@ -203,16 +205,17 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_team_kernel(const __nv_b
   int iter = 0;
   for (int64_t m = blockIdx.x * static_cast<int64_t>(teams) + team; m < M;
        m += static_cast<int64_t>(gridDim.x) * teams, ++iter) {
+    const bool row_ok = in_bounds(m, M, 0xB003);   // (a team-uniform test: no early exit before the barrier)
     const uint4* row = reinterpret_cast<const uint4*>(x + m * ldx);
     uint4 keep[kTeamVecs];
 #pragma unroll
     for (int j = 0; j < kTeamVecs; ++j) {
       const int v = tl + j * (32 * TW);
-      if (v < nv) keep[j] = __ldg(row + v);
+      if (row_ok && v < nv && in_bounds(v, nv, 0xB004)) keep[j] = __ldg(row + v);
     }
     float a;
     if (CHAIN && amax_in != nullptr) {   // uniform over the kernel
-      a = __uint_as_float(amax_in[m]);
+      a = row_ok ? __uint_as_float(amax_in[m]) : 0.0f;
     } else {
       uint32_t mb = 0;
 #pragma unroll
@@ -230,12 +233,12 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_team_kernel(const __nv_b
     }
     const float s = absmax_scale<QT>(a);
     const float rcp = __frcp_rn(s);
-    if (tl == 0) scale[m] = s;
+    if (row_ok && tl == 0) scale[m] = s;
     uint2* out = reinterpret_cast<uint2*>(q + m * ldq);
 #pragma unroll
     for (int j = 0; j < kTeamVecs; ++j) {
       const int v = tl + j * (32 * TW);
-      if (v < nv) out[v] = encode8<QT>(keep[j], s, rcp);
+      if (row_ok && v < nv) out[v] = encode8<QT>(keep[j], s, rcp);
     }
   }
 }
@@ -248,7 +251,7 @@ __global__ void __launch_bounds__(256) absmax_kernel(const uint4* __restrict__ w
   uint32_t mb = 0;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nvec;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    mb = absmax8(__ldg(w + i), mb);
+    if (in_bounds(i, nvec, 0xB005)) mb = absmax8(__ldg(w + i), mb);
   const float a = block_max(bf2_absmax_final(mb), red);
   if (threadIdx.x == 0) atomicMax(amax_bits, __float_as_uint(a));
 }
@@ -263,7 +266,7 @@ __global__ void __launch_bounds__(256) quantize_tensor_kernel(const uint4* __res
   if (blockIdx.x == 0 && threadIdx.x == 0) scale[0] = s;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nvec;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    q[i] = encode8<QT>(__ldg(w + i), s, rcp);
+    if (in_bounds(i, nvec, 0xB005)) q[i] = encode8<QT>(__ldg(w + i), s, rcp);
 }
 
 // fp32 -> E4M3FN codes with the quantizers' conversion.
@@ -271,6 +274,12 @@ __global__ void e4m3_encode_kernel(const float* __restrict__ x, int64_t n, uint8
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
     y[i] = static_cast<uint8_t>(cvt_e4m3x2(x[i], 0.0f) & 0xFFu);
+}
+
+// Index-check self test: a check one past the end of an extent (no memory
+// is touched): the debug build records kDevBounds at site 0xBFFF.
+__global__ void selftest_bounds_kernel(int64_t extent) {
+  if (!in_bounds(extent, extent, 0xBFFFu)) return;
 }
 
 // Bounded-wait self test: one thread waits on a barrier that nothing

@@ -1388,6 +1388,7 @@ w8a8_status w8a8_device_status(w8a8_stream_t stream, int reset) {
   }
   if (v == kDevOk) return W8A8_OK;
   if (v == kDevTimeout) return fail(W8A8_ERR_DEVICE_TIMEOUT, "device wait ran out (site 0x%x)", site);
+  if (v == kDevBounds) return fail(W8A8_ERR_DEVICE_BOUNDS, "device index check failed (site 0x%x)", site);
   return fail(W8A8_ERR_CUDA, "device status %u (site 0x%x)", v, site);
 }
 
@@ -1409,6 +1410,17 @@ w8a8_status w8a8_selftest_wait(uint64_t limit_ns, w8a8_stream_t stream) {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "selftest launch");
 }
+
+w8a8_status w8a8_selftest_bounds(w8a8_stream_t stream) {
+  W8A8_TRACE();
+  w8a8_status st = current_device(nullptr, nullptr);
+  if (st != W8A8_OK) return st;
+  selftest_bounds_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(1024);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? W8A8_OK : cuda_fail(e, "selftest launch");
+}
+
+int w8a8_debug_checks(void) { return W8A8_DEBUG_CHECKS; }
 
 w8a8_status w8a8_e4m3_encode(const float* x, int64_t n, uint8_t* y, w8a8_stream_t stream) {
   W8A8_TRACE();

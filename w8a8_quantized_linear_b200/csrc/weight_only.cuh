@@ -33,6 +33,7 @@ __global__ void __launch_bounds__(256) dequant_e4m3_bf16_kernel(const uint2* __r
   const float s = __ldg(scale);
   const float2 s2 = make_float2(s, s), up = make_float2(0x1p120f, 0x1p120f);
   for (int64_t i = blockIdx.x * 256ll + threadIdx.x; i < n8; i += static_cast<int64_t>(gridDim.x) * 256) {
+    if (!in_bounds(i, n8, 0xB501)) break;
     const uint2 c = __ldg(q + i);
     const uint32_t cw[2] = {c.x, c.y};
     uint32_t o[4];
