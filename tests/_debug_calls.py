@@ -60,5 +60,9 @@ def run_all(w8, dev):
         for M in (200, 600):
             out["svdq_%s_%d" % (qt, M)] = w8.svdq_linear_fwd(x(M, 512, 25), prep["rq"], prep["r_scale"], prep["l1"],
                                                              prep["l2"], bias=bias(520)).cpu()
+    # rows longer than the one-pass input kernel holds: row quantizer + T product
+    prep = w8.svdq_prepare(workloads.rank_spike_weight(136, 3088, 8, 0.5, 0.02, 26).to(dev), 8, "int8")
+    out["svdq_long_rows"] = w8.svdq_linear_fwd(x(45, 3088, 27), prep["rq"], prep["r_scale"], prep["l1"],
+                                               prep["l2"]).cpu()
     torch.cuda.synchronize()
     return out

@@ -20,6 +20,7 @@
 #include "q8_0.cuh"
 #include "gemv.cuh"
 #include "weight_only.cuh"
+#include "svdq_input.cuh"
 
 namespace w8a8 {
 namespace {
@@ -908,15 +909,32 @@ static w8a8_status svdq_fwd_impl(const void* x, int64_t M, int64_t N, int64_t K,
   void* xq = c.take(static_cast<size_t>(M * K));
   float* sx = static_cast<float*>(c.take(static_cast<size_t>(M) * 4));
   auto* t = static_cast<__nv_bfloat16*>(c.take(static_cast<size_t>(M) * r * 2));
-  const int tsplit = t_splits(M, K);
+  const bool one_pass = K <= kSiMaxK;   // 32 rows fit in one CTA's shared memory
+  const int tsplit = one_pass ? 1 : t_splits(M, K);
   SplitWs tsk;
   if (tsplit > 1) {
     tsk.splits = tsplit;
     tsk.partial = static_cast<uint32_t*>(
         c.take(static_cast<size_t>(tsplit) * static_cast<size_t>(M) * static_cast<size_t>(r) * 4));
   }
-  {
-    // the row quantizer, then T = bf16(X L1) as a bf16 tensor-core GEMM, L1
+  if (one_pass) {
+    // codes, scales and T = bf16(X L1) in one pass over X
+    alignas(64) CUtensorMap tl1;
+    if ((st = make_map(&tl1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, l1, r, K, static_cast<int64_t>(r) * 2, 32, kSiKC,
+                       CU_TENSOR_MAP_SWIZZLE_64B)) != W8A8_OK)
+      return st;
+    static std::atomic<uint64_t> si_smem_set{0};
+    int dev = 0;
+    if ((st = current_device(&dev, nullptr)) != W8A8_OK) return st;
+    auto kern = svdq_input_kernel<QT>;
+    cudaError_t e = set_smem_once(kern, si_smem_bytes(kSiMaxK), dev, si_smem_set);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(svdq_input)");
+    e = launch_pdl(kern, dim3(static_cast<unsigned>((M + kSiRows - 1) / kSiRows)), dim3(kSiThreads),
+                   si_smem_bytes(static_cast<int>(K)), s, static_cast<const __nv_bfloat16*>(x), tl1,
+                   static_cast<int>(M), static_cast<int>(K), r, static_cast<uint8_t*>(xq), sx, t);
+    if (e != cudaSuccess) return cuda_fail(e, "svdq input launch");
+  } else {
+    // longer rows: the row quantizer, then T = bf16(X L1) as a bf16 tensor-core GEMM, L1
     // [K, r] read MN-major, split along K when the rows make few tiles (fp32
     // partial sums, added in split order, then one bf16 rounding)
     if ((st = launch_quantize_rows(x, K, M, K, QT, xq, K, sx, s)) != W8A8_OK) return st;
