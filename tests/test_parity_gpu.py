@@ -287,7 +287,9 @@ def test_linear_fwd_int8_axis_bias_parity(w8, orc, M, N, K):
 # granularities and a bias: fewer tiles than pairs at (600, 520, 512),
 # (1024, 1024, 1024) and the ragged (777, 264, 384); two full rounds over the
 # 74 pairs and a partial third at (4096, 3072, 256)
-PAIR_SHAPES = [(600, 520, 512), (1024, 1024, 1024), (777, 264, 384), (4096, 3072, 256)]
+# CTA-pair forwards; (520, 9000): two rounds of tiles over the 74 pairs, the
+# last tile 40 columns wide.
+PAIR_SHAPES = [(600, 520, 512), (1024, 1024, 1024), (777, 264, 384), (4096, 3072, 256), (520, 9000, 512)]
 
 
 @pytest.mark.parametrize("qt", ["int8", "e4m3"])
