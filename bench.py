@@ -533,7 +533,8 @@ def run_case(args):
     import w8a8_quantized_linear_b200 as w8
     dev = torch.device("cuda", 0)
     if args.case in ("requant", "gguf_m1", "gguf_m64", "svdq", "requant_e4m3", "gguf_f_m1", "gguf_f_m4608",
-                     "svdq_e4m3", "wo_float8", "wo_gguf", "gguf_m512", "q8_0_quant", "q8_0_dequant"):
+                     "svdq_e4m3", "wo_float8", "wo_gguf", "gguf_m512", "q8_0_quant", "q8_0_dequant",
+                     "float_w8a8", "float_w8a8_int8"):
         return run_other_case(args, torch, workloads, w8, dev)
     wl = workloads.dit_mlp()
     if args.case in ("up", "dgrad_up"):
@@ -567,7 +568,9 @@ def run_other_case(args, torch, workloads, w8, dev):
     gguf_f_m1 / gguf_f_m4608: the GGUF A8 float forward at M = 1 / 4608;
     svdq / svdq_e4m3: the SVDQuant r = 32 forward at 4608 x 3072 x 3072 with
     an int8 / e4m3 residual; wo_float8 / wo_gguf: the weight-only forwards
-    on the DiT up-projection (dequantize to bf16, then the bf16 Linear)."""
+    on the DiT up-projection (dequantize to bf16, then the bf16 Linear);
+    float_w8a8 / float_w8a8_int8: the float W8A8 forward with bias at 4096 x
+    3072 x 3072 (e4m3), and the same shape with int8 codes."""
     if args.case in ("q8_0_quant", "q8_0_dequant"):
         # the standalone Q8_0 quantize / dequantize, 2^26 fp32 values (256 MiB,
         # twice the L2; the bench extras time 2^28)
@@ -586,6 +589,12 @@ def run_other_case(args, torch, workloads, w8, dev):
         else:
             blk = w8.q8_0_quantize(g["w_f32"].reshape(-1).to(dev))
             fn = lambda: w8.gguf_linear_fwd(x, blk, MLP)
+    elif args.case in ("float_w8a8", "float_w8a8_int8"):
+        d = workloads.float_w8a8()
+        qt = "e4m3" if args.case == "float_w8a8" else "int8"
+        wq, sw = w8.quantize_weight(d["w"].to(dev), qt, "tensor")
+        x, bias = d["x"].to(dev), d["bias"].to(dev)
+        fn = lambda: w8.linear_fwd(x, wq, sw, bias=bias)
     elif args.case in ("svdq", "svdq_e4m3"):
         d = workloads.svdquant()
         prep = w8.svdq_prepare(d["w"].to(dev), d["r"], "e4m3" if args.case == "svdq_e4m3" else "int8")
@@ -925,7 +934,8 @@ def main():
     ap.add_argument("--no-extras", dest="extras", action="store_false")
     ap.add_argument("--case", choices=["up", "down", "dgrad_down", "dgrad_up", "requant", "gguf_m1", "gguf_m64", "svdq",
                                        "requant_e4m3", "gguf_f_m1", "gguf_f_m4608", "svdq_e4m3", "wo_float8",
-                                       "wo_gguf", "gguf_m512", "q8_0_quant", "q8_0_dequant"],
+                                       "wo_gguf", "gguf_m512", "q8_0_quant", "q8_0_dequant", "float_w8a8",
+                                       "float_w8a8_int8"],
                     default=None, help="run only one of the step's four quantize+GEMM pairs, or one other kernel "
                                        "of the path (for profiling), no JSON")
     args = ap.parse_args()
