@@ -533,12 +533,14 @@ def test_svdq_parity_pairs(w8, orc, M, N, K, r):
     _svdq_check(w8, orc, x, w, r, bias=bias)
 
 
-@pytest.mark.parametrize("M,K,r,qt", [(33, 3072, 32, 0), (65, 3072, 24, 1), (33, 3088, 8, 0), (97, 1040, 16, 1)])
+@pytest.mark.parametrize("M,K,r,qt", [(33, 3072, 32, 0), (65, 3072, 24, 1), (33, 3088, 8, 0), (97, 1040, 16, 1),
+                                      (1, 16, 8, 0), (31, 48, 32, 1)])
 def test_svdq_input_row_lengths(w8, orc, M, K, r, qt):
     """Rows up to 3072 columns: codes, scales and T come from one pass over X
     (32 rows per CTA held on chip; a CTA with one row); K = 3088 takes the
     row quantizer and the T product; K = 1040 ends in a partial block of 64
-    columns."""
+    columns; K = 16 and 48 give one k-step to one or three of the eight
+    k-groups (the others add zero partial sums)."""
     x = workloads.with_outlier_channels((M, K), 1.0, seed=M + K)
     w = workloads.rank_spike_weight(136, K, 8, 0.5, 0.02, seed=K + r)
     _svdq_check(w8, orc, x, w, r, bias=workloads.normal((136,), 0.01, seed=77), qt=qt)

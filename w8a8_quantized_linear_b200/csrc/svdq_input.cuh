@@ -75,6 +75,12 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t add
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(addr));
 }
+// Column of the partial-sum array red[k-group][row][32] where rank column c
+// of `row` is kept: c ^ (8 (row & 3) + ((row >> 2) & 1)).  An MMA warp's
+// store of one accumulator element (rows r0 + lane / 4, columns 8 j + 2 (lane
+// % 4) + e) then hits 32 distinct banks.
+__device__ __forceinline__ int si_red_col(int row, int c) { return c ^ (8 * (row & 3) + ((row >> 2) & 1)); }
+
 __device__ __forceinline__ void si_bar() {   // every warp of the block
   asm volatile("bar.sync 1, %0;" ::"n"(kSiThreads) : "memory");
 }
@@ -155,7 +161,8 @@ __global__ void __launch_bounds__(kSiThreads, 1)
         mbar_arrive(&xfull[c]);
       }
     }
-  } else if (warp < kSiMmaWarps) {
+  }
+  if (warp < kSiMmaWarps) {
     // ---- T partial sums and row absmax, as the X chunks and L1 blocks land
     const int h = warp & 1, g = warp >> 1;
     const uint32_t xs_u = smem_u32(xs), ring_u = smem_u32(ring);
@@ -207,33 +214,37 @@ __global__ void __launch_bounds__(kSiThreads, 1)
       atomicMax(&amax[16 * h + (lane >> 2) + 8], __float_as_uint(ahi));
     }
     si_bar();   // every MMA warp is past its last L1 block: the ring becomes `red`
-    float* rp = red + g * (kSiRows * 32) + (16 * h + (lane >> 2)) * 32 + 2 * (lane & 3);
+    float* rg = red + g * (kSiRows * 32);
+    const int r0 = 16 * h + (lane >> 2), c0 = 2 * (lane & 3);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      rp[8 * j] = acc[j][0];
-      rp[8 * j + 1] = acc[j][1];
-      rp[8 * 32 + 8 * j] = acc[j][2];
-      rp[8 * 32 + 8 * j + 1] = acc[j][3];
+      rg[r0 * 32 + si_red_col(r0, 8 * j + c0)] = acc[j][0];
+      rg[r0 * 32 + si_red_col(r0, 8 * j + c0 + 1)] = acc[j][1];
+      rg[(r0 + 8) * 32 + si_red_col(r0 + 8, 8 * j + c0)] = acc[j][2];
+      rg[(r0 + 8) * 32 + si_red_col(r0 + 8, 8 * j + c0 + 1)] = acc[j][3];
     }
-  }
-  if (warp >= kSiMmaWarps) si_bar();   // (the MMA warps arrived above)
-  if (threadIdx.x < kSiRows) {
-    const float sc = absmax_scale<QT>(__uint_as_float(amax[threadIdx.x]));
-    srow[threadIdx.x] = sc;
-    rrow[threadIdx.x] = __frcp_rn(sc);
-    const int m = m0 + threadIdx.x;
-    if (m < M && in_bounds(m, M, 0xB601)) scale[m] = sc;
+  } else {
+    si_bar();   // (the MMA warps arrive above)
+    if (warp == kSiMmaWarps) {
+      // the row scales (every absmax is in), while the MMA warps store their sums
+      const float sc = absmax_scale<QT>(__uint_as_float(amax[lane]));
+      srow[lane] = sc;
+      rrow[lane] = __frcp_rn(sc);
+      const int m = m0 + lane;
+      if (m < M && in_bounds(m, M, 0xB601)) scale[m] = sc;
+    }
   }
   si_bar();
   if (threadIdx.x < kSiRows * 32 / 2) {
     // T: two ranks per thread, the k-groups' partial sums in order 0..7
     const int e = 2 * threadIdx.x;
     const int row = e >> 5, col = e & 31;
+    const int p0 = row * 32 + si_red_col(row, col), p1 = row * 32 + si_red_col(row, col + 1);
     float v0 = 0.0f, v1 = 0.0f;
 #pragma unroll
     for (int gg = 0; gg < kSiKGroups; ++gg) {
-      v0 += red[gg * (kSiRows * 32) + e];
-      v1 += red[gg * (kSiRows * 32) + e + 1];
+      v0 += red[gg * (kSiRows * 32) + p0];
+      v1 += red[gg * (kSiRows * 32) + p1];
     }
     const int m = m0 + row;
     if (m < M && col < r && in_bounds(static_cast<int64_t>(m) * r + col + 1, static_cast<int64_t>(M) * r, 0xB602))
