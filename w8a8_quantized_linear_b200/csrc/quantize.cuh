@@ -243,15 +243,37 @@ __global__ void __launch_bounds__(256, 4) quantize_rows_team_kernel(const __nv_b
   }
 }
 
+// 16-byte read-only loads with an L2 eviction priority (an L2 cache policy
+// from createpolicy): the tensor-wise quantizer reads W twice, and marks
+// its first pass's lines to stay in L2 and its second pass's to go first.
+__device__ __forceinline__ uint4 ldg_policy(const uint4* p, uint64_t policy) {
+  uint4 v;
+  asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(policy));
+  return v;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 // Tensor-wise weight quantization, pass 1: global absmax of W (as the bit
 // pattern of a non-negative float, so an unsigned atomicMax orders it).
 __global__ void __launch_bounds__(256) absmax_kernel(const uint4* __restrict__ w, int64_t nvec,
                                                      unsigned* __restrict__ amax_bits) {
   __shared__ float red[32];
   uint32_t mb = 0;
+  const uint64_t keep = policy_evict_last();   // pass 2 reads W again
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nvec;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    if (in_bounds(i, nvec, 0xB005)) mb = absmax8(__ldg(w + i), mb);
+    if (in_bounds(i, nvec, 0xB005)) mb = absmax8(ldg_policy(w + i, keep), mb);
   const float a = block_max(bf2_absmax_final(mb), red);
   if (threadIdx.x == 0) atomicMax(amax_bits, __float_as_uint(a));
 }
@@ -264,9 +286,10 @@ __global__ void __launch_bounds__(256) quantize_tensor_kernel(const uint4* __res
   const float s = absmax_scale<QT>(__uint_as_float(*amax_bits));
   const float rcp = __frcp_rn(s);
   if (blockIdx.x == 0 && threadIdx.x == 0) scale[0] = s;
+  const uint64_t drop = policy_evict_first();   // W's last read
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nvec;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    if (in_bounds(i, nvec, 0xB005)) q[i] = encode8<QT>(__ldg(w + i), s, rcp);
+    if (in_bounds(i, nvec, 0xB005)) q[i] = encode8<QT>(ldg_policy(w + i, drop), s, rcp);
 }
 
 // fp32 -> E4M3FN codes with the quantizers' conversion.
