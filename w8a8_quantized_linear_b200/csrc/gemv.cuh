@@ -108,25 +108,43 @@ __global__ void __launch_bounds__(kGemvThreads, 4) gemv_int8_kernel(const __nv_b
 // ---------------------------------------------------------------------------
 // The e4m3 forward for a few tokens (M <= kGemvE4m3MaxRows), e.g. GGUF A8
 // float at decode: e4m3 has no exact CUDA-core dot product like dp4a, so the
-// codes are decoded to fp32 and multiplied there.  Every block quantizes the
-// M rows to e4m3 (the row quantizer's arithmetic) and keeps their values,
-// times 2^112, in shared memory; a warp per weight row decodes each weight
-// code with integer operations to its value times 2^-120 (e4m3_top_byte_scaled)
-// and accumulates fl(w a 2^-8) products - exact: 4-bit by 4-bit significands,
-// no subnormal - in fp32.  acc * 2^8 (exact) then takes the GEMM epilogue's
-// fp32 RN steps.  The sum is in another order than the tensor cores', within
-// the fp8 bound.
+// codes are multiplied as 16-bit floats.  Every block quantizes the M rows to
+// e4m3 (the row quantizer's arithmetic) and keeps their values as f16 in
+// shared memory (every e4m3 value is an f16 value); a warp per weight row
+// converts each pair of weight codes to an f16 pair (cvt.rn.f16x2.e4m3x2,
+// exact) and accumulates with the mixed-precision fma.rn.f32.f16: the product
+// of two f16 operands is exact in fp32 (4-bit by 4-bit significands here), so
+// each step is one fp32 RN add, in k order.  acc then takes the GEMM
+// epilogue's fp32 RN steps.  The sum is in another order than the tensor
+// cores', within the fp8 bound.
 //
 // Shared layout: the activations of row m, in 16-value units U (16 U .. 16 U
-// + 15), with the 4 float4 quads of unit U stored at ((U / 32) * 4 + quad) *
-// 128 + (U % 32) * 4, so that the 32 lanes of a warp (lane l takes units l,
-// l + 32, ...) read 32 consecutive float4: no bank conflict.
+// + 15) of two 16-byte halves (8 f16 each), half h of unit U at byte
+// (((U / 32) * 2 + h) * 32 + U % 32) * 16, so that the 32 lanes of a warp
+// (lane l takes units l, l + 32, ...) read 32 consecutive 16-byte words: no
+// bank conflict.
 constexpr int kGemvE4m3MaxRows = 4;
-constexpr int kGemvE4m3SmemBytes = 128 * 1024;   // M * (K rounded up to 512) * 4
+constexpr int kGemvE4m3SmemBytes = 128 * 1024;   // M * (K rounded up to 512) * 4 (f16 needs half)
 
-__device__ __forceinline__ int gemv_e4m3_slot(int k) {   // float index of value k within its row
-  const int u = k >> 4, quad = (k >> 2) & 3;
-  return (((u >> 5) * 4 + quad) << 7) + ((u & 31) << 2) + (k & 3);
+__device__ __forceinline__ int gemv_e4m3_half_off(int u, int h) {   // byte offset of half h of unit u
+  return ((((u >> 5) * 2 + h) << 5) + (u & 31)) << 4;
+}
+// Two e4m3 codes (bits 15..0 of v; the code in bits 7..0 comes first) -> their
+// values as an f16 pair, the first in the low half.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
+  uint32_t h2;
+  asm("{\n\t.reg .b16 lo;\n\tcvt.u16.u32 lo, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}" : "=r"(h2) : "r"(v));
+  return h2;
+}
+// acc + w.lo a.lo, then + w.hi a.hi: fp32 fma of f16 operands (exact products
+// of e4m3 values), one RN rounding each.
+__device__ __forceinline__ float fma_f16x2_f32(uint32_t w2, uint32_t a2, float acc) {
+  float r;
+  asm("{\n\t.reg .b16 w0, w1, a0, a1;\n\tmov.b32 {w0, w1}, %1;\n\tmov.b32 {a0, a1}, %2;\n\t"
+      "fma.rn.f32.f16 %0, w0, a0, %3;\n\tfma.rn.f32.f16 %0, w1, a1, %0;\n\t}"
+      : "=f"(r)
+      : "r"(w2), "r"(a2), "f"(acc));
+  return r;
 }
 
 // blocks per SM: as many as the registers allow (the weight stream needs
@@ -141,13 +159,12 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_e4m3_min_blocks<M>()) gemv_
                                                                  const __nv_bfloat16* __restrict__ bias,
                                                                  __nv_bfloat16* __restrict__ y) {
   extern __shared__ __align__(16) uint8_t gemv_smem[];
-  float* const act = reinterpret_cast<float*>(gemv_smem);
   __shared__ float red[32];
   __shared__ float sx[kGemvE4m3MaxRows];
   griddep_launch();
   griddep_wait();   // x may be the previous kernel's output
   const int nv = K >> 3;             // 8-value vectors per row
-  const int row_f = ((K + 511) >> 9) << 9;   // floats per row in shared memory
+  const int row_b = (((K + 511) >> 9) << 9) * 2;   // bytes per row in shared memory
   for (int m = 0; m < M; ++m) {
     const uint4* row = reinterpret_cast<const uint4*>(x + m * ldx);
     uint32_t mb = 0;
@@ -158,27 +175,11 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_e4m3_min_blocks<M>()) gemv_
     const float yr = __frcp_rn(s);
     if (threadIdx.x == 0) sx[m] = s;
     for (int v = threadIdx.x; v < nv; v += kGemvThreads) {
+      // values 8 v .. 8 v + 7: half (v & 1) of unit v / 2
       const uint2 c = encode8<1>(__ldg(row + v), s, yr);
-      const uint32_t cw[2] = {c.x, c.y};
-      float f[8];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        // code value * 2^-120, then * 2^116 * 2^116 = value * 2^112 (exact)
-        f[4 * j] = e4m3_top_byte_scaled(cw[j] << 24);
-        f[4 * j + 1] = e4m3_top_byte_scaled(cw[j] << 16);
-        f[4 * j + 2] = e4m3_top_byte_scaled(cw[j] << 8);
-        f[4 * j + 3] = e4m3_top_byte_scaled(cw[j]);
-      }
-      float* dst = act + m * row_f;
-#pragma unroll
-      for (int i = 0; i < 8; i += 4) {
-        float4 q4;
-        q4.x = __fmul_rn(__fmul_rn(f[i], 0x1p116f), 0x1p116f);
-        q4.y = __fmul_rn(__fmul_rn(f[i + 1], 0x1p116f), 0x1p116f);
-        q4.z = __fmul_rn(__fmul_rn(f[i + 2], 0x1p116f), 0x1p116f);
-        q4.w = __fmul_rn(__fmul_rn(f[i + 3], 0x1p116f), 0x1p116f);
-        *reinterpret_cast<float4*>(dst + gemv_e4m3_slot(8 * v + i)) = q4;
-      }
+      const uint4 h = make_uint4(e4m3x2_to_f16x2(c.x), e4m3x2_to_f16x2(c.x >> 16), e4m3x2_to_f16x2(c.y),
+                                 e4m3x2_to_f16x2(c.y >> 16));
+      *reinterpret_cast<uint4*>(gemv_smem + m * row_b + gemv_e4m3_half_off(v >> 1, v & 1)) = h;
     }
   }
   __syncthreads();
@@ -201,26 +202,25 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_e4m3_min_blocks<M>()) gemv_
         const int U = base + 32 * u;
         if (U < nu) {
           const uint32_t cw[4] = {w8[u].x, w8[u].y, w8[u].z, w8[u].w};
-          float wv[16];
+          uint32_t wh[8];   // f16 pairs of codes 2 i, 2 i + 1 of the unit
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            wv[4 * j] = e4m3_top_byte_scaled(cw[j] << 24);
-            wv[4 * j + 1] = e4m3_top_byte_scaled(cw[j] << 16);
-            wv[4 * j + 2] = e4m3_top_byte_scaled(cw[j] << 8);
-            wv[4 * j + 3] = e4m3_top_byte_scaled(cw[j]);
+            wh[2 * j] = e4m3x2_to_f16x2(cw[j]);
+            wh[2 * j + 1] = e4m3x2_to_f16x2(cw[j] >> 16);
           }
-          const int slot = (((U >> 5) * 4) << 7) + ((U & 31) << 2);
 #pragma unroll
           for (int m = 0; m < M; ++m) {
-            const float* ar = act + m * row_f + slot;
-#pragma unroll
-            for (int quad = 0; quad < 4; ++quad) {
-              const float4 a4 = *reinterpret_cast<const float4*>(ar + quad * 128);
-              acc[m] = __fmaf_rn(wv[4 * quad], a4.x, acc[m]);
-              acc[m] = __fmaf_rn(wv[4 * quad + 1], a4.y, acc[m]);
-              acc[m] = __fmaf_rn(wv[4 * quad + 2], a4.z, acc[m]);
-              acc[m] = __fmaf_rn(wv[4 * quad + 3], a4.w, acc[m]);
-            }
+            const uint8_t* ar = gemv_smem + m * row_b;
+            const uint4 a0 = *reinterpret_cast<const uint4*>(ar + gemv_e4m3_half_off(U, 0));
+            const uint4 a1 = *reinterpret_cast<const uint4*>(ar + gemv_e4m3_half_off(U, 1));
+            acc[m] = fma_f16x2_f32(wh[0], a0.x, acc[m]);
+            acc[m] = fma_f16x2_f32(wh[1], a0.y, acc[m]);
+            acc[m] = fma_f16x2_f32(wh[2], a0.z, acc[m]);
+            acc[m] = fma_f16x2_f32(wh[3], a0.w, acc[m]);
+            acc[m] = fma_f16x2_f32(wh[4], a1.x, acc[m]);
+            acc[m] = fma_f16x2_f32(wh[5], a1.y, acc[m]);
+            acc[m] = fma_f16x2_f32(wh[6], a1.z, acc[m]);
+            acc[m] = fma_f16x2_f32(wh[7], a1.w, acc[m]);
           }
         }
       }
@@ -235,8 +235,7 @@ __global__ void __launch_bounds__(kGemvThreads, gemv_e4m3_min_blocks<M>()) gemv_
 #pragma unroll
       for (int m = 1; m < M; ++m)
         if (lane == m) a = acc[m];
-      float f = __fmul_rn(a, 256.0f);   // the products carried 2^-8
-      f = __fmul_rn(__fmul_rn(f, sx[lane]), axis ? __ldg(s_col + n) : sw0);
+      float f = __fmul_rn(__fmul_rn(a, sx[lane]), axis ? __ldg(s_col + n) : sw0);
       if (bias != nullptr) f = __fadd_rn(f, __bfloat162float(bias[n]));
       if (in_bounds(static_cast<int64_t>(lane) * N + n, static_cast<int64_t>(M) * N, 0xB302))
         y[static_cast<int64_t>(lane) * N + n] = __float2bfloat16_rn(f);
