@@ -124,7 +124,8 @@ __global__ void __launch_bounds__(kGemvThreads, 4) gemv_int8_kernel(const __nv_b
 // (lane l takes units l, l + 32, ...) read 32 consecutive 16-byte words: no
 // bank conflict.
 constexpr int kGemvE4m3MaxRows = 4;
-constexpr int kGemvE4m3SmemBytes = 128 * 1024;   // M * (K rounded up to 512) * 4 (f16 needs half)
+constexpr int kGemvE4m3SmemBytes = 128 * 1024;   // the K limit: M * (K rounded up to 512) * 4 <= this
+                                                 // (the f16 activations take half)
 
 __device__ __forceinline__ int gemv_e4m3_half_off(int u, int h) {   // byte offset of half h of unit u
   return ((((u >> 5) * 2 + h) << 5) + (u & 31)) << 4;

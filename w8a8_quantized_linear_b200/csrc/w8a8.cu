@@ -760,7 +760,7 @@ static w8a8_status launch_gemv_e4m3(const void* x, int64_t M, int64_t N, int64_t
   w8a8_status s = current_device(&dev, &sms);
   if (s != W8A8_OK) return s;
   static std::atomic<uint64_t> smem_set[kGemvE4m3MaxRows] = {};
-  const size_t smem = static_cast<size_t>(M * ((K + 511) / 512) * 512 * 4);
+  const size_t smem = static_cast<size_t>(M * ((K + 511) / 512) * 512 * 2);   // f16 activations
   const int64_t reg_cap = M == 1 ? 4 : (M == 2 ? 3 : 2);   // gemv_e4m3_min_blocks
   int64_t per_sm = static_cast<int64_t>(200 * 1024) / static_cast<int64_t>(smem + 1024);
   per_sm = per_sm < 1 ? 1 : (per_sm > reg_cap ? reg_cap : per_sm);
