@@ -600,6 +600,29 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
         mbar_arrive(lr_ready);
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(lr_ready, local & 1, abort_flag, 0x600u, limit))) break;
       }
+      // Transposed form: the token scales of this warp's first chunk, the
+      // weight row's scale and its bias are loaded before the wait, so that
+      // their latency overlaps the MMAs.
+      float sx_first[32];
+      float swr = 0.0f, br = 0.0f;
+      if constexpr (EPI == kEpiScaleT) {
+        const int nc = n0 + group * 32;
+        if (nc + 32 <= N) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            const float4 f = __ldg(reinterpret_cast<const float4*>(ep.s_row + nc + j));
+            sx_first[j] = f.x; sx_first[j + 1] = f.y; sx_first[j + 2] = f.z; sx_first[j + 3] = f.w;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) sx_first[j] = (nc + j < N) ? __ldg(ep.s_row + nc + j) : 0.0f;
+        }
+        const int row = m0 + quarter * 32 + lane;   // n
+        if (row < M) {
+          swr = ep.s_col_axis ? __ldg(ep.s_col + row) : __ldg(ep.s_col);
+          if (ep.bias != nullptr) br = __bfloat162float(ep.bias[row]);
+        }
+      }
       // Every lane polls; the warp then agrees (and reconverges) before the
       // warp-collective tcgen05.ld, also when the wait ran out.
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&tfull[acc], acc_phase, abort_flag, 0x400u | acc, limit))) break;
@@ -616,15 +639,18 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
         // writing 32 consecutive n; split partial sums go to partial[split][m][n].
         const int row = m0 + quarter * 32 + lane;   // n
         const bool row_ok = row < M;
-        const float swr = row_ok ? (ep.s_col_axis ? ep.s_col[row] : ep.s_col[0]) : 0.0f;
-        const float br = (ep.bias != nullptr && row_ok) ? __bfloat162float(ep.bias[row]) : 0.0f;
   #pragma unroll 1
         for (int c = group; c < BN / 32; c += kGroups) {
           const int nc = n0 + c * 32;               // first token of the chunk
           if (nc >= N) break;                       // warp-uniform
           float sxc[32];
+          if (c == group) {
   #pragma unroll
-          for (int j = 0; j < 32; ++j) sxc[j] = (nc + j < N) ? __ldg(ep.s_row + nc + j) : 0.0f;
+            for (int j = 0; j < 32; ++j) sxc[j] = sx_first[j];
+          } else {
+  #pragma unroll
+            for (int j = 0; j < 32; ++j) sxc[j] = (nc + j < N) ? __ldg(ep.s_row + nc + j) : 0.0f;
+          }
           uint32_t r[32];
           tmem_ld_x32(tmem + lane_base + static_cast<uint32_t>(acc * BN + c * 32), r);
           tmem_ld_wait();
