@@ -100,9 +100,9 @@ struct GemmCfg {
   static constexpr int kEpiWarps = 8;   // two per TMEM lane quarter, splitting the column chunks
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
   // per epilogue warp, two 32 x 32 bf16 staging buffers for the TMA store
-  // (none in the transposed form, which stores directly)
+  // (in the transposed form a block is staged transposed)
   static constexpr int kOutBufBytes = 32 * 32 * 2;
-  static constexpr int kOutBytes = (EPI == kEpiScaleT) ? 0 : kEpiWarps * 2 * kOutBufBytes;
+  static constexpr int kOutBytes = kEpiWarps * 2 * kOutBufBytes;
   static constexpr int kFixedBytes = 1024 + ((kLrBytes + 1023) & ~1023) + kOutBytes + 256;
   static constexpr int kStagesFit = (232448 - kFixedBytes) / kStageBytes;
   // as many pipeline stages as the shared memory holds (4 for 128x256 tiles,
@@ -661,7 +661,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
                 if (nc + j < N && in_bounds((static_cast<int64_t>(split) * N + nc + j) * M + row,
                                             static_cast<int64_t>(splits) * N * M, 0xB103))
                   pcol[static_cast<int64_t>(nc + j) * M] = r[j];
-            } else {
+            } else if (!ep.tma_store) {
               for (int j = 0; j < 32; ++j) {
                 if (nc + j < N && in_bounds(static_cast<int64_t>(nc + j) * ep.ldy + row,
                                             static_cast<int64_t>(N) * ep.ldy, 0xB106)) {
@@ -672,6 +672,29 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, EPI>::kThreads, 1)
                 }
               }
             }
+          }
+          if (splits == 1 && ep.tma_store) {
+            // the 32 tokens x 32 weight rows block, staged transposed (token j's
+            // 64-byte row, this lane's column, 64-byte swizzle) and stored by
+            // TMA; rows and columns past the output are clipped by the copy
+            uint8_t* buf = sOut + e * 2 * C::kOutBufBytes + (out_iter & 1) * C::kOutBufBytes;
+            if (lane == 0) bulk_wait_read<1>();   // this buffer's previous store has read it
+            __syncwarp();
+  #pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              float a = (KIND == kKindI8) ? __int2float_rn(static_cast<int>(r[j])) : __uint_as_float(r[j]);
+              a = __fmul_rn(__fmul_rn(a, sxc[j]), swr);
+              if (ep.bias != nullptr) a = __fadd_rn(a, br);
+              const uint32_t chunk = static_cast<uint32_t>(lane >> 3) ^ static_cast<uint32_t>((j >> 1) & 3);
+              *reinterpret_cast<__nv_bfloat16*>(buf + j * 64 + (chunk << 4) + (lane & 7) * 2) = __float2bfloat16_rn(a);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmY, buf, m0 + quarter * 32, nc);
+              bulk_commit();
+            }
+            ++out_iter;
           }
         }
       } else {

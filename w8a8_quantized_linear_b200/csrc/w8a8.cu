@@ -168,13 +168,10 @@ template <int KIND, bool B_MN, int BN, int EPI>
 w8a8_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, int64_t M, int64_t N, int64_t Kc,
                         EpiParams ep, cudaStream_t st) {
   alignas(64) CUtensorMap ty;
-  if constexpr (EPI == kEpiScaleT) {   // direct transposed stores, no output map
-    std::memset(&ty, 0, sizeof(ty));
-    ep.tma_store = 0;
-  } else {
-    w8a8_status ms = make_out_map(&ty, &ep, M, N);
-    if (ms != W8A8_OK) return ms;
-  }
+  // the transposed form's rows are y's columns (weight rows) and its columns
+  // y's rows (tokens)
+  w8a8_status ms = (EPI == kEpiScaleT) ? make_out_map(&ty, &ep, N, M) : make_out_map(&ty, &ep, M, N);
+  if (ms != W8A8_OK) return ms;
   using C = GemmCfg<KIND, BN, EPI>;
   static std::atomic<uint64_t> smem_set{0};
   int dev = 0, sms = 0;
