@@ -58,7 +58,10 @@ def test_sizes(L):
     assert L.w8a8_workspace_bytes(1, 3, 40, 16, 0) == 256 + 256  # N padded to 48 -> 144 bytes
     # SVDQuant: codes, row scales, T [M, r] bf16, then T's split-K partial sums
     # (36 row tiles over a 3072-long contraction: 4 splits, [4, 4608, 32] fp32)
-    assert L.w8a8_workspace_bytes(2, 4608, 3072, 3072, 32) == 4608 * 3072 + 4608 * 4 + 4608 * 32 * 2 + 4 * 4608 * 32 * 4
+    # SVDQuant: rows of up to 3072 take the one-pass input kernel (no split
+    # partial sums); longer rows the split T product (4 splits at 4608 rows)
+    assert L.w8a8_workspace_bytes(2, 4608, 3072, 3072, 32) == 4608 * 3072 + 4608 * 4 + 4608 * 32 * 2
+    assert L.w8a8_workspace_bytes(2, 4608, 3072, 6144, 32) == 4608 * 6144 + 4608 * 4 + 4608 * 32 * 2 + 4 * 4608 * 32 * 4
     assert L.w8a8_workspace_bytes(2, 200, 320, 256, 32) == 200 * 256 + 1024 + 200 * 32 * 2   # unsplit
     assert L.w8a8_workspace_bytes(3, 10, 10, 16, 0) == 256
     # few output tiles, long contraction: split-K partial sums follow

@@ -429,13 +429,14 @@ int t_splits(int64_t M, int64_t K) {
   return s < 2 ? 1 : static_cast<int>(s);
 }
 // Workspace of svdq_linear_fwd: codes [M, K], row scales [M], T [M, r]
-// bf16, then T's split-K partial sums [S, M, r] fp32 when split.
+// bf16, then T's split-K partial sums [S, M, r] fp32 when split (rows longer
+// than the one-pass input kernel takes).
 size_t ws_svdq(int64_t M, int64_t K, int r) {
   Carve c(nullptr);
   c.take(static_cast<size_t>(M * K));
   c.take(static_cast<size_t>(M) * 4);
   c.take(static_cast<size_t>(M) * r * 2);
-  const int s = t_splits(M, K);
+  const int s = K <= kSiMaxK ? 1 : t_splits(M, K);
   if (s > 1) c.take(static_cast<size_t>(s) * static_cast<size_t>(M) * static_cast<size_t>(r) * 4);
   return c.off;
 }
